@@ -1,0 +1,425 @@
+"""Benchmark: streaming block-causal sink + sliding-window attention at 720p on B200.
+
+One step = one steady-state chunk of the 720p stream: two denoise-step forwards (attention of
+the chunk's 3180 queries over condition + sink + window + current keys) and the commit of the
+chunk into the ring cache (append/evict copy + visibility-table rebuild).  The metric is the
+attention TFLOP/s over the timed steps (algorithmic FLOPs: 4 * B * H * T * N_vis * d per
+forward, visible keys only), with ms per chunk and the fraction of the measured dense bf16 peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference] [--config 720p]
+
+Under torchrun (N > 1) every rank runs an independent replica (the path has no exchange step);
+the time is the max over ranks and the value sums all ranks' FLOPs.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from block_causal_attention_sliding_b200 import synth  # noqa: E402
+from block_causal_attention_sliding_b200.configs import WORKLOADS  # noqa: E402
+
+METRIC = "attention TFLOP/s and ms/chunk at 720p, % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            uuid = None
+        self.target = uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.target:
+            cmd += ["-i", self.target]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ---------------------------------------------------------------------------- distributed plumbing
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _init_dist(world, backend="nccl"):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max_time(dist, seconds: float, device) -> float:
+    """Max over ranks of a device-timed interval (seconds)."""
+    if dist is None:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index] if device.type == "cuda" else None)
+
+
+# ---------------------------------------------------------------------------- CPU baseline (oracle)
+
+def cpu_baseline(wl, k: int, rows: int, repeats: int = 1):
+    """Time the FP64 oracle on a bounded sample of one steady-state forward: `rows` query rows
+    for every head, over all visible keys.  Returns (TFLOP/s, seconds, flops, threads)."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    Kc, Vc = synth.cond_inputs(wl)
+    hist_K = [None] * k
+    hist_V = [None] * k
+    vis = [c for c in range(k) if oracle.visible(k, wl.W, wl.sink, c)]
+    for c in vis:
+        _, K, V = synth.chunk_inputs(wl, c, wl.steps - 1)
+        hist_K[c], hist_V[c] = K, V
+    Q, K, V = synth.chunk_inputs(wl, k, 0)
+    sel = np.linspace(0, wl.T - 1, rows).astype(np.int32)
+    nvis = wl.n_vis(k)
+    flops = 4.0 * wl.B * wl.H * rows * nvis * wl.d
+    best = None
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink, k=k, Kc=Kc, Vc=Vc,
+                         hist_K=hist_K, hist_V=hist_V, Q=Q, K_cur=K, V_cur=V, rows=sel)
+        dt = time.perf_counter() - t0
+        best = dt if best is None else min(best, dt)
+    return flops / best / 1e12, best, flops, oracle.num_threads()
+
+
+# ---------------------------------------------------------------------------- the CUDA arm
+
+def run_cuda(args, wl, world, rank, local):
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+
+    dist = _init_dist(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = _peaks()
+
+    h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                               out_dtype=torch.bfloat16, device=dev)
+    Kc, Vc = synth.cond_inputs(wl, seed=rank, device=dev)
+    h.set_cond(Kc, Vc)
+    # a pool of distinct input sets, resident in HBM; together with the 160 MB cache the
+    # working set of every step is far larger than the 126 MB L2
+    pool = []
+    for i in range(args.pool):
+        per_step = [synth.chunk_inputs(wl, 1000 + i, s, seed=rank, device=dev) for s in range(wl.steps)]
+        pool.append(per_step)
+    outs = [torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev) for _ in range(wl.steps)]
+
+    def step(i, ev=None):
+        inputs = pool[i % len(pool)]
+        for s, (Q, K, V) in enumerate(inputs):
+            if ev is not None:
+                ev[2 * s].record(stream)
+            h.forward(Q, K, V, out=outs[s])
+            if ev is not None:
+                ev[2 * s + 1].record(stream)
+        Q, K, V = inputs[-1]
+        h.append_chunk(K, V)
+
+    # reach the steady state (sink + full window visible), untimed
+    for i in range(wl.steady_k()):
+        step(i)
+    k_start = wl.steady_k()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert h.status() == 0
+
+    # timed region: K steps, per-forward events for the attention kernel's own time
+    fwd_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * wl.steps)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(i, fwd_events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(dist, dev)
+    elapsed = start.elapsed_time(end) / 1e3
+    t_max = reduce_max_time(dist, elapsed, dev)
+    fwd_ms = [fwd_events[i][2 * s].elapsed_time(fwd_events[i][2 * s + 1])
+              for i in range(args.steps) for s in range(wl.steps)]
+    status = h.status()
+
+    flops_fwd = wl.flops_forward(k_start)
+    flops_step = wl.steps * flops_fwd
+    total_flops = flops_step * args.steps * world
+    value = total_flops / t_max / 1e12
+    fwd_avg = sum(fwd_ms) / len(fwd_ms) / 1e3
+    achieved = flops_fwd / fwd_avg / 1e12
+
+    # ---- e2e: the same steps through the public API with host buffers (pinned), copies timed
+    host_in = [[t.cpu().pin_memory() for t in per_step] for per_step in pool[0]]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    dev_in = [[torch.empty_like(t) for t in per_step] for per_step in pool[0]]
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        for s in range(wl.steps):
+            for dst, src in zip(dev_in[s], host_in[s]):
+                dst.copy_(src, non_blocking=True)
+            Q, K, V = dev_in[s]
+            h.forward(Q, K, V, out=outs[s])
+            host_out[s].copy_(outs[s], non_blocking=True)
+        h.append_chunk(dev_in[-1][1], dev_in[-1][2])
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_t = reduce_max_time(dist, e0.elapsed_time(e1) / 1e3, dev)
+    bi = sum(t.numel() * t.element_size() for per_step in host_in for t in per_step)
+    bo = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_value = flops_step * e2e_steps * world / e2e_t / 1e12
+
+    # ---- side measurements (untimed for the metric): append/evict and the split-K path
+    paths = {}
+    if rank == 0:
+        paths = side_paths(h, wl, pool, dev, stream, peaks)
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline:
+            try:
+                v, secs, fl, thr = cpu_baseline(wl, k_start, rows=args.cpu_rows)
+                cpu = {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
+                       "sample": f"FP64 oracle, one steady-state forward (k={k_start}), {args.cpu_rows} query "
+                                 f"rows x {wl.H} heads over all {wl.n_vis(k_start)} visible keys "
+                                 f"({fl / 1e9:.2f} GFLOP in {secs:.2f} s)"}
+            except Exception as e:   # the baseline never blocks the GPU line
+                cpu = {"value": None, "unit": UNIT, "cores": None, "kind": "oracle", "sample": f"failed: {e}"}
+        peak = peaks["bf16_tflops"]
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_max / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "d": wl.d, "T": wl.T, "n_cond": wl.n_cond,
+                       "W": wl.W, "sink": wl.sink, "N_vis": wl.n_vis(k_start),
+                       "step": "one steady-state chunk: 2 forwards + append/evict + table",
+                       "gflop_per_forward": round(flops_fwd / 1e9, 2),
+                       "l2": f"inputs larger than L2: {len(pool)} resident input sets of "
+                             f"{sum(t.numel() * 2 for t in pool[0][0]) * wl.steps / 2 ** 20:.0f} MiB plus the "
+                             f"{h.workspace_bytes() / 2 ** 20:.0f} MiB cache, cycled per step",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "pct_of_peak": round(100.0 * value / world / peak, 2),
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,2>", "achieved": round(achieved, 2),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": None, "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                         "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                         "launch_ms_avg": round(fwd_avg * 1e3, 4)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                    "steps": e2e_steps, "ms_per_step": round(e2e_t / e2e_steps * 1e3, 4)},
+            "gpu_launches": args.steps * (wl.steps + 2),
+            "clocks": clk,
+            "device_status": status,
+            "paths": paths,
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def side_paths(h, wl, pool, dev, stream, peaks):
+    """Append/evict (HBM-bound copy) and the split-K short-query path, timed alone."""
+    out = {}
+    reps = 50
+    Q, K, V = pool[0][-1]
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        h.append_chunk(K, V)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    nbytes = 2 * 2 * K.numel() * K.element_size()          # K and V, read + write
+    out["append"] = {"us": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
+                     "frac_hbm": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 3), "bytes": nbytes,
+                     "note": "includes the table-build launch"}
+    k = wl.steady_k()
+    nvis = wl.n_vis(k)
+    dec = {}
+    for nq in (16, 64, 128):
+        q = Q[:, :nq].contiguous()
+        o = torch.empty((wl.B, nq, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            h.forward(q, K, V, out=o)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            h.forward(q, K, V, out=o)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        kv_bytes = 2 * wl.B * wl.H * nvis * wl.d * 2
+        dec[str(nq)] = {"us": round(t * 1e6, 2), "GB/s": round(kv_bytes / t / 1e9, 1),
+                        "frac_hbm": round(kv_bytes / t / 1e9 / peaks["hbm_gbs"], 3)}
+    out["split_k"] = dec
+    return out
+
+
+# ---------------------------------------------------------------------------- the reference arm
+
+def run_reference(args, wl, world, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded sample of the same
+    workload (a few query rows of one steady-state forward, all heads, all visible keys)."""
+    if rank != 0:
+        return
+    k = wl.steady_k()
+    for _ in range(args.warmup):
+        cpu_baseline(wl, k, rows=2)
+    t_total, fl_total, thr = 0.0, 0.0, 1
+    for _ in range(args.steps):
+        v, secs, fl, thr = cpu_baseline(wl, k, rows=args.ref_rows)
+        t_total += secs
+        fl_total += fl
+    value = fl_total / t_total / 1e12
+    full_step = wl.steps * wl.flops_forward(k)
+    ms_per_chunk = full_step / (fl_total / t_total) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_chunk, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "d": wl.d, "T": wl.T, "n_cond": wl.n_cond,
+                   "W": wl.W, "sink": wl.sink, "N_vis": wl.n_vis(k),
+                   "note": "ms_per_step extrapolated from the sampled rows to a full chunk"},
+        "cpu_baseline": {"kind": "oracle", "cores": thr, "value": value, "unit": UNIT,
+                         "sample": f"per step {args.ref_rows} query rows x {wl.H} heads of one steady-state "
+                                   f"forward over {wl.n_vis(k)} keys"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--config", default="720p", choices=sorted(WORKLOADS))
+    ap.add_argument("--pool", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.config]
+    world, rank, local = _dist_env()
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        sys.exit(1)
+    run_cuda(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

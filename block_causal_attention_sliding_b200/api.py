@@ -1,0 +1,131 @@
+"""Python face of libswattn: one handle = one layer's bounded KV cache on one GPU.
+
+PyTorch provides the device memory (the workspace and the caller's tensors) and the stream;
+the library's kernels do every step of the computation.  Calls enqueue on the current torch
+stream and never synchronise, so a chunk step can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native as N
+
+
+def _stream_ptr(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return int(t.data_ptr())
+
+
+class SlidingWindowAttention:
+    """Streaming block-causal attention over [condition ; sink ; window ; current chunk]."""
+
+    def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
+                 sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
+                 max_short_q: int = 0, device=None):
+        self._lib = N.lib()
+        cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
+                             sink=int(bool(sink)),
+                             out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
+                             scale=0.0 if scale is None else float(scale), max_short_q=max_short_q)
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+        h = ctypes.c_void_p()
+        N.check(self._lib.sw_attn_create_ex(ctypes.byref(cfg), ctypes.byref(h)))
+        self._h = h
+        self.B, self.H, self.d, self.T, self.W, self.n_cond, self.sink = B, H, d, T, W, n_cond, bool(sink)
+        self.out_dtype = out_dtype
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        nbytes = int(self._lib.sw_attn_workspace_bytes(h))
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            N.check(self._lib.sw_attn_bind_workspace(h, self.workspace.data_ptr(), nbytes, _stream_ptr()))
+        self.table_ints = int(self._lib.sw_attn_table_ints(h))
+
+    # -- stream control
+    def set_cond(self, K_cond: torch.Tensor, V_cond: torch.Tensor, stream=None) -> None:
+        shape = (self.B, self.n_cond, self.H, self.d)
+        for name, t in (("K_cond", K_cond), ("V_cond", V_cond)):
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        N.check(self._lib.sw_attn_set_cond(self._h, _dev_ptr(K_cond, "K_cond", torch.bfloat16),
+                                           _dev_ptr(V_cond, "V_cond", torch.bfloat16), _stream_ptr(stream)))
+
+    def append_chunk(self, K: torch.Tensor, V: torch.Tensor, stream=None) -> None:
+        shape = (self.B, self.T, self.H, self.d)
+        for name, t in (("K", K), ("V", V)):
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        N.check(self._lib.sw_attn_append_chunk(self._h, _dev_ptr(K, "K", torch.bfloat16),
+                                               _dev_ptr(V, "V", torch.bfloat16), _stream_ptr(stream)))
+
+    def forward(self, Q: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if Q.dim() != 4 or Q.shape[0] != self.B or Q.shape[2] != self.H or Q.shape[3] != self.d:
+            raise ValueError(f"Q must be [B, n_q, H, d] = [{self.B}, n_q, {self.H}, {self.d}]")
+        n_q = int(Q.shape[1])
+        kv_shape = (self.B, self.T, self.H, self.d)
+        for name, t in (("K_cur", K_cur), ("V_cur", V_cur)):
+            if tuple(t.shape) != kv_shape:
+                raise ValueError(f"{name} must have shape {kv_shape}, got {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty((self.B, n_q, self.H, self.d), dtype=self.out_dtype, device=Q.device)
+        elif tuple(out.shape) != tuple(Q.shape) or out.dtype != self.out_dtype:
+            raise ValueError("out must match Q's shape and the handle's out_dtype")
+        N.check(self._lib.sw_attn_forward(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
+                                          _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+                                          _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                          _dev_ptr(out, "out"), n_q, _stream_ptr(stream)))
+        return out
+
+    __call__ = forward
+
+    def reset(self, stream=None) -> None:
+        N.check(self._lib.sw_attn_reset(self._h, _stream_ptr(stream)))
+
+    # -- inspection
+    def table(self, stream=None) -> torch.Tensor:
+        t = torch.empty(self.table_ints, dtype=torch.int32, device=self.device)
+        N.check(self._lib.sw_attn_get_table(self._h, t.data_ptr(), _stream_ptr(stream)))
+        return t
+
+    def status(self) -> int:
+        v = ctypes.c_int32(0)
+        N.check(self._lib.sw_attn_get_status(self._h, ctypes.byref(v)))
+        return int(v.value)
+
+    def workspace_bytes(self) -> int:
+        return int(self._lib.sw_attn_workspace_bytes(self._h))
+
+    def cache_views(self):
+        """(K_cache, V_cache) as [B, H, S, T, d] bf16 views of the workspace (for inspection)."""
+        S = self.W + (1 if self.sink else 0)
+        ko, vo = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        N.check(self._lib.sw_attn_cache_offsets(self._h, ctypes.byref(ko), ctypes.byref(vo)))
+        n = 2 * self.B * self.H * S * self.T * self.d
+        shape = (self.B, self.H, S, self.T, self.d)
+        kc = self.workspace[ko.value: ko.value + n].view(torch.bfloat16).view(shape)
+        vc = self.workspace[vo.value: vo.value + n].view(torch.bfloat16).view(shape)
+        return kc, vc
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sw_attn_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,124 @@
+// cache_kernels.cu -- the bounded KV cache: visibility/slot table builder and the
+// append/evict copy into the ring buffer.
+//
+// The cache keeps the condition tokens, a pinned first chunk (global sink) and the W most
+// recent chunks; a finished chunk's clean K/V are written into it right after the chunk
+// completes, so memory and per-chunk work stay constant (agifrontier tutorial "JoyAI-Video-
+// Edit：单卡720p 30帧，两步蒸馏攻克流式视频编辑", sections "从双向编辑到分块因果架构的蜕变" and
+// "软硬件协同部署"; neurohive review "JoyAI-Video-Edit", section "Чанки и борьба с дрейфом").
+#include "swattn_internal.h"
+
+namespace swattn {
+
+// Ring slot of committed chunk c: the sink owns slot 0; window chunks rotate through the
+// remaining W slots, so chunk c lands where chunk c - W (the one leaving the window) was.
+__device__ __forceinline__ int ring_slot(int c, int W, int sink) {
+    if (sink) {
+        if (c == 0) return 0;
+        return W > 0 ? 1 + (c - 1) % W : -1;
+    }
+    return W > 0 ? c % W : -1;
+}
+
+// K1: advance the counter (after an append) and write the visibility table of the active
+// chunk k: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...], in the order
+// condition, sink, window ascending, current.  One thread: a few dozen integers.
+__global__ void table_build_kernel(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+                                   int reset) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int32_t* tab = state + kStateHeaderInts;
+    if (reset) {
+        state[0] = 0;
+        state[1] = 0;
+    }
+    int k = state[0];
+    if (advance) {
+        if (k >= (1 << 30)) {
+            state[1] |= SW_STATUS_OVERFLOW;
+        } else {
+            k += 1;
+            state[0] = k;
+        }
+    }
+    const int cap = table_ints_for(W);
+    int pos = 3, nseg = 0, nvis = 0;
+    auto put = [&](int kind, int chunk, int slot, int n) {
+        tab[pos++] = kind; tab[pos++] = chunk; tab[pos++] = slot; tab[pos++] = n;
+        ++nseg; nvis += n;
+    };
+    if (n_cond > 0) put(0, -1, -1, n_cond);
+    const int first_win = k - W > 0 ? k - W : 0;
+    if (sink && k >= 1 && first_win > 0) put(1, 0, 0, T);      // sink outside the window
+    for (int j = first_win; j < k; ++j) put(1, j, ring_slot(j, W, sink), T);
+    put(2, k, -1, T);
+    tab[0] = k; tab[1] = nseg; tab[2] = nvis;
+    for (int i = pos; i < cap; ++i) tab[i] = -1;
+}
+
+cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+                               cudaStream_t stream) {
+    table_build_kernel<<<1, 32, 0, stream>>>(state, W, sink, n_cond, T, advance, 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
+                               cudaStream_t stream) {
+    table_build_kernel<<<1, 32, 0, stream>>>(state, W, sink, n_cond, T, 0, 1);
+    return cudaGetLastError();
+}
+
+// K2: copy K and V of one chunk from the user layout [B, N, H, d] into the head-major cache
+// layout [B][H][rows_per_bh][d] at row offset slot * N.  One thread moves 16 bytes; threads
+// run over the source in order (coalesced 16-byte loads), and each group of d/8 threads
+// writes one contiguous d-row of the destination (coalesced 16-byte stores).
+__global__ void __launch_bounds__(256) relayout_kernel(const uint4* __restrict__ srcK,
+                                                       const uint4* __restrict__ srcV,
+                                                       uint4* __restrict__ dstK,
+                                                       uint4* __restrict__ dstV, int B, int N,
+                                                       int H, int vec_per_row, int rows_per_bh,
+                                                       int ring, int W, int sink, int S,
+                                                       int32_t* state) {
+    int slot = 0;
+    if (ring) {
+        slot = ring_slot(state[0], W, sink);
+        if (slot < 0) return;                 // W = 0: nothing is kept for this chunk
+        if (slot >= S) {                      // cannot happen; recorded, never trapped
+            if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+                atomicOr(state + 1, SW_STATUS_BAD_SLOT);
+            return;
+        }
+    }
+    const uint4* __restrict__ src = blockIdx.y == 0 ? srcK : srcV;
+    uint4* __restrict__ dst = blockIdx.y == 0 ? dstK : dstV;
+    const long long total = (long long)B * N * H * vec_per_row;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int v = (int)(i % vec_per_row);
+        long long r = i / vec_per_row;              // source row index over (b, t, h)
+        const int h = (int)(r % H);
+        r /= H;
+        const int t = (int)(r % N);
+        const int b = (int)(r / N);
+        const long long drow = ((long long)b * H + h) * rows_per_bh + (long long)slot * N + t;
+        dst[drow * vec_per_row + v] = __ldg(src + i);
+    }
+}
+
+cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
+                            int H, int d, int rows_per_bh, int ring, int W, int sink, int S,
+                            int32_t* state, cudaStream_t stream) {
+    const int vec_per_row = d / 8;
+    const long long total = (long long)B * N * H * vec_per_row;
+    long long blocks = (total + 255) / 256;
+    // enough blocks to fill the GPU several times over, grid-stride beyond that
+    const long long cap = 148LL * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    dim3 grid((unsigned)blocks, 2);
+    relayout_kernel<<<grid, 256, 0, stream>>>(
+        static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
+        static_cast<uint4*>(dstV), B, N, H, vec_per_row, rows_per_bh, ring, W, sink, S, state);
+    return cudaGetLastError();
+}
+
+}  // namespace swattn

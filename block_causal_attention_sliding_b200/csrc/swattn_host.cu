@@ -1,0 +1,332 @@
+// swattn_host.cu -- the C ABI: argument checks, workspace layout, TMA tensor maps, launches.
+//
+// Calls only enqueue work on the caller's stream (no synchronisation, no allocation), so a
+// chunk step can be captured in a CUDA graph; the chunk counter and the visibility table
+// live on the device for the same reason.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "swattn_internal.h"
+
+using namespace swattn;
+
+struct sw_attn {
+    sw_attn_config cfg;
+    int S = 0;                 // ring slots = W + sink
+    int table_ints = 0;
+    int max_splits = 1;
+    int short_q = 0;           // n_q <= short_q uses the split-K path (0: never)
+    size_t off_kcache = 0, off_vcache = 0, off_kcond = 0, off_vcond = 0, off_opart = 0, off_ml = 0;
+    size_t total = 0;
+    char* ws = nullptr;
+    size_t ws_bytes = 0;
+    int device = -1;
+    int num_sms = 148;
+    bool cond_set = false;
+    CUtensorMap tm_cache_k, tm_cache_v, tm_cond_k, tm_cond_v;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(SW_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// bf16 tiled map, 128-byte swizzle, boxes of 64 columns; out-of-range rows read as zero.
+int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
+           const uint32_t* box, const char* what) {
+    auto fn = encode_fn();
+    if (!fn) return fail(SW_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    uint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr),
+                    reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides),
+                    reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SW_ECUDA, "tensor map for %s: CUresult %d", what, (int)r);
+    return SW_OK;
+}
+
+// user layout [B, N, H, d]: dims {d, H, N, B}; box 64 x 1 x 128 x 1 (128 rows of one head)
+int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, const char* what) {
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)N * H * d * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)kBlockN, 1};
+    return encode(m, ptr, 4, dims, strides, box, what);
+}
+
+int check_cfg(const sw_attn_config& c) {
+    if (c.B < 1 || c.H < 1) return fail(SW_ESHAPE, "B and H must be >= 1 (B=%d H=%d)", c.B, c.H);
+    if (c.d != 64 && c.d != 128) return fail(SW_ESHAPE, "d must be 64 or 128 (d=%d)", c.d);
+    if (c.tokens_per_chunk < 1) return fail(SW_ESHAPE, "tokens_per_chunk must be >= 1");
+    if (c.W < 0 || c.W > kMaxW) return fail(SW_ESHAPE, "W must be in [0, %d] (W=%d)", kMaxW, c.W);
+    if (c.n_cond < 0) return fail(SW_ESHAPE, "n_cond must be >= 0");
+    if (c.sink != 0 && c.sink != 1) return fail(SW_EINVAL, "sink must be 0 or 1");
+    if (c.out_dtype != SW_OUT_BF16 && c.out_dtype != SW_OUT_F32) return fail(SW_EINVAL, "bad out_dtype");
+    if (c.max_short_q > kMaxShortQ) return fail(SW_ESHAPE, "max_short_q must be <= %d", kMaxShortQ);
+    if (!std::isfinite(c.scale)) return fail(SW_EINVAL, "scale must be finite");
+    const double elems = (double)c.B * c.H * (c.W + 1) * c.tokens_per_chunk * c.d;
+    if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
+        (double)c.n_cond * c.H * c.B > 2.0e9)
+        return fail(SW_ESHAPE, "problem too large");
+    return SW_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sw_attn_last_error(void) { return g_err.c_str(); }
+
+int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
+    g_err.clear();
+    if (!cfg || !out) return fail(SW_EINVAL, "null argument");
+    *out = nullptr;
+    int rc = check_cfg(*cfg);
+    if (rc) return rc;
+    sw_attn* h = new (std::nothrow) sw_attn();
+    if (!h) return fail(SW_EINVAL, "out of host memory");
+    h->cfg = *cfg;
+    if (h->cfg.scale <= 0.f) h->cfg.scale = 1.0f / std::sqrt((float)cfg->d);
+    h->short_q = cfg->max_short_q == 0 ? kMaxShortQ : (cfg->max_short_q < 0 ? 0 : cfg->max_short_q);
+    h->S = cfg->W + (cfg->sink ? 1 : 0);
+    h->table_ints = table_ints_for(cfg->W);
+    const int bh = cfg->B * cfg->H;
+    h->max_splits = std::max(1, std::min(kMaxSplits, (148 + bh - 1) / bh));   // B200: 148 SMs
+    const size_t B = cfg->B, H = cfg->H, d = cfg->d, T = cfg->tokens_per_chunk;
+    size_t off = align_up(sizeof(int32_t) * (kStateHeaderInts + h->table_ints), 1024);
+    h->off_kcache = off; off = align_up(off + B * H * h->S * T * d * 2, 1024);
+    h->off_vcache = off; off = align_up(off + B * H * h->S * T * d * 2, 1024);
+    h->off_kcond = off;  off = align_up(off + B * H * cfg->n_cond * d * 2, 1024);
+    h->off_vcond = off;  off = align_up(off + B * H * cfg->n_cond * d * 2, 1024);
+    h->off_opart = off;
+    if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * d * 4, 1024);
+    h->off_ml = off;
+    if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * 2 * 4, 1024);
+    h->total = off;
+    *out = h;
+    return SW_OK;
+}
+
+int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_attn_t** out) {
+    sw_attn_config c;
+    std::memset(&c, 0, sizeof c);
+    c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
+    c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0;
+    return sw_attn_create_ex(&c, out);
+}
+
+size_t sw_attn_workspace_bytes(const sw_attn_t* h) { return h ? h->total : 0; }
+
+int sw_attn_table_ints(const sw_attn_t* h) { return h ? h->table_ints : 0; }
+
+void sw_attn_destroy(sw_attn_t* h) { delete h; }
+
+int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stream) {
+    g_err.clear();
+    if (!h || !dev_ptr) return fail(SW_EINVAL, "null argument");
+    if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u) return fail(SW_EALIGN, "workspace must be 256-byte aligned");
+    if (bytes < h->total) return fail(SW_ESHAPE, "workspace too small: %zu < %zu", bytes, h->total);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    const sw_attn_config& c = h->cfg;
+    char* ws = static_cast<char*>(dev_ptr);
+    int rc;
+    if (h->S > 0) {
+        // ring [B][H][S][T][d]: dims {d, T, S, H, B}; rows past T read as zero
+        const uint64_t dims[5] = {(uint64_t)c.d, (uint64_t)c.tokens_per_chunk, (uint64_t)h->S, (uint64_t)c.H,
+                                  (uint64_t)c.B};
+        const uint64_t row = (uint64_t)c.d * 2;
+        const uint64_t strides[4] = {row, row * c.tokens_per_chunk, row * c.tokens_per_chunk * h->S,
+                                     row * c.tokens_per_chunk * h->S * c.H};
+        const uint32_t box[5] = {64, (uint32_t)kBlockN, 1, 1, 1};
+        if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, strides, box, "K cache"))) return rc;
+        if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, strides, box, "V cache"))) return rc;
+    }
+    if (c.n_cond > 0) {
+        const uint64_t dims[4] = {(uint64_t)c.d, (uint64_t)c.n_cond, (uint64_t)c.H, (uint64_t)c.B};
+        const uint64_t row = (uint64_t)c.d * 2;
+        const uint64_t strides[3] = {row, row * c.n_cond, row * c.n_cond * c.H};
+        const uint32_t box[4] = {64, (uint32_t)kBlockN, 1, 1};
+        if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, strides, box, "K cond"))) return rc;
+        if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, strides, box, "V cond"))) return rc;
+    }
+    e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, c.sink, c.n_cond, c.tokens_per_chunk,
+                           static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state reset launch");
+    h->ws = ws;
+    h->ws_bytes = bytes;
+    h->device = dev;
+    h->num_sms = sms;
+    h->cond_set = c.n_cond == 0;
+    return SW_OK;
+}
+
+int sw_attn_reset(sw_attn_t* h, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    const sw_attn_config& c = h->cfg;
+    cudaError_t e = launch_state_reset(reinterpret_cast<int32_t*>(h->ws), c.W, c.sink, c.n_cond,
+                                       c.tokens_per_chunk, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "state reset launch");
+}
+
+int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    const sw_attn_config& c = h->cfg;
+    if (c.n_cond == 0) return SW_OK;
+    if (!K_cond || !V_cond) return fail(SW_EINVAL, "null condition tensor");
+    if (!aligned16(K_cond) || !aligned16(V_cond)) return fail(SW_EALIGN, "condition tensors must be 16-byte aligned");
+    cudaError_t e = launch_relayout(K_cond, V_cond, h->ws + h->off_kcond, h->ws + h->off_vcond, c.B, c.n_cond,
+                                    c.H, c.d, c.n_cond, 0, c.W, c.sink, h->S, reinterpret_cast<int32_t*>(h->ws),
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "condition copy launch");
+    h->cond_set = true;
+    return SW_OK;
+}
+
+int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (!K || !V) return fail(SW_EINVAL, "null K or V");
+    if (!aligned16(K) || !aligned16(V)) return fail(SW_EALIGN, "K and V must be 16-byte aligned");
+    const sw_attn_config& c = h->cfg;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    cudaError_t e;
+    if (h->S > 0) {
+        e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
+                            h->S * c.tokens_per_chunk, 1, c.W, c.sink, h->S, state, st);
+        if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    }
+    e = launch_table_build(state, c.W, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
+}
+
+int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out, int n_q,
+                    void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
+    if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
+    const sw_attn_config& c = h->cfg;
+    if (n_q < 1 || n_q > c.tokens_per_chunk)
+        return fail(SW_ESHAPE, "n_q must be in [1, %d] (n_q=%d)", c.tokens_per_chunk, n_q);
+    if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
+        return fail(SW_EALIGN, "Q, K_cur, V_cur and out must be 16-byte aligned");
+    AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    int rc;
+    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
+    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
+    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
+    // maps for regions this handle does not have are never read; fill them with a valid map
+    p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
+    p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
+    p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
+    p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    p.out = out;
+    p.table = state + kStateHeaderInts;
+    p.status = state + 1;
+    p.B = c.B;
+    p.H = c.H;
+    p.n_q = n_q;
+    p.out_f32 = c.out_dtype == SW_OUT_F32;
+    p.scale_log2 = c.scale * 1.4426950408889634f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (n_q <= h->short_q) {
+        const int bh = c.B * c.H;
+        int splits = h->num_sms / bh;
+        splits = std::max(1, std::min(splits, h->max_splits));
+        p.splits = splits;
+        p.o_part = reinterpret_cast<float*>(h->ws + h->off_opart);
+        p.ml_part = reinterpret_cast<float*>(h->ws + h->off_ml);
+        e = launch_attention(p, c.d, 1, splits, st);
+        if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
+        e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
+        if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    } else {
+        p.splits = 0;
+        const int grid_x = (n_q + 2 * kBlockM - 1) / (2 * kBlockM);
+        e = launch_attention(p, c.d, 2, grid_x, st);
+        if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    }
+    return SW_OK;
+}
+
+int sw_attn_get_table(const sw_attn_t* h, int32_t* dev_table, void* stream) {
+    g_err.clear();
+    if (!h || !dev_table) return fail(SW_EINVAL, "null argument");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    cudaError_t e = cudaMemcpyAsync(dev_table, h->ws + sizeof(int32_t) * kStateHeaderInts,
+                                    sizeof(int32_t) * h->table_ints, cudaMemcpyDeviceToDevice,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "table copy");
+}
+
+int sw_attn_cache_offsets(const sw_attn_t* h, size_t* k_offset, size_t* v_offset) {
+    g_err.clear();
+    if (!h || !k_offset || !v_offset) return fail(SW_EINVAL, "null argument");
+    *k_offset = h->off_kcache;
+    *v_offset = h->off_vcache;
+    return SW_OK;
+}
+
+int sw_attn_get_status(sw_attn_t* h, int32_t* host_status) {
+    g_err.clear();
+    if (!h || !host_status) return fail(SW_EINVAL, "null argument");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    e = cudaMemcpy(host_status, h->ws + sizeof(int32_t), sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "status copy");
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// swattn_internal.h -- shared between the C-ABI host code and the kernel launchers.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "swattn.h"
+
+namespace swattn {
+
+constexpr int kBlockM = 128;       // query rows per Q tile (MMA M)
+constexpr int kBlockN = 128;       // keys per K/V tile (MMA N of QK^T, K of PV)
+constexpr int kMaxW = 64;          // largest window supported
+constexpr int kStateHeaderInts = 16;   // [0] chunks committed, [1] status bits, rest reserved
+constexpr int kMaxShortQ = 128;    // split-K path handles one Q tile per (b, h)
+constexpr int kMaxSplits = 64;
+
+__host__ __device__ inline int table_ints_for(int W) { return 3 + 4 * (W + 3); }
+
+// Device-side state layout: int32 words at the start of the workspace.
+//   state[0] = chunks committed (= index k of the active chunk)
+//   state[1] = status bits (SW_STATUS_*)
+//   state[kStateHeaderInts ...] = visibility table (table_ints_for(W) entries)
+
+// Everything a launch of the attention kernel needs.  Passed by value as a __grid_constant__
+// parameter, so the tensor maps live in parameter space as TMA requires.
+struct alignas(64) AttnParams {
+    CUtensorMap tm_q;        // Q       [B, n_q, H, d]   dims {d, H, n_q, B}
+    CUtensorMap tm_kcur;     // K_cur   [B, T, H, d]     dims {d, H, T, B}
+    CUtensorMap tm_vcur;     // V_cur
+    CUtensorMap tm_cache_k;  // K ring  [B][H][S][T][d]  dims {d, T, S, H, B}
+    CUtensorMap tm_cache_v;
+    CUtensorMap tm_cond_k;   // K cond  [B][H][n_cond][d] dims {d, n_cond, H, B}
+    CUtensorMap tm_cond_v;
+    void* out;               // [B, n_q, H, d] bf16 or f32 (full mode)
+    float* o_part;           // split mode: [splits][B*H][kBlockM][d] unnormalised fp32
+    float* ml_part;          // split mode: [splits][B*H][kBlockM][2] (row max log2-scaled, row sum)
+    const int32_t* table;    // device visibility table
+    int32_t* status;         // device status word
+    int B, H, n_q;
+    int out_f32;
+    int splits;              // 0: full mode (normalised output); >= 1: split-K partials
+    float scale_log2;        // softmax scale * log2(e)
+};
+
+// kernel launchers (defined in the .cu files)
+cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+                               cudaStream_t stream);
+cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
+                               cudaStream_t stream);
+// Copy [B, N, H, d] bf16 K and V into [B][H][rows_per_bh][d] regions at row offset
+// slot * N (slot from the device counter when `ring` is set, else 0).
+cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
+                            int H, int d, int rows_per_bh, int ring, int W, int sink, int S,
+                            int32_t* state, cudaStream_t stream);
+cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
+                             cudaStream_t stream);
+cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
+                           int n_q, int d, int splits, int out_f32, cudaStream_t stream);
+
+}  // namespace swattn

@@ -1,0 +1,167 @@
+/*
+ * swattn.h -- C ABI of libswattn: streaming block-causal sink + sliding-window attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  A chunk-wise autoregressive video diffusion transformer splits the
+ * stream into aligned chunks (one latent frame = 8 video frames; source and target tokens);
+ * attention is bidirectional inside a chunk and causal across chunks, and the active chunk
+ * sees only a fixed window of the W most recent history chunks plus the first chunk, kept
+ * permanently as a global sink (agifrontier tutorial "JoyAI-Video-Edit：单卡720p 30帧，
+ * 两步蒸馏攻克流式视频编辑", section "从双向编辑到分块因果架构的蜕变"; neurohive review
+ * "JoyAI-Video-Edit", section "Чанки и борьба с дрейфом").  Condition tokens from the MLLM
+ * encoder are always-visible keys (neurohive, section "Архитектура JoyAI-Video-Edit").  After
+ * a chunk finishes, its clean K/V are written to the cache, which keeps "global sink + sliding
+ * local window" so memory and time stay flat (tutorial, section "软硬件协同部署").
+ *
+ * For active chunk k (= number of chunks committed so far), per stream b and head h:
+ *   Hist(k) = { j : max(0, k-W) <= j <= k-1 }  U  ({0} if sink and k >= 1)
+ *   keys    = [condition tokens ; chunks of Hist(k) ; the current chunk's K_cur]
+ *   out[i]  = softmax_j(scale * q_i . k_j) . V        over those keys only
+ * The result is exact masked softmax attention; the cache only decides which keys exist.
+ *
+ * Conventions for every call:
+ *   - Tensors are device memory allocated by the caller (e.g. PyTorch), bf16, contiguous,
+ *     in the user layout [B, N, H, d] (N = tokens), 16-byte aligned.  The library never
+ *     takes ownership of them; the caller keeps them alive until the stream has run the work.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls only
+ *     enqueue work on it and never synchronise, except sw_attn_get_status.
+ *   - Return value 0 on success, a negative SW_E* code otherwise; sw_attn_last_error()
+ *     then returns a message (thread-local, valid until the next call on that thread).
+ *   - Problems found on the device (a wait that ran out, an impossible slot) set bits in a
+ *     status word on the device; kernels never trap.  Read it with sw_attn_get_status.
+ *   - One handle holds one layer's cache.  Calls on one handle must be ordered on one stream.
+ */
+#ifndef SWATTN_H
+#define SWATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SW_API __attribute__((visibility("default")))
+#else
+#define SW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sw_attn sw_attn_t;   /* opaque handle, created and destroyed by the caller */
+
+/* return codes */
+#define SW_OK       0
+#define SW_EINVAL  (-1)   /* null handle or pointer, bad enum, bad number */
+#define SW_ESHAPE  (-2)   /* unsupported or inconsistent size */
+#define SW_EALIGN  (-3)   /* pointer or size not aligned as required */
+#define SW_ESTATE  (-4)   /* call not valid in the handle's state (no workspace, no cond) */
+#define SW_ECUDA   (-5)   /* a CUDA runtime or driver call failed */
+
+/* device status bits (sw_attn_get_status) */
+#define SW_STATUS_TIMEOUT    0x1   /* a bounded wait inside a kernel ran out; output invalid */
+#define SW_STATUS_BAD_SLOT   0x2   /* slot index out of range (never expected) */
+#define SW_STATUS_OVERFLOW   0x4   /* chunk counter overflow */
+
+/* output dtypes */
+#define SW_OUT_BF16 0
+#define SW_OUT_F32  1
+
+typedef struct {
+    int   B;                 /* independent streams (batch), >= 1 */
+    int   H;                 /* heads, >= 1 */
+    int   d;                 /* head dim: 64 or 128 */
+    int   tokens_per_chunk;  /* T = source + target tokens of one chunk, >= 1 */
+    int   W;                 /* window: most recent history chunks kept, 0..64 */
+    int   n_cond;            /* condition tokens (always visible), >= 0 */
+    int   sink;              /* 1: chunk 0 is pinned as the global sink */
+    int   out_dtype;         /* SW_OUT_BF16 or SW_OUT_F32 */
+    float scale;             /* softmax scale; <= 0 selects 1/sqrt(d) */
+    int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128 */
+} sw_attn_config;
+
+/*
+ * Create a handle with B = 1, sink on, bf16 output, scale 1/sqrt(d).  Host only: allocates
+ * no device memory and makes no CUDA call.  *out receives the handle.
+ */
+SW_API int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_attn_t **out);
+
+/* Same, with every option (see sw_attn_config).  Host only. */
+SW_API int sw_attn_create_ex(const sw_attn_config *cfg, sw_attn_t **out);
+
+/*
+ * Bytes of device memory the handle needs: the K and V ring caches [B][H][S][T][d] bf16 with
+ * S = W + sink slots, the condition K/V [B][H][n_cond][d] bf16, the split-K partials, the
+ * chunk counter, the status word and the visibility table.  Constant for the handle's life.
+ * Returns 0 for a NULL handle.
+ */
+SW_API size_t sw_attn_workspace_bytes(const sw_attn_t *h);
+
+/*
+ * Give the handle its device memory (allocated and owned by the caller, >= 256-byte aligned,
+ * at least sw_attn_workspace_bytes bytes, on the current device).  Enqueues on `stream`:
+ * zeroing of the counter and status, and the table build for chunk 0.  Cache contents are
+ * left as they are (unused slots are never read).  May be called again to move the handle
+ * to new memory; that also resets the stream to chunk 0 and forgets the condition tokens.
+ */
+SW_API int sw_attn_bind_workspace(sw_attn_t *h, void *dev_ptr, size_t bytes, void *stream);
+
+/*
+ * Copy the condition keys and values (each [B, n_cond, H, d] bf16) into the handle's
+ * condition region.  Required before the first forward when n_cond > 0; may be called
+ * again between chunks (a prompt change).  K_cond/V_cond are read by the enqueued copy.
+ */
+SW_API int sw_attn_set_cond(sw_attn_t *h, const void *K_cond, const void *V_cond, void *stream);
+
+/*
+ * Commit the finished chunk c (c = chunks committed so far, tracked on the device): copy its
+ * K and V ([B, T, H, d] bf16) into ring slot slot(c) -- slot 0 for the sink, then slots
+ * rotating over the window, each new chunk evicting the one that leaves the window -- then
+ * advance the counter and rebuild the visibility table.  With W = 0 the copy of chunks c >= 1
+ * is skipped (only the counter advances).
+ */
+SW_API int sw_attn_append_chunk(sw_attn_t *h, const void *K, const void *V, void *stream);
+
+/*
+ * Attention of the active chunk: Q [B, n_q, H, d], K_cur and V_cur [B, T, H, d] (bf16) and
+ * out [B, n_q, H, d] (bf16 or fp32, per the handle's out_dtype).  Keys are the condition
+ * tokens, the visible cached chunks and K_cur.  n_q == T is the chunk's full query set;
+ * 1 <= n_q <= max_short_q uses the split-K short-query path (queries are the first n_q rows);
+ * other n_q in (max_short_q, T] use the full path.  Reads the visibility table on the device.
+ */
+SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const void *V_cur,
+                    void *out, int n_q, void *stream);
+
+/* Number of int32 entries of the visibility table (3 + 4 * (W + 3)). */
+SW_API int sw_attn_table_ints(const sw_attn_t *h);
+
+/*
+ * Copy the device visibility table for the active chunk into dev_table (device memory,
+ * sw_attn_table_ints entries): [k, n_segments, N_vis, then per segment (kind, chunk_id,
+ * slot, n_tokens)], kind 0 = condition, 1 = cached chunk, 2 = current chunk; order:
+ * condition, sink, window chunks ascending, current; unused entries are -1.
+ */
+SW_API int sw_attn_get_table(const sw_attn_t *h, int32_t *dev_table, void *stream);
+
+/*
+ * Byte offsets, inside the bound workspace, of the K and V ring caches ([B][H][S][T][d] bf16,
+ * S = W + sink slots; slot 0 holds the sink when it is on).  For inspection and tests.
+ */
+SW_API int sw_attn_cache_offsets(const sw_attn_t *h, size_t *k_offset, size_t *v_offset);
+
+/* Synchronise the device, then read the device status bits into *host_status. */
+SW_API int sw_attn_get_status(sw_attn_t *h, int32_t *host_status);
+
+/* Start a new stream on the same handle: counter and status to 0, table for chunk 0. */
+SW_API int sw_attn_reset(sw_attn_t *h, void *stream);
+
+/* Free the handle (host memory only; the workspace stays the caller's). NULL is ignored. */
+SW_API void sw_attn_destroy(sw_attn_t *h);
+
+/* Message for the last failed call on this thread ("" if none). */
+SW_API const char *sw_attn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWATTN_H */

@@ -1,0 +1,92 @@
+"""Shared helpers for the GPU parity tests: stream a workload through the CUDA library and the
+FP64 oracle on the same seeded inputs, and compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from block_causal_attention_sliding_b200 import synth
+from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+
+MAX_ABS = 1e-2      # tolerances on fp32 output, against the FP64 oracle
+MEAN_REL = 2e-3     # mean-relative = sum |got - ref| / sum |ref|
+
+
+def compare(got: np.ndarray, ref: np.ndarray, max_abs: float = MAX_ABS, mean_rel: float = MEAN_REL):
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), "non-finite output"
+    d = np.abs(got.astype(np.float64) - ref)
+    ma = float(d.max())
+    mr = float(d.sum() / max(np.abs(ref).sum(), 1e-300))
+    assert ma <= max_abs and mr <= mean_rel, f"max-abs {ma:.3e} (<= {max_abs}), mean-rel {mr:.3e} (<= {mean_rel})"
+    return ma, mr
+
+
+def sample_rows(n_q: int, n: int, seed: int) -> np.ndarray:
+    """Rows that always include both ends and the 128-row tile edges, plus random ones."""
+    fixed = {0, 1, n_q - 1, n_q - 2}
+    for e in range(128, n_q, 128):
+        fixed.update({e - 1, e})
+    fixed = sorted(r for r in fixed if 0 <= r < n_q)
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(n_q, size=min(n_q, max(0, n - len(fixed))), replace=False)
+    return np.array(sorted(set(fixed) | set(int(x) for x in extra)), dtype=np.int32)
+
+
+def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink=None, n_cond=None):
+    return SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W if W is None else W,
+                                  n_cond=wl.n_cond if n_cond is None else n_cond,
+                                  sink=wl.sink if sink is None else sink, out_dtype=out_dtype,
+                                  max_short_q=max_short_q, device=dev)
+
+
+def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, n_q=None,
+                     out_dtype=torch.float32, max_short_q=0, poison=False, seed=0,
+                     tol=(MAX_ABS, MEAN_REL), keep_last=None, gen_on_device=False):
+    """Stream `chunks` chunks (2 forwards then an append each).  At the chunks in `check_at`
+    (all if None) compare the CUDA output with the oracle, on all rows or on sampled rows.
+    With gen_on_device the seeded draws use the GPU generator (faster for big shapes); the
+    oracle then reads host copies of exactly those bf16 values.
+    Returns a list of (k, step, max_abs, mean_rel)."""
+    h = make_handle(wl, dev, out_dtype=out_dtype, max_short_q=max_short_q)
+    if poison:
+        kc, vc = h.cache_views()
+        kc.fill_(float("nan"))
+        vc.fill_(float("nan"))
+    gdev = dev if gen_on_device else "cpu"
+    Kc, Vc = synth.cond_inputs(wl, seed=seed, device=gdev)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    Kc, Vc = Kc.cpu(), Vc.cpu()
+    hist_K, hist_V = [], []
+    results = []
+    nq = wl.T if n_q is None else n_q
+    for k in range(chunks):
+        for step in range(wl.steps):
+            Q, K, V = synth.chunk_inputs(wl, k, step, seed=seed, n_q=nq, device=gdev)
+            out = h.forward(Q.to(dev), K.to(dev), V.to(dev))
+            if check_at is None or k in check_at:
+                Q = Q.cpu()
+                r = rows
+                if r is None and n_rows is not None:
+                    r = sample_rows(nq, n_rows, seed=1000 * k + step)
+                ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
+                                       k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V, Q=Q,
+                                       K_cur=K.cpu(), V_cur=V.cpu(), rows=r)
+                got = out.float().cpu().numpy()
+                if r is not None:
+                    got = got[:, r]
+                ma, mr = compare(got, ref, *tol)
+                results.append((k, step, ma, mr))
+        h.append_chunk(K.to(dev), V.to(dev))
+        hist_K.append(K.cpu())
+        hist_V.append(V.cpu())
+        if keep_last is not None:
+            # only the sink and the most recent chunks are ever visible; drop the rest from
+            # host memory (the oracle raises if a dropped chunk turns out to be visible)
+            for c in range(1, max(1, len(hist_K) - keep_last)):
+                hist_K[c] = None
+                hist_V[c] = None
+    torch.cuda.synchronize()
+    assert h.status() == 0, f"device status {h.status():#x}"
+    return results

@@ -1,0 +1,121 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every declared symbol, and
+its host-only calls (create, workspace sizing, argument checks) behave as documented."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from block_causal_attention_sliding_b200 import build as B
+    B.build()
+    from block_causal_attention_sliding_b200 import _native
+    return _native
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "swattn.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"SW_API\s+[\w\s\*]*?\b(sw_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = _declared_symbols()
+    for name in ("sw_attn_create", "sw_attn_append_chunk", "sw_attn_forward"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(native):
+    L = native.lib()
+    syms = _declared_symbols()
+    assert sorted(native.EXPORTS) == syms
+    for name in syms:
+        assert hasattr(L, name), name
+
+
+def _create(native, **kw):
+    cfg = dict(B=1, H=24, d=128, tokens_per_chunk=3180, W=3, n_cond=256, sink=1, out_dtype=0,
+               scale=0.0, max_short_q=0)
+    cfg.update(kw)
+    c = native.SwAttnConfig(**cfg)
+    h = ctypes.c_void_p()
+    rc = native.lib().sw_attn_create_ex(ctypes.byref(c), ctypes.byref(h))
+    return rc, h
+
+
+def test_create_and_workspace_bytes(native):
+    L = native.lib()
+    rc, h = _create(native)
+    assert rc == 0 and h.value
+    ws = L.sw_attn_workspace_bytes(h)
+    # ring K+V: 2 * 24 heads * 4 slots * 3180 * 128 * 2 B; cond K+V: 2 * 24 * 256 * 128 * 2 B
+    ring = 2 * 24 * 4 * 3180 * 128 * 2
+    cond = 2 * 24 * 256 * 128 * 2
+    assert ring + cond <= ws <= ring + cond + 16 * 2 ** 20
+    assert L.sw_attn_table_ints(h) == 3 + 4 * (3 + 3)
+    ko, vo = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.sw_attn_cache_offsets(h, ctypes.byref(ko), ctypes.byref(vo)) == 0
+    assert ko.value % 1024 == 0 and vo.value - ko.value >= ring // 2
+    L.sw_attn_destroy(h)
+    # the simple constructor: B = 1, sink on
+    h2 = ctypes.c_void_p()
+    assert L.sw_attn_create(24, 128, 3180, 3, 256, ctypes.byref(h2)) == 0
+    assert L.sw_attn_workspace_bytes(h2) == ws
+    L.sw_attn_destroy(h2)
+
+
+def test_workspace_constant_in_stream_length(native):
+    """Cache memory depends on W, not on how many chunks will be streamed."""
+    L = native.lib()
+    sizes = []
+    for W in (1, 3, 6):
+        rc, h = _create(native, W=W)
+        assert rc == 0
+        sizes.append(L.sw_attn_workspace_bytes(h))
+        L.sw_attn_destroy(h)
+    assert sizes[0] < sizes[1] < sizes[2]
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), -2), (dict(d=0), -2), (dict(H=0), -2), (dict(B=0), -2),
+    (dict(tokens_per_chunk=0), -2), (dict(W=-1), -2), (dict(W=65), -2), (dict(n_cond=-3), -2),
+    (dict(sink=2), -1), (dict(out_dtype=7), -1), (dict(max_short_q=129), -2),
+    (dict(scale=float("inf")), -1),
+])
+def test_create_rejects_bad_config(native, kw, code):
+    rc, h = _create(native, **kw)
+    assert rc == code
+    assert not h.value
+    assert native.lib().sw_attn_last_error().decode()
+
+
+def test_calls_before_workspace_fail_cleanly(native):
+    L = native.lib()
+    rc, h = _create(native, H=2, d=64, tokens_per_chunk=16, W=1, n_cond=8)
+    assert rc == 0
+    dummy = ctypes.c_void_p(0x1000)
+    assert L.sw_attn_forward(h, dummy, dummy, dummy, dummy, 16, None) == native.SW_ESTATE
+    assert b"workspace" in L.sw_attn_last_error()
+    assert L.sw_attn_append_chunk(h, dummy, dummy, None) == native.SW_ESTATE
+    assert L.sw_attn_set_cond(h, dummy, dummy, None) == native.SW_ESTATE
+    assert L.sw_attn_reset(h, None) == native.SW_ESTATE
+    st = ctypes.c_int32()
+    assert L.sw_attn_get_status(h, ctypes.byref(st)) == native.SW_ESTATE
+    # bind: null and misaligned pointers and short buffers are refused before any CUDA call
+    assert L.sw_attn_bind_workspace(h, None, 1 << 20, None) == native.SW_EINVAL
+    assert L.sw_attn_bind_workspace(h, ctypes.c_void_p(0x1008), 1 << 30, None) == native.SW_EALIGN
+    assert L.sw_attn_bind_workspace(h, ctypes.c_void_p(0x10000), 16, None) == native.SW_ESHAPE
+    L.sw_attn_destroy(h)
+
+
+def test_null_handle(native):
+    L = native.lib()
+    assert L.sw_attn_workspace_bytes(None) == 0
+    assert L.sw_attn_forward(None, None, None, None, None, 1, None) == native.SW_EINVAL
+    L.sw_attn_destroy(None)   # ignored

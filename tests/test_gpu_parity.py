@@ -1,0 +1,202 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the FP64 oracle.
+
+Tables and cache contents are compared bit for bit; attention outputs (fp32) within
+max-abs 1e-2 and mean-relative 2e-3.  Full rows for the small workloads (several 128-row
+tiles with ragged tails), sampled rows -- always including both ends and every tile edge --
+for the 480p, 720p and stress workloads, in the same launch configuration the benchmark uses.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_causal_attention_sliding_b200 import synth
+from block_causal_attention_sliding_b200.configs import WORKLOADS, Workload
+
+from parity_util import compare, make_handle, stream_and_check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_causal_attention_sliding_b200 import build as B
+    B.build()
+    oracle.build()
+    d = torch.device("cuda", 0)
+    torch.cuda.set_device(d)
+    return d
+
+
+# a workload spanning several tiles with ragged tails everywhere: T = 300 = 128 + 128 + 44,
+# n_cond = 40, two streams, three heads
+RAGGED = Workload("ragged", B=2, H=3, d=128, T=300, n_cond=40, W=2, sink=True, chunks=6, steps=2)
+
+
+# ------------------------------------------------------------------ K1 tables (bit-exact)
+
+@pytest.mark.parametrize("name", ["tiny", "480p", "720p", "long720p", "stress"])
+def test_tables_every_chunk(dev, name):
+    wl = WORKLOADS[name]
+    # the table depends only on W, sink, n_cond and T; a one-head, d=64 handle is enough
+    small = dataclasses.replace(wl, B=1, H=1, d=64)
+    h = make_handle(small, dev)
+    z = torch.zeros((1, small.T, 1, 64), dtype=torch.bfloat16, device=dev)
+    for k in range(wl.chunks):
+        got = h.table().cpu().numpy()
+        ref = oracle.table(k, wl.W, wl.sink, wl.n_cond, wl.T)
+        np.testing.assert_array_equal(got[: len(ref)], ref)
+        assert (got[len(ref):] == -1).all()
+        h.append_chunk(z, z)
+    assert h.status() == 0
+
+
+@pytest.mark.parametrize("W,sink,n_cond", [(0, True, 8), (0, False, 0), (1, False, 3), (5, True, 0),
+                                           (64, True, 2)])
+def test_tables_other_windows(dev, W, sink, n_cond):
+    wl = Workload("t", B=1, H=1, d=64, T=5, n_cond=n_cond, W=W, sink=sink, chunks=80, steps=1)
+    h = make_handle(wl, dev)
+    z = torch.zeros((1, 5, 1, 64), dtype=torch.bfloat16, device=dev)
+    for k in range(wl.chunks):
+        got = h.table().cpu().numpy()
+        ref = oracle.table(k, W, sink, n_cond, 5)
+        np.testing.assert_array_equal(got[: len(ref)], ref)
+        h.append_chunk(z, z)
+    h.reset()
+    np.testing.assert_array_equal(h.table().cpu().numpy()[:7 if n_cond else 3 + 4],
+                                  oracle.table(0, W, sink, n_cond, 5))
+
+
+# ------------------------------------------------------------------ K2 ring cache (bit-exact)
+
+@pytest.mark.parametrize("W,sink", [(3, True), (2, False), (0, True), (1, True)])
+def test_cache_contents_match_ring_model(dev, W, sink):
+    B, H, d, T = 2, 3, 64, 40
+    wl = Workload("c", B=B, H=H, d=d, T=T, n_cond=0, W=W, sink=sink, chunks=12, steps=1)
+    h = make_handle(wl, dev)
+    kc, vc = h.cache_views()
+    kc.fill_(float("nan"))
+    vc.fill_(float("nan"))
+    ring = oracle.Ring(B=B, H=H, d=d, T=T, n_cond=0, W=W, sink=sink, Kc=None, Vc=None)
+    chunks = {}
+    for c in range(wl.chunks):
+        K = synth.draw((B, T, H, d), 77 + 2 * c)
+        V = synth.draw((B, T, H, d), 78 + 2 * c)
+        chunks[c] = (K, V)
+        h.append_chunk(K.to(dev), V.to(dev))
+        ring.append(K, V)
+        torch.cuda.synchronize()
+        for s, held in enumerate(ring.slot_chunks()):
+            gk = kc[:, :, s].cpu()          # [B, H, T, d]
+            gv = vc[:, :, s].cpu()
+            if held < 0:
+                assert torch.isnan(gk.float()).all() and torch.isnan(gv.float()).all()
+            else:
+                ek, ev = chunks[held]
+                assert torch.equal(gk.view(torch.int16), ek.permute(0, 2, 1, 3).contiguous().view(torch.int16))
+                assert torch.equal(gv.view(torch.int16), ev.permute(0, 2, 1, 3).contiguous().view(torch.int16))
+    assert h.status() == 0
+
+
+# ------------------------------------------------------------------ K3 / K4 attention
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("max_short_q", [-1, 0])
+def test_tiny_full_stream(dev, out_dtype, max_short_q):
+    """Every chunk and both denoise steps of the tiny workload, all rows; -1 forces the full
+    path, 0 lets the 16 queries take the split-K path."""
+    wl = WORKLOADS["tiny"]
+    tol = (1e-2, 2e-3) if out_dtype == torch.float32 else (2e-2, 4e-3)
+    res = stream_and_check(wl, dev, chunks=wl.chunks, out_dtype=out_dtype, max_short_q=max_short_q, tol=tol)
+    assert len(res) == wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("max_short_q", [-1, 0])
+def test_ragged_multi_tile(dev, d, max_short_q):
+    wl = dataclasses.replace(RAGGED, d=d)
+    stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=max_short_q)
+
+
+@pytest.mark.parametrize("W,sink,n_cond", [(0, False, 40), (0, True, 0), (4, False, 7), (1, True, 130)])
+def test_ragged_other_windows(dev, W, sink, n_cond):
+    wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
+    stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1)
+
+
+def test_stale_slots_poisoned_with_nan(dev):
+    """Unused and not-yet-filled ring slots hold NaN: they are never read."""
+    wl = dataclasses.replace(RAGGED, W=4, chunks=4)
+    stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1, poison=True)
+
+
+def test_permutation_within_chunk(dev):
+    """Permuting the current chunk's keys (with their values) leaves the output unchanged."""
+    wl = RAGGED
+    h = make_handle(wl, dev)
+    Kc, Vc = synth.cond_inputs(wl)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    for k in range(3):
+        _, K, V = synth.chunk_inputs(wl, k, 0)
+        h.append_chunk(K.to(dev), V.to(dev))
+    Q, K, V = synth.chunk_inputs(wl, 3, 0)
+    perm = torch.randperm(wl.T, generator=torch.Generator().manual_seed(3))
+    a = h.forward(Q.to(dev), K.to(dev), V.to(dev)).cpu().numpy()
+    b = h.forward(Q.to(dev), K[:, perm].contiguous().to(dev), V[:, perm].contiguous().to(dev)).cpu().numpy()
+    compare(b, a.astype(np.float64), 2e-3, 5e-4)
+
+
+def test_480p_sampled(dev):
+    wl = WORKLOADS["480p"]
+    res = stream_and_check(wl, dev, chunks=wl.chunks, check_at={0, 1, 2, 3, 4, 15}, n_rows=48,
+                           keep_last=wl.W + 1, gen_on_device=True)
+    assert len(res) == 12
+
+
+def test_720p_sampled(dev):
+    """The 720p workload in the benchmark's launch configuration, chunks 0, 1, W, W+1, W+2
+    and the last of 32."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check(wl, dev, chunks=wl.chunks, check_at={0, 1, 3, 4, 5, 31}, n_rows=40,
+                           keep_last=wl.W + 1, gen_on_device=True)
+    assert len(res) == 12
+
+
+def test_stress_sampled(dev):
+    """Four streams, 32 heads, W = 6, 512 condition tokens, 1% sigma-4 key outliers."""
+    wl = WORKLOADS["stress"]
+    res = stream_and_check(wl, dev, chunks=9, check_at={0, 7, 8}, n_rows=12, keep_last=wl.W + 1,
+                           gen_on_device=True)
+    assert len(res) == 6
+
+
+@pytest.mark.parametrize("n_q", [1, 16, 64, 128])
+def test_short_queries_720p(dev, n_q):
+    """Split-K path: n_q queries against the steady-state 720p cache."""
+    wl = WORKLOADS["720p"]
+    stream_and_check(wl, dev, chunks=6, check_at={0, 5}, n_q=n_q, keep_last=wl.W + 1, gen_on_device=True)
+
+
+def test_long_horizon_constant_memory(dev):
+    """225 chunks: the device table stays exact, memory does not grow, the last chunk matches
+    the oracle on sampled rows."""
+    wl = WORKLOADS["long720p"]
+    torch.cuda.synchronize()
+    res = None
+    before = None
+    h = make_handle(wl, dev)
+    ws = h.workspace_bytes()
+    del h
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated(dev)
+    res = stream_and_check(wl, dev, chunks=wl.chunks, check_at={wl.chunks - 1}, n_rows=24,
+                           keep_last=wl.W + 1, gen_on_device=True)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated(dev) <= before + 4096
+    assert len(res) == 2 and ws > 0
