@@ -186,7 +186,7 @@ def run_cuda(args, wl, world, rank, local):
     peaks = _peaks()
 
     h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
-                               out_dtype=torch.bfloat16, device=dev)
+                               out_dtype=torch.bfloat16, schedule=args.schedule, device=dev)
     Kc, Vc = synth.cond_inputs(wl, seed=rank, device=dev)
     h.set_cond(Kc, Vc)
     # a pool of distinct input sets, resident in HBM; together with the 160 MB cache the
@@ -303,9 +303,12 @@ def run_cuda(args, wl, world, rank, local):
                        "l2": f"inputs larger than L2: {len(pool)} resident input sets of "
                              f"{sum(t.numel() * 2 for t in pool[0][0]) * wl.steps / 2 ** 20:.0f} MiB plus the "
                              f"{h.workspace_bytes() / 2 ** 20:.0f} MiB cache, cycled per step",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "schedule": args.schedule},
             "pct_of_peak": round(100.0 * value / world / peak, 2),
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,2>", "achieved": round(achieved, 2),
+            "roofline": {"bound": "tensor",
+                         "kernel": "attn_persistent_kernel<128>" if args.schedule == "persistent"
+                         else "attn_fwd_kernel<128,2>", "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "traffic": None, "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                          "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
@@ -407,6 +410,7 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", choices=["persistent", "grid"], default="persistent")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -33,12 +33,13 @@ class SlidingWindowAttention:
 
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
-                 max_short_q: int = 0, device=None):
+                 max_short_q: int = 0, schedule: str = "persistent", device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
                              out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
-                             scale=0.0 if scale is None else float(scale), max_short_q=max_short_q)
+                             scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
+                             schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID}[schedule])
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()

@@ -1,0 +1,281 @@
+// attn_common.cuh -- pieces shared by the attention kernels: tile geometry, the shared-memory
+// control block, bounded waits, the tile schedule over the visibility table, the TMA loads of
+// one K or V tile, the tcgen05 issue of S = Q K^T and O += P V, and one softmax step.
+#pragma once
+#include "ptx.cuh"
+#include "swattn_internal.h"
+
+namespace swattn {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: far above any legitimate wait
+constexpr int kBoxCols = 64;                        // 128-byte swizzle atom = 64 bf16
+constexpr int kBoxBytes = kBlockM * kBoxCols * 2;   // 16 KB: one TMA box (128 rows x 64 cols)
+constexpr float kRescaleThreshold = 8.0f;           // log2 units: rescale O when max grows > 2^8
+
+template <int D>
+struct TileCfg {
+    static constexpr int kBoxes = D / kBoxCols;
+    static constexpr int kTileBytes = kBoxes * kBoxBytes;   // one 128-row tile of Q, K or V
+    static constexpr int kStages = D == 128 ? 4 : 6;
+};
+
+struct SmemCtl {
+    uint64_t q_full;
+    uint64_t q_empty;
+    uint64_t kv_full[8];
+    uint64_t kv_empty[8];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_full[2];
+    uint64_t o_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int n_seg;
+    int n_tiles;
+    int merge_flag[2];
+    int seg_kind[kMaxW + 3];
+    int seg_slot[kMaxW + 3];
+    int seg_ntok[kMaxW + 3];
+    int seg_tile0[kMaxW + 4];   // first tile index of each segment; [n_seg] = total
+};
+
+template <int D, int NQ>
+struct AttnLayout {
+    using C = TileCfg<D>;
+    static constexpr int kQBytes = NQ * C::kTileBytes;
+    static constexpr int kKVBytes = C::kStages * C::kTileBytes;
+    static constexpr int kCtlOffset = kQBytes + kKVBytes;
+    static constexpr int kSmemBytes = kCtlOffset + (int)sizeof(SmemCtl) + 1024;  // + align slack
+    static constexpr int kThreads = 64 + NQ * 128;    // producer, MMA, NQ softmax warpgroups
+    static constexpr int kTmemNeed = NQ * (kBlockN + D);
+    static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
+};
+
+// Bounded wait that also honours the CTA abort flag; raises the flag on a timeout.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* flag) {
+    const bool ok = mbar_wait(bar, parity, flag, kWaitLimitNs);
+    if (!ok) *flag = 1;
+    return ok;
+}
+
+// Bounded wait used while draining: ignores the abort flag (copies in flight always land).
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+    int never = 0;
+    (void)mbar_wait(bar, parity, &never, kWaitLimitNs);
+}
+
+// Warp-uniform wait for the softmax warps.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* flag) {
+    const bool ok = wait_or_abort(bar, parity, flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Copy the table's segment list into shared memory (one thread).  Returns false on a table
+// that cannot be right; the caller then processes nothing and the status word says why.
+__device__ __forceinline__ void load_table(SmemCtl* ctl, const int32_t* table, int32_t* status) {
+    const int n_seg = table[1];
+    int ok = n_seg >= 1 && n_seg <= kMaxW + 3;
+    int tiles = 0;
+    if (ok) {
+        for (int s = 0; s < n_seg; ++s) {
+            const int32_t* e = table + 3 + 4 * s;
+            const int kind = e[0], slot = e[2], ntok = e[3];
+            if (kind < 0 || kind > 2 || ntok <= 0) ok = 0;
+            ctl->seg_kind[s] = kind;
+            ctl->seg_slot[s] = slot;
+            ctl->seg_ntok[s] = ntok;
+            ctl->seg_tile0[s] = tiles;
+            tiles += (ntok + kBlockN - 1) / kBlockN;
+        }
+        ctl->seg_tile0[n_seg] = tiles;
+    }
+    if (!ok) {
+        atomicOr(status, SW_STATUS_BAD_SLOT);
+        ctl->n_seg = 0;
+        ctl->n_tiles = 0;
+    } else {
+        ctl->n_seg = n_seg;
+        ctl->n_tiles = tiles;
+    }
+}
+
+// Which segment key tile j belongs to, its first key row, and how many of its rows are keys.
+__device__ __forceinline__ void tile_of(const SmemCtl* ctl, int j, int& seg, int& row0, int& valid) {
+    int s = 0;
+    while (s + 1 < ctl->n_seg && ctl->seg_tile0[s + 1] <= j) ++s;
+    seg = s;
+    row0 = (j - ctl->seg_tile0[s]) * kBlockN;
+    const int rem = ctl->seg_ntok[s] - row0;
+    valid = rem < kBlockN ? rem : kBlockN;
+}
+
+// TMA loads of one 128-row K (kv = 0) or V (kv = 1) tile of key tile j of (b, h) into dst,
+// completing on bar: condition tokens, a ring slot, or the caller's current chunk.
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl* ctl, int j, int kv,
+                                             int h, int b, uint32_t dst, uint32_t bar) {
+    int seg, row0, valid;
+    tile_of(ctl, j, seg, row0, valid);
+    const int kind = ctl->seg_kind[seg];
+    const int slot = ctl->seg_slot[seg];
+#pragma unroll
+    for (int c = 0; c < TileCfg<D>::kBoxes; ++c) {
+        const uint32_t d = dst + c * kBoxBytes;
+        if (kind == 0)
+            tma_load_4d(d, kv ? &p.tm_cond_v : &p.tm_cond_k, bar, c * kBoxCols, row0, h, b);
+        else if (kind == 1)
+            tma_load_5d(d, kv ? &p.tm_cache_v : &p.tm_cache_k, bar, c * kBoxCols, row0, slot, h, b);
+        else
+            tma_load_4d(d, kv ? &p.tm_vcur : &p.tm_kcur, bar, c * kBoxCols, h, row0, b);
+    }
+}
+
+// S[tS] = Q(q_tile) K(k_tile)^T: M = 128 queries, N = 128 keys, K = D, bf16 -> fp32.
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;   // 16 columns = 32 bytes
+        mma_ss(tS, smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
+               idesc, ks > 0 ? 1u : 0u);
+    }
+}
+
+// O[tO] (+)= P[tP] V(v_tile): P (bf16 pairs in TMEM) is the A operand, V is MN-major in shared
+// memory (16 key rows per step = 2 KB; the two 64-column boxes are 16 KB apart).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_tile, bool accumulate) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
+#pragma unroll
+    for (int ks = 0; ks < kBlockN / 16; ++ks)
+        mma_ts(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
+               (accumulate || ks > 0) ? 1u : 0u);
+}
+
+// One online-softmax step for this thread's query row over one key tile:
+//   read the S row from TMEM, mask keys past the segment's end, update the reference max
+//   (lazily: only when it grows by more than 2^kRescaleThreshold), write P = exp2(s*sl2 - m)
+//   as bf16 pairs over the S columns, add the same rounded weights to l, and rescale the
+//   O row in TMEM when the reference moved (after waiting for the previous PV).
+// The caller has waited for S and arrives on p_full afterwards.  Returns false on abort.
+template <int D>
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
+                                             uint32_t o_full_bar, uint32_t prev_pv_parity, float sl2,
+                                             float& m_ref, float& l, volatile int* abort_flag) {
+    uint32_t sr[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+    tmem_wait_ld_dep(sr[0]);
+    reg_fence(sr[1]);
+    reg_fence(sr[2]);
+    reg_fence(sr[3]);
+    if (valid < kBlockN) {
+        // last tile of a segment: keys past its end read as zero; mask them out
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+    const float m_new = mx * sl2;
+    float f = 1.f;            // factor that takes O and l to the new reference max
+    bool rescale = false;     // warp-uniform: does this warp rescale O this tile
+    if (first) {
+        m_ref = m_new;
+    } else {
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+            f = ex2_approx(m_ref - m_new);
+            m_ref = m_new;
+        }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][i]), sl2, -m_ref));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][i + 1]), sl2, -m_ref));
+                const uint32_t pp = pack_bf16x2(p0, p1);
+                // the row sum adds the same bf16-rounded weights the PV MMA multiplies, so
+                // out is an exact weighted mean of V under those weights
+                sum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
+                pk[cc * 16 + (i >> 1)] = pp;
+            }
+        }
+        tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
+    }
+    l = l * f + sum;
+    if (rescale) {
+        // done once the S row is dead (low register pressure); it must land before this
+        // tile's PV, which the caller's p_full arrival releases
+        if (!warp_wait(o_full_bar, prev_pv_parity, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld_dep(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(tO + c * 32, o);
+        }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    return true;
+}
+
+// Write one output row (32 columns at a time from registers), bf16 or fp32.
+template <int D>
+__device__ __forceinline__ void store_row_chunk(void* out, int out_f32, size_t orow, int c,
+                                                const uint32_t (&o)[32], float scale) {
+    if (out_f32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + orow * D + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]) * scale, __uint_as_float(o[4 * i + 1]) * scale,
+                                 __uint_as_float(o[4 * i + 2]) * scale, __uint_as_float(o[4 * i + 3]) * scale);
+    } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + orow * D + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(
+                pack_bf16x2(__uint_as_float(o[8 * i + 0]) * scale, __uint_as_float(o[8 * i + 1]) * scale),
+                pack_bf16x2(__uint_as_float(o[8 * i + 2]) * scale, __uint_as_float(o[8 * i + 3]) * scale),
+                pack_bf16x2(__uint_as_float(o[8 * i + 4]) * scale, __uint_as_float(o[8 * i + 5]) * scale),
+                pack_bf16x2(__uint_as_float(o[8 * i + 6]) * scale, __uint_as_float(o[8 * i + 7]) * scale));
+    }
+}
+
+__device__ __forceinline__ void init_barriers(SmemCtl* ctl, int stages) {
+    mbar_init(smem_u32(&ctl->q_full), 1);
+    mbar_init(smem_u32(&ctl->q_empty), 1);
+    for (int s = 0; s < stages; ++s) {
+        mbar_init(smem_u32(&ctl->kv_full[s]), 1);
+        mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+        mbar_init(smem_u32(&ctl->s_full[q]), 1);
+        mbar_init(smem_u32(&ctl->p_full[q]), 128);
+        mbar_init(smem_u32(&ctl->o_full[q]), 1);
+        mbar_init(smem_u32(&ctl->o_empty[q]), 128);
+    }
+    mbar_init(smem_u32(&ctl->drain), 1);
+    ctl->abort_flag = 0;
+    fence_mbar_init();
+}
+
+}  // namespace swattn

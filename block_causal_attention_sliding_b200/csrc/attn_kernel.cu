@@ -1,4 +1,6 @@
-// attn_kernel.cu -- fused attention of the active chunk over the bounded cache (sm_100a).
+// attn_kernel.cu -- fused attention of the active chunk over the bounded cache (sm_100a):
+// the one-work-item-per-CTA kernel (grid over query blocks, heads and streams), its split-K
+// mode for short query sets, and the split-K combine.
 //
 // out = softmax(scale * Q K^T) V over the keys the visibility table lists: condition tokens,
 // the sink, the window chunks and the current chunk (block-causal: bidirectional inside the
@@ -12,81 +14,15 @@
 //               zero-filled by TMA.  A ring of kStages shared-memory tiles.
 //   warp 1      MMA issuer (one thread): S_q = Q_q K^T into TMEM (tcgen05, bf16 in, fp32
 //               accumulate), then O_q += P_q V with P read from TMEM.
-//   warps 4..   one warpgroup per Q tile (thread = query row = TMEM lane): online softmax in
+//   warps 2..   one warpgroup per Q tile (thread = query row = TMEM lane): online softmax in
 //               fp32 registers -- row max, lazy rescale of O only when the max grows by more
 //               than 2^8, exp2, row sum -- writes P as bf16 into the S columns.
 // The two Q tiles share every K/V tile, and while one warpgroup runs its softmax the tensor
 // core works on the other tile.  In split mode (short query sets) a CTA takes one Q tile and
 // a slice of the key tiles, and writes unnormalised partials that a combine kernel merges.
-#include "ptx.cuh"
-#include "swattn_internal.h"
+#include "attn_common.cuh"
 
 namespace swattn {
-
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: far above any legitimate wait
-constexpr int kBoxCols = 64;                        // 128-byte swizzle atom = 64 bf16
-constexpr int kBoxBytes = kBlockM * kBoxCols * 2;   // 16 KB: one TMA box (128 rows x 64 cols)
-constexpr float kRescaleThreshold = 8.0f;           // log2 units: rescale O when max grows > 2^8
-
-template <int D>
-struct TileCfg {
-    static constexpr int kBoxes = D / kBoxCols;
-    static constexpr int kTileBytes = kBoxes * kBoxBytes;   // one 128-row tile of Q, K or V
-    static constexpr int kStages = D == 128 ? 4 : 6;
-};
-
-struct SmemCtl {
-    uint64_t q_full;
-    uint64_t kv_full[8];
-    uint64_t kv_empty[8];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_full[2];
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort_flag;
-    int n_seg;
-    int n_tiles;
-    int seg_kind[kMaxW + 3];
-    int seg_slot[kMaxW + 3];
-    int seg_ntok[kMaxW + 3];
-    int seg_tile0[kMaxW + 4];   // first tile index of each segment; [n_seg] = total
-};
-
-template <int D, int NQ>
-struct AttnLayout {
-    using C = TileCfg<D>;
-    static constexpr int kQBytes = NQ * C::kTileBytes;
-    static constexpr int kKVBytes = C::kStages * C::kTileBytes;
-    static constexpr int kCtlOffset = kQBytes + kKVBytes;
-    static constexpr int kSmemBytes = kCtlOffset + (int)sizeof(SmemCtl) + 1024;  // + align slack
-    static constexpr int kThreads = 128 + NQ * 128;
-    static constexpr int kTmemNeed = NQ * (kBlockN + D);
-    static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
-};
-
-// Bounded wait that also honours the CTA abort flag; raises the flag on a timeout.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* flag) {
-    const bool ok = mbar_wait(bar, parity, flag, kWaitLimitNs);
-    if (!ok) *flag = 1;
-    return ok;
-}
-
-// Bounded wait used while draining: ignores the abort flag (copies in flight always land).
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-    int never = 0;
-    (void)mbar_wait(bar, parity, &never, kWaitLimitNs);
-}
-
-// Which segment tile j belongs to, its first key row, and how many of its 128 rows are keys.
-__device__ __forceinline__ void tile_of(const SmemCtl* ctl, int j, int& seg, int& row0, int& valid) {
-    int s = 0;
-    while (s + 1 < ctl->n_seg && ctl->seg_tile0[s + 1] <= j) ++s;
-    seg = s;
-    row0 = (j - ctl->seg_tile0[s]) * kBlockN;
-    const int rem = ctl->seg_ntok[s] - row0;
-    valid = rem < kBlockN ? rem : kBlockN;
-}
 
 template <int D, int NQ>
 __global__ void __launch_bounds__(AttnLayout<D, NQ>::kThreads, 1)
@@ -113,50 +49,12 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
 
     // ---------------------------------------------------------------- set-up
     if (warp == 0) {
-        if (lane == 0) {
-            mbar_init(smem_u32(&ctl->q_full), 1);
-            for (int s = 0; s < kStages; ++s) {
-                mbar_init(smem_u32(&ctl->kv_full[s]), 1);
-                mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
-            }
-            for (int q = 0; q < 2; ++q) {
-                mbar_init(smem_u32(&ctl->s_full[q]), 1);
-                mbar_init(smem_u32(&ctl->p_full[q]), 128);
-                mbar_init(smem_u32(&ctl->o_full[q]), 1);
-            }
-            mbar_init(smem_u32(&ctl->drain), 1);
-            ctl->abort_flag = 0;
-            fence_mbar_init();
-        }
+        if (lane == 0) init_barriers(ctl, kStages);
         __syncwarp();
         tmem_alloc(smem_u32(&ctl->tmem_base), L::kTmemCols);
         tmem_relinquish();
     } else if (warp == 2 && lane == 0) {
-        // copy the visibility table's segment list into shared memory
-        const int n_seg = p.table[1];
-        int ok = n_seg >= 1 && n_seg <= kMaxW + 3;
-        int tiles = 0;
-        if (ok) {
-            for (int s = 0; s < n_seg; ++s) {
-                const int* e = p.table + 3 + 4 * s;
-                const int kind = e[0], slot = e[2], ntok = e[3];
-                if (kind < 0 || kind > 2 || ntok <= 0) ok = 0;
-                ctl->seg_kind[s] = kind;
-                ctl->seg_slot[s] = slot;
-                ctl->seg_ntok[s] = ntok;
-                ctl->seg_tile0[s] = tiles;
-                tiles += (ntok + kBlockN - 1) / kBlockN;
-            }
-            ctl->seg_tile0[n_seg] = tiles;
-        }
-        if (!ok) {
-            atomicOr(p.status, SW_STATUS_BAD_SLOT);
-            ctl->n_seg = 0;
-            ctl->n_tiles = 0;
-        } else {
-            ctl->n_seg = n_seg;
-            ctl->n_tiles = tiles;
-        }
+        load_table(ctl, p.table, p.status);
     } else if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_kcur);
@@ -177,23 +75,22 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
     }
     const int n = t1 - t0;                          // key tiles this CTA processes
     const int m0 = split_mode ? 0 : blockIdx.x * NQ * kBlockM;
+    // Q tiles of this CTA that hold at least one query row (the last CTA of a head may own
+    // a single tile); tiles past n_q are neither loaded nor computed
+    const int live = min(NQ, (p.n_q - m0 + kBlockM - 1) / kBlockM);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && n > 0) {
             const uint32_t qbar = smem_u32(&ctl->q_full);
-            mbar_arrive_expect_tx(qbar, NQ * kTileBytes);
-            for (int qt = 0; qt < NQ; ++qt)
+            mbar_arrive_expect_tx(qbar, live * kTileBytes);
+            for (int qt = 0; qt < live; ++qt)
                 for (int c = 0; c < C::kBoxes; ++c)
                     tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), &p.tm_q, qbar,
                                 c * kBoxCols, h, m0 + qt * kBlockM, b);
             uint32_t it = 0;
             bool ok = true;
             for (int j = t0; j < t1 && ok; ++j) {
-                int seg, row0, valid;
-                tile_of(ctl, j, seg, row0, valid);
-                const int kind = ctl->seg_kind[seg];
-                const int slot = ctl->seg_slot[seg];
                 for (int kv = 0; kv < 2; ++kv, ++it) {
                     const int s = it % kStages;
                     const uint32_t r = it / kStages;
@@ -203,17 +100,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                     }
                     const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
                     mbar_arrive_expect_tx(fbar, kTileBytes);
-                    const uint32_t dst = smem_u32(kv_smem + s * kTileBytes);
-                    for (int c = 0; c < C::kBoxes; ++c) {
-                        const uint32_t d = dst + c * kBoxBytes;
-                        if (kind == 0)
-                            tma_load_4d(d, kv ? &p.tm_cond_v : &p.tm_cond_k, fbar, c * kBoxCols, row0, h, b);
-                        else if (kind == 1)
-                            tma_load_5d(d, kv ? &p.tm_cache_v : &p.tm_cache_k, fbar, c * kBoxCols, row0,
-                                        slot, h, b);
-                        else
-                            tma_load_4d(d, kv ? &p.tm_vcur : &p.tm_kcur, fbar, c * kBoxCols, h, row0, b);
-                    }
+                    load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
                 }
             }
             // never leave while copies are in flight: the last fill of every stage has landed
@@ -228,36 +115,14 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
             const uint32_t q_base = smem_u32(q_smem);
             const uint32_t kv_base = smem_u32(kv_smem);
-            auto issue_s = [&](int qt, int s) {
-                const uint32_t tS = tmem + qt * kBlockN;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(q_base + qt * kTileBytes + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(kv_base + s * kTileBytes + off, 16, 1024);
-                    mma_ss(tS, a, bd, idesc_s, ks > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_pv = [&](int qt, int s, bool acc) {
-                const uint32_t tS = tmem + qt * kBlockN;
-                const uint32_t tO = tmem + NQ * kBlockN + qt * D;
-#pragma unroll
-                for (int ks = 0; ks < kBlockN / 16; ++ks) {
-                    const uint64_t bd = smem_desc_sw128(kv_base + s * kTileBytes + ks * 16 * 128,
-                                                        kBoxBytes, 1024);
-                    mma_ts(tO, tS + ks * 8, bd, idesc_o, (acc || ks > 0) ? 1u : 0u);
-                }
-            };
             bool ok = wait_or_abort(smem_u32(&ctl->q_full), 0, abort_flag);
             if (ok) ok = wait_or_abort(smem_u32(&ctl->kv_full[0]), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                for (int qt = 0; qt < NQ; ++qt) {
-                    issue_s(qt, 0);
+                for (int qt = 0; qt < live; ++qt) {
+                    issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base);
                     mma_commit(smem_u32(&ctl->s_full[qt]));
                 }
                 mma_commit(smem_u32(&ctl->kv_empty[0]));
@@ -270,10 +135,11 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                     ok = false;
                     break;
                 }
-                for (int qt = 0; qt < NQ && ok; ++qt) {
+                for (int qt = 0; qt < live && ok; ++qt) {
                     if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), jj & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(qt, sV, jj > 0);
+                    issue_pv<D>(tmem + NQ * kBlockN + qt * D, tmem + qt * kBlockN, kv_base + sV * kTileBytes,
+                                jj > 0);
                     mma_commit(smem_u32(&ctl->o_full[qt]));
                     if (more) {
                         if (qt == 0 &&
@@ -281,11 +147,10 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                             ok = false;
                             break;
                         }
-                        // P_q lives in the S_q columns: the next S_q may only be written once
-                        // this tile's PV has read P.
-                        if (!wait_or_abort(smem_u32(&ctl->o_full[qt]), jj & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        issue_s(qt, sK);
+                        // P_q lives in the S_q columns.  MMAs issued by this thread run in
+                        // issue order on the tensor pipe, so the PV above reads P_q before
+                        // this S_q overwrites it.
+                        issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
                         mma_commit(smem_u32(&ctl->s_full[qt]));
                     }
                 }
@@ -297,86 +162,29 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             mma_commit(smem_u32(&ctl->drain));
             wait_drain(smem_u32(&ctl->drain), 0);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 2 && ((warp - 2) >> 2) < live) {
         // ------------------------------------------------------------ softmax warpgroups
-        const int qt = (warp - 4) >> 2;
-        const int wq = warp & 3;                       // TMEM lane quarter of this warp
+        // warps 2..5 own Q tile 0 and warps 6..9 Q tile 1; a warp may only touch the TMEM lane
+        // quarter warp % 4, and each group of four consecutive warps covers all four quarters
+        const int qt = (warp - 2) >> 2;
+        const int wq = warp & 3;
         const int row = wq * 32 + lane;                // query row inside the tile
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         const uint32_t tS = lane_base + qt * kBlockN;
         const uint32_t tO = lane_base + NQ * kBlockN + qt * D;
-        const float sl2 = p.scale_log2;
+        const uint32_t o_bar = smem_u32(&ctl->o_full[qt]);
         float m_ref = -INFINITY;   // reference max, log2-scaled
-        float l = 0.f;             // row sum of exp2(s*sl2 - m_ref)
+        float l = 0.f;             // row sum of the bf16-rounded exp2(s*sl2 - m_ref)
         bool ok = true;
         for (int jj = 0; jj < n; ++jj) {
             int seg, row0, valid;
             tile_of(ctl, t0 + jj, seg, row0, valid);
-            ok = wait_or_abort(smem_u32(&ctl->s_full[qt]), jj & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
+            ok = warp_wait(smem_u32(&ctl->s_full[qt]), jj & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-            tmem_wait_ld_dep(sr[0]);
-            reg_fence(sr[1]);
-            reg_fence(sr[2]);
-            reg_fence(sr[3]);
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float v = __uint_as_float(sr[c][i]);
-                    if (c * 32 + i >= valid) v = -INFINITY;
-                    sr[c][i] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
-                }
-            const float m_new = mx * sl2;
-            if (jj == 0) {
-                m_ref = m_new;
-            } else {
-                const bool need = m_new > m_ref + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    float f = 1.f;
-                    if (need) {
-                        f = ex2_approx(m_ref - m_new);
-                        m_ref = m_new;
-                    }
-                    l *= f;
-                    ok = wait_or_abort(smem_u32(&ctl->o_full[qt]), (jj - 1) & 1, abort_flag);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-                        tmem_wait_ld_dep(o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                        tmem_st32(tO + c * 32, o);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            float sum = 0.f;
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][i]), sl2, -m_ref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][i + 1]), sl2, -m_ref));
-                    sum += p0 + p1;
-                    pk[c >> 1][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
-                }
-            l += sum;
-            tmem_st32(tS, pk[0]);
-            tmem_st32(tS + 32, pk[1]);
-            tmem_wait_st();
-            tc_fence_before();
+            ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (jj - 1) & 1, p.scale_log2, m_ref, l,
+                                 abort_flag);
+            if (!ok) break;
             mbar_arrive(smem_u32(&ctl->p_full[qt]));
         }
         // ------------------------------------------------------------ epilogue
@@ -390,49 +198,27 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                 p.ml_part[prow * 2 + 0] = -INFINITY;
                 p.ml_part[prow * 2 + 1] = 0.f;
             }
-        } else if (ok) {
-            ok = wait_or_abort(smem_u32(&ctl->o_full[qt]), (n - 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
-                tc_fence_after();
-                const float inv = 1.f / l;
+        } else if (ok && warp_wait(o_bar, (n - 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = 1.f / l;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + c * 32, o);
-                    tmem_wait_ld_dep(o);
-                    if (split_mode) {
-                        const size_t prow = ((size_t)blockIdx.x * p.B * p.H + bh) * kBlockM + row;
-                        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + c * 32);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld_dep(o);
+                if (split_mode) {
+                    const size_t prow = ((size_t)blockIdx.x * p.B * p.H + bh) * kBlockM + row;
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + c * 32);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
-                        if (c == 0) {
-                            p.ml_part[prow * 2 + 0] = m_ref;
-                            p.ml_part[prow * 2 + 1] = l;
-                        }
-                    } else if (m_row < p.n_q) {
-                        const size_t orow = ((size_t)b * p.n_q + m_row) * p.H + h;
-                        if (p.out_f32) {
-                            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D + c * 32);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv,
-                                                     __uint_as_float(o[4 * i + 1]) * inv,
-                                                     __uint_as_float(o[4 * i + 2]) * inv,
-                                                     __uint_as_float(o[4 * i + 3]) * inv);
-                        } else {
-                            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D + c * 32);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                dst[i] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
-                        }
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                    if (c == 0) {
+                        p.ml_part[prow * 2 + 0] = m_ref;
+                        p.ml_part[prow * 2 + 1] = l;
                     }
+                } else if (m_row < p.n_q) {
+                    store_row_chunk<D>(p.out, p.out_f32, ((size_t)b * p.n_q + m_row) * p.H + h, c, o, inv);
                 }
             }
         }

@@ -1,0 +1,377 @@
+// attn_persistent.cu -- the full-chunk attention as a persistent, load-balanced kernel.
+//
+// Same computation and warp roles as attn_fwd_kernel (TMA producer, one-thread tcgen05 MMA
+// issuer, one softmax warpgroup per 128-row Q tile), but the grid is one CTA per SM and the
+// work is cut evenly.  Work items are (pair of Q tiles, key tile) of every (b, h), costed by
+// the number of live Q tiles (1 or 2), laid out in one line; CTA g takes the items whose
+// start cost falls in [g C / G, (g+1) C / G).  Each SM therefore does the same amount of
+// tensor work whatever the number of query blocks, so there is no partial last wave.
+//
+// A pair whose key tiles are cut between CTAs ("split piece") is merged without any
+// inter-CTA waiting: every piece writes its unnormalised O row block and its (max, sum)
+// to a scratch slot, then bumps a per-pair counter; the piece that sees the counter reach
+// npieces - 1 is last, reads the others' partials (log-sum-exp merge) and writes the output,
+// then clears the counter for the next launch.
+//
+// Within a CTA, consecutive pieces overlap: the producer streams the next piece's Q and K/V
+// while the softmax warpgroups finish the previous piece's epilogue; the first P V of a
+// piece waits only until the epilogue has read the previous O out of TMEM.
+#include "attn_common.cuh"
+
+namespace swattn {
+
+struct Piece {
+    int bh;     // stream * H + head
+    int pair;   // index of the Q-tile pair within the head (rows pair * 256 ...)
+    int live;   // Q tiles of the pair that hold queries (1 or 2)
+    int j0, j1; // key tiles [j0, j1) of this piece
+};
+
+// Next piece of the range [cur, c1) of the cost line (nqt Q tiles per head, nt key tiles).
+__device__ __forceinline__ bool next_piece(long long& cur, long long c1, int nqt, int nt, Piece& pc) {
+    const long long per_bh = (long long)nqt * nt;
+    while (cur < c1) {
+        const int bh = (int)(cur / per_bh);
+        const long long r = cur - (long long)bh * per_bh;
+        const int i = (int)(r / (2LL * nt));
+        const int lv = min(2, nqt - 2 * i);
+        const long long ps = (long long)bh * per_bh + 2LL * i * nt;
+        const int j0 = (int)((cur - ps + lv - 1) / lv);     // first item starting at or after cur
+        if (j0 >= nt) {
+            cur = ps + (long long)lv * nt;
+            continue;
+        }
+        const long long e = (c1 - ps + lv - 1) / lv;       // first item starting at or after c1
+        const int j1 = (int)(e < nt ? e : nt);
+        cur = ps + (long long)lv * j1;
+        pc.bh = bh;
+        pc.pair = i;
+        pc.live = lv;
+        pc.j0 = j0;
+        pc.j1 = j1;
+        return true;
+    }
+    return false;
+}
+
+// The CTA whose cost range [g C / G, (g+1) C / G) contains cost position s.
+__device__ __forceinline__ int cta_of(long long s, long long C, int G) {
+    return (int)(((s + 1) * G - 1) / C);
+}
+
+// Barrier over the 128 threads of softmax warpgroup qt (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void wg_bar(int qt) {
+    if (qt == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+    else asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnLayout<D, 2>::kThreads, 1)
+attn_persistent_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int NQ = 2;
+    using C = TileCfg<D>;
+    using L = AttnLayout<D, NQ>;
+    constexpr int kStages = C::kStages;
+    constexpr int kTileBytes = C::kTileBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* q_smem = base;
+    uint8_t* kv_smem = base + L::kQBytes;
+    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(base + L::kCtlOffset);
+    volatile int* abort_flag = &ctl->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (warp == 0) {
+        if (lane == 0) init_barriers(ctl, kStages);
+        __syncwarp();
+        tmem_alloc(smem_u32(&ctl->tmem_base), L::kTmemCols);
+        tmem_relinquish();
+    } else if (warp == 2 && lane == 0) {
+        load_table(ctl, p.table, p.status);
+    } else if (warp == 1 && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_kcur);
+        tma_prefetch_desc(&p.tm_vcur);
+        tma_prefetch_desc(&p.tm_cache_k);
+        tma_prefetch_desc(&p.tm_cache_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = ctl->tmem_base;
+    const int G = gridDim.x;
+    const int g = blockIdx.x;
+    const int nt = ctl->n_tiles;
+    const int nqt = (p.n_q + kBlockM - 1) / kBlockM;
+    const long long Ctot = (long long)p.B * p.H * nqt * nt;
+    const long long c0 = (long long)g * Ctot / G;
+    const long long c1 = (long long)(g + 1) * Ctot / G;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && nt > 0) {
+            const uint32_t qbar = smem_u32(&ctl->q_full);
+            long long cur = c0;
+            Piece pc;
+            uint32_t it = 0;
+            int pi = 0;
+            bool ok = true;
+            while (ok && next_piece(cur, c1, nqt, nt, pc)) {
+                const int b = pc.bh / p.H, h = pc.bh % p.H;
+                const int m0 = pc.pair * NQ * kBlockM;
+                // the Q buffers are reused: wait until every S MMA of the previous piece is done
+                if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(qbar, pc.live * kTileBytes);
+                for (int qt = 0; qt < pc.live; ++qt)
+                    for (int c = 0; c < C::kBoxes; ++c)
+                        tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), &p.tm_q, qbar,
+                                    c * kBoxCols, h, m0 + qt * kBlockM, b);
+                ++pi;
+                for (int j = pc.j0; j < pc.j1 && ok; ++j) {
+                    for (int kv = 0; kv < 2; ++kv, ++it) {
+                        const int s = it % kStages;
+                        const uint32_t r = it / kStages;
+                        if (!wait_or_abort(smem_u32(&ctl->kv_empty[s]), (r & 1) ^ 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
+                        mbar_arrive_expect_tx(fbar, kTileBytes);
+                        load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                    }
+                }
+            }
+            for (int s = 0; s < kStages; ++s) {
+                if (it > (uint32_t)s) {
+                    const uint32_t uses = (it - 1 - s) / kStages + 1;
+                    wait_drain(smem_u32(&ctl->kv_full[s]), (uses - 1) & 1);
+                }
+            }
+            if (pi > 0) wait_drain(qbar, (pi - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nt > 0) {
+            const uint32_t q_base = smem_u32(q_smem);
+            const uint32_t kv_base = smem_u32(kv_smem);
+            long long cur = c0;
+            Piece pc;
+            uint32_t it = 0;          // K/V tiles consumed so far (ring position)
+            int pi = 0;               // pieces started
+            uint32_t tcnt[2] = {0, 0};   // key tiles processed per Q tile (p_full phases)
+            uint32_t ucnt[2] = {0, 0};   // pieces finished per Q tile (o_empty phases)
+            bool ok = true;
+            while (ok && next_piece(cur, c1, nqt, nt, pc)) {
+                const int n = pc.j1 - pc.j0;
+                const int live = pc.live;
+                if (!wait_or_abort(smem_u32(&ctl->q_full), pi & 1, abort_flag)) break;
+                ++pi;
+                const int s0 = it % kStages;
+                if (!wait_or_abort(smem_u32(&ctl->kv_full[s0]), (it / kStages) & 1, abort_flag)) break;
+                tc_fence_after();
+                for (int qt = 0; qt < live; ++qt) {
+                    issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + s0 * kTileBytes);
+                    mma_commit(smem_u32(&ctl->s_full[qt]));
+                }
+                if (n == 1) mma_commit(smem_u32(&ctl->q_empty));
+                mma_commit(smem_u32(&ctl->kv_empty[s0]));
+                for (int jj = 0; jj < n && ok; ++jj) {
+                    const uint32_t itV = it + 2 * jj + 1, itK = it + 2 * jj + 2;
+                    const int sV = itV % kStages, sK = itK % kStages;
+                    const bool more = jj + 1 < n;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int qt = 0; qt < live && ok; ++qt) {
+                        if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (jj == 0 && ucnt[qt] > 0) {
+                            // the previous piece's O must be out of TMEM before it is overwritten
+                            if (!wait_or_abort(smem_u32(&ctl->o_empty[qt]), (ucnt[qt] - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        issue_pv<D>(tmem + NQ * kBlockN + qt * D, tmem + qt * kBlockN, kv_base + sV * kTileBytes,
+                                    jj > 0);
+                        mma_commit(smem_u32(&ctl->o_full[qt]));
+                        ++tcnt[qt];
+                        if (more) {
+                            if (qt == 0 &&
+                                !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            // in issue order after the PV that reads P_q from the same columns
+                            issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
+                            mma_commit(smem_u32(&ctl->s_full[qt]));
+                        }
+                    }
+                    if (!ok) break;
+                    if (more && jj + 2 == n) mma_commit(smem_u32(&ctl->q_empty));   // last S issued
+                    mma_commit(smem_u32(&ctl->kv_empty[sV]));
+                    if (more) mma_commit(smem_u32(&ctl->kv_empty[sK]));
+                }
+                for (int qt = 0; qt < live; ++qt) ++ucnt[qt];
+                it += 2 * n;
+            }
+            mma_commit(smem_u32(&ctl->drain));
+            wait_drain(smem_u32(&ctl->drain), 0);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int qt = (warp - 2) >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t tS = lane_base + qt * kBlockN;
+        const uint32_t tO = lane_base + NQ * kBlockN + qt * D;
+        const uint32_t o_bar = smem_u32(&ctl->o_full[qt]);
+        long long cur = c0;
+        Piece pc;
+        int pi = 0;
+        uint32_t tcnt = 0;
+        bool ok = nt > 0;
+        while (ok && next_piece(cur, c1, nqt, nt, pc)) {
+            const bool first_in_cta = pi == 0;
+            ++pi;
+            if (qt >= pc.live) continue;
+            const int n = pc.j1 - pc.j0;
+            float m_ref = -INFINITY, l = 0.f;
+            for (int jj = 0; jj < n; ++jj) {
+                int seg, row0, valid;
+                tile_of(ctl, pc.j0 + jj, seg, row0, valid);
+                ok = warp_wait(smem_u32(&ctl->s_full[qt]), tcnt & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (tcnt - 1) & 1, p.scale_log2, m_ref, l,
+                                     abort_flag);
+                if (!ok) break;
+                mbar_arrive(smem_u32(&ctl->p_full[qt]));
+                ++tcnt;
+            }
+            if (!ok) break;
+            // ---------------------------------------------------- epilogue of this piece
+            ok = warp_wait(o_bar, (tcnt - 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t o[D / 32][32];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+            tmem_wait_ld_dep(o[0]);
+#pragma unroll
+            for (int c = 1; c < D / 32; ++c) reg_fence(o[c]);
+            tc_fence_before();
+            mbar_arrive(smem_u32(&ctl->o_empty[qt]));   // O may now be overwritten
+
+            const int b = pc.bh / p.H, h = pc.bh % p.H;
+            const int m_row = pc.pair * NQ * kBlockM + qt * kBlockM + row;
+            const size_t orow = ((size_t)b * p.n_q + m_row) * p.H + h;
+            if (pc.j0 == 0 && pc.j1 == nt) {
+                const float inv = 1.f / l;
+                if (m_row < p.n_q) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(p.out, p.out_f32, orow, c, o[c], inv);
+                }
+                continue;
+            }
+            // split piece: publish the partial, then the last of the pair's pieces merges
+            const long long ps = (long long)pc.bh * nqt * nt + 2LL * pc.pair * nt;
+            const int g_first = cta_of(ps, Ctot, G);
+            const int g_last = cta_of(ps + (long long)pc.live * (nt - 1), Ctot, G);
+            const int npieces = g_last - g_first + 1;
+            const int slot = first_in_cta ? 2 * g : 2 * g + 1;
+            float* so = p.sk_o + ((size_t)slot * 2 + qt) * D * kBlockM;     // [D][128 rows]
+            float* sml = p.sk_ml + ((size_t)slot * 2 + qt) * kBlockM * 2;   // [128 rows][2]
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) so[(c * 32 + i) * kBlockM + row] = __uint_as_float(o[c][i]);
+            sml[row * 2 + 0] = m_ref;
+            sml[row * 2 + 1] = l;
+            __threadfence();
+            wg_bar(qt);
+            int* cnt = p.sk_cnt + ((size_t)pc.bh * p.sk_pairs + pc.pair) * 2 + qt;
+            if (row == 0) ctl->merge_flag[qt] = atomicAdd(cnt, 1);
+            wg_bar(qt);
+            if (ctl->merge_flag[qt] != npieces - 1) continue;     // another piece will merge
+            __threadfence();
+            // the pair's first piece is CTA g_first's last piece unless it opens that CTA's range
+            bool opens_first = false;
+            {
+                long long cf = (long long)g_first * Ctot / G;
+                Piece fp;
+                if (next_piece(cf, (long long)(g_first + 1) * Ctot / G, nqt, nt, fp))
+                    opens_first = fp.bh == pc.bh && fp.pair == pc.pair;
+            }
+            float M = m_ref;
+            for (int gg = g_first; gg <= g_last; ++gg) {
+                if (gg == g) continue;
+                const int sl = (gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1;
+                M = fmaxf(M, __ldcg(p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2));
+            }
+            const float ws = ex2_approx(m_ref - M);
+            float L_ = l * ws;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[c][i] = __float_as_uint(__uint_as_float(o[c][i]) * ws);
+            for (int gg = g_first; gg <= g_last; ++gg) {
+                if (gg == g) continue;
+                const int sl = (gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1;
+                const float* pml = p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2;
+                const float w = ex2_approx(__ldcg(pml) - M);
+                L_ += w * __ldcg(pml + 1);
+                const float* po = p.sk_o + ((size_t)sl * 2 + qt) * D * kBlockM + row;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[c][i] = __float_as_uint(fmaf(w, __ldcg(po + (c * 32 + i) * kBlockM), __uint_as_float(o[c][i])));
+            }
+            const float inv = 1.f / L_;
+            if (m_row < p.n_q) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(p.out, p.out_f32, orow, c, o[c], inv);
+            }
+            if (row == 0) atomicExch(cnt, 0);   // all pieces have arrived: ready for the next launch
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+    if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
+}
+
+template <int D>
+static cudaError_t launch_persistent_d(const AttnParams& p, int ctas, cudaStream_t stream) {
+    using L = AttnLayout<D, 2>;
+    auto kern = attn_persistent_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, L::kThreads, L::kSmemBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream) {
+    if (ctas < 1 || ctas > kMaxPersistentCtas) return cudaErrorInvalidValue;
+    if (d == 128) return launch_persistent_d<128>(p, ctas, stream);
+    if (d == 64) return launch_persistent_d<64>(p, ctas, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace swattn

@@ -61,9 +61,18 @@ cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int 
     return cudaGetLastError();
 }
 
+__global__ void zero_kernel(int32_t* p, long long n) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        p[i] = 0;
+}
+
 cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
-                               cudaStream_t stream) {
+                               int32_t* counters, long long n_counters, cudaStream_t stream) {
     table_build_kernel<<<1, 32, 0, stream>>>(state, W, sink, n_cond, T, 0, 1);
+    if (n_counters > 0) {
+        const long long blocks = (n_counters + 255) / 256;
+        zero_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(counters, n_counters);
+    }
     return cudaGetLastError();
 }
 

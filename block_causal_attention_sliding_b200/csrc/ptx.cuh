@@ -62,6 +62,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// ------------------------------------------------------------------ register split
+
+// Warpgroup-wide register re-allocation.  The sum over warpgroups of the new counts must stay
+// within the block's launch allocation (threads x registers at launch), or an increase waits.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ TMA (tiled, no multicast)
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {

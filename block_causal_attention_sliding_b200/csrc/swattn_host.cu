@@ -24,6 +24,9 @@ struct sw_attn {
     int max_splits = 1;
     int short_q = 0;           // n_q <= short_q uses the split-K path (0: never)
     size_t off_kcache = 0, off_vcache = 0, off_kcond = 0, off_vcond = 0, off_opart = 0, off_ml = 0;
+    size_t off_sk_o = 0, off_sk_ml = 0, off_sk_cnt = 0;
+    int sk_pairs = 0;
+    long long n_counters = 0;
     size_t total = 0;
     char* ws = nullptr;
     size_t ws_bytes = 0;
@@ -101,6 +104,7 @@ int check_cfg(const sw_attn_config& c) {
     if (c.out_dtype != SW_OUT_BF16 && c.out_dtype != SW_OUT_F32) return fail(SW_EINVAL, "bad out_dtype");
     if (c.max_short_q > kMaxShortQ) return fail(SW_ESHAPE, "max_short_q must be <= %d", kMaxShortQ);
     if (!std::isfinite(c.scale)) return fail(SW_EINVAL, "scale must be finite");
+    if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID) return fail(SW_EINVAL, "bad schedule");
     const double elems = (double)c.B * c.H * (c.W + 1) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
         (double)c.n_cond * c.H * c.B > 2.0e9)
@@ -139,6 +143,12 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * d * 4, 1024);
     h->off_ml = off;
     if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * 2 * 4, 1024);
+    // persistent schedule: two partial slots per CTA and one counter per (b, h, pair, Q tile)
+    h->sk_pairs = (cfg->tokens_per_chunk + 2 * kBlockM - 1) / (2 * kBlockM);
+    h->n_counters = (long long)bh * h->sk_pairs * 2;
+    h->off_sk_o = off;   off = align_up(off + (size_t)2 * kMaxPersistentCtas * 2 * d * kBlockM * 4, 1024);
+    h->off_sk_ml = off;  off = align_up(off + (size_t)2 * kMaxPersistentCtas * 2 * kBlockM * 2 * 4, 1024);
+    h->off_sk_cnt = off; off = align_up(off + (size_t)h->n_counters * 4, 1024);
     h->total = off;
     *out = h;
     return SW_OK;
@@ -148,7 +158,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     sw_attn_config c;
     std::memset(&c, 0, sizeof c);
     c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
-    c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0;
+    c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_PERSISTENT;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -192,6 +202,7 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, strides, box, "V cond"))) return rc;
     }
     e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, c.sink, c.n_cond, c.tokens_per_chunk,
+                           reinterpret_cast<int32_t*>(ws + h->off_sk_cnt), h->n_counters,
                            static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state reset launch");
     h->ws = ws;
@@ -208,7 +219,8 @@ int sw_attn_reset(sw_attn_t* h, void* stream) {
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     const sw_attn_config& c = h->cfg;
     cudaError_t e = launch_state_reset(reinterpret_cast<int32_t*>(h->ws), c.W, c.sink, c.n_cond,
-                                       c.tokens_per_chunk, static_cast<cudaStream_t>(stream));
+                                       c.tokens_per_chunk, reinterpret_cast<int32_t*>(h->ws + h->off_sk_cnt),
+                                       h->n_counters, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "state reset launch");
 }
 
@@ -292,11 +304,26 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
         e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
         if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-    } else {
+    } else if (c.schedule == SW_SCHED_GRID) {
         p.splits = 0;
         const int grid_x = (n_q + 2 * kBlockM - 1) / (2 * kBlockM);
         e = launch_attention(p, c.d, 2, grid_x, st);
         if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    } else {
+        p.splits = 0;
+        p.sk_o = reinterpret_cast<float*>(h->ws + h->off_sk_o);
+        p.sk_ml = reinterpret_cast<float*>(h->ws + h->off_sk_ml);
+        p.sk_cnt = reinterpret_cast<int32_t*>(h->ws + h->off_sk_cnt);
+        p.sk_pairs = h->sk_pairs;
+        // one CTA per SM, but never so many that a CTA's share of the cost line is shorter than
+        // two items at the fewest key tiles a chunk can have (condition + current only)
+        const long long nqt = (n_q + kBlockM - 1) / kBlockM;
+        const long long nt_min = (c.n_cond + kBlockN - 1) / kBlockN + (c.tokens_per_chunk + kBlockN - 1) / kBlockN;
+        const long long c_min = (long long)c.B * c.H * nqt * nt_min;
+        long long ctas = std::min<long long>(h->num_sms, kMaxPersistentCtas);
+        ctas = std::max<long long>(1, std::min<long long>(ctas, c_min / 2));
+        e = launch_persistent(p, c.d, (int)ctas, st);
+        if (e != cudaSuccess) return cuda_fail(e, "persistent attention launch");
     }
     return SW_OK;
 }

@@ -15,6 +15,7 @@ constexpr int kMaxW = 64;          // largest window supported
 constexpr int kStateHeaderInts = 16;   // [0] chunks committed, [1] status bits, rest reserved
 constexpr int kMaxShortQ = 128;    // split-K path handles one Q tile per (b, h)
 constexpr int kMaxSplits = 64;
+constexpr int kMaxPersistentCtas = 160;   // >= SMs of a B200 (148)
 
 __host__ __device__ inline int table_ints_for(int W) { return 3 + 4 * (W + 3); }
 
@@ -42,13 +43,18 @@ struct alignas(64) AttnParams {
     int out_f32;
     int splits;              // 0: full mode (normalised output); >= 1: split-K partials
     float scale_log2;        // softmax scale * log2(e)
+    // persistent kernel: partials of pieces whose key tiles are cut between CTAs
+    float* sk_o;             // [2 * kMaxPersistentCtas slots][2 Q tiles][d][128 rows] fp32
+    float* sk_ml;            // [slots][2][128 rows][2] (row max log2-scaled, row sum)
+    int32_t* sk_cnt;         // [B*H][sk_pairs][2] arrival counters, zero between launches
+    int sk_pairs;            // Q-tile pairs per (b, h) the counters are sized for
 };
 
 // kernel launchers (defined in the .cu files)
 cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int T, int advance,
                                cudaStream_t stream);
 cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
-                               cudaStream_t stream);
+                               int32_t* counters, long long n_counters, cudaStream_t stream);
 // Copy [B, N, H, d] bf16 K and V into [B][H][rows_per_bh][d] regions at row offset
 // slot * N (slot from the device counter when `ring` is set, else 0).
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
@@ -56,6 +62,7 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
                             int32_t* state, cudaStream_t stream);
 cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
                              cudaStream_t stream);
+cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream);
 cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
                            int n_q, int d, int splits, int out_f32, cudaStream_t stream);
 

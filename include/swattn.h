@@ -76,8 +76,14 @@ typedef struct {
     int   sink;              /* 1: chunk 0 is pinned as the global sink */
     int   out_dtype;         /* SW_OUT_BF16 or SW_OUT_F32 */
     float scale;             /* softmax scale; <= 0 selects 1/sqrt(d) */
-    int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128 */
+    int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128,
+                                negative disables the split-K path */
+    int   schedule;          /* full path: SW_SCHED_PERSISTENT (default) or SW_SCHED_GRID */
 } sw_attn_config;
+
+/* schedules of the full path */
+#define SW_SCHED_PERSISTENT 0   /* one CTA per SM, key tiles cut evenly (stream-K) */
+#define SW_SCHED_GRID       1   /* one CTA per 256 query rows of each (b, h) */
 
 /*
  * Create a handle with B = 1, sink on, bf16 output, scale 1/sqrt(d).  Host only: allocates
