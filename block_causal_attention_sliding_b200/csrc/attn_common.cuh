@@ -11,6 +11,25 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: far above any legitim
 constexpr int kBoxCols = 64;                        // 128-byte swizzle atom = 64 bf16
 constexpr int kBoxBytes = kBlockM * kBoxCols * 2;   // 16 KB: one TMA box (128 rows x 64 cols)
 constexpr float kRescaleThreshold = 8.0f;           // log2 units: rescale O when max grows > 2^8
+// One in kPolyEvery pairs of exponentials runs on the FMA pipe (exp2_poly) instead of MUFU
+// (0: none).  At two Q tiles per CTA the exponentials alone keep MUFU as busy as the tensor
+// core, but the softmax step is bound by issue and latency first; measured, not assumed.
+#ifndef SWATTN_POLY_EVERY
+#define SWATTN_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = SWATTN_POLY_EVERY;
+// Publish P in two halves (PV of the first 64 keys overlaps the exponentials of the rest).
+#ifndef SWATTN_SPLIT_P
+#define SWATTN_SPLIT_P 1
+#endif
+constexpr bool kSplitP = SWATTN_SPLIT_P != 0;
+// MMA issuer serves whichever Q tile is ready (1) or strictly alternates between them (0).
+// Measured on B200: polling both tiles costs the softmax warps that share the MMA warp's
+// sub-partition more issue slots than it saves, so alternating is the default.
+#ifndef SWATTN_DYNAMIC_MMA
+#define SWATTN_DYNAMIC_MMA 0
+#endif
+constexpr bool kDynamicMma = SWATTN_DYNAMIC_MMA != 0;
 
 template <int D>
 struct TileCfg {
@@ -25,6 +44,7 @@ struct SmemCtl {
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
     uint64_t s_full[2];
+    uint64_t p_half[2];         // first 64 keys of P written (PV may start on them)
     uint64_t p_full[2];
     uint64_t o_full[2];
     uint64_t o_empty[2];
@@ -63,6 +83,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     int never = 0;
     (void)mbar_wait(bar, parity, &never, kWaitLimitNs);
+}
+
+// One arrival per warp: the warp's lanes finish their work (and tcgen05 fences) first.  128
+// single-thread arrivals on one barrier word serialise for hundreds of cycles.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Warp-uniform wait for the softmax warps.
@@ -154,16 +181,33 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_ti
                (accumulate || ks > 0) ? 1u : 0u);
 }
 
+// Half of O += P V: keys [64 half, 64 half + 64) of the tile (4 MMA steps of 16 keys).
+template <int D>
+__device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t v_tile, int half,
+                                              bool accumulate) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
+#pragma unroll
+    for (int k = 0; k < kBlockN / 32; ++k) {
+        const int ks = half * (kBlockN / 32) + k;
+        mma_ts(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
+               (accumulate || ks > 0) ? 1u : 0u);
+    }
+}
+
 // One online-softmax step for this thread's query row over one key tile:
 //   read the S row from TMEM, mask keys past the segment's end, update the reference max
 //   (lazily: only when it grows by more than 2^kRescaleThreshold), write P = exp2(s*sl2 - m)
 //   as bf16 pairs over the S columns, add the same rounded weights to l, and rescale the
 //   O row in TMEM when the reference moved (after waiting for the previous PV).
-// The caller has waited for S and arrives on p_full afterwards.  Returns false on abort.
+// P is published in two halves: the warp arrives on p_half_bar once keys 0..63 are written
+// (the PV of those keys may then start) and the caller arrives on p_full after the return.
+// A warp that must rescale O first publishes nothing early: its O rescale has to land before
+// any PV of this tile.  The caller has waited for S.  Returns false on abort.
 template <int D>
 __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
-                                             uint32_t o_full_bar, uint32_t prev_pv_parity, float sl2,
-                                             float& m_ref, float& l, volatile int* abort_flag) {
+                                             uint32_t o_full_bar, uint32_t prev_pv_parity,
+                                             uint32_t p_half_bar, float sl2, float& m_ref, float& l,
+                                             volatile int* abort_flag) {
     uint32_t sr[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
@@ -179,12 +223,19 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
             for (int i = 0; i < 32; ++i)
                 if (c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
     }
-    float mx = -INFINITY;
+    // row max as an 8-way tree: independent accumulators keep the dependent chain short
+    float mxa[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mxa[a] = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
-    const float m_new = mx * sl2;
+        for (int i = 0; i < 32; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], __uint_as_float(sr[c][i]));
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int a = 0; a < w; ++a) mxa[a] = fmaxf(mxa[a], mxa[a + w]);
+    const float m_new = mxa[0] * sl2;
     float f = 1.f;            // factor that takes O and l to the new reference max
     bool rescale = false;     // warp-uniform: does this warp rescale O this tile
     if (first) {
@@ -197,7 +248,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
             m_ref = m_new;
         }
     }
-    float sum = 0.f;
+    float suma[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) suma[a] = 0.f;
+    const float neg_m = -m_ref;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -206,21 +260,39 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
             const int c = 2 * half + cc;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][i]), sl2, -m_ref));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][i + 1]), sl2, -m_ref));
+                const float x0 = fmaf(__uint_as_float(sr[c][i]), sl2, neg_m);
+                const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), sl2, neg_m);
+                const bool poly = kPolyEvery > 0 && ((i >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+                const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+                const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
                 const uint32_t pp = pack_bf16x2(p0, p1);
                 // the row sum adds the same bf16-rounded weights the PV MMA multiplies, so
-                // out is an exact weighted mean of V under those weights
-                sum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
+                // out is an exact weighted mean of V under those weights (8 accumulators)
+                const int a = (i >> 1) & 7;
+                suma[a] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
                 pk[cc * 16 + (i >> 1)] = pp;
             }
         }
         tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
+        if (half == 0 && !rescale && kSplitP) {
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(p_half_bar);
+        }
     }
-    l = l * f + sum;
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int a = 0; a < w; ++a) suma[a] += suma[a + w];
+    l = l * f + suma[0];
+    if (!rescale && !kSplitP) {
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(p_half_bar);
+    }
     if (rescale) {
         // done once the S row is dead (low register pressure); it must land before this
-        // tile's PV, which the caller's p_full arrival releases
+        // tile's PV, which waits for p_half (arrived below) and p_full
         if (!warp_wait(o_full_bar, prev_pv_parity, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll 1
@@ -232,6 +304,9 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
             tmem_st32(tO + c * 32, o);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(p_half_bar);
     }
     tmem_wait_st();
     tc_fence_before();
@@ -269,9 +344,10 @@ __device__ __forceinline__ void init_barriers(SmemCtl* ctl, int stages) {
     }
     for (int q = 0; q < 2; ++q) {
         mbar_init(smem_u32(&ctl->s_full[q]), 1);
-        mbar_init(smem_u32(&ctl->p_full[q]), 128);
+        mbar_init(smem_u32(&ctl->p_half[q]), 4);    // one arrival per softmax warp
+        mbar_init(smem_u32(&ctl->p_full[q]), 4);
         mbar_init(smem_u32(&ctl->o_full[q]), 1);
-        mbar_init(smem_u32(&ctl->o_empty[q]), 128);
+        mbar_init(smem_u32(&ctl->o_empty[q]), 4);
     }
     mbar_init(smem_u32(&ctl->drain), 1);
     ctl->abort_flag = 0;

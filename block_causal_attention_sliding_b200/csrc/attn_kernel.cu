@@ -127,36 +127,119 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                 }
                 mma_commit(smem_u32(&ctl->kv_empty[0]));
             }
-            for (int jj = 0; jj < n && ok; ++jj) {
-                const uint32_t itV = 2 * jj + 1, itK = 2 * jj + 2;
-                const int sV = itV % kStages, sK = itK % kStages;
-                const bool more = jj + 1 < n;
-                if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                for (int qt = 0; qt < live && ok; ++qt) {
-                    if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), jj & 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_pv<D>(tmem + NQ * kBlockN + qt * D, tmem + qt * kBlockN, kv_base + sV * kTileBytes,
-                                jj > 0);
-                    mma_commit(smem_u32(&ctl->o_full[qt]));
-                    if (more) {
-                        if (qt == 0 &&
-                            !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
-                            ok = false;
-                            break;
+            if (kDynamicMma) {
+                // One small state machine per Q tile, polled without blocking: PV of the first
+                // half of P (needs V_j and p_half), PV of the second half (p_full), then S of the
+                // next tile (needs K_j+1).  Whichever tile is ready is served, so one softmax
+                // warpgroup never waits behind the other.  Per tile the issue order is unchanged
+                // (PV_j before S_j+1 over the same columns).  A K or V stage is released once
+                // every live tile has issued the MMAs that read it.
+                int jq[2] = {0, 0}, ph[2] = {0, 0};
+                // per tile j mod 4: how many Q tiles have issued the MMAs reading V_j / K_j,
+                // as 2-bit fields of one register each (no local memory)
+                uint32_t cntV = 0, cntK = 0;
+                int remaining = ok ? live : 0;
+                uint32_t idle = 0;
+                uint64_t t_idle = 0;
+                while (remaining > 0) {
+                    bool prog = false;
+#pragma unroll
+                    for (int qt = 0; qt < NQ; ++qt) {
+                        if (qt >= live || jq[qt] >= n) continue;
+                        const int j = jq[qt];
+                        const uint32_t itV = 2 * j + 1, itK = 2 * j + 2;
+                        const int sV = itV % kStages, sK = itK % kStages;
+                        const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
+                        if (ph[qt] == 0 && mbar_test(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1) &&
+                            mbar_test(smem_u32(&ctl->p_half[qt]), j & 1)) {
+                            tc_fence_after();
+                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, j > 0);
+                            ph[qt] = 1;
+                            prog = true;
                         }
-                        // P_q lives in the S_q columns.  MMAs issued by this thread run in
-                        // issue order on the tensor pipe, so the PV above reads P_q before
-                        // this S_q overwrites it.
-                        issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
-                        mma_commit(smem_u32(&ctl->s_full[qt]));
+                        if (ph[qt] == 1 && mbar_test(smem_u32(&ctl->p_full[qt]), j & 1)) {
+                            tc_fence_after();
+                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                            mma_commit(smem_u32(&ctl->o_full[qt]));
+                            const int shV = 2 * (j & 3);
+                            cntV += 1u << shV;
+                            if ((int)((cntV >> shV) & 3u) == live) {
+                                mma_commit(smem_u32(&ctl->kv_empty[sV]));
+                                cntV &= ~(3u << shV);
+                            }
+                            if (j + 1 < n) {
+                                ph[qt] = 2;
+                            } else {
+                                jq[qt] = n;
+                                --remaining;
+                            }
+                            prog = true;
+                        }
+                        if (ph[qt] == 2 && mbar_test(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1)) {
+                            tc_fence_after();
+                            issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
+                            mma_commit(smem_u32(&ctl->s_full[qt]));
+                            const int shK = 2 * ((j + 1) & 3);
+                            cntK += 1u << shK;
+                            if ((int)((cntK >> shK) & 3u) == live) {
+                                mma_commit(smem_u32(&ctl->kv_empty[sK]));
+                                cntK &= ~(3u << shK);
+                            }
+                            jq[qt] = j + 1;
+                            ph[qt] = 0;
+                            prog = true;
+                        }
                     }
+                    if (prog) {
+                        idle = 0;
+                        continue;
+                    }
+                    // nothing ready: back off briefly, and give up after the wait limit
+                    if (*abort_flag) break;
+                    if (idle++ == 0) t_idle = globaltimer_ns();
+                    else if ((idle & 255) == 0 && globaltimer_ns() - t_idle > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    __nanosleep(20);
                 }
-                if (!ok) break;
-                mma_commit(smem_u32(&ctl->kv_empty[sV]));
-                if (more) mma_commit(smem_u32(&ctl->kv_empty[sK]));
+            } else {
+                for (int jj = 0; jj < n && ok; ++jj) {
+                    const uint32_t itV = 2 * jj + 1, itK = 2 * jj + 2;
+                    const int sV = itV % kStages, sK = itK % kStages;
+                    const bool more = jj + 1 < n;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int qt = 0; qt < live && ok; ++qt) {
+                        // P arrives in two halves; the PV of the first 64 keys overlaps the softmax
+                        // of the other 64
+                        const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
+                        if (!wait_or_abort(smem_u32(&ctl->p_half[qt]), jj & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                        if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), jj & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                        mma_commit(smem_u32(&ctl->o_full[qt]));
+                        if (more) {
+                            if (qt == 0 &&
+                                !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            // P_q lives in the S_q columns.  MMAs issued by this thread run in
+                            // issue order on the tensor pipe, so the PV above reads P_q before
+                            // this S_q overwrites it.
+                            issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
+                            mma_commit(smem_u32(&ctl->s_full[qt]));
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&ctl->kv_empty[sV]));
+                    if (more) mma_commit(smem_u32(&ctl->kv_empty[sK]));
+                }
             }
             // every MMA issued has completed before the CTA can release TMEM
             mma_commit(smem_u32(&ctl->drain));
@@ -182,10 +265,10 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             ok = warp_wait(smem_u32(&ctl->s_full[qt]), jj & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (jj - 1) & 1, p.scale_log2, m_ref, l,
-                                 abort_flag);
+            ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (jj - 1) & 1, smem_u32(&ctl->p_half[qt]),
+                                 p.scale_log2, m_ref, l, abort_flag);
             if (!ok) break;
-            mbar_arrive(smem_u32(&ctl->p_full[qt]));
+            warp_arrive(smem_u32(&ctl->p_full[qt]));
         }
         // ------------------------------------------------------------ epilogue
         const int m_row = m0 + qt * kBlockM + row;

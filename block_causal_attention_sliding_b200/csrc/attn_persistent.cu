@@ -189,7 +189,8 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     for (int qt = 0; qt < live && ok; ++qt) {
-                        if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                        const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
+                        if (!wait_or_abort(smem_u32(&ctl->p_half[qt]), tcnt[qt] & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -202,8 +203,13 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                             }
                             tc_fence_after();
                         }
-                        issue_pv<D>(tmem + NQ * kBlockN + qt * D, tmem + qt * kBlockN, kv_base + sV * kTileBytes,
-                                    jj > 0);
+                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                        if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                         mma_commit(smem_u32(&ctl->o_full[qt]));
                         ++tcnt[qt];
                         if (more) {
@@ -254,10 +260,10 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 ok = warp_wait(smem_u32(&ctl->s_full[qt]), tcnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (tcnt - 1) & 1, p.scale_log2, m_ref, l,
-                                     abort_flag);
+                ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (tcnt - 1) & 1, smem_u32(&ctl->p_half[qt]),
+                                     p.scale_log2, m_ref, l, abort_flag);
                 if (!ok) break;
-                mbar_arrive(smem_u32(&ctl->p_full[qt]));
+                warp_arrive(smem_u32(&ctl->p_full[qt]));
                 ++tcnt;
             }
             if (!ok) break;
@@ -272,7 +278,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 #pragma unroll
             for (int c = 1; c < D / 32; ++c) reg_fence(o[c]);
             tc_fence_before();
-            mbar_arrive(smem_u32(&ctl->o_empty[qt]));   // O may now be overwritten
+            warp_arrive(smem_u32(&ctl->o_empty[qt]));   // O may now be overwritten
 
             const int b = pc.bh / p.H, h = pc.bh % p.H;
             const int m_row = pc.pair * NQ * kBlockM + qt * kBlockM + row;
@@ -314,21 +320,20 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 if (next_piece(cf, (long long)(g_first + 1) * Ctot / G, nqt, nt, fp))
                     opens_first = fp.bh == pc.bh && fp.pair == pc.pair;
             }
-            float M = m_ref;
+            // merge every piece -- this one's too, read back -- in slot order, so the result
+            // does not depend on which piece happened to arrive last
+            float M = -INFINITY;
             for (int gg = g_first; gg <= g_last; ++gg) {
-                if (gg == g) continue;
-                const int sl = (gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1;
+                const int sl = gg == g ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
                 M = fmaxf(M, __ldcg(p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2));
             }
-            const float ws = ex2_approx(m_ref - M);
-            float L_ = l * ws;
+            float L_ = 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) o[c][i] = __float_as_uint(__uint_as_float(o[c][i]) * ws);
+                for (int i = 0; i < 32; ++i) o[c][i] = 0u;
             for (int gg = g_first; gg <= g_last; ++gg) {
-                if (gg == g) continue;
-                const int sl = (gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1;
+                const int sl = gg == g ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
                 const float* pml = p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2;
                 const float w = ex2_approx(__ldcg(pml) - M);
                 L_ += w * __ldcg(pml + 1);

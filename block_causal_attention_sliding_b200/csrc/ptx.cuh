@@ -47,6 +47,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up (returns false) when the
 // CTA-wide abort flag is raised or when `limit_ns` of wall time has passed, so no kernel can
 // spin forever on a barrier that will never complete.
@@ -231,6 +242,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe, for x <= 8 (inputs below -125, including -inf, give ~2^-125).
+// Cody-Waite split x = j + f with j = round(x) (adding 1.5 * 2^23 rounds to an integer in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic minimax polynomial (relative error
+// below 7.5e-5, coefficients fitted by Remez exchange for this kernel); 2^j is added straight
+// into the exponent field: the low bits of t shifted left by 23 are exactly j << 23.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float magic = 12582912.f;
+    const float t = x + magic;
+    const float f = x - (t - magic);
+    float p = fmaf(0.0551716685f, f, 0.242611125f);
+    p = fmaf(p, f, 0.693260968f);
+    p = fmaf(p, f, 0.999928057f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -143,8 +143,8 @@ def test_persistent_split_shapes(dev, H, T):
 
 
 def test_persistent_repeatable(dev):
-    """The merge counters return to zero after every launch: repeated forwards on the same
-    inputs give bit-identical output."""
+    """The merge counters return to zero after every launch, and split pieces are merged in a
+    fixed order whichever arrives last: repeated forwards give bit-identical output."""
     wl = RAGGED
     h = make_handle(wl, dev, max_short_q=-1)
     Kc, Vc = synth.cond_inputs(wl)
@@ -175,7 +175,9 @@ def test_permutation_within_chunk(dev):
     perm = torch.randperm(wl.T, generator=torch.Generator().manual_seed(3))
     a = h.forward(Q.to(dev), K.to(dev), V.to(dev)).cpu().numpy()
     b = h.forward(Q.to(dev), K[:, perm].contiguous().to(dev), V[:, perm].contiguous().to(dev)).cpu().numpy()
-    compare(b, a.astype(np.float64), 2e-3, 5e-4)
+    # the same keys fall into other tiles, so lazy-rescale points and bf16 rounding of P
+    # differ: equal within the parity tolerance, not bit for bit
+    compare(b, a.astype(np.float64))
 
 
 def test_480p_sampled(dev):

@@ -1,0 +1,65 @@
+"""Host-side checks of arithmetic the CUDA kernels use (no GPU needed).
+
+exp2_poly (csrc/ptx.cuh) replaces a share of the MUFU exponentials with FMA-pipe arithmetic:
+a Cody-Waite split x = j + f, |f| <= 1/2, a cubic for 2^f, and j added into the exponent bits.
+Its bound is pinned here by replaying the same float32 steps (fused multiply-adds rounded once)
+against numpy's exp2 in float64 over the whole input range the softmax can produce.
+"""
+from __future__ import annotations
+
+import os
+import re
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _poly_constants():
+    src = open(os.path.join(ROOT, "block_causal_attention_sliding_b200", "csrc", "ptx.cuh")).read()
+    body = src[src.index("float exp2_poly(float x)"):]
+    body = body[: body.index("}")]
+    lo = float(re.search(r"fmaxf\(x, (-?[0-9.]+)f\)", body).group(1))
+    magic = float(re.search(r"magic = ([0-9.]+)f", body).group(1))
+    coef = [float(v) for v in re.findall(r"fmaf\([a-z]*,?\s*([0-9.]+)f", body)]
+    c3, c2 = [float(v) for v in re.search(r"fmaf\(([0-9.]+)f, f, ([0-9.]+)f\)", body).groups()]
+    c1 = float(re.search(r"fmaf\(p, f, ([0-9.]+)f\);\s*p = fmaf\(p, f, ([0-9.]+)f\)", body).group(1))
+    c0 = float(re.search(r"fmaf\(p, f, ([0-9.]+)f\);\s*return", body).group(1))
+    assert coef  # the source still has the fused steps this test replays
+    return lo, magic, (np.float32(c0), np.float32(c1), np.float32(c2), np.float32(c3))
+
+
+def _fma32(a, b, c):
+    # float32 fused multiply-add: exact product and sum in float64, one rounding to float32
+    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
+
+
+def exp2_poly_replay(x):
+    lo, magic, (c0, c1, c2, c3) = _poly_constants()
+    x = np.maximum(x.astype(np.float32), np.float32(lo))
+    m = np.float32(magic)
+    t = (x + m).astype(np.float32)
+    f = (x - (t - m).astype(np.float32)).astype(np.float32)
+    p = _fma32(np.full_like(f, c3), f, np.full_like(f, c2))
+    p = _fma32(p, f, np.full_like(f, c1))
+    p = _fma32(p, f, np.full_like(f, c0))
+    bits = p.view(np.int32).astype(np.int64) + (t.view(np.int32).astype(np.int64) << 23)
+    return (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+
+
+def test_exp2_poly_relative_error_bound():
+    x = np.concatenate([np.linspace(-125.0, 8.0, 2_000_001, dtype=np.float32),
+                        np.float32(np.random.default_rng(0).uniform(-30, 8, 1_000_000))])
+    got = exp2_poly_replay(x).astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(got - ref) / ref
+    # well below bf16's half-ulp (2^-9 ~ 2e-3), the precision P is stored in
+    assert rel.max() < 1.0e-4, rel.max()
+
+
+def test_exp2_poly_masked_and_extremes():
+    x = np.array([-np.inf, -1e30, -200.0, -125.0, 0.0, 1.0, 8.0], dtype=np.float32)
+    got = exp2_poly_replay(x)
+    assert np.all(np.isfinite(got)) and np.all(got >= 0)
+    assert got[0] < 1e-37 and got[1] < 1e-37 and got[2] < 1e-37      # masked keys weigh ~0
+    np.testing.assert_allclose(got[4:], [1.0, 2.0, 256.0], rtol=1e-4)
