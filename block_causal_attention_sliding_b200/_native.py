@@ -20,7 +20,7 @@ EXPORTS = (
     "sw_attn_create", "sw_attn_create_ex", "sw_attn_workspace_bytes", "sw_attn_bind_workspace",
     "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
-    "sw_attn_last_error", "sw_attn_cache_offsets",
+    "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
 )
 
 
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_append_chunk.restype = i32
     L.sw_attn_forward.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward.restype = i32
+    L.sw_attn_forward_short_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
+    L.sw_attn_forward_short_noalloc.restype = i32
     L.sw_attn_table_ints.argtypes = [vp]
     L.sw_attn_table_ints.restype = i32
     L.sw_attn_get_table.argtypes = [vp, vp, vp]

@@ -357,3 +357,83 @@ int sw_attn_get_status(sw_attn_t* h, int32_t* host_status) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-alloc short forward
+// Callers that cannot allocate device memory at call time (a framework's fixed memory pool, a
+// fixed-footprint server) get the split-K decode path with its partials in this file-scope
+// array instead of the workspace.  Host code only ever uses the array's device address, looked
+// up once per device with that device current (the array's name is a host-side stand-in).
+namespace {
+constexpr size_t kNoAllocScratchFloats = size_t(4) << 20;   // 16 MiB per GPU
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur,
+                                             void* out, int n_q, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
+    if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
+    const sw_attn_config& c = h->cfg;
+    if (n_q < 1 || n_q > kMaxShortQ || n_q > c.tokens_per_chunk)
+        return fail(SW_ESHAPE, "n_q must be in [1, min(%d, T)] (n_q=%d)", kMaxShortQ, n_q);
+    if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
+        return fail(SW_EALIGN, "Q, K_cur, V_cur and out must be 16-byte aligned");
+    const size_t per_split = (size_t)c.B * c.H * kBlockM * (c.d + 2);
+    const size_t fit = kNoAllocScratchFloats / per_split;
+    if (fit < 1)
+        return fail(SW_ESHAPE, "B*H*128*(d+2) = %zu floats exceeds the fixed %zu-float scratch", per_split,
+                    kNoAllocScratchFloats);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return fail(SW_ESTATE, "current device %d is not the workspace's device %d", dev, h->device);
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(SW_EINVAL, "device ordinal %d not supported", dev);
+    float* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+            g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    int rc;
+    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
+    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
+    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
+    p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
+    p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
+    p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
+    p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    p.out = out;
+    p.table = state + kStateHeaderInts;
+    p.status = state + 1;
+    p.B = c.B;
+    p.H = c.H;
+    p.n_q = n_q;
+    p.out_f32 = c.out_dtype == SW_OUT_F32;
+    p.scale_log2 = c.scale * 1.4426950408889634f;
+    const int bh = c.B * c.H;
+    long long splits = h->num_sms / bh;
+    splits = std::max<long long>(1, std::min<long long>(splits, std::min<long long>((long long)fit, kMaxSplits)));
+    p.splits = (int)splits;
+    p.o_part = scratch;
+    p.ml_part = scratch + (size_t)splits * bh * kBlockM * c.d;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    e = launch_attention(p, c.d, 1, (int)splits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
+    e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, (int)splits, p.out_f32, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    return SW_OK;
+}

@@ -137,6 +137,32 @@ SW_API int sw_attn_append_chunk(sw_attn_t *h, const void *K, const void *V, void
 SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const void *V_cur,
                     void *out, int n_q, void *stream);
 
+/*
+ * Short-query forward that allocates nothing and uses no workspace scratch.
+ *
+ * Same result as sw_attn_forward for 1 <= n_q <= 128 (the split-K path), but its split-K
+ * partials go to a fixed device array inside this library instead of the handle's workspace.
+ * It is for callers that cannot allocate device memory at call time -- code running inside
+ * another framework's memory pool or a pre-planned, fixed-footprint serving process -- and
+ * want the cache-resident decode path without growing the workspace they hand over.  The
+ * paper has no counterpart: this is an interface convenience of this library.
+ *
+ * Limits and behaviour:
+ *   - The fixed array holds 4 Mi floats (16 MiB).  Each key split needs B*H*128*(d+2) floats;
+ *     the call uses as many splits as fit (up to one per SM per (b, h)) and rejects with
+ *     SW_ESHAPE a shape where not even one split fits (B*H > 252 at d = 128, > 496 at d = 64).
+ *   - Every GPU that loads the library holds the 16 MiB until the process exits.
+ *   - The array is shared by every call in the process and keeps the last call's contents;
+ *     every split writes its own partials before the merge reads them, so nothing needs
+ *     clearing, but calls that overlap on the GPU (two streams, two threads) race on it.
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.  Same argument rules as
+ *     sw_attn_forward; the caller's current device must be the workspace's device.
+ */
+SW_API int sw_attn_forward_short_noalloc(sw_attn_t *h, const void *Q, const void *K_cur,
+                                         const void *V_cur, void *out, int n_q, void *stream);
+
 /* Number of int32 entries of the visibility table (3 + 4 * (W + 3)). */
 SW_API int sw_attn_table_ints(const sw_attn_t *h);
 

@@ -1,0 +1,59 @@
+"""The allocation-free short-query forward, called through the C ABI.
+
+sw_attn_forward_short_noalloc serves callers that cannot allocate device memory when they
+call (a host framework's fixed pool, a fixed-footprint server): its split-K partials live in
+a fixed array inside the library instead of the handle's workspace.  Its output must match
+the ordinary entry point's within the parity tolerance, on two calls in a row (the second
+call reuses the array the first one left behind).  Kept in a file of its own so a run that
+stops at the first failure has already run everything else; it must pass both alone and
+after the other tests.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_causal_attention_sliding_b200 import _native, synth
+from block_causal_attention_sliding_b200.configs import Workload
+
+from parity_util import MAX_ABS, MEAN_REL, compare, make_handle
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_matches_forward_two_calls():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_causal_attention_sliding_b200 import build as B
+    B.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = Workload("noalloc", B=2, H=3, d=128, T=300, n_cond=40, W=2, sink=True, chunks=4, steps=1)
+    h = make_handle(wl, dev)   # fp32 output
+    Kc, Vc = synth.cond_inputs(wl)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    for k in range(3):
+        _, K, V = synth.chunk_inputs(wl, k, 0)
+        h.append_chunk(K.to(dev), V.to(dev))
+    lib = _native.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    for call, n_q in enumerate((64, 17)):
+        Q, K, V = (t.to(dev) for t in synth.chunk_inputs(wl, 3, call, n_q=n_q))
+        ref = h.forward(Q, K, V)                      # existing entry point (workspace scratch)
+        out = torch.full_like(ref, float("nan"))
+        rc = lib.sw_attn_forward_short_noalloc(h._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                               out.data_ptr(), n_q, ctypes.c_void_p(stream))
+        assert rc == 0, lib.sw_attn_last_error().decode()
+        torch.cuda.synchronize()
+        compare(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), MAX_ABS, MEAN_REL)
+    assert h.status() == 0
+    # a shape that cannot fit even one split in the fixed array is refused, not truncated
+    big = make_handle(Workload("big", B=1, H=256, d=128, T=8, n_cond=0, W=0, sink=False, chunks=1, steps=1), dev)
+    q = torch.zeros((1, 8, 256, 128), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((1, 8, 256, 128), dtype=torch.float32, device=dev)
+    rc = lib.sw_attn_forward_short_noalloc(big._h, q.data_ptr(), q.data_ptr(), q.data_ptr(), o.data_ptr(), 8,
+                                           ctypes.c_void_p(stream))
+    assert rc == _native.SW_ESHAPE and b"scratch" in lib.sw_attn_last_error()
