@@ -223,14 +223,16 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
             for (int i = 0; i < 32; ++i)
                 if (c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
     }
-    // row max as an 8-way tree: independent accumulators keep the dependent chain short
+    // row max as an 8-way tree of three-input maxes: independent accumulators keep the
+    // dependent chain short, two elements per instruction
     float mxa[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) mxa[a] = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], __uint_as_float(sr[c][i]));
+        for (int i = 0; i < 32; i += 2)
+            mxa[(i >> 1) & 7] = fmax3(mxa[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
 #pragma unroll
     for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
@@ -269,7 +271,7 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
                 // the row sum adds the same bf16-rounded weights the PV MMA multiplies, so
                 // out is an exact weighted mean of V under those weights (8 accumulators)
                 const int a = (i >> 1) & 7;
-                suma[a] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xFFFF0000u);
+                suma[a] = add_bf16x2_f32(pp, suma[a]);
                 pk[cc * 16 + (i >> 1)] = pp;
             }
         }

@@ -2,20 +2,21 @@
 //
 // Same computation and warp roles as attn_fwd_kernel (TMA producer, one-thread tcgen05 MMA
 // issuer, one softmax warpgroup per 128-row Q tile), but the grid is one CTA per SM and the
-// work is cut evenly.  Work items are (pair of Q tiles, key tile) of every (b, h), costed by
-// the number of live Q tiles (1 or 2), laid out in one line; CTA g takes the items whose
-// start cost falls in [g C / G, (g+1) C / G).  Each SM therefore does the same amount of
-// tensor work whatever the number of query blocks, so there is no partial last wave.
-//
-// A pair whose key tiles are cut between CTAs ("split piece") is merged without any
-// inter-CTA waiting: every piece writes its unnormalised O row block and its (max, sum)
-// to a scratch slot, then bumps a per-pair counter; the piece that sees the counter reach
-// npieces - 1 is last, reads the others' partials (log-sum-exp merge) and writes the output,
-// then clears the counter for the next launch.
+// work is dealt out in two phases:
+//   1. whole pairs of Q tiles, round-robin (CTA g takes pairs g, g + G, ...) for as many full
+//      rounds as there are -- like the one-CTA-per-pair grid, so the CTAs running together
+//      share a handful of heads and their K/V stay in L2;
+//   2. the leftover pairs (fewer than G) as one line of (pair, key tile) items costed by the
+//      number of live Q tiles, cut evenly between the CTAs ("stream-K"), so no SM idles while
+//      a partial last wave runs.
+// A pair whose key tiles are cut between CTAs ("split piece") is merged without any inter-CTA
+// waiting: every piece writes its unnormalised O rows and (max, sum) to a scratch slot, then
+// bumps a per-pair counter; the piece that sees the counter reach npieces - 1 is last, merges
+// all pieces in slot order (log-sum-exp) and writes the output, then clears the counter.
 //
 // Within a CTA, consecutive pieces overlap: the producer streams the next piece's Q and K/V
-// while the softmax warpgroups finish the previous piece's epilogue; the first P V of a
-// piece waits only until the epilogue has read the previous O out of TMEM.
+// while the softmax warpgroups finish the previous piece's epilogue; the first P V of a piece
+// waits only until the epilogue has read the previous O out of TMEM.
 #include "attn_common.cuh"
 
 namespace swattn {
@@ -25,38 +26,80 @@ struct Piece {
     int pair;   // index of the Q-tile pair within the head (rows pair * 256 ...)
     int live;   // Q tiles of the pair that hold queries (1 or 2)
     int j0, j1; // key tiles [j0, j1) of this piece
+    bool sk;    // from the stream-K phase (may be split) rather than a whole-pair round
 };
 
-// Next piece of the range [cur, c1) of the cost line (nqt Q tiles per head, nt key tiles).
-__device__ __forceinline__ bool next_piece(long long& cur, long long c1, int nqt, int nt, Piece& pc) {
-    const long long per_bh = (long long)nqt * nt;
-    while (cur < c1) {
-        const int bh = (int)(cur / per_bh);
-        const long long r = cur - (long long)bh * per_bh;
-        const int i = (int)(r / (2LL * nt));
-        const int lv = min(2, nqt - 2 * i);
-        const long long ps = (long long)bh * per_bh + 2LL * i * nt;
-        const int j0 = (int)((cur - ps + lv - 1) / lv);     // first item starting at or after cur
-        if (j0 >= nt) {
-            cur = ps + (long long)lv * nt;
+// The two-phase schedule, identical in every role of every CTA.
+struct Sched {
+    int nqt, nt, npairs, P, G, g, rounds, p0, Gsk;
+    long long Csk, c0, c1;   // stream-K line length and this CTA's range of it
+    __device__ int live(int p) const { return min(2, nqt - 2 * (p % npairs)); }
+    // cost position of pair p (p >= p0) on the stream-K line: 2 nt per pair, nt for the
+    // single-tile last pair of a head (when nqt is odd)
+    __device__ long long cstart(int p) const {
+        return 2LL * nt * (p - p0) - (long long)(nqt & 1) * nt * (p / npairs - p0 / npairs);
+    }
+    __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
+        nqt = nqt_; nt = nt_; npairs = (nqt + 1) / 2; P = BH * npairs; G = G_; g = g_;
+        rounds = P / G;
+        p0 = rounds * G;
+        Csk = P > p0 ? cstart(P) : 0;
+        // every stream-K CTA gets at least two cost units, so a pair's pieces sit in
+        // consecutive CTAs that all hold one of its key tiles
+        Gsk = Csk > 0 ? (int)min((long long)G, max(1LL, Csk / 2)) : 0;
+        set_range(g);
+    }
+    __device__ void set_range(int cta) {
+        c0 = cta < Gsk ? (long long)cta * Csk / Gsk : 0;
+        c1 = cta < Gsk ? (long long)(cta + 1) * Csk / Gsk : 0;
+    }
+    // the stream-K CTA whose range holds cost position s
+    __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
+};
+
+struct PieceIt {
+    int r = 0;             // whole-pair rounds done
+    long long cur = -1;    // stream-K cursor (-1: not started)
+    int p = 0;             // stream-K pair the cursor is in
+};
+
+__device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
+    if (it.r < s.rounds) {
+        const int p = s.g + it.r * s.G;
+        ++it.r;
+        pc.bh = p / s.npairs;
+        pc.pair = p % s.npairs;
+        pc.live = s.live(p);
+        pc.j0 = 0;
+        pc.j1 = s.nt;
+        pc.sk = false;
+        return true;
+    }
+    if (it.cur < 0) {
+        it.cur = s.c0;
+        it.p = s.p0;
+    }
+    while (it.cur < s.c1) {
+        while (it.p + 1 < s.P && s.cstart(it.p + 1) <= it.cur) ++it.p;
+        const long long ps = s.cstart(it.p);
+        const int lv = s.live(it.p);
+        const int j0 = (int)((it.cur - ps + lv - 1) / lv);     // first item starting at or after cur
+        if (j0 >= s.nt) {
+            it.cur = ps + (long long)lv * s.nt;
             continue;
         }
-        const long long e = (c1 - ps + lv - 1) / lv;       // first item starting at or after c1
-        const int j1 = (int)(e < nt ? e : nt);
-        cur = ps + (long long)lv * j1;
-        pc.bh = bh;
-        pc.pair = i;
+        const long long e = (s.c1 - ps + lv - 1) / lv;        // first item starting at or after c1
+        const int j1 = (int)(e < s.nt ? e : s.nt);
+        it.cur = ps + (long long)lv * j1;
+        pc.bh = it.p / s.npairs;
+        pc.pair = it.p % s.npairs;
         pc.live = lv;
         pc.j0 = j0;
         pc.j1 = j1;
+        pc.sk = true;
         return true;
     }
     return false;
-}
-
-// The CTA whose cost range [g C / G, (g+1) C / G) contains cost position s.
-__device__ __forceinline__ int cta_of(long long s, long long C, int G) {
-    return (int)(((s + 1) * G - 1) / C);
 }
 
 // Barrier over the 128 threads of softmax warpgroup qt (ids 1 and 2; 0 is __syncthreads).
@@ -104,24 +147,22 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
     tc_fence_after();
 
     const uint32_t tmem = ctl->tmem_base;
-    const int G = gridDim.x;
     const int g = blockIdx.x;
     const int nt = ctl->n_tiles;
     const int nqt = (p.n_q + kBlockM - 1) / kBlockM;
-    const long long Ctot = (long long)p.B * p.H * nqt * nt;
-    const long long c0 = (long long)g * Ctot / G;
-    const long long c1 = (long long)(g + 1) * Ctot / G;
+    Sched sched;
+    sched.init(nqt, nt, p.B * p.H, (int)gridDim.x, g);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && nt > 0) {
             const uint32_t qbar = smem_u32(&ctl->q_full);
-            long long cur = c0;
+            PieceIt pit;
             Piece pc;
             uint32_t it = 0;
             int pi = 0;
             bool ok = true;
-            while (ok && next_piece(cur, c1, nqt, nt, pc)) {
+            while (ok && next_piece(sched, pit, pc)) {
                 const int b = pc.bh / p.H, h = pc.bh % p.H;
                 const int m0 = pc.pair * NQ * kBlockM;
                 // the Q buffers are reused: wait until every S MMA of the previous piece is done
@@ -159,14 +200,14 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
         if (lane == 0 && nt > 0) {
             const uint32_t q_base = smem_u32(q_smem);
             const uint32_t kv_base = smem_u32(kv_smem);
-            long long cur = c0;
+            PieceIt pit;
             Piece pc;
             uint32_t it = 0;          // K/V tiles consumed so far (ring position)
             int pi = 0;               // pieces started
             uint32_t tcnt[2] = {0, 0};   // key tiles processed per Q tile (p_full phases)
             uint32_t ucnt[2] = {0, 0};   // pieces finished per Q tile (o_empty phases)
             bool ok = true;
-            while (ok && next_piece(cur, c1, nqt, nt, pc)) {
+            while (ok && next_piece(sched, pit, pc)) {
                 const int n = pc.j1 - pc.j0;
                 const int live = pc.live;
                 if (!wait_or_abort(smem_u32(&ctl->q_full), pi & 1, abort_flag)) break;
@@ -243,14 +284,14 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
         const uint32_t tS = lane_base + qt * kBlockN;
         const uint32_t tO = lane_base + NQ * kBlockN + qt * D;
         const uint32_t o_bar = smem_u32(&ctl->o_full[qt]);
-        long long cur = c0;
+        PieceIt pit;
         Piece pc;
-        int pi = 0;
+        int sk_pi = 0;            // stream-K pieces seen (the first and last may be split)
         uint32_t tcnt = 0;
         bool ok = nt > 0;
-        while (ok && next_piece(cur, c1, nqt, nt, pc)) {
-            const bool first_in_cta = pi == 0;
-            ++pi;
+        while (ok && next_piece(sched, pit, pc)) {
+            const bool first_sk = pc.sk && sk_pi == 0;
+            if (pc.sk) ++sk_pi;
             if (qt >= pc.live) continue;
             const int n = pc.j1 - pc.j0;
             float m_ref = -INFINITY, l = 0.f;
@@ -292,11 +333,12 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 continue;
             }
             // split piece: publish the partial, then the last of the pair's pieces merges
-            const long long ps = (long long)pc.bh * nqt * nt + 2LL * pc.pair * nt;
-            const int g_first = cta_of(ps, Ctot, G);
-            const int g_last = cta_of(ps + (long long)pc.live * (nt - 1), Ctot, G);
+            const int pidx = pc.bh * sched.npairs + pc.pair;
+            const long long ps = sched.cstart(pidx);
+            const int g_first = sched.cta_of(ps);
+            const int g_last = sched.cta_of(ps + (long long)pc.live * (nt - 1));
             const int npieces = g_last - g_first + 1;
-            const int slot = first_in_cta ? 2 * g : 2 * g + 1;
+            const int slot = first_sk ? 2 * g : 2 * g + 1;
             float* so = p.sk_o + ((size_t)slot * 2 + qt) * D * kBlockM;     // [D][128 rows]
             float* sml = p.sk_ml + ((size_t)slot * 2 + qt) * kBlockM * 2;   // [128 rows][2]
 #pragma unroll
@@ -312,13 +354,17 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             wg_bar(qt);
             if (ctl->merge_flag[qt] != npieces - 1) continue;     // another piece will merge
             __threadfence();
-            // the pair's first piece is CTA g_first's last piece unless it opens that CTA's range
+            // the pair's first piece is CTA g_first's last piece unless it opens that CTA's
+            // stream-K range
             bool opens_first = false;
             {
-                long long cf = (long long)g_first * Ctot / G;
+                Sched sf = sched;
+                sf.g = g_first;
+                sf.set_range(g_first);
+                PieceIt fit;
+                fit.r = sf.rounds;
                 Piece fp;
-                if (next_piece(cf, (long long)(g_first + 1) * Ctot / G, nqt, nt, fp))
-                    opens_first = fp.bh == pc.bh && fp.pair == pc.pair;
+                if (next_piece(sf, fit, fp)) opens_first = fp.bh == pc.bh && fp.pair == pc.pair;
             }
             // merge every piece -- this one's too, read back -- in slot order, so the result
             // does not depend on which piece happened to arrive last

@@ -260,6 +260,23 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// max(a, b, c) in one instruction (three-input max, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// acc + lo + hi, where lo/hi are the two bf16 halves of a packed pair, widened exactly by the
+// mixed-precision adds (bf16 operand, fp32 accumulate; sm_100).
+__device__ __forceinline__ float add_bf16x2_f32(uint32_t pp, float acc) {
+    float d;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.f32.bf16 %0, lo, %2;\n\tadd.f32.bf16 %0, hi, %0;\n\t}"
+        : "=f"(d) : "r"(pp), "f"(acc));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t*>(&v);
