@@ -216,12 +216,15 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                         // P arrives in two halves; the PV of the first 64 keys overlaps the softmax
                         // of the other 64
                         const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
-                        if (!wait_or_abort(smem_u32(&ctl->p_half[qt]), jj & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                        if (kSplitP) {
+                            if (!wait_or_abort(smem_u32(&ctl->p_half[qt]), jj & 1, abort_flag)) { ok = false; break; }
+                            tc_fence_after();
+                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                        }
                         if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), jj & 1, abort_flag)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                        if (kSplitP) issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                        else issue_pv<D>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
                         mma_commit(smem_u32(&ctl->o_full[qt]));
                         if (more) {
                             if (qt == 0 &&

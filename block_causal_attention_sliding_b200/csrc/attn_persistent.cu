@@ -231,7 +231,8 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                     }
                     for (int qt = 0; qt < live && ok; ++qt) {
                         const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
-                        if (!wait_or_abort(smem_u32(&ctl->p_half[qt]), tcnt[qt] & 1, abort_flag)) {
+                        if (!wait_or_abort(smem_u32(kSplitP ? &ctl->p_half[qt] : &ctl->p_full[qt]), tcnt[qt] & 1,
+                                           abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -244,13 +245,17 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                             }
                             tc_fence_after();
                         }
-                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
-                        if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
-                            ok = false;
-                            break;
+                        if (kSplitP) {
+                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                            if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                        } else {
+                            issue_pv<D>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
                         }
-                        tc_fence_after();
-                        issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                         mma_commit(smem_u32(&ctl->o_full[qt]));
                         ++tcnt[qt];
                         if (more) {
