@@ -120,13 +120,13 @@ def _dist_env():
     return world, rank, local
 
 
-def _init_dist(world, backend="nccl"):
+def _init_dist(world, backend="nccl", timeout_s=120):
     if world <= 1:
         return None
     import datetime
     import torch.distributed as dist
     os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
     return dist
 
 
@@ -137,6 +137,14 @@ def reduce_max_time(dist, seconds: float, device) -> float:
     t = torch.tensor([seconds], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(dist, elapsed_s: float, flops_per_rank: float, device):
+    """Whole-job throughput of independent replicas: every rank's FLOPs over the slowest rank's
+    device time.  Returns (t_max seconds, TFLOP/s)."""
+    world = 1 if dist is None else dist.get_world_size()
+    t_max = reduce_max_time(dist, elapsed_s, device)
+    return t_max, flops_per_rank * world / t_max / 1e12
 
 
 def barrier(dist, device):
@@ -233,15 +241,13 @@ def run_cuda(args, wl, world, rank, local):
     clk = clocks.stop()
     barrier(dist, dev)
     elapsed = start.elapsed_time(end) / 1e3
-    t_max = reduce_max_time(dist, elapsed, dev)
     fwd_ms = [fwd_events[i][2 * s].elapsed_time(fwd_events[i][2 * s + 1])
               for i in range(args.steps) for s in range(wl.steps)]
     status = h.status()
 
     flops_fwd = wl.flops_forward(k_start)
     flops_step = wl.steps * flops_fwd
-    total_flops = flops_step * args.steps * world
-    value = total_flops / t_max / 1e12
+    t_max, value = aggregate(dist, elapsed, flops_step * args.steps, dev)
     fwd_avg = sum(fwd_ms) / len(fwd_ms) / 1e3
     achieved = flops_fwd / fwd_avg / 1e12
 
@@ -270,10 +276,9 @@ def run_cuda(args, wl, world, rank, local):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_t = reduce_max_time(dist, e0.elapsed_time(e1) / 1e3, dev)
+    e2e_t, e2e_value = aggregate(dist, e0.elapsed_time(e1) / 1e3, flops_step * e2e_steps, dev)
     bi = sum(t.numel() * t.element_size() for per_step in host_in for t in per_step)
     bo = sum(t.numel() * t.element_size() for t in host_out)
-    e2e_value = flops_step * e2e_steps * world / e2e_t / 1e12
 
     # ---- side measurements (untimed for the metric): append/evict and the split-K path
     paths = {}

@@ -21,6 +21,7 @@ EXPORTS = (
     "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
+    "sw_attn_selftest_timeout",
 )
 
 
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_forward.restype = i32
     L.sw_attn_forward_short_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward_short_noalloc.restype = i32
+    L.sw_attn_selftest_timeout.argtypes = [vp, ctypes.c_int64, vp]
+    L.sw_attn_selftest_timeout.restype = i32
     L.sw_attn_table_ints.argtypes = [vp]
     L.sw_attn_table_ints.restype = i32
     L.sw_attn_get_table.argtypes = [vp, vp, vp]

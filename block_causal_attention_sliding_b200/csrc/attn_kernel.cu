@@ -346,6 +346,26 @@ cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, in
     return cudaErrorInvalidValue;
 }
 
+// ------------------------------------------------------------------ failure-detection self-test
+// Waits on a barrier that nothing completes, with the kernels' own bounded wait; records the
+// timeout in the status word like a stalled attention kernel would.
+__global__ void selftest_timeout_kernel(int32_t* status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        flag = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(smem_u32(&bar), 0, &flag, limit_ns)) atomicOr(status, SW_STATUS_TIMEOUT);
+}
+
+cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream) {
+    selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ split-K combine (K4)
 // out[row] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (log-sum-exp merge).
 // One warp per (b, h, row); each lane owns d/32 consecutive columns.

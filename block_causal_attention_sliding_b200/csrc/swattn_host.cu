@@ -346,6 +346,16 @@ int sw_attn_cache_offsets(const sw_attn_t* h, size_t* k_offset, size_t* v_offset
     return SW_OK;
 }
 
+int sw_attn_selftest_timeout(sw_attn_t* h, int64_t limit_ns, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (limit_ns < 1000000 || limit_ns > 2000000000LL) return fail(SW_EINVAL, "limit_ns must be in [1e6, 2e9]");
+    cudaError_t e = launch_selftest_timeout(reinterpret_cast<int32_t*>(h->ws) + 1, (uint64_t)limit_ns,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "self-test launch");
+}
+
 int sw_attn_get_status(sw_attn_t* h, int32_t* host_status) {
     g_err.clear();
     if (!h || !host_status) return fail(SW_EINVAL, "null argument");

@@ -180,6 +180,15 @@ SW_API int sw_attn_get_table(const sw_attn_t *h, int32_t *dev_table, void *strea
  */
 SW_API int sw_attn_cache_offsets(const sw_attn_t *h, size_t *k_offset, size_t *v_offset);
 
+/*
+ * Failure-detection self-test.  Enqueues one tiny kernel that waits on an mbarrier nothing
+ * will ever complete, through the same bounded wait every attention kernel uses, with a limit
+ * of limit_ns (1e6 .. 2e9 ns) instead of the kernels' 1 s.  When the wait gives up it sets
+ * SW_STATUS_TIMEOUT in the device status word and returns; the context stays usable.  Shows
+ * that a stalled pipeline ends in an error status rather than a hang.  sw_attn_reset clears it.
+ */
+SW_API int sw_attn_selftest_timeout(sw_attn_t *h, int64_t limit_ns, void *stream);
+
 /* Synchronise the device, then read the device status bits into *host_status. */
 SW_API int sw_attn_get_status(sw_attn_t *h, int32_t *host_status);
 
