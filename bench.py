@@ -47,6 +47,31 @@ def _peaks():
         return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
+# DRAM traffic of one attention launch from an ncu capture of the 720p steady-state forward
+# (dram__bytes_read.sum + dram__bytes_write.sum).  It is reported only while the kernel's
+# sources hash to what was captured; any change to them makes the figure stale (null).
+PROFILED_TRAFFIC = {
+    ("720p", "persistent"): {"bytes": 231_825_152 + 15_539_968,
+                             "sources_sha256": "75b2ce8dfb965622cfeac19874c819df137a526da860d020af3611c2444ce9fc"},
+}
+KERNEL_SOURCES = ("attn_persistent.cu", "attn_common.cuh", "ptx.cuh", "swattn_internal.h")
+
+
+def _profiled_traffic(workload: str, schedule: str):
+    import hashlib
+    rec = PROFILED_TRAFFIC.get((workload, schedule))
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        try:
+            with open(os.path.join(ROOT, "block_causal_attention_sliding_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    return rec["bytes"] if h.hexdigest() == rec["sources_sha256"] else None
+
+
 # ---------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -315,7 +340,7 @@ def run_cuda(args, wl, world, rank, local):
                          "kernel": "attn_persistent_kernel<128>" if args.schedule == "persistent"
                          else "attn_fwd_kernel<128,2>", "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": None, "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                         "traffic": _profiled_traffic(wl.name, args.schedule), "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                          "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                          "launch_ms_avg": round(fwd_avg * 1e3, 4)},
             "cpu_baseline": cpu,
