@@ -198,16 +198,14 @@ __device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t
 //   read the S row from TMEM, mask keys past the segment's end, update the reference max
 //   (lazily: only when it grows by more than 2^kRescaleThreshold), write P = exp2(s*sl2 - m)
 //   as bf16 pairs over the S columns, add the same rounded weights to l, and rescale the
-//   O row in TMEM when the reference moved (after waiting for the previous PV).
+//   O row in TMEM when the reference moved.
 // P is published in two halves: the warp arrives on p_half_bar once keys 0..63 are written
 // (the PV of those keys may then start) and the caller arrives on p_full after the return.
 // A warp that must rescale O first publishes nothing early: its O rescale has to land before
-// any PV of this tile.  The caller has waited for S.  Returns false on abort.
+// any PV of this tile.  The caller has waited for S.
 template <int D>
-__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
-                                             uint32_t o_full_bar, uint32_t prev_pv_parity,
-                                             uint32_t p_half_bar, float sl2, float& m_ref, float& l,
-                                             volatile int* abort_flag) {
+__device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
+                                             uint32_t p_half_bar, float sl2, float& m_ref, float& l) {
     uint32_t sr[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
@@ -294,9 +292,9 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
     }
     if (rescale) {
         // done once the S row is dead (low register pressure); it must land before this
-        // tile's PV, which waits for p_half (arrived below) and p_full
-        if (!warp_wait(o_full_bar, prev_pv_parity, abort_flag)) return false;
-        tc_fence_after();
+        // tile's PV, which waits for p_half (arrived below) and p_full.  The previous PV into
+        // O has completed: it was issued before this tile's S, whose completion the caller
+        // has waited for, and the tensor pipe completes one thread's MMAs in issue order.
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -312,7 +310,6 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int valid
     }
     tmem_wait_st();
     tc_fence_before();
-    return true;
 }
 
 // Write one output row (32 columns at a time from registers), bf16 or fp32.

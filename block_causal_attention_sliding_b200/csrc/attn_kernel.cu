@@ -160,7 +160,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                         if (ph[qt] == 1 && mbar_test(smem_u32(&ctl->p_full[qt]), j & 1)) {
                             tc_fence_after();
                             issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
-                            mma_commit(smem_u32(&ctl->o_full[qt]));
+                            if (j + 1 == n) mma_commit(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
                             const int shV = 2 * (j & 3);
                             cntV += 1u << shV;
                             if ((int)((cntV >> shV) & 3u) == live) {
@@ -225,7 +225,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                         tc_fence_after();
                         if (kSplitP) issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                         else issue_pv<D>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
-                        mma_commit(smem_u32(&ctl->o_full[qt]));
+                        if (!more) mma_commit(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
                         if (more) {
                             if (qt == 0 &&
                                 !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
@@ -268,9 +268,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             ok = warp_wait(smem_u32(&ctl->s_full[qt]), jj & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (jj - 1) & 1, smem_u32(&ctl->p_half[qt]),
-                                 p.scale_log2, m_ref, l, abort_flag);
-            if (!ok) break;
+            softmax_step<D>(tS, tO, valid, jj == 0, smem_u32(&ctl->p_half[qt]), p.scale_log2, m_ref, l);
             warp_arrive(smem_u32(&ctl->p_full[qt]));
         }
         // ------------------------------------------------------------ epilogue
@@ -284,7 +282,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                 p.ml_part[prow * 2 + 0] = -INFINITY;
                 p.ml_part[prow * 2 + 1] = 0.f;
             }
-        } else if (ok && warp_wait(o_bar, (n - 1) & 1, abort_flag)) {
+        } else if (ok && warp_wait(o_bar, 0, abort_flag)) {   // o_full completes once, after the last PV
             tc_fence_after();
             const float inv = 1.f / l;
 #pragma unroll 1

@@ -102,7 +102,21 @@ __device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& p
     return false;
 }
 
+// All-of-group vote over the 128 threads of softmax warpgroup qt (barrier ids 3 and 4): true
+// iff every thread passes true.  Taken once per piece, after the piece's waits, so a warp
+// whose wait gave up never leaves its group mates blocked in a barrier.
+__device__ __forceinline__ bool wg_all(int qt, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v), "r"(3 + qt) : "memory");
+    return r != 0;
+}
+
 // Barrier over the 128 threads of softmax warpgroup qt (ids 1 and 2; 0 is __syncthreads).
+// Used only after wg_all has found every warp of the group healthy for this piece, and no
+// wait sits between the two, so no warp can be stranded in it.
 __device__ __forceinline__ void wg_bar(int qt) {
     if (qt == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
     else asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -256,8 +270,8 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                         } else {
                             issue_pv<D>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
                         }
-                        mma_commit(smem_u32(&ctl->o_full[qt]));
                         ++tcnt[qt];
+                        if (!more) mma_commit(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
                         if (more) {
                             if (qt == 0 &&
                                 !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
@@ -292,7 +306,8 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
         PieceIt pit;
         Piece pc;
         int sk_pi = 0;            // stream-K pieces seen (the first and last may be split)
-        uint32_t tcnt = 0;
+        uint32_t tcnt = 0;        // key tiles processed (s_full phases)
+        uint32_t ucnt = 0;        // pieces processed (o_full phases: one per piece)
         bool ok = nt > 0;
         while (ok && next_piece(sched, pit, pc)) {
             const bool first_sk = pc.sk && sk_pi == 0;
@@ -306,15 +321,16 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 ok = warp_wait(smem_u32(&ctl->s_full[qt]), tcnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                ok = softmax_step<D>(tS, tO, valid, jj == 0, o_bar, (tcnt - 1) & 1, smem_u32(&ctl->p_half[qt]),
-                                     p.scale_log2, m_ref, l, abort_flag);
-                if (!ok) break;
+                softmax_step<D>(tS, tO, valid, jj == 0, smem_u32(&ctl->p_half[qt]), p.scale_log2, m_ref, l);
                 warp_arrive(smem_u32(&ctl->p_full[qt]));
                 ++tcnt;
             }
-            if (!ok) break;
             // ---------------------------------------------------- epilogue of this piece
-            ok = warp_wait(o_bar, (tcnt - 1) & 1, abort_flag);
+            if (ok) ok = warp_wait(o_bar, ucnt & 1, abort_flag);
+            ++ucnt;
+            // every warp of the group reaches this point once per piece, failed or not, and
+            // all of them go on (or leave) together
+            ok = wg_all(qt, ok);
             if (!ok) break;
             tc_fence_after();
             uint32_t o[D / 32][32];
