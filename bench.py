@@ -337,8 +337,9 @@ def run_cuda(args, wl, world, rank, local):
                        "schedule": args.schedule},
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
-                         "kernel": "attn_persistent_kernel<128>" if args.schedule == "persistent"
-                         else "attn_fwd_kernel<128,2>", "achieved": round(achieved, 2),
+                         "kernel": {"persistent": "attn_persistent_kernel<128>", "tri": "attn_tri_kernel<128>",
+                                    "grid": "attn_fwd_kernel<128,2>"}[args.schedule],
+                         "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "traffic": _profiled_traffic(wl.name, args.schedule), "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                          "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
@@ -440,7 +441,7 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", choices=["persistent", "grid"], default="persistent")
+    ap.add_argument("--schedule", choices=["persistent", "grid", "tri"], default="persistent")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -39,7 +39,8 @@ class SlidingWindowAttention:
                              sink=int(bool(sink)),
                              out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
                              scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
-                             schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID}[schedule])
+                             schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
+                                       "tri": N.SW_SCHED_TRI}[schedule])
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()

@@ -1,0 +1,713 @@
+// attn_tri.cu -- the full-chunk attention with three S buffers per 128-row Q tile.
+//
+// Work unit: one 128-row Q tile of one (b, h) against all its visible key tiles (or a slice of
+// them, see the schedule).  Tensor memory holds three S accumulators and O:
+//     S0 | S1 | S2 | O        (3 x 128 + D <= 512 columns)
+// so S of key tile u + 3 is computed while the softmax of tiles u + 1 and u + 2 runs, and the
+// softmax never waits on the PV -> next-S round trip of its own tile.  P (bf16 pairs) is
+// written over the first 64 columns of its S buffer; the next S into that buffer is issued
+// after the PV that reads P, and one thread's MMAs complete in issue order.
+//
+// Warps: 0 = TMA producer, 1 = tcgen05 MMA issuer, 2..5 = softmax group A, 6..9 = group B,
+// 10 = helper that turns TMA completions into words the MMA issuer can poll.
+// Key tiles alternate between the groups (global tile counter u: group u & 1), so one group's
+// exponentials overlap the other's tensor-memory loads and row maxima, and the two groups
+// share the SM's MUFU units.  All tiles of a Q tile accumulate into one O, so the groups keep
+// one reference max per row: the group of tile u reads the reference of tile u - 1 from the
+// other group (a tagged shared-memory word), raises it lazily (only when the tile's max is
+// more than 2^8 above it), publishes it for tile u + 1, and -- when it moved -- rescales O
+// after PV(u - 1) has completed and before PV(u) may start.  Each group keeps its own row sum
+// relative to the last reference it used; the epilogue brings both to the final reference.
+//
+// K and V tiles flow through two shared-memory rings (K: 2 stages, V: 3 at d = 128), loaded in
+// the order the MMA issuer consumes them: K(0), K(1), K(2), then V(0), K(3), V(1), K(4), ...
+// A K stage is refilled once S of its previous tile has completed (s_full), a V stage once PV
+// of its previous tile has (o_full): with at most three stages per ring, neither barrier can
+// run two phases ahead of the producer, so no separate release commits are needed.
+//
+// The MMA issuer never waits on an mbarrier: a wait in the thread that issues tcgen05.mma
+// stalls the tensor pipe until its queued MMAs and commits have drained.  It polls shared
+// words instead (acquire loads), once per key tile, and commits twice per key tile.
+//
+// Schedule (persistent, one CTA per SM): whole Q tiles round-robin (CTA g takes units g,
+// g + G, ...) for the full rounds, so the CTAs running together cover a few heads and their
+// K/V stay in L2; the leftover units are laid on one line of (unit, key tile) items cut
+// evenly between the CTAs (stream-K).  A unit whose key tiles are cut between CTAs is merged
+// by its last-arriving piece, reading all pieces in slot order (deterministic).
+#include "attn_common.cuh"
+
+namespace swattn {
+
+namespace tri {
+
+constexpr int kSBufs = 3;
+
+template <int D>
+struct Cfg {
+    static constexpr int kTileBytes = TileCfg<D>::kTileBytes;
+    static constexpr int kKSt = D == 128 ? 2 : 3;    // K ring stages (at most 3, see above)
+    static constexpr int kVSt = 3;                  // V ring stages (at most 3)
+    static constexpr int kQBytes = kTileBytes;
+    static constexpr int kKVBytes = (kKSt + kVSt) * kTileBytes;
+    static_assert(kKSt <= 3 && kVSt <= 3 && kKSt + kVSt <= 8, "ring stages");
+    static constexpr int kCtlOffset = kQBytes + kKVBytes;
+    static constexpr int kThreads = 64 + 2 * 128 + 32;   // + the load-completion helper warp
+    static constexpr int kTmemCols = 512;
+    static constexpr int kOCol = kSBufs * kBlockN;      // O after the three S buffers
+    static_assert(kSBufs * kBlockN + D <= kTmemCols, "tensor memory budget");
+};
+
+// Barriers and exchange words of the three-buffer pipeline (the K/V ring, Q, the visibility
+// table, the TMEM base and the abort flag live in the common SmemCtl).
+struct Ext {
+    uint64_t s_full[kSBufs];     // S(u) in buffer u % 3 complete                (1 commit)
+    uint64_t o_full[kSBufs];     // PV(u) complete, on barrier u % 3              (1 commit)
+    uint64_t ep;                 // both groups' row sums are published           (8 warps)
+    // Signals the MMA issuer polls with plain acquire loads (an mbarrier wait in the issuing
+    // thread stalls the tensor pipe until its queued MMAs and commits have drained):
+    uint32_t k_seq;              // K of key tiles 0..u have landed once k_seq >= u + 1 (helper)
+    uint32_t v_seq;              // V likewise                                        (helper)
+    uint32_t q_seq;              // Q of piece pi has landed once q_seq == pi + 1     (helper)
+    // P(u) written (and O ready for PV(u)): +1 per warp of the tile's group, so 4 (u / 3 + 1)
+    // once tile u in buffer u % 3 is done
+    uint32_t p_cnt[kSBufs];
+    uint32_t oe_cnt;             // +1 per softmax warp once the piece's O has been read
+    // reference max of tile u for tile u + 1: (tag u + 1) << 32 | float bits, slot u & 1
+    unsigned long long ref[2][kBlockM];
+    float lsum[2][2][kBlockM];   // [piece parity][group][row] row sums at the final reference
+};
+
+template <int D>
+constexpr int smem_bytes() {
+    return ((Cfg<D>::kCtlOffset + (int)sizeof(SmemCtl) + 15) & ~15) + (int)sizeof(Ext) + 1024;
+}
+
+// The two-phase schedule over units (one Q tile of one (b, h)), identical in every role.
+struct Sched {
+    int nqt, nt, U, G, g, rounds, u0, Gsk;
+    long long Csk, c0, c1;   // stream-K line length and this CTA's range of it
+    __device__ long long cstart(int u) const { return (long long)(u - u0) * nt; }
+    __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
+        nqt = nqt_; nt = nt_; U = BH * nqt; G = G_; g = g_;
+        rounds = U / G;
+        u0 = rounds * G;
+        Csk = (long long)(U - u0) * nt;
+        // at least two items per stream-K CTA
+        Gsk = Csk > 0 ? (int)min((long long)G, max(1LL, Csk / 2)) : 0;
+        set_range(g);
+    }
+    __device__ void set_range(int cta) {
+        c0 = cta < Gsk ? (long long)cta * Csk / Gsk : 0;
+        c1 = cta < Gsk ? (long long)(cta + 1) * Csk / Gsk : 0;
+    }
+    __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
+};
+
+struct Piece {
+    int unit;     // bh * nqt + q tile
+    int j0, j1;   // key tiles [j0, j1)
+    bool sk;      // from the stream-K phase (may be split)
+};
+
+struct PieceIt {
+    int r = 0;
+    long long cur = -1;
+};
+
+__device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
+    if (it.r < s.rounds) {
+        pc.unit = s.g + it.r * s.G;
+        ++it.r;
+        pc.j0 = 0;
+        pc.j1 = s.nt;
+        pc.sk = false;
+        return true;
+    }
+    if (it.cur < 0) it.cur = s.c0;
+    if (it.cur >= s.c1) return false;
+    const int u = s.u0 + (int)(it.cur / s.nt);
+    const int j0 = (int)(it.cur % s.nt);
+    const long long left = s.c1 - it.cur;
+    const int j1 = (int)min((long long)s.nt, j0 + left);
+    it.cur += j1 - j0;
+    pc.unit = u;
+    pc.j0 = j0;
+    pc.j1 = j1;
+    pc.sk = true;
+    return true;
+}
+
+// Acquire load of a shared word.
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(a)) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
+    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
+}
+
+// One release increment per warp, after the warp's lanes have finished (and fenced) their work.
+__device__ __forceinline__ void warp_signal(uint32_t* cnt) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(cnt)) : "memory");
+}
+
+// The MMA issuer's wait: poll until the counter reaches target (wrap-safe), bounded like every
+// other wait.  Returns false on abort or timeout (raising the abort flag on a timeout).
+__device__ __forceinline__ bool poll_reach(const uint32_t* a, uint32_t target, volatile int* abort_flag) {
+    if ((int32_t)(ld_acquire(a) - target) >= 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if ((int32_t)(ld_acquire(a) - target) >= 0) return true;
+        if ((it & 15u) == 15u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Publish v under tag for the other group's thread of the same row.
+__device__ __forceinline__ void ref_put(unsigned long long* a, float v, uint32_t tag) {
+    const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
+    asm volatile("st.relaxed.cta.shared.b64 [%0], %1;" ::"r"(smem_u32(a)), "l"(w) : "memory");
+}
+
+// Bounded wait for the value published under tag; false (warp-uniform) on abort or timeout,
+// which raises the CTA abort flag like every other wait.
+__device__ __forceinline__ bool ref_get(const unsigned long long* a, uint32_t tag, float& v,
+                                        volatile int* abort_flag) {
+    const uint32_t addr = smem_u32(a);
+    bool ok = false;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        unsigned long long w;
+        asm volatile("ld.relaxed.cta.shared.b64 %0, [%1];" : "=l"(w) : "r"(addr) : "memory");
+        if ((uint32_t)(w >> 32) == tag) {
+            v = __uint_as_float((uint32_t)w);
+            ok = true;
+            break;
+        }
+        if ((it & 31u) == 31u) {
+            if (*abort_flag) break;
+            const uint64_t t = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = t;
+            } else if (t - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                break;
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// All-of-both-groups vote (256 softmax threads, barrier id 2): true iff every thread passes
+// true.  Taken once per piece after the piece's waits, so a warp whose wait gave up never
+// leaves the others blocked in a barrier.
+__device__ __forceinline__ bool vote_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 2, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+
+// bar.sync over the 256 softmax threads (id 1); used only after vote_all found them healthy.
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+}  // namespace tri
+
+namespace tri {
+
+// One online-softmax step of this thread's query row over key tile u (the caller has waited
+// for S(u)).  `first`: u opens the piece (no previous reference, O is overwritten by PV(u)).
+// ref_prev / ref_mine: the reference words of tiles u - 1 and u.  m_g, l_g: this group's
+// reference of its last tile in the piece and its row sum relative to it (has_g: the group
+// has had a tile in this piece).  P is published once it is written in full and O, if the
+// reference moved, has been rescaled.
+// Returns false on abort.
+template <int D>
+__device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid, bool first, uint32_t u,
+                                             const unsigned long long* ref_prev, unsigned long long* ref_mine,
+                                             uint32_t o_full_prev, uint32_t o_full_prev_parity,
+                                             uint32_t* p_cnt, float sl2, float& m_g, float& l_g,
+                                             bool& has_g, volatile int* abort_flag) {
+    uint32_t sr[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+    tmem_wait_ld_dep(sr[0]);
+    reg_fence(sr[1]);
+    reg_fence(sr[2]);
+    reg_fence(sr[3]);
+    if (valid < kBlockN) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
+    }
+    float mxa[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mxa[a] = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            mxa[(i >> 1) & 7] = fmax3(mxa[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int a = 0; a < w; ++a) mxa[a] = fmaxf(mxa[a], mxa[a + w]);
+    const float m_loc = mxa[0] * sl2;
+    float m_new = m_loc;
+    float f_o = 1.f;          // factor taking O from the reference of tile u - 1 to m_new
+    bool rescale = false;     // warp-uniform: this warp rescales O before PV(u)
+    if (!first) {
+        float m_prev;
+        if (!ref_get(ref_prev, u, m_prev, abort_flag)) return false;
+        const bool need = m_loc > m_prev + kRescaleThreshold;
+        m_new = need ? m_loc : m_prev;
+        if (need) f_o = ex2_approx(m_prev - m_new);
+        rescale = __any_sync(0xffffffffu, need);
+    }
+    ref_put(ref_mine, m_new, u + 1);     // as early as possible: the other group waits on it
+    if (has_g) l_g *= ex2_approx(m_g - m_new);
+    m_g = m_new;
+    has_g = true;
+    float suma[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) suma[a] = 0.f;
+    const float neg_m = -m_new;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float x0 = fmaf(__uint_as_float(sr[c][i]), sl2, neg_m);
+                const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), sl2, neg_m);
+                const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+                // the row sum adds the same bf16-rounded weights the PV MMA multiplies
+                const int a = (i >> 1) & 7;
+                suma[a] = add_bf16x2_f32(pp, suma[a]);
+                pk[cc * 16 + (i >> 1)] = pp;
+            }
+        }
+        tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
+    }
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int a = 0; a < w; ++a) suma[a] += suma[a + w];
+    l_g += suma[0];
+    if (rescale) {
+        // O holds the sum up to PV(u - 1), relative to the reference of tile u - 1: wait for
+        // PV(u - 1) to complete, scale, and only then let PV(u) start
+        if (!warp_wait(o_full_prev, o_full_prev_parity, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld_dep(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f_o);
+            tmem_st32(tO + c * 32, o);
+        }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    warp_signal(p_cnt);   // P(u) written and O ready for PV(u)
+    return true;
+}
+
+}  // namespace tri
+
+template <int D>
+__global__ void __launch_bounds__(tri::Cfg<D>::kThreads, 1)
+attn_tri_kernel(const __grid_constant__ AttnParams p) {
+    using C = tri::Cfg<D>;
+    constexpr int kTileBytes = C::kTileBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* q_smem = base;
+    uint8_t* kv_smem = base + C::kQBytes;
+    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(base + C::kCtlOffset);
+    tri::Ext* ex = reinterpret_cast<tri::Ext*>(base + ((C::kCtlOffset + (int)sizeof(SmemCtl) + 15) & ~15));
+    volatile int* abort_flag = &ctl->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i < 2 * kBlockM; i += blockDim.x) (&ex->ref[0][0])[i] = 0ull;   // tags start at 1
+    if (threadIdx.x == 64) {
+        for (int b = 0; b < tri::kSBufs; ++b) ex->p_cnt[b] = 0;
+        ex->k_seq = ex->v_seq = ex->q_seq = 0;
+        ex->oe_cnt = 0;
+    }
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int b = 0; b < tri::kSBufs; ++b) {
+                mbar_init(smem_u32(&ex->s_full[b]), 1);
+                mbar_init(smem_u32(&ex->o_full[b]), 1);
+            }
+            mbar_init(smem_u32(&ex->ep), 8);
+            init_barriers(ctl, C::kKSt + C::kVSt);   // Q, the K/V rings, drain; fences every init above
+        }
+        __syncwarp();
+        tmem_alloc(smem_u32(&ctl->tmem_base), C::kTmemCols);
+        tmem_relinquish();
+    } else if (warp == 2 && lane == 0) {
+        load_table(ctl, p.table, p.status);
+    } else if (warp == 1 && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_kcur);
+        tma_prefetch_desc(&p.tm_vcur);
+        tma_prefetch_desc(&p.tm_cache_k);
+        tma_prefetch_desc(&p.tm_cache_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = ctl->tmem_base;
+    const int nt = ctl->n_tiles;
+    const int nqt = (p.n_q + kBlockM - 1) / kBlockM;
+    tri::Sched sched;
+    sched.init(nqt, nt, p.B * p.H, (int)gridDim.x, blockIdx.x);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && nt > 0) {
+            const uint32_t qbar = smem_u32(&ctl->q_full);
+            tri::PieceIt pit;
+            tri::Piece pc;
+            uint32_t t = 0;    // key tiles of all pieces so far (global tile index base)
+            int pi = 0;
+            bool ok = true;
+            while (ok && tri::next_piece(sched, pit, pc)) {
+                const int bh = pc.unit / nqt, qtile = pc.unit % nqt;
+                const int b = bh / p.H, h = bh % p.H;
+                // the Q buffer is reused: every S MMA of the previous piece has completed
+                if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(qbar, kTileBytes);
+                for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
+                    tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * kBoxCols, h, qtile * kBlockM, b);
+                ++pi;
+                const int n = pc.j1 - pc.j0;
+                // K(u): its stage last held K(u - kKSt), free once S(u - kKSt) has completed
+                auto load_k = [&](int jrel) -> bool {
+                    const uint32_t u = t + jrel;
+                    if (u >= (uint32_t)C::kKSt) {
+                        const uint32_t v = u - C::kKSt;
+                        if (!wait_or_abort(smem_u32(&ex->s_full[v % tri::kSBufs]), (v / tri::kSBufs) & 1, abort_flag))
+                            return false;
+                    }
+                    const int st = u % C::kKSt;
+                    const uint32_t fbar = smem_u32(&ctl->kv_full[st]);
+                    mbar_arrive_expect_tx(fbar, kTileBytes);
+                    load_kv_tile<D>(p, ctl, pc.j0 + jrel, 0, h, b, smem_u32(kv_smem + st * kTileBytes), fbar);
+                    return true;
+                };
+                // V(u): its stage last held V(u - kVSt), free once PV(u - kVSt) has completed
+                auto load_v = [&](int jrel) -> bool {
+                    const uint32_t u = t + jrel;
+                    if (u >= (uint32_t)C::kVSt) {
+                        const uint32_t v = u - C::kVSt;
+                        if (!wait_or_abort(smem_u32(&ex->o_full[v % tri::kSBufs]), (v / tri::kSBufs) & 1, abort_flag))
+                            return false;
+                    }
+                    const int st = C::kKSt + (int)(u % C::kVSt);
+                    const uint32_t fbar = smem_u32(&ctl->kv_full[st]);
+                    mbar_arrive_expect_tx(fbar, kTileBytes);
+                    load_kv_tile<D>(p, ctl, pc.j0 + jrel, 1, h, b, smem_u32(kv_smem + st * kTileBytes), fbar);
+                    return true;
+                };
+                // consumption order: K(0..2), then V(jj), K(jj + 3)
+                for (int k = 0; k < min(3, n) && ok; ++k) ok = load_k(k);
+                for (int jj = 0; jj < n && ok; ++jj) {
+                    ok = load_v(jj);
+                    if (ok && jj + 3 < n) ok = load_k(jj + 3);
+                }
+                t += n;
+            }
+            // never leave while copies are in flight: the last fill of every stage has landed
+            for (int st = 0; st < C::kKSt; ++st)
+                if (t > (uint32_t)st) wait_drain(smem_u32(&ctl->kv_full[st]), (((t - 1 - st) / C::kKSt) & 1));
+            for (int st = 0; st < C::kVSt; ++st)
+                if (t > (uint32_t)st)
+                    wait_drain(smem_u32(&ctl->kv_full[C::kKSt + st]), (((t - 1 - st) / C::kVSt) & 1));
+            if (pi > 0) wait_drain(qbar, (pi - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // Per key tile u: one poll point (V(u), P(u), K(u + 3)), PV(u), commit o_full, S(u + 3)
+        // into the same buffer, commit s_full.
+        if (lane == 0 && nt > 0) {
+            const uint32_t q_base = smem_u32(q_smem);
+            const uint32_t kv_base = smem_u32(kv_smem);
+            const uint32_t tO = tmem + C::kOCol;
+            tri::PieceIt pit;
+            tri::Piece pc;
+            uint32_t t = 0;    // key tiles of all pieces so far (S buffer u % 3, phase u / 3)
+            int pi = 0;        // pieces done
+            bool ok = true;
+            while (ok && tri::next_piece(sched, pit, pc)) {
+                const int n = pc.j1 - pc.j0;
+                if (!tri::poll_reach(&ex->q_seq, pi + 1, abort_flag)) break;
+                for (int k = 0; k < min(3, n) && ok; ++k) {
+                    const uint32_t u = t + k;
+                    if (!tri::poll_reach(&ex->k_seq, u + 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // buffer u % 3 last held P(u - 3), read by a PV issued before this S
+                    issue_s<D>(tmem + (u % tri::kSBufs) * kBlockN, q_base, kv_base + (u % C::kKSt) * kTileBytes);
+                    mma_commit(smem_u32(&ex->s_full[u % tri::kSBufs]));
+                    if (k == n - 1) mma_commit(smem_u32(&ctl->q_empty));   // last S of the piece
+                }
+                for (int jj = 0; jj < n && ok; ++jj) {
+                    const uint32_t u = t + jj, bu = u % tri::kSBufs;
+                    const bool more = jj + 3 < n;
+                    if (!tri::poll_reach(&ex->v_seq, u + 1, abort_flag) ||
+                        !tri::poll_reach(&ex->p_cnt[bu], 4 * (u / tri::kSBufs + 1), abort_flag) ||
+                        (more && !tri::poll_reach(&ex->k_seq, u + 4, abort_flag)) ||
+                        // the previous piece's O must be out of TMEM before PV(u) overwrites it
+                        (jj == 0 && pi > 0 && !tri::poll_reach(&ex->oe_cnt, 8 * pi, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tP = tmem + bu * kBlockN;
+                    issue_pv<D>(tO, tP, kv_base + (C::kKSt + u % C::kVSt) * kTileBytes, jj > 0);
+                    mma_commit(smem_u32(&ex->o_full[bu]));   // PV(u) done: V stage, rescale, epilogue
+                    if (more) {
+                        // S(u + 3) into the same buffer, in issue order after PV(u) read P(u)
+                        issue_s<D>(tP, q_base, kv_base + ((u + 3) % C::kKSt) * kTileBytes);
+                        mma_commit(smem_u32(&ex->s_full[bu]));
+                        if (jj + 3 == n - 1) mma_commit(smem_u32(&ctl->q_empty));
+                    }
+                }
+                ++pi;
+                t += n;
+            }
+            // every MMA issued has completed before the CTA can release TMEM
+            mma_commit(smem_u32(&ctl->drain));
+            wait_drain(smem_u32(&ctl->drain), 0);
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ completion helper
+        // Follows the producer's sequence: Q of each piece, then K and V of every key tile in
+        // consumption order; publishes each completion as a word the MMA issuer polls.  Never
+        // more than one phase behind a barrier: a stage is refilled only after the MMA issuer
+        // has seen the word for its previous fill.
+        if (lane == 0 && nt > 0) {
+            tri::PieceIt pit;
+            tri::Piece pc;
+            uint32_t t = 0;
+            int pi = 0;
+            bool ok = true;
+            while (ok && tri::next_piece(sched, pit, pc)) {
+                if (!wait_or_abort(smem_u32(&ctl->q_full), pi & 1, abort_flag)) break;
+                ++pi;
+                tri::st_release(&ex->q_seq, pi);
+                const int n = pc.j1 - pc.j0;
+                auto done_k = [&](int jrel) -> bool {
+                    const uint32_t u = t + jrel;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_full[u % C::kKSt]), (u / C::kKSt) & 1, abort_flag)) return false;
+                    tri::st_release(&ex->k_seq, u + 1);
+                    return true;
+                };
+                auto done_v = [&](int jrel) -> bool {
+                    const uint32_t u = t + jrel;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_full[C::kKSt + u % C::kVSt]), (u / C::kVSt) & 1, abort_flag))
+                        return false;
+                    tri::st_release(&ex->v_seq, u + 1);
+                    return true;
+                };
+                for (int k = 0; k < min(3, n) && ok; ++k) ok = done_k(k);
+                for (int jj = 0; jj < n && ok; ++jj) {
+                    ok = done_v(jj);
+                    if (ok && jj + 3 < n) ok = done_k(jj + 3);
+                }
+                t += n;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax groups
+        const int sw = warp - 2;          // 0..7
+        const int g = sw >> 2;            // group: key tiles u with u & 1 == g
+        const int wq = warp & 3;          // TMEM lane quarter (fixed by the warp's slot)
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t tO = lane_base + C::kOCol;
+        tri::PieceIt pit;
+        tri::Piece pc;
+        int sk_pi = 0;            // stream-K pieces seen (the first and last may be split)
+        uint32_t t = 0;           // key tiles of all pieces so far
+        uint32_t ucnt = 0;        // pieces done (ep phases)
+        bool ok = nt > 0;
+        while (ok && tri::next_piece(sched, pit, pc)) {
+            const bool first_sk = pc.sk && sk_pi == 0;
+            if (pc.sk) ++sk_pi;
+            const int n = pc.j1 - pc.j0;
+            float m_g = 0.f, l_g = 0.f;
+            bool has_g = false;
+            for (int jj = (int)((g + t) & 1); jj < n; jj += 2) {
+                const uint32_t u = t + jj, bu = u % tri::kSBufs;
+                int seg, row0, valid;
+                tile_of(ctl, pc.j0 + jj, seg, row0, valid);
+                ok = warp_wait(smem_u32(&ex->s_full[bu]), (u / tri::kSBufs) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t up = u - 1;   // unused when jj == 0
+                ok = tri::softmax_tile<D>(lane_base + bu * kBlockN, tO, valid, jj == 0, u, &ex->ref[up & 1][row],
+                                          &ex->ref[u & 1][row], smem_u32(&ex->o_full[up % tri::kSBufs]),
+                                          (up / tri::kSBufs) & 1, &ex->p_cnt[bu], p.scale_log2, m_g,
+                                          l_g, has_g, abort_flag);
+                if (!ok) break;
+            }
+            // ---------------------------------------------------- epilogue of this piece
+            const uint32_t tl = t + n - 1;   // the piece's last key tile
+            const int par = ucnt & 1;
+            float m_fin = m_g;
+            if (ok && (int)(tl & 1) != g) ok = tri::ref_get(&ex->ref[tl & 1][row], tl + 1, m_fin, abort_flag);
+            float l_row = 0.f;
+            if (ok) {
+                ex->lsum[par][g][row] = has_g ? l_g * ex2_approx(m_g - m_fin) : 0.f;
+                warp_arrive(smem_u32(&ex->ep));
+                ok = warp_wait(smem_u32(&ex->ep), par, abort_flag);
+            }
+            if (ok) {
+                l_row = ex->lsum[par][0][row] + ex->lsum[par][1][row];
+                // PV(tl - 3) has completed (S(tl) was seen before the exchange), so o_full of
+                // buffer tl % 3 is at most one phase behind the one awaited
+                ok = warp_wait(smem_u32(&ex->o_full[tl % tri::kSBufs]), (tl / tri::kSBufs) & 1, abort_flag);
+            }
+            ok = tri::vote_all(ok);
+            ++ucnt;
+            t += n;
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t o[D / 64][32];   // this group's half of the O columns
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_ld32(tO + g * (D / 2) + c * 32, o[c]);
+            tmem_wait_ld_dep(o[0]);
+#pragma unroll
+            for (int c = 1; c < D / 64; ++c) reg_fence(o[c]);
+            tc_fence_before();
+            tri::warp_signal(&ex->oe_cnt);   // O may now be overwritten
+
+            const int bh = pc.unit / nqt, qtile = pc.unit % nqt;
+            const int b = bh / p.H, h = bh % p.H;
+            const int m_row = qtile * kBlockM + row;
+            const size_t orow = ((size_t)b * p.n_q + m_row) * p.H + h;
+            if (pc.j0 == 0 && pc.j1 == nt) {
+                const float inv = 1.f / l_row;
+                if (m_row < p.n_q) {
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c)
+                        store_row_chunk<D>(p.out, p.out_f32, orow, g * (D / 64) + c, o[c], inv);
+                }
+                continue;
+            }
+            // split piece: publish the partial, then the last of the unit's pieces merges
+            const long long ps = sched.cstart(pc.unit);
+            const int g_first = sched.cta_of(ps);
+            const int g_last = sched.cta_of(ps + nt - 1);
+            const int npieces = g_last - g_first + 1;
+            const int cta = blockIdx.x;
+            const int slot = first_sk ? 2 * cta : 2 * cta + 1;
+            float* so = p.sk_o + (size_t)slot * 2 * D * kBlockM;       // [D][128 rows]
+            float* sml = p.sk_ml + (size_t)slot * 2 * kBlockM * 2;     // [128 rows][2]
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) so[(g * (D / 2) + c * 32 + i) * kBlockM + row] = __uint_as_float(o[c][i]);
+            if (g == 0) {
+                sml[row * 2 + 0] = m_fin;
+                sml[row * 2 + 1] = l_row;
+            }
+            __threadfence();
+            tri::softmax_bar();
+            int* cnt = p.sk_cnt + (size_t)bh * (2 * p.sk_pairs) + qtile;
+            if (sw == 0 && lane == 0) ctl->merge_flag[0] = atomicAdd(cnt, 1);
+            tri::softmax_bar();
+            if (ctl->merge_flag[0] != npieces - 1) continue;     // another piece will merge
+            __threadfence();
+            // the unit's first piece is CTA g_first's first stream-K piece iff g_first's range
+            // opens inside this unit; every later CTA's piece of it opens that CTA's range
+            tri::Sched sf = sched;
+            sf.set_range(g_first);
+            const bool opens_first = sf.u0 + (int)(sf.c0 / nt) == pc.unit;
+            float M = -INFINITY;
+            for (int gg = g_first; gg <= g_last; ++gg) {
+                const int sl = gg == cta ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
+                M = fmaxf(M, __ldcg(p.sk_ml + (size_t)sl * 2 * kBlockM * 2 + row * 2));
+            }
+            float L_ = 0.f;
+            for (int gg = g_first; gg <= g_last; ++gg) {
+                const int sl = gg == cta ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
+                const float* pml = p.sk_ml + (size_t)sl * 2 * kBlockM * 2 + row * 2;
+                L_ += ex2_approx(__ldcg(pml) - M) * __ldcg(pml + 1);
+            }
+            const float inv = 1.f / L_;
+#pragma unroll 1
+            for (int c = 0; c < D / 64; ++c) {      // 32 columns at a time
+                uint32_t acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = 0u;
+                for (int gg = g_first; gg <= g_last; ++gg) {
+                    const int sl = gg == cta ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
+                    const float w = ex2_approx(__ldcg(p.sk_ml + (size_t)sl * 2 * kBlockM * 2 + row * 2) - M);
+                    const float* po = p.sk_o + (size_t)sl * 2 * D * kBlockM + (g * (D / 2) + c * 32) * kBlockM + row;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        acc[i] = __float_as_uint(fmaf(w, __ldcg(po + i * kBlockM), __uint_as_float(acc[i])));
+                }
+                if (m_row < p.n_q) store_row_chunk<D>(p.out, p.out_f32, orow, g * (D / 64) + c, acc, inv);
+            }
+            if (sw == 0 && lane == 0) atomicExch(cnt, 0);   // all pieces arrived: ready for the next launch
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
+}
+
+template <int D>
+static cudaError_t launch_tri_d(const AttnParams& p, int ctas, cudaStream_t stream) {
+    constexpr int smem = tri::smem_bytes<D>();
+    static_assert(smem <= 227 * 1024, "shared memory budget");
+    auto kern = attn_tri_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, tri::Cfg<D>::kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tri(const AttnParams& p, int d, int ctas, cudaStream_t stream) {
+    if (ctas < 1 || ctas > kMaxPersistentCtas) return cudaErrorInvalidValue;
+    if (d == 128) return launch_tri_d<128>(p, ctas, stream);
+    if (d == 64) return launch_tri_d<64>(p, ctas, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace swattn

@@ -104,7 +104,8 @@ int check_cfg(const sw_attn_config& c) {
     if (c.out_dtype != SW_OUT_BF16 && c.out_dtype != SW_OUT_F32) return fail(SW_EINVAL, "bad out_dtype");
     if (c.max_short_q > kMaxShortQ) return fail(SW_ESHAPE, "max_short_q must be <= %d", kMaxShortQ);
     if (!std::isfinite(c.scale)) return fail(SW_EINVAL, "scale must be finite");
-    if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID) return fail(SW_EINVAL, "bad schedule");
+    if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID && c.schedule != SW_SCHED_TRI)
+        return fail(SW_EINVAL, "bad schedule");
     const double elems = (double)c.B * c.H * (c.W + 1) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
         (double)c.n_cond * c.H * c.B > 2.0e9)
@@ -322,6 +323,11 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         const long long c_min = (long long)c.B * c.H * nqt * nt_min;
         long long ctas = std::min<long long>(h->num_sms, kMaxPersistentCtas);
         ctas = std::max<long long>(1, std::min<long long>(ctas, c_min / 2));
+        if (c.schedule == SW_SCHED_TRI) {
+            e = launch_tri(p, c.d, (int)ctas, st);
+            if (e != cudaSuccess) return cuda_fail(e, "three-buffer attention launch");
+            return SW_OK;
+        }
         e = launch_persistent(p, c.d, (int)ctas, st);
         if (e != cudaSuccess) return cuda_fail(e, "persistent attention launch");
     }

@@ -78,12 +78,15 @@ typedef struct {
     float scale;             /* softmax scale; <= 0 selects 1/sqrt(d) */
     int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128,
                                 negative disables the split-K path */
-    int   schedule;          /* full path: SW_SCHED_PERSISTENT (default) or SW_SCHED_GRID */
+    int   schedule;          /* full path: SW_SCHED_PERSISTENT (default), SW_SCHED_GRID or
+                                SW_SCHED_TRI */
 } sw_attn_config;
 
 /* schedules of the full path */
 #define SW_SCHED_PERSISTENT 0   /* one CTA per SM, key tiles cut evenly (stream-K) */
 #define SW_SCHED_GRID       1   /* one CTA per 256 query rows of each (b, h) */
+#define SW_SCHED_TRI        2   /* one CTA per SM, one 128-row Q tile per unit, three S
+                                   accumulators in tensor memory, stream-K leftover */
 
 /*
  * Create a handle with B = 1, sink on, bf16 output, scale 1/sqrt(d).  Host only: allocates

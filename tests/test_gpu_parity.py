@@ -117,7 +117,7 @@ def test_tiny_full_stream(dev, out_dtype, max_short_q):
     assert len(res) == wl.chunks * wl.steps
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
 @pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("max_short_q", [-1, 0])
 def test_ragged_multi_tile(dev, d, max_short_q, schedule):
@@ -127,26 +127,29 @@ def test_ragged_multi_tile(dev, d, max_short_q, schedule):
     stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=max_short_q, schedule=schedule)
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
 @pytest.mark.parametrize("W,sink,n_cond", [(0, False, 40), (0, True, 0), (4, False, 7), (1, True, 130)])
 def test_ragged_other_windows(dev, W, sink, n_cond, schedule):
     wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
     stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1, schedule=schedule)
 
 
-@pytest.mark.parametrize("H,T", [(1, 300), (1, 129), (5, 640), (2, 1400)])
-def test_persistent_split_shapes(dev, H, T):
-    """Shapes whose cost line cuts pairs into 2, 3 or more pieces (one head: a handful of CTAs
-    share every pair)."""
+@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+@pytest.mark.parametrize("H,T", [(1, 300), (1, 129), (5, 640), (2, 1400), (7, 3180)])
+def test_persistent_split_shapes(dev, H, T, schedule):
+    """Shapes whose cost line cuts units into 2, 3 or more pieces (one head: a handful of CTAs
+    share every unit), and one with whole rounds before the stream-K leftover."""
     wl = Workload("split", B=1, H=H, d=128, T=T, n_cond=64, W=1, sink=True, chunks=4, steps=2)
-    stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1)
+    stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1, schedule=schedule,
+                     check_at=None if T < 3000 else {0, 3}, n_rows=None if T < 3000 else 48)
 
 
-def test_persistent_repeatable(dev):
+@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+def test_persistent_repeatable(dev, schedule):
     """The merge counters return to zero after every launch, and split pieces are merged in a
     fixed order whichever arrives last: repeated forwards give bit-identical output."""
     wl = RAGGED
-    h = make_handle(wl, dev, max_short_q=-1)
+    h = make_handle(wl, dev, max_short_q=-1, schedule=schedule)
     Kc, Vc = synth.cond_inputs(wl)
     h.set_cond(Kc.to(dev), Vc.to(dev))
     Q, K, V = (t.to(dev) for t in synth.chunk_inputs(wl, 0, 0))
@@ -194,6 +197,21 @@ def test_720p_sampled(dev):
     res = stream_and_check(wl, dev, chunks=wl.chunks, check_at={0, 1, 3, 4, 5, 31}, n_rows=40,
                            keep_last=wl.W + 1, gen_on_device=True)
     assert len(res) == 12
+
+
+def test_720p_sampled_tri(dev):
+    """The 720p workload on the three-buffer kernel: chunks 0, W+1 and the last of 12."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check(wl, dev, chunks=12, check_at={0, 4, 11}, n_rows=40, keep_last=wl.W + 1,
+                           gen_on_device=True, schedule="tri")
+    assert len(res) == 6
+
+
+def test_stress_sampled_tri(dev):
+    wl = WORKLOADS["stress"]
+    res = stream_and_check(wl, dev, chunks=8, check_at={7}, n_rows=12, keep_last=wl.W + 1,
+                           gen_on_device=True, schedule="tri")
+    assert len(res) == 2
 
 
 def test_stress_sampled(dev):
