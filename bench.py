@@ -268,6 +268,9 @@ def run_cuda(args, wl, world, rank, local):
     elapsed = start.elapsed_time(end) / 1e3
     fwd_ms = [fwd_events[i][2 * s].elapsed_time(fwd_events[i][2 * s + 1])
               for i in range(args.steps) for s in range(wl.steps)]
+    # per chunk: from one step's first forward to the next step's (the last one to `end`)
+    chunk_ms = [fwd_events[i][0].elapsed_time(fwd_events[i + 1][0]) for i in range(args.steps - 1)]
+    chunk_ms.append(fwd_events[-1][0].elapsed_time(end))
     status = h.status()
 
     flops_fwd = wl.flops_forward(k_start)
@@ -307,8 +310,18 @@ def run_cuda(args, wl, world, rank, local):
 
     # ---- side measurements (untimed for the metric): append/evict and the split-K path
     paths = {}
+    ws_bytes = h.workspace_bytes()
+    sched = h.schedule_for()   # the schedule the timed forwards ran with
     if rank == 0:
         paths = side_paths(h, wl, pool, dev, stream, peaks)
+        paths["chunk_ms"] = {"median": round(statistics.median(chunk_ms), 4),
+                             "p95": round(sorted(chunk_ms)[min(len(chunk_ms) - 1, int(0.95 * len(chunk_ms)))], 4),
+                             "chunks": len(chunk_ms)}
+        if not args.no_extra:
+            h.close()
+            h = None
+            paths["long_horizon"] = long_horizon(args, dev, stream, pool)
+            paths["workloads"] = other_workloads(args, dev, stream, peaks)
 
     if rank == 0:
         cpu = None
@@ -332,16 +345,16 @@ def run_cuda(args, wl, world, rank, local):
                        "gflop_per_forward": round(flops_fwd / 1e9, 2),
                        "l2": f"inputs larger than L2: {len(pool)} resident input sets of "
                              f"{sum(t.numel() * 2 for t in pool[0][0]) * wl.steps / 2 ** 20:.0f} MiB plus the "
-                             f"{h.workspace_bytes() / 2 ** 20:.0f} MiB cache, cycled per step",
+                             f"{ws_bytes / 2 ** 20:.0f} MiB cache, cycled per step",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "schedule": args.schedule},
+                       "schedule": sched},
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
                          "kernel": {"persistent": "attn_persistent_kernel<128>", "tri": "attn_tri_kernel<128>",
-                                    "grid": "attn_fwd_kernel<128,2>"}[args.schedule],
+                                    "grid": "attn_fwd_kernel<128,2>"}[sched],
                          "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": _profiled_traffic(wl.name, args.schedule), "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                         "traffic": _profiled_traffic(wl.name, sched), "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                          "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                          "launch_ms_avg": round(fwd_avg * 1e3, 4)},
             "cpu_baseline": cpu,
@@ -353,9 +366,115 @@ def run_cuda(args, wl, world, rank, local):
             "paths": paths,
         }
         print(json.dumps(line), flush=True)
-    h.close()
+    if h is not None:
+        h.close()
     if dist is not None:
         dist.destroy_process_group()
+
+
+def long_horizon(args, dev, stream, pool):
+    """The 225-chunk 720p stream.  (1) On one fresh handle, chunk by chunk: per-chunk device time
+    (2 forwards + append) and the device memory in use (allocator and driver view) after every
+    chunk, which must not change.  (2) Drift = mean time of chunks 200-224 over chunks 5-29,
+    minus 1, measured clock-neutrally: one handle advanced to chunk 5 and one to chunk 200 run
+    their chunks alternately, so both see the same SM clock (a sequential run also sees the
+    clock fall as the part heats under its power cap; that figure is given too)."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    wl = WORKLOADS["long720p"]
+    h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                               out_dtype=torch.bfloat16, schedule=args.schedule, device=dev)
+    Kc, Vc = synth.cond_inputs(wl, seed=7, device=dev)
+    h.set_cond(Kc, Vc)
+    outs = [torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev) for _ in range(wl.steps)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(wl.chunks + 1)]
+    torch.cuda.synchronize(dev)
+    alloc, free = [], []
+    for c in range(wl.chunks):
+        ev[c].record(stream)
+        inputs = pool[c % len(pool)]
+        for s, (Q, K, V) in enumerate(inputs):
+            h.forward(Q, K, V, out=outs[s])
+        h.append_chunk(inputs[-1][1], inputs[-1][2])
+        alloc.append(torch.cuda.memory_allocated(dev))
+        free.append(torch.cuda.mem_get_info(dev)[0])
+    ev[wl.chunks].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = [ev[c].elapsed_time(ev[c + 1]) for c in range(wl.chunks)]
+    early, late = ms[5:30], ms[200:225]
+    drift_seq = (sum(late) / len(late)) / (sum(early) / len(early)) - 1.0
+    steady = ms[wl.W + 1:]
+    res = {"chunks": wl.chunks, "drift_sequential": round(drift_seq, 4),
+           "ms_median": round(statistics.median(steady), 4),
+           "ms_p95": round(sorted(steady)[int(0.95 * (len(steady) - 1))], 4),
+           "allocated_bytes_constant": len(set(alloc)) == 1, "driver_free_bytes_constant": len(set(free)) == 1,
+           "workspace_bytes": h.workspace_bytes(), "status": h.status()}
+    h.close()
+    # clock-neutral drift: chunks 5-29 and 200-224 interleaved on two handles
+    hs = []
+    for start in (5, 200):
+        hx = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                    out_dtype=torch.bfloat16, schedule=args.schedule, device=dev)
+        hx.set_cond(Kc, Vc)
+        for _ in range(start):
+            hx.append_chunk(pool[0][-1][1], pool[0][-1][2])
+        hs.append(hx)
+    t_ms = [[], []]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    for c in range(25):
+        for which, hx in enumerate(hs):
+            inputs = pool[c % len(pool)]
+            e0.record(stream)
+            for s, (Q, K, V) in enumerate(inputs):
+                hx.forward(Q, K, V, out=outs[s])
+            hx.append_chunk(inputs[-1][1], inputs[-1][2])
+            e1.record(stream)
+            e1.synchronize()
+            t_ms[which].append(e0.elapsed_time(e1))
+    drift = (sum(t_ms[1]) / 25) / (sum(t_ms[0]) / 25) - 1.0
+    res.update({"drift": round(drift, 4), "target": "<= 0.02",
+                "ms_chunks_5_29": round(sum(t_ms[0]) / 25, 4), "ms_chunks_200_224": round(sum(t_ms[1]) / 25, 4),
+                "status_interleaved": max(hx.status() for hx in hs)})
+    for hx in hs:
+        hx.close()
+    return res
+
+
+def other_workloads(args, dev, stream, peaks):
+    """Steady-state forward throughput of the other attention workloads (480p, stress): the
+    stream is advanced to the steady state (sink and full window visible), then forwards are
+    timed with CUDA events."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    res = {}
+    for name in ("480p", "stress"):
+        wl = WORKLOADS[name]
+        h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                   out_dtype=torch.bfloat16, schedule=args.schedule, device=dev)
+        Kc, Vc = synth.cond_inputs(wl, seed=3, device=dev)
+        h.set_cond(Kc, Vc)
+        Q, K, V = synth.chunk_inputs(wl, 0, 0, seed=3, device=dev)
+        for _ in range(wl.steady_k()):
+            h.append_chunk(K, V)
+        out = torch.empty_like(Q)
+        for _ in range(3):
+            h.forward(Q, K, V, out=out)
+        torch.cuda.synchronize(dev)
+        reps = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            h.forward(Q, K, V, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        k = wl.steady_k()
+        tf = wl.flops_forward(k) / t / 1e12
+        res[name] = {"schedule": h.schedule_for(), "ms_per_forward": round(t * 1e3, 4), "TFLOP/s": round(tf, 2),
+                     "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "N_vis": wl.n_vis(k),
+                     "status": h.status()}
+        h.close()
+        del Q, K, V, out, Kc, Vc
+    return res
 
 
 def side_paths(h, wl, pool, dev, stream, peaks):
@@ -441,7 +560,9 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", choices=["persistent", "grid", "tri"], default="persistent")
+    ap.add_argument("--schedule", choices=["auto", "persistent", "grid", "tri"], default="auto")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the long-horizon and other-workload side measurements")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswattn.s
 SW_OK, SW_EINVAL, SW_ESHAPE, SW_EALIGN, SW_ESTATE, SW_ECUDA = 0, -1, -2, -3, -4, -5
 SW_STATUS_TIMEOUT, SW_STATUS_BAD_SLOT, SW_STATUS_OVERFLOW = 0x1, 0x2, 0x4
 SW_OUT_BF16, SW_OUT_F32 = 0, 1
-SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI = 0, 1, 2
+SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
 
 # every symbol include/swattn.h declares
 EXPORTS = (
@@ -21,7 +21,7 @@ EXPORTS = (
     "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
-    "sw_attn_selftest_timeout",
+    "sw_attn_selftest_timeout", "sw_attn_schedule_for",
 )
 
 
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_forward_short_noalloc.restype = i32
     L.sw_attn_selftest_timeout.argtypes = [vp, ctypes.c_int64, vp]
     L.sw_attn_selftest_timeout.restype = i32
+    L.sw_attn_schedule_for.argtypes = [vp, i32]
+    L.sw_attn_schedule_for.restype = i32
     L.sw_attn_table_ints.argtypes = [vp]
     L.sw_attn_table_ints.restype = i32
     L.sw_attn_get_table.argtypes = [vp, vp, vp]

@@ -33,14 +33,14 @@ class SlidingWindowAttention:
 
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
-                 max_short_q: int = 0, schedule: str = "persistent", device=None):
+                 max_short_q: int = 0, schedule: str = "auto", device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
                              out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
                              scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
                              schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
-                                       "tri": N.SW_SCHED_TRI}[schedule])
+                                       "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule])
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()
@@ -54,6 +54,13 @@ class SlidingWindowAttention:
             self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
             N.check(self._lib.sw_attn_bind_workspace(h, self.workspace.data_ptr(), nbytes, _stream_ptr()))
         self.table_ints = int(self._lib.sw_attn_table_ints(h))
+
+    def schedule_for(self, n_q: int | None = None) -> str:
+        """The schedule a full-path forward of n_q queries (default T) runs with."""
+        r = int(self._lib.sw_attn_schedule_for(self._h, self.T if n_q is None else n_q))
+        if r < 0:
+            N.check(r)
+        return {N.SW_SCHED_PERSISTENT: "persistent", N.SW_SCHED_GRID: "grid", N.SW_SCHED_TRI: "tri"}[r]
 
     # -- stream control
     def set_cond(self, K_cond: torch.Tensor, V_cond: torch.Tensor, stream=None) -> None:

@@ -77,16 +77,19 @@ cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int 
 }
 
 // K2: copy K and V of one chunk from the user layout [B, N, H, d] into the head-major cache
-// layout [B][H][rows_per_bh][d] at row offset slot * N.  One thread moves 16 bytes; threads
-// run over the source in order (coalesced 16-byte loads), and each group of d/8 threads
-// writes one contiguous d-row of the destination (coalesced 16-byte stores).
-__global__ void __launch_bounds__(256) relayout_kernel(const uint4* __restrict__ srcK,
+// layout [B][H][rows_per_bh][d] at row offset slot * N.
+// One block per token row (b, t) of K or V (blockIdx.y = 0 / 1): the row's H x d bf16 values are
+// contiguous in the caller's [B, N, H, d] layout, and head h's d values go to row
+// slot * N + t of the (b, h) panel of the destination.  Thread k of the block moves 16-byte
+// vector k of the row (head k / vpr, vector k % vpr), looping when H * vpr exceeds the block,
+// so consecutive threads read consecutive bytes and write whole 16-byte pieces of 2d-byte
+// destination rows.  No division in the copy loop (vpr is a power of two).
+__global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__ srcK,
                                                        const uint4* __restrict__ srcV,
                                                        uint4* __restrict__ dstK,
-                                                       uint4* __restrict__ dstV, int B, int N,
-                                                       int H, int vec_per_row, int rows_per_bh,
-                                                       int ring, int W, int sink, int S,
-                                                       int32_t* state) {
+                                                       uint4* __restrict__ dstV, int N, int H,
+                                                       int vpr_log2, int rows_per_bh, int ring,
+                                                       int W, int sink, int S, int32_t* state) {
     int slot = 0;
     if (ring) {
         slot = ring_slot(state[0], W, sink);
@@ -99,34 +102,34 @@ __global__ void __launch_bounds__(256) relayout_kernel(const uint4* __restrict__
     }
     const uint4* __restrict__ src = blockIdx.y == 0 ? srcK : srcV;
     uint4* __restrict__ dst = blockIdx.y == 0 ? dstK : dstV;
-    const long long total = (long long)B * N * H * vec_per_row;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-        const int v = (int)(i % vec_per_row);
-        long long r = i / vec_per_row;              // source row index over (b, t, h)
-        const int h = (int)(r % H);
-        r /= H;
-        const int t = (int)(r % N);
-        const int b = (int)(r / N);
-        const long long drow = ((long long)b * H + h) * rows_per_bh + (long long)slot * N + t;
-        dst[drow * vec_per_row + v] = __ldg(src + i);
+    const int row = blockIdx.x;                     // b * N + t
+    const int b = row / N, t = row - b * N;
+    const int vpr = 1 << vpr_log2;
+    const int per_row = H << vpr_log2;
+    const uint4* s_row = src + (size_t)row * per_row;
+    const size_t drow0 = (size_t)b * H * rows_per_bh + (size_t)slot * N + t;   // head 0's row
+    for (int k = threadIdx.x; k < per_row; k += blockDim.x) {
+        const int h = k >> vpr_log2, v = k & (vpr - 1);
+        dst[(drow0 + (size_t)h * rows_per_bh) * vpr + v] = __ldg(s_row + k);
     }
 }
 
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int W, int sink, int S,
                             int32_t* state, cudaStream_t stream) {
-    const int vec_per_row = d / 8;
-    const long long total = (long long)B * N * H * vec_per_row;
-    long long blocks = (total + 255) / 256;
-    // enough blocks to fill the GPU several times over, grid-stride beyond that
-    const long long cap = 148LL * 16;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    dim3 grid((unsigned)blocks, 2);
-    relayout_kernel<<<grid, 256, 0, stream>>>(
+    const int vpr = d / 8;                          // 16-byte vectors per head row
+    int vpr_log2 = 0;
+    while ((1 << vpr_log2) < vpr) ++vpr_log2;
+    if ((1 << vpr_log2) != vpr) return cudaErrorInvalidValue;   // d is 64 or 128
+    const long long rows = (long long)B * N;
+    if (rows < 1) return cudaSuccess;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int per_row = H * vpr;
+    const int threads = per_row >= 512 ? 512 : ((per_row + 31) / 32) * 32;
+    dim3 grid((unsigned)rows, 2);
+    relayout_kernel<<<grid, threads, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
-        static_cast<uint4*>(dstV), B, N, H, vec_per_row, rows_per_bh, ring, W, sink, S, state);
+        static_cast<uint4*>(dstV), N, H, vpr_log2, rows_per_bh, ring, W, sink, S, state);
     return cudaGetLastError();
 }
 

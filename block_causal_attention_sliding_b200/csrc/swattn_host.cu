@@ -104,7 +104,8 @@ int check_cfg(const sw_attn_config& c) {
     if (c.out_dtype != SW_OUT_BF16 && c.out_dtype != SW_OUT_F32) return fail(SW_EINVAL, "bad out_dtype");
     if (c.max_short_q > kMaxShortQ) return fail(SW_ESHAPE, "max_short_q must be <= %d", kMaxShortQ);
     if (!std::isfinite(c.scale)) return fail(SW_EINVAL, "scale must be finite");
-    if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID && c.schedule != SW_SCHED_TRI)
+    if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID && c.schedule != SW_SCHED_TRI &&
+        c.schedule != SW_SCHED_AUTO)
         return fail(SW_EINVAL, "bad schedule");
     const double elems = (double)c.B * c.H * (c.W + 1) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
@@ -159,7 +160,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     sw_attn_config c;
     std::memset(&c, 0, sizeof c);
     c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
-    c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_PERSISTENT;
+    c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_AUTO;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -260,6 +261,23 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
 }
 
+// The full-path schedule of a forward of n_q queries.  Auto: with fewer pairs of 128-row Q tiles
+// than SMs, the two-tile persistent schedule would cut every pair between CTAs, and one Q tile
+// per unit (the three-buffer kernel) balances better; otherwise the two-tile kernel, whose K/V
+// tiles each serve two Q tiles, is faster.
+static int resolve_schedule(const sw_attn_t* h, int n_q) {
+    const sw_attn_config& c = h->cfg;
+    if (c.schedule != SW_SCHED_AUTO) return c.schedule;
+    const long long pairs = (long long)c.B * c.H * ((n_q + 2 * kBlockM - 1) / (2 * kBlockM));
+    return pairs < h->num_sms ? SW_SCHED_TRI : SW_SCHED_PERSISTENT;
+}
+
+int sw_attn_schedule_for(const sw_attn_t* h, int n_q) {
+    g_err.clear();
+    if (!h || n_q < 1) return fail(SW_EINVAL, "null handle or n_q < 1");
+    return resolve_schedule(h, n_q);
+}
+
 int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out, int n_q,
                     void* stream) {
     g_err.clear();
@@ -305,7 +323,7 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
         e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
         if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-    } else if (c.schedule == SW_SCHED_GRID) {
+    } else if (resolve_schedule(h, n_q) == SW_SCHED_GRID) {
         p.splits = 0;
         const int grid_x = (n_q + 2 * kBlockM - 1) / (2 * kBlockM);
         e = launch_attention(p, c.d, 2, grid_x, st);
@@ -323,7 +341,7 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         const long long c_min = (long long)c.B * c.H * nqt * nt_min;
         long long ctas = std::min<long long>(h->num_sms, kMaxPersistentCtas);
         ctas = std::max<long long>(1, std::min<long long>(ctas, c_min / 2));
-        if (c.schedule == SW_SCHED_TRI) {
+        if (resolve_schedule(h, n_q) == SW_SCHED_TRI) {
             e = launch_tri(p, c.d, (int)ctas, st);
             if (e != cudaSuccess) return cuda_fail(e, "three-buffer attention launch");
             return SW_OK;

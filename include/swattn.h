@@ -78,8 +78,8 @@ typedef struct {
     float scale;             /* softmax scale; <= 0 selects 1/sqrt(d) */
     int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128,
                                 negative disables the split-K path */
-    int   schedule;          /* full path: SW_SCHED_PERSISTENT (default), SW_SCHED_GRID or
-                                SW_SCHED_TRI */
+    int   schedule;          /* full path: SW_SCHED_AUTO (default), SW_SCHED_PERSISTENT,
+                                SW_SCHED_GRID or SW_SCHED_TRI */
 } sw_attn_config;
 
 /* schedules of the full path */
@@ -87,6 +87,9 @@ typedef struct {
 #define SW_SCHED_GRID       1   /* one CTA per 256 query rows of each (b, h) */
 #define SW_SCHED_TRI        2   /* one CTA per SM, one 128-row Q tile per unit, three S
                                    accumulators in tensor memory, stream-K leftover */
+#define SW_SCHED_AUTO       3   /* per launch: SW_SCHED_TRI when the pairs of 128-row Q tiles
+                                   (B * H * ceil(n_q / 256)) are fewer than the SMs, else
+                                   SW_SCHED_PERSISTENT (see sw_attn_schedule_for) */
 
 /*
  * Create a handle with B = 1, sink on, bf16 output, scale 1/sqrt(d).  Host only: allocates
@@ -191,6 +194,13 @@ SW_API int sw_attn_cache_offsets(const sw_attn_t *h, size_t *k_offset, size_t *v
  * that a stalled pipeline ends in an error status rather than a hang.  sw_attn_reset clears it.
  */
 SW_API int sw_attn_selftest_timeout(sw_attn_t *h, int64_t limit_ns, void *stream);
+
+/*
+ * The schedule a full-path forward of n_q queries runs with on this handle (SW_SCHED_PERSISTENT,
+ * SW_SCHED_GRID or SW_SCHED_TRI; SW_SCHED_AUTO resolved as described above).  Host only, no
+ * CUDA call.  Returns the schedule, or SW_EINVAL for a null handle or n_q < 1.
+ */
+SW_API int sw_attn_schedule_for(const sw_attn_t* h, int n_q);
 
 /* Synchronise the device, then read the device status bits into *host_status. */
 SW_API int sw_attn_get_status(sw_attn_t *h, int32_t *host_status);

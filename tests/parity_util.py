@@ -35,7 +35,7 @@ def sample_rows(n_q: int, n: int, seed: int) -> np.ndarray:
 
 
 def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink=None, n_cond=None,
-                schedule="persistent"):
+                schedule="auto"):
     return SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W if W is None else W,
                                   n_cond=wl.n_cond if n_cond is None else n_cond,
                                   sink=wl.sink if sink is None else sink, out_dtype=out_dtype,
@@ -44,7 +44,7 @@ def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink
 
 def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, n_q=None,
                      out_dtype=torch.float32, max_short_q=0, poison=False, seed=0,
-                     tol=(MAX_ABS, MEAN_REL), keep_last=None, gen_on_device=False, schedule="persistent"):
+                     tol=(MAX_ABS, MEAN_REL), keep_last=None, gen_on_device=False, schedule="auto"):
     """Stream `chunks` chunks (2 forwards then an append each).  At the chunks in `check_at`
     (all if None) compare the CUDA output with the oracle, on all rows or on sampled rows.
     With gen_on_device the seeded draws use the GPU generator (faster for big shapes); the

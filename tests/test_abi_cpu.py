@@ -120,3 +120,31 @@ def test_null_handle(native):
     assert L.sw_attn_workspace_bytes(None) == 0
     assert L.sw_attn_forward(None, None, None, None, None, 1, None) == native.SW_EINVAL
     L.sw_attn_destroy(None)   # ignored
+
+
+def test_schedule_resolution(native):
+    """Auto picks the two-tile persistent kernel when there are at least as many 128-row Q-tile
+    pairs as SMs (148 before a device is bound), the three-buffer kernel otherwise; explicit
+    schedules are returned as given.  Host only."""
+    L = native.lib()
+    cases = [
+        (dict(schedule=native.SW_SCHED_AUTO), 3180, native.SW_SCHED_PERSISTENT),        # 24 x 13 = 312 pairs
+        (dict(schedule=native.SW_SCHED_AUTO, H=16, tokens_per_chunk=1400), 1400, native.SW_SCHED_TRI),  # 96
+        (dict(schedule=native.SW_SCHED_GRID), 3180, native.SW_SCHED_GRID),
+        (dict(schedule=native.SW_SCHED_TRI), 3180, native.SW_SCHED_TRI),
+    ]
+    for kw, n_q, want in cases:
+        rc, h = _create(native, **kw)
+        assert rc == 0
+        assert L.sw_attn_schedule_for(h, n_q) == want, (kw, n_q)
+        L.sw_attn_destroy(h)
+    # the boundary: 147 pairs -> tri, 148 pairs -> persistent (H heads x 1 pair with n_q <= 256)
+    for H, want in ((147, native.SW_SCHED_TRI), (148, native.SW_SCHED_PERSISTENT)):
+        rc, h = _create(native, schedule=native.SW_SCHED_AUTO, H=H, tokens_per_chunk=256, n_cond=0)
+        assert rc == 0
+        assert L.sw_attn_schedule_for(h, 256) == want
+        L.sw_attn_destroy(h)
+    rc, h = _create(native, schedule=native.SW_SCHED_AUTO)
+    assert L.sw_attn_schedule_for(h, 0) == native.SW_EINVAL
+    assert L.sw_attn_schedule_for(None, 10) == native.SW_EINVAL
+    L.sw_attn_destroy(h)
