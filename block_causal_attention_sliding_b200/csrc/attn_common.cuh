@@ -252,6 +252,7 @@ __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid
 #pragma unroll
     for (int a = 0; a < 8; ++a) suma[a] = 0.f;
     const float neg_m = -m_ref;
+    const uint64_t sl2_2 = bcast2(sl2), neg_m2 = bcast2(neg_m);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -260,8 +261,9 @@ __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid
             const int c = 2 * half + cc;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float x0 = fmaf(__uint_as_float(sr[c][i]), sl2, neg_m);
-                const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), sl2, neg_m);
+                // x = s * scale * log2(e) - m for two columns in one packed FMA
+                float x0, x1;
+                fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
                 const bool poly = kPolyEvery > 0 && ((i >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
                 const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
                 const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);

@@ -285,6 +285,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid
 #pragma unroll
     for (int a = 0; a < 8; ++a) suma[a] = 0.f;
     const float neg_m = -m_new;
+    const uint64_t sl2_2 = bcast2(sl2), neg_m2 = bcast2(neg_m);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -293,8 +294,8 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid
             const int c = 2 * half + cc;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float x0 = fmaf(__uint_as_float(sr[c][i]), sl2, neg_m);
-                const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), sl2, neg_m);
+                float x0, x1;   // s * scale * log2(e) - m for two columns in one packed FMA
+                fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
                 const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
                 // the row sum adds the same bf16-rounded weights the PV MMA multiplies
                 const int a = (i >> 1) & 7;

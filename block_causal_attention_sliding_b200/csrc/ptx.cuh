@@ -260,6 +260,21 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// (x0, x1) = (a0 * s + b, a1 * s + b) as one packed two-lane fp32 FMA (the sm_100 f32x2 form;
+// each lane rounds exactly like a scalar fmaf).  s2 and b2 hold the broadcast operands.
+__device__ __forceinline__ void fma2_bcast(float& x0, float& x1, float a0, float a1, uint64_t s2, uint64_t b2) {
+    asm("{\n\t.reg .b64 a, d;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 d, a, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(x0), "=f"(x1) : "f"(a0), "f"(a1), "l"(s2), "l"(b2));
+}
+
+// v in both lanes of a packed f32x2 operand.
+__device__ __forceinline__ uint64_t bcast2(float v) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
+
 // max(a, b, c) in one instruction (three-input max, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
