@@ -493,7 +493,8 @@ def other_workloads(args, dev, stream, peaks):
 
 
 def side_paths(h, wl, pool, dev, stream, peaks):
-    """Append/evict (HBM-bound copy) and the split-K short-query path, timed alone."""
+    """Append/evict (HBM-bound copy), the split-K short-query path and the joint forward with
+    condition-stream queries, timed alone."""
     out = {}
     reps = 50
     Q, K, V = pool[0][-1]
@@ -528,6 +529,29 @@ def side_paths(h, wl, pool, dev, stream, peaks):
         dec[str(nq)] = {"us": round(t * 1e6, 2), "GB/s": round(kv_bytes / t / 1e9, 1),
                         "frac_hbm": round(kv_bytes / t / 1e9 / peaks["hbm_gbs"], 3)}
     out["split_k"] = dec
+    # the joint forward: the chunk's T queries and the n_cond condition-stream queries in one
+    # launch, against the two as separate forwards
+    Qc = synth.cond_queries(wl, 0, 0, seed=5, device=dev)
+    o = torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+    oc = torch.empty((wl.B, wl.n_cond, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    t_joint = timed(lambda: h.forward_joint(Q, Qc, K, V, out=o, out_cond=oc))
+    t_sep = timed(lambda: (h.forward(Q, K, V, out=o), h.forward(Qc, K, V, out=oc)))
+    fl = wl.flops_forward(k, wl.T + wl.n_cond)
+    out["joint"] = {"queries": f"{wl.T} chunk + {wl.n_cond} condition", "ms": round(t_joint * 1e3, 4),
+                    "TFLOP/s": round(fl / t_joint / 1e12, 2), "frac_of_peak": round(fl / t_joint / 1e12 / peaks["bf16_tflops"], 4),
+                    "separate_forwards_ms": round(t_sep * 1e3, 4)}
     return out
 
 

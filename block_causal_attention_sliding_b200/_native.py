@@ -18,7 +18,8 @@ SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
 # every symbol include/swattn.h declares
 EXPORTS = (
     "sw_attn_create", "sw_attn_create_ex", "sw_attn_workspace_bytes", "sw_attn_bind_workspace",
-    "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_table_ints",
+    "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_forward_joint",
+    "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
     "sw_attn_selftest_timeout", "sw_attn_schedule_for",
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_append_chunk.restype = i32
     L.sw_attn_forward.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward.restype = i32
+    L.sw_attn_forward_joint.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    L.sw_attn_forward_joint.restype = i32
     L.sw_attn_forward_short_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward_short_noalloc.restype = i32
     L.sw_attn_selftest_timeout.argtypes = [vp, ctypes.c_int64, vp]

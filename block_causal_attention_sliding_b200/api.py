@@ -100,6 +100,32 @@ class SlidingWindowAttention:
 
     __call__ = forward
 
+    def forward_joint(self, Q: torch.Tensor, Q_cond: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
+                      out: torch.Tensor | None = None, out_cond: torch.Tensor | None = None,
+                      stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+        """The chunk's queries (all T rows) and the condition-stream queries ([B, n_cond, H, d]) over
+        the same visible keys, in one launch (sw_attn_forward_joint).  Returns (out, out_cond)."""
+        q_shape = (self.B, self.T, self.H, self.d)
+        qc_shape = (self.B, self.n_cond, self.H, self.d)
+        for name, t, shp in (("Q", Q, q_shape), ("K_cur", K_cur, q_shape), ("V_cur", V_cur, q_shape),
+                             ("Q_cond", Q_cond, qc_shape)):
+            if tuple(t.shape) != shp:
+                raise ValueError(f"{name} must have shape {shp}, got {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty(q_shape, dtype=self.out_dtype, device=Q.device)
+        if out_cond is None:
+            out_cond = torch.empty(qc_shape, dtype=self.out_dtype, device=Q.device)
+        for name, t, shp in (("out", out, q_shape), ("out_cond", out_cond, qc_shape)):
+            if tuple(t.shape) != shp or t.dtype != self.out_dtype:
+                raise ValueError(f"{name} must be {shp} in the handle's out_dtype")
+        N.check(self._lib.sw_attn_forward_joint(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
+                                                _dev_ptr(Q_cond, "Q_cond", torch.bfloat16),
+                                                _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+                                                _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                                _dev_ptr(out, "out"), _dev_ptr(out_cond, "out_cond"),
+                                                _stream_ptr(stream)))
+        return out, out_cond
+
     def reset(self, stream=None) -> None:
         N.check(self._lib.sw_attn_reset(self._h, _stream_ptr(stream)))
 

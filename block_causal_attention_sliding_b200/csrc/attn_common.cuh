@@ -137,6 +137,25 @@ __device__ __forceinline__ void tile_of(const SmemCtl* ctl, int j, int& seg, int
     valid = rem < kBlockN ? rem : kBlockN;
 }
 
+// Query tiles of a launch: the chunk's n_q queries in tiles 0 .. ceil(n_q / 128) - 1, then (joint
+// forward) the n_qc condition-stream queries, which attend over the same visible keys.
+struct QSrc {
+    const CUtensorMap* tm;   // tensor map of the tile's query tensor
+    int row0;                // first query row of the tile in that tensor
+    int rows;                // rows of that tensor (n_q or n_qc)
+    void* out;               // output tensor of the same rows
+};
+
+__device__ __forceinline__ int q_tiles(const AttnParams& p) {
+    return (p.n_q + kBlockM - 1) / kBlockM + (p.n_qc + kBlockM - 1) / kBlockM;
+}
+
+__device__ __forceinline__ QSrc q_src(const AttnParams& p, int u) {
+    const int nv = (p.n_q + kBlockM - 1) / kBlockM;
+    if (u < nv) return QSrc{&p.tm_q, u * kBlockM, p.n_q, p.out};
+    return QSrc{&p.tm_qc, (u - nv) * kBlockM, p.n_qc, p.out_c};
+}
+
 // TMA loads of one 128-row K (kv = 0) or V (kv = 1) tile of key tile j of (b, h) into dst,
 // completing on bar: condition tokens, a ring slot, or the caller's current chunk.
 template <int D>

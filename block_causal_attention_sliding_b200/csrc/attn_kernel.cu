@@ -57,6 +57,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
         load_table(ctl, p.table, p.status);
     } else if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_qc);
         tma_prefetch_desc(&p.tm_kcur);
         tma_prefetch_desc(&p.tm_vcur);
         tma_prefetch_desc(&p.tm_cache_k);
@@ -74,20 +75,22 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
         t1 = (int)((long long)(blockIdx.x + 1) * n_tiles / p.splits);
     }
     const int n = t1 - t0;                          // key tiles this CTA processes
-    const int m0 = split_mode ? 0 : blockIdx.x * NQ * kBlockM;
+    const int u0 = split_mode ? 0 : blockIdx.x * NQ;   // first Q tile of this CTA
     // Q tiles of this CTA that hold at least one query row (the last CTA of a head may own
     // a single tile); tiles past n_q are neither loaded nor computed
-    const int live = min(NQ, (p.n_q - m0 + kBlockM - 1) / kBlockM);
+    const int live = min(NQ, q_tiles(p) - u0);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && n > 0) {
             const uint32_t qbar = smem_u32(&ctl->q_full);
             mbar_arrive_expect_tx(qbar, live * kTileBytes);
-            for (int qt = 0; qt < live; ++qt)
+            for (int qt = 0; qt < live; ++qt) {
+                const QSrc qs = q_src(p, u0 + qt);
                 for (int c = 0; c < C::kBoxes; ++c)
-                    tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), &p.tm_q, qbar,
-                                c * kBoxCols, h, m0 + qt * kBlockM, b);
+                    tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), qs.tm, qbar,
+                                c * kBoxCols, h, qs.row0, b);
+            }
             uint32_t it = 0;
             bool ok = true;
             for (int j = t0; j < t1 && ok; ++j) {
@@ -272,7 +275,8 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             warp_arrive(smem_u32(&ctl->p_full[qt]));
         }
         // ------------------------------------------------------------ epilogue
-        const int m_row = m0 + qt * kBlockM + row;
+        const QSrc qs = q_src(p, u0 + qt);
+        const int m_row = qs.row0 + row;
         if (n == 0) {
             // split mode with an empty slice: neutral partials
             if (split_mode) {
@@ -301,8 +305,8 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                         p.ml_part[prow * 2 + 0] = m_ref;
                         p.ml_part[prow * 2 + 1] = l;
                     }
-                } else if (m_row < p.n_q) {
-                    store_row_chunk<D>(p.out, p.out_f32, ((size_t)b * p.n_q + m_row) * p.H + h, c, o, inv);
+                } else if (m_row < qs.rows) {
+                    store_row_chunk<D>(qs.out, p.out_f32, ((size_t)b * qs.rows + m_row) * p.H + h, c, o, inv);
                 }
             }
         }

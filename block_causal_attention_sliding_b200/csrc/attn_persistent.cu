@@ -50,6 +50,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
         load_table(ctl, p.table, p.status);
     } else if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_qc);
         tma_prefetch_desc(&p.tm_kcur);
         tma_prefetch_desc(&p.tm_vcur);
         tma_prefetch_desc(&p.tm_cache_k);
@@ -62,7 +63,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
     const uint32_t tmem = ctl->tmem_base;
     const int g = blockIdx.x;
     const int nt = ctl->n_tiles;
-    const int nqt = (p.n_q + kBlockM - 1) / kBlockM;
+    const int nqt = q_tiles(p);
     Sched sched;
     sched.init(nqt, nt, p.B * p.H, (int)gridDim.x, g);
 
@@ -77,14 +78,15 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             bool ok = true;
             while (ok && next_piece(sched, pit, pc)) {
                 const int b = pc.bh / p.H, h = pc.bh % p.H;
-                const int m0 = pc.pair * NQ * kBlockM;
                 // the Q buffers are reused: wait until every S MMA of the previous piece is done
                 if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(qbar, pc.live * kTileBytes);
-                for (int qt = 0; qt < pc.live; ++qt)
+                for (int qt = 0; qt < pc.live; ++qt) {
+                    const QSrc qs = q_src(p, pc.pair * NQ + qt);
                     for (int c = 0; c < C::kBoxes; ++c)
-                        tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), &p.tm_q, qbar,
-                                    c * kBoxCols, h, m0 + qt * kBlockM, b);
+                        tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), qs.tm, qbar,
+                                    c * kBoxCols, h, qs.row0, b);
+                }
                 ++pi;
                 for (int j = pc.j0; j < pc.j1 && ok; ++j) {
                     for (int kv = 0; kv < 2; ++kv, ++it) {
@@ -242,13 +244,14 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             warp_arrive(smem_u32(&ctl->o_empty[qt]));   // O may now be overwritten
 
             const int b = pc.bh / p.H, h = pc.bh % p.H;
-            const int m_row = pc.pair * NQ * kBlockM + qt * kBlockM + row;
-            const size_t orow = ((size_t)b * p.n_q + m_row) * p.H + h;
+            const QSrc qs = q_src(p, pc.pair * NQ + qt);
+            const int m_row = qs.row0 + row;
+            const size_t orow = ((size_t)b * qs.rows + m_row) * p.H + h;
             if (pc.j0 == 0 && pc.j1 == nt) {
                 const float inv = 1.f / l;
-                if (m_row < p.n_q) {
+                if (m_row < qs.rows) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(p.out, p.out_f32, orow, c, o[c], inv);
+                    for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(qs.out, p.out_f32, orow, c, o[c], inv);
                 }
                 continue;
             }
@@ -311,9 +314,9 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                         o[c][i] = __float_as_uint(fmaf(w, __ldcg(po + (c * 32 + i) * kBlockM), __uint_as_float(o[c][i])));
             }
             const float inv = 1.f / L_;
-            if (m_row < p.n_q) {
+            if (m_row < qs.rows) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(p.out, p.out_f32, orow, c, o[c], inv);
+                for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(qs.out, p.out_f32, orow, c, o[c], inv);
             }
             if (row == 0) atomicExch(cnt, 0);   // all pieces have arrived: ready for the next launch
         }

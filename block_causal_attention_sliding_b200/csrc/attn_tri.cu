@@ -373,6 +373,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
         load_table(ctl, p.table, p.status);
     } else if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_qc);
         tma_prefetch_desc(&p.tm_kcur);
         tma_prefetch_desc(&p.tm_vcur);
         tma_prefetch_desc(&p.tm_cache_k);
@@ -384,7 +385,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
 
     const uint32_t tmem = ctl->tmem_base;
     const int nt = ctl->n_tiles;
-    const int nqt = (p.n_q + kBlockM - 1) / kBlockM;
+    const int nqt = q_tiles(p);
     tri::Sched sched;
     sched.init(nqt, nt, p.B * p.H, (int)gridDim.x, blockIdx.x);
 
@@ -403,8 +404,9 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                 // the Q buffer is reused: every S MMA of the previous piece has completed
                 if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(qbar, kTileBytes);
+                const QSrc qs = q_src(p, qtile);
                 for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
-                    tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * kBoxCols, h, qtile * kBlockM, b);
+                    tma_load_4d(smem_u32(q_smem + c * kBoxBytes), qs.tm, qbar, c * kBoxCols, h, qs.row0, b);
                 ++pi;
                 const int n = pc.j1 - pc.j0;
                 // K(u): its stage last held K(u - kKSt), free once S(u - kKSt) has completed
@@ -613,14 +615,15 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
 
             const int bh = pc.unit / nqt, qtile = pc.unit % nqt;
             const int b = bh / p.H, h = bh % p.H;
-            const int m_row = qtile * kBlockM + row;
-            const size_t orow = ((size_t)b * p.n_q + m_row) * p.H + h;
+            const QSrc qs = q_src(p, qtile);
+            const int m_row = qs.row0 + row;
+            const size_t orow = ((size_t)b * qs.rows + m_row) * p.H + h;
             if (pc.j0 == 0 && pc.j1 == nt) {
                 const float inv = 1.f / l_row;
-                if (m_row < p.n_q) {
+                if (m_row < qs.rows) {
 #pragma unroll
                     for (int c = 0; c < D / 64; ++c)
-                        store_row_chunk<D>(p.out, p.out_f32, orow, g * (D / 64) + c, o[c], inv);
+                        store_row_chunk<D>(qs.out, p.out_f32, orow, g * (D / 64) + c, o[c], inv);
                 }
                 continue;
             }
@@ -678,7 +681,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                     for (int i = 0; i < 32; ++i)
                         acc[i] = __float_as_uint(fmaf(w, __ldcg(po + i * kBlockM), __uint_as_float(acc[i])));
                 }
-                if (m_row < p.n_q) store_row_chunk<D>(p.out, p.out_f32, orow, g * (D / 64) + c, acc, inv);
+                if (m_row < qs.rows) store_row_chunk<D>(qs.out, p.out_f32, orow, g * (D / 64) + c, acc, inv);
             }
             if (sw == 0 && lane == 0) atomicExch(cnt, 0);   // all pieces arrived: ready for the next launch
         }

@@ -146,7 +146,8 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->off_ml = off;
     if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * 2 * 4, 1024);
     // persistent schedule: two partial slots per CTA and one counter per (b, h, pair, Q tile)
-    h->sk_pairs = (cfg->tokens_per_chunk + 2 * kBlockM - 1) / (2 * kBlockM);
+    // (a joint forward adds the condition queries' Q tiles after the chunk's)
+    h->sk_pairs = ((cfg->tokens_per_chunk + kBlockM - 1) / kBlockM + (cfg->n_cond + kBlockM - 1) / kBlockM + 1) / 2;
     h->n_counters = (long long)bh * h->sk_pairs * 2;
     h->off_sk_o = off;   off = align_up(off + (size_t)2 * kMaxPersistentCtas * 2 * d * kBlockM * 4, 1024);
     h->off_sk_ml = off;  off = align_up(off + (size_t)2 * kMaxPersistentCtas * 2 * kBlockM * 2 * 4, 1024);
@@ -261,21 +262,85 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
 }
 
-// The full-path schedule of a forward of n_q queries.  Auto: with fewer pairs of 128-row Q tiles
-// than SMs, the two-tile persistent schedule would cut every pair between CTAs, and one Q tile
-// per unit (the three-buffer kernel) balances better; otherwise the two-tile kernel, whose K/V
-// tiles each serve two Q tiles, is faster.
-static int resolve_schedule(const sw_attn_t* h, int n_q) {
+// The full-path schedule of a forward over nqt Q tiles of 128 rows.  Auto: with fewer pairs of
+// tiles than SMs, the three-buffer kernel (one tile per unit balances better); else persistent.
+static int resolve_schedule_tiles(const sw_attn_t* h, long long nqt) {
     const sw_attn_config& c = h->cfg;
     if (c.schedule != SW_SCHED_AUTO) return c.schedule;
-    const long long pairs = (long long)c.B * c.H * ((n_q + 2 * kBlockM - 1) / (2 * kBlockM));
+    const long long pairs = (long long)c.B * c.H * ((nqt + 1) / 2);
     return pairs < h->num_sms ? SW_SCHED_TRI : SW_SCHED_PERSISTENT;
+}
+
+static int resolve_schedule(const sw_attn_t* h, int n_q) {
+    return resolve_schedule_tiles(h, (n_q + kBlockM - 1) / kBlockM);
 }
 
 int sw_attn_schedule_for(const sw_attn_t* h, int n_q) {
     g_err.clear();
     if (!h || n_q < 1) return fail(SW_EINVAL, "null handle or n_q < 1");
     return resolve_schedule(h, n_q);
+}
+
+// Tensor maps, pointers and scalars every forward shares (the chunk's own n_q queries).
+static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const void* K_cur, const void* V_cur,
+                       void* out, int n_q) {
+    const sw_attn_config& c = h->cfg;
+    std::memset(&p, 0, sizeof p);
+    int rc;
+    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
+    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
+    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
+    // maps for regions this handle does not have are never read; fill them with a valid map
+    p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
+    p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
+    p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
+    p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
+    p.tm_qc = p.tm_q;   // no condition queries unless a joint forward sets them
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    p.out = out;
+    p.out_c = nullptr;
+    p.table = state + kStateHeaderInts;
+    p.status = state + 1;
+    p.B = c.B;
+    p.H = c.H;
+    p.n_q = n_q;
+    p.n_qc = 0;
+    p.out_f32 = c.out_dtype == SW_OUT_F32;
+    p.scale_log2 = c.scale * 1.4426950408889634f;
+    return SW_OK;
+}
+
+// Full-path launch over all Q tiles of p (the chunk's, then any condition queries'), with the
+// schedule the handle resolves for that many tiles.
+static int launch_full(sw_attn_t* h, AttnParams& p, cudaStream_t st) {
+    const sw_attn_config& c = h->cfg;
+    const long long nqt = (p.n_q + kBlockM - 1) / kBlockM + (p.n_qc + kBlockM - 1) / kBlockM;
+    const int sched = resolve_schedule_tiles(h, nqt);
+    cudaError_t e;
+    p.splits = 0;
+    if (sched == SW_SCHED_GRID) {
+        e = launch_attention(p, c.d, 2, (int)((nqt + 1) / 2), st);
+        if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+        return SW_OK;
+    }
+    p.sk_o = reinterpret_cast<float*>(h->ws + h->off_sk_o);
+    p.sk_ml = reinterpret_cast<float*>(h->ws + h->off_sk_ml);
+    p.sk_cnt = reinterpret_cast<int32_t*>(h->ws + h->off_sk_cnt);
+    p.sk_pairs = h->sk_pairs;
+    // one CTA per SM, but never so many that a CTA's share of the cost line is shorter than
+    // two items at the fewest key tiles a chunk can have (condition + current only)
+    const long long nt_min = (c.n_cond + kBlockN - 1) / kBlockN + (c.tokens_per_chunk + kBlockN - 1) / kBlockN;
+    const long long c_min = (long long)c.B * c.H * nqt * nt_min;
+    long long ctas = std::min<long long>(h->num_sms, kMaxPersistentCtas);
+    ctas = std::max<long long>(1, std::min<long long>(ctas, c_min / 2));
+    if (sched == SW_SCHED_TRI) {
+        e = launch_tri(p, c.d, (int)ctas, st);
+        if (e != cudaSuccess) return cuda_fail(e, "three-buffer attention launch");
+        return SW_OK;
+    }
+    e = launch_persistent(p, c.d, (int)ctas, st);
+    if (e != cudaSuccess) return cuda_fail(e, "persistent attention launch");
+    return SW_OK;
 }
 
 int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out, int n_q,
@@ -291,27 +356,9 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
         return fail(SW_EALIGN, "Q, K_cur, V_cur and out must be 16-byte aligned");
     AttnParams p;
-    std::memset(&p, 0, sizeof p);
     int rc;
-    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
-    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
-    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
-    // maps for regions this handle does not have are never read; fill them with a valid map
-    p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
-    p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
-    p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
-    p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
-    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
-    p.out = out;
-    p.table = state + kStateHeaderInts;
-    p.status = state + 1;
-    p.B = c.B;
-    p.H = c.H;
-    p.n_q = n_q;
-    p.out_f32 = c.out_dtype == SW_OUT_F32;
-    p.scale_log2 = c.scale * 1.4426950408889634f;
+    if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, n_q))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
     if (n_q <= h->short_q) {
         const int bh = c.B * c.H;
         int splits = h->num_sms / bh;
@@ -319,37 +366,34 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         p.splits = splits;
         p.o_part = reinterpret_cast<float*>(h->ws + h->off_opart);
         p.ml_part = reinterpret_cast<float*>(h->ws + h->off_ml);
-        e = launch_attention(p, c.d, 1, splits, st);
+        cudaError_t e = launch_attention(p, c.d, 1, splits, st);
         if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
         e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
         if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-    } else if (resolve_schedule(h, n_q) == SW_SCHED_GRID) {
-        p.splits = 0;
-        const int grid_x = (n_q + 2 * kBlockM - 1) / (2 * kBlockM);
-        e = launch_attention(p, c.d, 2, grid_x, st);
-        if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    } else {
-        p.splits = 0;
-        p.sk_o = reinterpret_cast<float*>(h->ws + h->off_sk_o);
-        p.sk_ml = reinterpret_cast<float*>(h->ws + h->off_sk_ml);
-        p.sk_cnt = reinterpret_cast<int32_t*>(h->ws + h->off_sk_cnt);
-        p.sk_pairs = h->sk_pairs;
-        // one CTA per SM, but never so many that a CTA's share of the cost line is shorter than
-        // two items at the fewest key tiles a chunk can have (condition + current only)
-        const long long nqt = (n_q + kBlockM - 1) / kBlockM;
-        const long long nt_min = (c.n_cond + kBlockN - 1) / kBlockN + (c.tokens_per_chunk + kBlockN - 1) / kBlockN;
-        const long long c_min = (long long)c.B * c.H * nqt * nt_min;
-        long long ctas = std::min<long long>(h->num_sms, kMaxPersistentCtas);
-        ctas = std::max<long long>(1, std::min<long long>(ctas, c_min / 2));
-        if (resolve_schedule(h, n_q) == SW_SCHED_TRI) {
-            e = launch_tri(p, c.d, (int)ctas, st);
-            if (e != cudaSuccess) return cuda_fail(e, "three-buffer attention launch");
-            return SW_OK;
-        }
-        e = launch_persistent(p, c.d, (int)ctas, st);
-        if (e != cudaSuccess) return cuda_fail(e, "persistent attention launch");
+        return SW_OK;
     }
-    return SW_OK;
+    return launch_full(h, p, st);
+}
+
+int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const void* K_cur, const void* V_cur,
+                          void* out, void* out_cond, void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
+    const sw_attn_config& c = h->cfg;
+    if (c.n_cond < 1) return fail(SW_ESHAPE, "a joint forward needs n_cond >= 1 condition tokens");
+    if (!Q || !Q_cond || !K_cur || !V_cur || !out || !out_cond) return fail(SW_EINVAL, "null tensor");
+    if (!aligned16(Q) || !aligned16(Q_cond) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out) ||
+        !aligned16(out_cond))
+        return fail(SW_EALIGN, "Q, Q_cond, K_cur, V_cur, out and out_cond must be 16-byte aligned");
+    AttnParams p;
+    int rc;
+    if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, c.tokens_per_chunk))) return rc;
+    if ((rc = encode_user(&p.tm_qc, Q_cond, c.B, c.n_cond, c.H, c.d, "Q_cond"))) return rc;
+    p.out_c = out_cond;
+    p.n_qc = c.n_cond;
+    return launch_full(h, p, static_cast<cudaStream_t>(stream));
 }
 
 int sw_attn_get_table(const sw_attn_t* h, int32_t* dev_table, void* stream) {
@@ -440,24 +484,8 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
         scratch = g_noalloc_ptr[dev];
     }
     AttnParams p;
-    std::memset(&p, 0, sizeof p);
     int rc;
-    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
-    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
-    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
-    p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
-    p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
-    p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
-    p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
-    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
-    p.out = out;
-    p.table = state + kStateHeaderInts;
-    p.status = state + 1;
-    p.B = c.B;
-    p.H = c.H;
-    p.n_q = n_q;
-    p.out_f32 = c.out_dtype == SW_OUT_F32;
-    p.scale_log2 = c.scale * 1.4426950408889634f;
+    if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, n_q))) return rc;
     const int bh = c.B * c.H;
     long long splits = h->num_sms / bh;
     splits = std::max<long long>(1, std::min<long long>(splits, std::min<long long>((long long)fit, kMaxSplits)));

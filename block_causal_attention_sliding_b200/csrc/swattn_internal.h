@@ -34,12 +34,15 @@ struct alignas(64) AttnParams {
     CUtensorMap tm_cache_v;
     CUtensorMap tm_cond_k;   // K cond  [B][H][n_cond][d] dims {d, n_cond, H, B}
     CUtensorMap tm_cond_v;
+    CUtensorMap tm_qc;       // condition-stream queries [B, n_qc, H, d] (joint forward)
     void* out;               // [B, n_q, H, d] bf16 or f32 (full mode)
+    void* out_c;             // [B, n_qc, H, d] (joint forward)
     float* o_part;           // split mode: [splits][B*H][kBlockM][d] unnormalised fp32
     float* ml_part;          // split mode: [splits][B*H][kBlockM][2] (row max log2-scaled, row sum)
     const int32_t* table;    // device visibility table
     int32_t* status;         // device status word
     int B, H, n_q;
+    int n_qc;                // condition-stream query rows (0: none); their Q tiles follow the chunk's
     int out_f32;
     int splits;              // 0: full mode (normalised output); >= 1: split-K partials
     float scale_log2;        // softmax scale * log2(e)

@@ -8,15 +8,17 @@ bf16 inputs.  Recipe (stated once, used everywhere):
   * with ``outlier_p > 0`` every key row (b, token, h) is independently an outlier with that
     probability and is multiplied by 4 (an N(0, 16) draw), in K_cur, committed K and the
     condition K alike;
-  * tensor ids: Q = 0, K_cur = 1, V_cur = 2, condition K = 3, condition V = 4; condition
-    tensors use chunk 0, step 0.
+  * tensor ids: Q = 0, K_cur = 1, V_cur = 2, condition K = 3, condition V = 4, condition-stream
+    queries = 5; condition K/V use chunk 0, step 0 for the first prompt and chunk v, step 0 for
+    prompt version v (a prompt changed mid-stream); condition queries use the (chunk, step) of
+    the forward they belong to.
 The user layout is [B, N, H, d] contiguous.
 """
 from __future__ import annotations
 
 import torch
 
-TID_Q, TID_K, TID_V, TID_KC, TID_VC = 0, 1, 2, 3, 4
+TID_Q, TID_K, TID_V, TID_KC, TID_VC, TID_QC = 0, 1, 2, 3, 4, 5
 
 
 def stream_seed(seed: int, chunk: int, step: int, tensor_id: int) -> int:
@@ -50,9 +52,14 @@ def chunk_inputs(wl, chunk: int, step: int, *, seed: int = 0, n_q: int | None = 
     return Q, K, V
 
 
-def cond_inputs(wl, *, seed: int = 0, device="cpu"):
-    """Condition K, V [B, n_cond, H, d]."""
+def cond_inputs(wl, *, seed: int = 0, version: int = 0, device="cpu"):
+    """Condition K, V [B, n_cond, H, d] of prompt version `version` (0: the stream's first)."""
     shape = (wl.B, wl.n_cond, wl.H, wl.d)
-    Kc = draw(shape, stream_seed(seed, 0, 0, TID_KC), outlier_p=wl.outlier_p, device=device)
-    Vc = draw(shape, stream_seed(seed, 0, 0, TID_VC), device=device)
+    Kc = draw(shape, stream_seed(seed, version, 0, TID_KC), outlier_p=wl.outlier_p, device=device)
+    Vc = draw(shape, stream_seed(seed, version, 0, TID_VC), device=device)
     return Kc, Vc
+
+
+def cond_queries(wl, chunk: int, step: int, *, seed: int = 0, device="cpu"):
+    """Condition-stream queries Q_cond [B, n_cond, H, d] for one (chunk, step)."""
+    return draw((wl.B, wl.n_cond, wl.H, wl.d), stream_seed(seed, chunk, step, TID_QC), device=device)

@@ -144,6 +144,26 @@ SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const
                     void *out, int n_q, void *stream);
 
 /*
+ * Joint forward of the chunk's queries and the condition-stream queries, in one launch.
+ * In the MM-DiT the condition tokens form a stream of their own next to the video stream
+ * (neurohive review "JoyAI-Video-Edit", section "Архитектура JoyAI-Video-Edit": MM-DiT blocks
+ * with a condition stream and an image stream); their queries are read here as attending over
+ * the same keys as the active chunk's queries -- condition tokens, visible cached chunks and
+ * K_cur -- the plainest reading of one joint attention per chunk.
+ *   Q        [B, T, H, d] bf16   the chunk's queries (all T rows)
+ *   Q_cond   [B, n_cond, H, d]   the condition tokens' queries
+ *   K_cur, V_cur [B, T, H, d]    as in sw_attn_forward
+ *   out      [B, T, H, d], out_cond [B, n_cond, H, d]   (bf16 or fp32, per out_dtype)
+ * Both query sets run through the full path as one set of 128-row Q tiles (the chunk's first,
+ * then the condition queries'), so the launch stays full even where n_cond alone would not
+ * fill the GPU.  Needs n_cond >= 1 and the condition set (SW_ESHAPE / SW_ESTATE otherwise).
+ * A prompt change (tutorial, section "范式重塑：视频交互从“渲染等待”迈向“即拍即得”": prompts
+ * adjusted while streaming) is sw_attn_set_cond between chunks; the cached history is kept.
+ */
+SW_API int sw_attn_forward_joint(sw_attn_t *h, const void *Q, const void *Q_cond, const void *K_cur,
+                                 const void *V_cur, void *out, void *out_cond, void *stream);
+
+/*
  * Short-query forward that allocates nothing and uses no workspace scratch.
  *
  * Same result as sw_attn_forward for 1 <= n_q <= 128 (the split-K path), but its split-K

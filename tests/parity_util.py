@@ -91,3 +91,52 @@ def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, 
     torch.cuda.synchronize()
     assert h.status() == 0, f"device status {h.status():#x}"
     return results
+
+
+def stream_and_check_joint(wl, dev, *, chunks, check_at=None, n_rows=None, prompts=None,
+                           out_dtype=torch.float32, seed=0, schedule="auto", gen_on_device=False,
+                           keep_last=None, tol=(MAX_ABS, MEAN_REL)):
+    """Stream `chunks` chunks through the joint forward (the chunk's queries and the condition
+    queries in one launch; 2 steps, then an append each).  `prompts` maps a chunk index to a
+    prompt version: before that chunk the condition K/V are replaced (set_cond), and the oracle
+    uses the new ones from there on.  At the chunks in `check_at` (all if None) both outputs
+    are compared with the oracle, on all rows or on `n_rows` sampled rows of each.
+    Returns a list of (k, step, which, max_abs, mean_rel)."""
+    h = make_handle(wl, dev, out_dtype=out_dtype, schedule=schedule)
+    gdev = dev if gen_on_device else "cpu"
+    prompts = dict(prompts or {})
+    Kc, Vc = synth.cond_inputs(wl, seed=seed, device=gdev)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    Kc, Vc = Kc.cpu(), Vc.cpu()
+    hist_K, hist_V = [], []
+    results = []
+    for k in range(chunks):
+        if k in prompts:
+            Kc, Vc = synth.cond_inputs(wl, seed=seed, version=prompts[k], device=gdev)
+            h.set_cond(Kc.to(dev), Vc.to(dev))
+            Kc, Vc = Kc.cpu(), Vc.cpu()
+        for step in range(wl.steps):
+            Q, K, V = synth.chunk_inputs(wl, k, step, seed=seed, device=gdev)
+            Qc = synth.cond_queries(wl, k, step, seed=seed, device=gdev)
+            out, out_c = h.forward_joint(Q.to(dev), Qc.to(dev), K.to(dev), V.to(dev))
+            if check_at is None or k in check_at:
+                for which, q, o, n in (("chunk", Q, out, wl.T), ("cond", Qc, out_c, wl.n_cond)):
+                    r = None if n_rows is None else sample_rows(n, n_rows, seed=1000 * k + step)
+                    ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
+                                           k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V, Q=q.cpu(),
+                                           K_cur=K.cpu(), V_cur=V.cpu(), rows=r)
+                    got = o.float().cpu().numpy()
+                    if r is not None:
+                        got = got[:, r]
+                    ma, mr = compare(got, ref, *tol)
+                    results.append((k, step, which, ma, mr))
+        h.append_chunk(K.to(dev), V.to(dev))
+        hist_K.append(K.cpu())
+        hist_V.append(V.cpu())
+        if keep_last is not None:
+            for c in range(1, max(1, len(hist_K) - keep_last)):
+                hist_K[c] = None
+                hist_V[c] = None
+    torch.cuda.synchronize()
+    assert h.status() == 0, f"device status {h.status():#x}"
+    return results

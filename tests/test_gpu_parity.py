@@ -17,7 +17,7 @@ import oracle
 from block_causal_attention_sliding_b200 import synth
 from block_causal_attention_sliding_b200.configs import WORKLOADS, Workload
 
-from parity_util import compare, make_handle, stream_and_check
+from parity_util import compare, make_handle, stream_and_check, stream_and_check_joint
 
 pytestmark = pytest.mark.gpu
 
@@ -227,6 +227,47 @@ def test_short_queries_720p(dev, n_q):
     """Split-K path: n_q queries against the steady-state 720p cache."""
     wl = WORKLOADS["720p"]
     stream_and_check(wl, dev, chunks=6, check_at={0, 5}, n_q=n_q, keep_last=wl.W + 1, gen_on_device=True)
+
+
+# ------------------------------------------------------------------ condition-stream queries
+
+@pytest.mark.parametrize("schedule", ["auto", "persistent", "grid", "tri"])
+def test_joint_tiny_stream(dev, schedule):
+    """The tiny workload through the joint forward: the 16 chunk queries and the 8 condition
+    queries share one launch; every chunk and step, all rows of both outputs."""
+    wl = WORKLOADS["tiny"]
+    res = stream_and_check_joint(wl, dev, chunks=wl.chunks, schedule=schedule)
+    assert len(res) == 2 * wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("d,T,n_cond", [(128, 300, 40), (128, 256, 130), (64, 300, 200), (128, 129, 1)])
+def test_joint_ragged(dev, d, T, n_cond, schedule):
+    """Ragged tails in both query sets: the chunk's last Q tile and a condition tile share a
+    pair (T = 300, n_cond = 40: 3 + 1 tiles), two condition tiles form a pair (n_cond = 130),
+    an odd tile total (T = 300, n_cond = 200 at d = 64: 3 + 2 tiles), one condition query."""
+    wl = dataclasses.replace(RAGGED, d=d, T=T, n_cond=n_cond, chunks=4)
+    res = stream_and_check_joint(wl, dev, chunks=wl.chunks, schedule=schedule)
+    assert len(res) == 2 * wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+def test_prompt_change_mid_stream(dev, schedule):
+    """Prompt edits while streaming: the condition K/V are replaced before chunks 2 and 4;
+    both outputs follow the new condition from that chunk on, and the cached history (sink
+    and window) is unaffected."""
+    wl = dataclasses.replace(RAGGED, chunks=6)
+    res = stream_and_check_joint(wl, dev, chunks=wl.chunks, prompts={2: 1, 4: 2}, schedule=schedule)
+    assert len(res) == 2 * wl.chunks * wl.steps
+
+
+def test_joint_720p_sampled(dev):
+    """720p: 3180 chunk queries and 256 condition queries in one launch, sampled rows at
+    chunks 0 and W + 1, with a prompt change before chunk W + 1."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_joint(wl, dev, chunks=5, check_at={0, 4}, n_rows=40, prompts={4: 1},
+                                 keep_last=wl.W + 1, gen_on_device=True)
+    assert len(res) == 8
 
 
 def test_long_horizon_constant_memory(dev):
