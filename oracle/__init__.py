@@ -54,6 +54,14 @@ def _load():
     lib.swo_slot.restype = i32
     lib.swo_table.argtypes = [i32, i32, i32, i32, i32, vp, i32]
     lib.swo_table.restype = i32
+    lib.swo_num_slots_r.argtypes = [i32, i32]
+    lib.swo_num_slots_r.restype = i32
+    lib.swo_slot_r.argtypes = [i32, i32, i32]
+    lib.swo_slot_r.restype = i32
+    lib.swo_table_r.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
+    lib.swo_table_r.restype = i32
+    lib.swo_ring_create_r.argtypes = [i32] * 8 + [vp, vp]
+    lib.swo_ring_create_r.restype = vp
     lib.swo_attention.argtypes = [i32] * 8 + [vp, vp, vp, vp, vp, i32, vp, vp, dbl, vp, i32, vp]
     lib.swo_attention.restype = i32
     lib.swo_ring_create.argtypes = [i32] * 7 + [vp, vp]
@@ -92,19 +100,21 @@ def visible(k: int, W: int, sink: bool, j: int) -> bool:
     return bool(_load().swo_visible(k, W, int(sink), j))
 
 
-def num_slots(W: int, sink: bool) -> int:
-    return int(_load().swo_num_slots(W, int(sink)))
+def num_slots(W: int, sink: bool, R: int | None = None) -> int:
+    """Ring slots; R window slots (default W; W + 1 keeps a spare slot)."""
+    return int(_load().swo_num_slots_r(W if R is None else R, int(sink)))
 
 
-def slot(c: int, W: int, sink: bool) -> int:
-    return int(_load().swo_slot(c, W, int(sink)))
+def slot(c: int, W: int, sink: bool, R: int | None = None) -> int:
+    return int(_load().swo_slot_r(c, W if R is None else R, int(sink)))
 
 
-def table(k: int, W: int, sink: bool, n_cond: int, T: int) -> np.ndarray:
-    """Canonical visibility table: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...]."""
+def table(k: int, W: int, sink: bool, n_cond: int, T: int, R: int | None = None) -> np.ndarray:
+    """Canonical visibility table: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...];
+    slots of a ring with R window slots (default W)."""
     cap = 3 + 4 * (k + 3)
     out = np.zeros(cap, dtype=np.int32)
-    n = _load().swo_table(k, W, int(sink), n_cond, T, out.ctypes.data, cap)
+    n = _load().swo_table_r(k, W, W if R is None else R, int(sink), n_cond, T, out.ctypes.data, cap)
     if n < 0:
         raise RuntimeError("swo_table: capacity")
     return out[:n].copy()
@@ -154,16 +164,18 @@ def attention(*, H: int, d: int, T: int, n_cond: int, W: int, sink: bool, k: int
 class Ring:
     """The ring-buffer statement of the same attention (bounded cache with pinned sink)."""
 
-    def __init__(self, *, B: int, H: int, d: int, T: int, n_cond: int, W: int, sink: bool, Kc, Vc):
+    def __init__(self, *, B: int, H: int, d: int, T: int, n_cond: int, W: int, sink: bool, Kc, Vc,
+                 R: int | None = None):
         assert d <= 512
         self._lib = _load()
         self.B, self.H, self.d, self.T = B, H, d, T
+        R = W if R is None else R
         self._Kc, self._Vc = (_f32(Kc), _f32(Vc)) if n_cond > 0 else (None, None)
-        self._h = self._lib.swo_ring_create(B, H, d, T, n_cond, W, int(sink),
-                                            _ptr(self._Kc), _ptr(self._Vc))
+        self._h = self._lib.swo_ring_create_r(B, H, d, T, n_cond, W, R, int(sink),
+                                              _ptr(self._Kc), _ptr(self._Vc))
         if not self._h:
             raise MemoryError("swo_ring_create")
-        self.S = num_slots(W, sink)
+        self.S = num_slots(W, sink, R)
 
     def append(self, K, V) -> None:
         Kf, Vf = _f32(K), _f32(V)

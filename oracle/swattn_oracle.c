@@ -33,6 +33,10 @@
  *   - masked keys are skipped (never multiplied by zero), so NaN in them cannot leak.
  *   - ring slots: with the sink, slot(0)=0 and slot(c)=1+((c-1) mod W); without it
  *     slot(c)=c mod W.  W=0 keeps no window chunk.
+ *   - a ring may keep R = W + 1 window slots instead of W (the *_r functions): one slot then
+ *     holds the chunk that has just left the window, so the chunk being produced can be
+ *     written while its own forward still reads every visible chunk.  Which keys are visible
+ *     does not change, only where they are kept.
  *
  * Inputs are float32 arrays holding bf16-rounded values (exact in float32); all arithmetic
  * is in double.  Layouts are the user layout [B][N][H][d], row-major.
@@ -59,23 +63,35 @@ int swo_visible(int k, int W, int sink, int j)
     return 0;
 }
 
-/* Number of ring slots for the bounded cache. */
-int swo_num_slots(int W, int sink)
+/* Number of ring slots for the bounded cache with R window slots. */
+int swo_num_slots_r(int R, int sink)
 {
-    return W + (sink ? 1 : 0);
+    return R + (sink ? 1 : 0);
 }
 
-/* Ring slot holding committed chunk c; -1 if the chunk is never stored (W=0 cases). */
-int swo_slot(int c, int W, int sink)
+int swo_num_slots(int W, int sink)
+{
+    return swo_num_slots_r(W, sink);
+}
+
+/* Ring slot holding committed chunk c with R window slots; -1 if the chunk is never stored
+ * (R = 0: no window chunk is kept).  Window chunks rotate through the R slots, so chunk c
+ * takes the slot of chunk c - R. */
+int swo_slot_r(int c, int R, int sink)
 {
     if (c < 0) return -1;
     if (sink) {
         if (c == 0) return 0;
-        if (W == 0) return -1;
-        return 1 + (c - 1) % W;
+        if (R == 0) return -1;
+        return 1 + (c - 1) % R;
     }
-    if (W == 0) return -1;
-    return c % W;
+    if (R == 0) return -1;
+    return c % R;
+}
+
+int swo_slot(int c, int W, int sink)
+{
+    return swo_slot_r(c, W, sink);
 }
 
 /*
@@ -86,7 +102,7 @@ int swo_slot(int c, int W, int sink)
  * For kind 0 chunk_id = slot = -1; for kind 2 chunk_id = k and slot = -1.
  * Returns the number of ints written, or -1 if cap is too small.
  */
-int swo_table(int k, int W, int sink, int n_cond, int T, int32_t *out, int cap)
+int swo_table_r(int k, int W, int R, int sink, int n_cond, int T, int32_t *out, int cap)
 {
     int nseg = 0, nvis = 0, pos = 3, j;
     if (cap < 3) return -1;
@@ -98,7 +114,7 @@ int swo_table(int k, int W, int sink, int n_cond, int T, int32_t *out, int cap)
     for (j = 0; j < k; j++) {
         if (!swo_visible(k, W, sink, j)) continue;
         if (pos + 4 > cap) return -1;
-        out[pos++] = 1; out[pos++] = j; out[pos++] = swo_slot(j, W, sink); out[pos++] = T;
+        out[pos++] = 1; out[pos++] = j; out[pos++] = swo_slot_r(j, R, sink); out[pos++] = T;
         nseg++; nvis += T;
     }
     if (pos + 4 > cap) return -1;
@@ -106,6 +122,11 @@ int swo_table(int k, int W, int sink, int n_cond, int T, int32_t *out, int cap)
     nseg++; nvis += T;
     out[0] = k; out[1] = nseg; out[2] = nvis;
     return pos;
+}
+
+int swo_table(int k, int W, int sink, int n_cond, int T, int32_t *out, int cap)
+{
+    return swo_table_r(k, W, W, sink, n_cond, T, out, cap);
 }
 
 /* ---------------------------------------------------------------- dense oracle */
@@ -232,19 +253,20 @@ int swo_attention(int B, int H, int d, int T, int n_cond, int W, int sink, int k
  * streaming through the ring equals recomputation from the full history.
  */
 typedef struct {
-    int B, H, d, T, n_cond, W, sink, S, n_committed;
+    int B, H, d, T, n_cond, W, R, sink, S, n_committed;
     int *slot_chunk;     /* chunk id held by each slot, -1 if empty */
     float *K, *V;        /* [S][B][T][H][d] */
     float *Kc, *Vc;      /* [B][n_cond][H][d] */
 } swo_ring;
 
-void *swo_ring_create(int B, int H, int d, int T, int n_cond, int W, int sink,
-                      const float *Kc, const float *Vc)
+/* R window slots (R = W: the plain ring; R = W + 1: one spare slot). */
+void *swo_ring_create_r(int B, int H, int d, int T, int n_cond, int W, int R, int sink,
+                        const float *Kc, const float *Vc)
 {
     swo_ring *r = (swo_ring *)calloc(1, sizeof(swo_ring));
     if (!r) return NULL;
-    r->B = B; r->H = H; r->d = d; r->T = T; r->n_cond = n_cond; r->W = W; r->sink = sink;
-    r->S = W + (sink ? 1 : 0);
+    r->B = B; r->H = H; r->d = d; r->T = T; r->n_cond = n_cond; r->W = W; r->R = R; r->sink = sink;
+    r->S = R + (sink ? 1 : 0);
     const size_t chunk = (size_t)B * T * H * d;
     const size_t cond = (size_t)B * n_cond * H * d;
     r->slot_chunk = (int *)malloc(sizeof(int) * (size_t)(r->S > 0 ? r->S : 1));
@@ -261,6 +283,12 @@ void *swo_ring_create(int B, int H, int d, int T, int n_cond, int W, int sink,
     return r;
 }
 
+void *swo_ring_create(int B, int H, int d, int T, int n_cond, int W, int sink,
+                      const float *Kc, const float *Vc)
+{
+    return swo_ring_create_r(B, H, d, T, n_cond, W, W, sink, Kc, Vc);
+}
+
 void swo_ring_destroy(void *h)
 {
     swo_ring *r = (swo_ring *)h;
@@ -269,7 +297,8 @@ void swo_ring_destroy(void *h)
 }
 
 /* Commit the finished chunk: the sink slot is written once; later chunks overwrite the
- * oldest window chunk (the slot is freed by the chunk that leaves the window). */
+ * oldest window chunk, c - R (with R = W that is the chunk leaving the window now; with a
+ * spare slot, the one that left it a chunk ago), or take an empty slot. */
 void swo_ring_append(void *h, const float *K, const float *V)
 {
     swo_ring *r = (swo_ring *)h;
@@ -277,11 +306,11 @@ void swo_ring_append(void *h, const float *K, const float *V)
     int s = -1;
     if (r->sink && c == 0) {
         s = 0;
-    } else if (r->W > 0) {
-        /* choose the slot whose chunk leaves the window, else the first empty slot */
+    } else if (r->R > 0 && r->W > 0) {
+        /* choose the slot of the oldest window chunk, else the first empty slot */
         const int base = r->sink ? 1 : 0;
         for (int q = base; q < r->S; q++)
-            if (r->slot_chunk[q] >= 0 && r->slot_chunk[q] == c - r->W) { s = q; break; }
+            if (r->slot_chunk[q] >= 0 && r->slot_chunk[q] == c - r->R) { s = q; break; }
         if (s < 0)
             for (int q = base; q < r->S; q++)
                 if (r->slot_chunk[q] < 0) { s = q; break; }
@@ -297,7 +326,9 @@ void swo_ring_append(void *h, const float *K, const float *V)
 
 int swo_ring_slot_chunk(void *h, int s) { return ((swo_ring *)h)->slot_chunk[s]; }
 
-/* Attention of the active chunk over [cond ; occupied slots ; current]; all rows. */
+/* Attention of the active chunk over [cond ; occupied slots holding a window or sink chunk ;
+ * current]; all rows.  (With a spare slot, one occupied slot holds the chunk that has already
+ * left the window: it is skipped.) */
 int swo_ring_forward(void *h, const float *Q, int n_q, const float *Kcur, const float *Vcur,
                      double scale, double *out)
 {
@@ -322,7 +353,9 @@ int swo_ring_forward(void *h, const float *Q, int n_q, const float *Kcur, const 
                 int nrows, rstride_n;
                 if (part == 0) { Kb = r->Kc; Vb = r->Vc; nrows = nc; rstride_n = nc; }
                 else if (part == 1) {
-                    if (r->slot_chunk[s] < 0) continue;
+                    const int held = r->slot_chunk[s];
+                    if (held < 0) continue;
+                    if (held < r->n_committed - r->W && !(r->sink && held == 0)) continue;
                     Kb = r->K + (size_t)s * chunk; Vb = r->V + (size_t)s * chunk;
                     nrows = T; rstride_n = T;
                 } else { Kb = Kcur; Vb = Vcur; nrows = T; rstride_n = T; }

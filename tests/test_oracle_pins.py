@@ -73,6 +73,31 @@ def brute_slots(n_commits, W, sink):
     return where
 
 
+def brute_slots_spare(n_commits, W, sink):
+    """Physical slots of a ring that keeps one spare window slot (W + 1 in all, none for
+    W = 0), written while the chunk's own forward still reads its history: chunk c takes the
+    lowest window slot whose chunk is not visible to chunk c, or an empty one."""
+    R = W + 1 if W > 0 else 0
+    base = 1 if sink else 0
+    holder = [None] * (base + R)
+    where = {}
+    for c in range(n_commits):
+        if sink and c == 0:
+            holder[0] = 0
+            where[c] = 0
+            continue
+        if R == 0:
+            where[c] = -1
+            continue
+        vis = set(brute_visible(c, W, sink))
+        for s_ in range(base, base + R):
+            if holder[s_] is None or holder[s_] not in vis:
+                holder[s_] = c
+                where[c] = s_
+                break
+    return where
+
+
 def brute_attention(Kc, Vc, hist_K, hist_V, Q, Kcur, Vcur, W, sink, scale):
     B, n_q, H, d = Q.shape
     k = len(hist_K)
@@ -174,6 +199,28 @@ def test_tables_brute_force(oracle_mod, W, sink):
         sl = [where[j] for j in vis]
         assert all(0 <= s < oracle_mod.num_slots(W, sink) for s in sl)
         assert len(set(sl)) == len(sl)
+
+
+@pytest.mark.parametrize("sink", [True, False])
+@pytest.mark.parametrize("W", [0, 1, 2, 3, 5, 6])
+def test_tables_spare_slot(oracle_mod, W, sink):
+    """A ring with one spare window slot: the same visible chunks, other slots.  The slot
+    chunk k is committed into is never one that chunk k's own forward reads."""
+    R = W + 1 if W > 0 else 0
+    where = brute_slots_spare(40, W, sink)
+    for k in range(40):
+        vis = brute_visible(k, W, sink)
+        plain = oracle_mod.table(k, W, sink, n_cond=3, T=11)
+        tab = oracle_mod.table(k, W, sink, n_cond=3, T=11, R=R)
+        segs, psegs = tab[3:].reshape(-1, 4), plain[3:].reshape(-1, 4)
+        assert tab[:3].tolist() == plain[:3].tolist()
+        assert segs[:, [0, 1, 3]].tolist() == psegs[:, [0, 1, 3]].tolist()   # only slots differ
+        assert list(segs[1:-1, 2]) == [where[j] for j in vis]
+        sl = [where[j] for j in vis]
+        assert all(0 <= x < oracle_mod.num_slots(W, sink, R) for x in sl) and len(set(sl)) == len(sl)
+        own = oracle_mod.slot(k, W, sink, R)
+        assert own == where[k]
+        assert own not in sl or own < 0                                     # never read while written
 
 
 def test_ring_holds_exactly_hist(oracle_mod):
@@ -368,6 +415,28 @@ def test_streaming_equals_recompute(oracle_mod, B, H, d, T, n_cond, W, sink, n_c
                                      hist_V=[x if c in keep else None for c, x in enumerate(hv)],
                                      Q=Q, K_cur=Kn, V_cur=Vn)
             np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+        ring.append(Kn, Vn)
+        hk.append(Kn); hv.append(Vn)
+
+
+@pytest.mark.parametrize("W,sink", [(1, True), (2, False), (3, True), (0, True)])
+def test_spare_slot_ring_streaming_equals_recompute(oracle_mod, W, sink):
+    """The ring with a spare window slot holds one chunk that has left the window; its forward
+    skips it and equals the dense mask over the full history, every chunk."""
+    B, H, d, T, n_cond, n_chunks = 1, 2, 8, 5, 3, 10
+    R = W + 1 if W > 0 else 0
+    Kc, Vc, _, _, _ = _stream(B, H, d, T, n_cond, 0, seed=23)
+    ring = oracle_mod.Ring(B=B, H=H, d=d, T=T, n_cond=n_cond, W=W, sink=sink, Kc=Kc, Vc=Vc, R=R)
+    hk, hv = [], []
+    for k in range(n_chunks):
+        held = sorted(c for c in ring.slot_chunks() if c >= 0)
+        vis = brute_visible(k, W, sink)
+        assert set(vis) <= set(held) and len(held) <= len(vis) + 1
+        Q, Kn, Vn = _rand((B, T, H, d), 7 * k + 1), _rand((B, T, H, d), 7 * k + 2), _rand((B, T, H, d), 7 * k + 3)
+        a = ring.forward(Q, Kn, Vn)
+        b = oracle_mod.attention(H=H, d=d, T=T, n_cond=n_cond, W=W, sink=sink, k=k, Kc=Kc, Vc=Vc,
+                                 hist_K=hk, hist_V=hv, Q=Q, K_cur=Kn, V_cur=Vn)
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
         ring.append(Kn, Vn)
         hk.append(Kn); hv.append(Vn)
 
