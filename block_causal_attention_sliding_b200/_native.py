@@ -19,6 +19,7 @@ SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
 EXPORTS = (
     "sw_attn_create", "sw_attn_create_ex", "sw_attn_workspace_bytes", "sw_attn_bind_workspace",
     "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_forward_joint",
+    "sw_attn_forward_commit",
     "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
@@ -30,7 +31,7 @@ class SwAttnConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("tokens_per_chunk", ctypes.c_int), ("W", ctypes.c_int), ("n_cond", ctypes.c_int),
                 ("sink", ctypes.c_int), ("out_dtype", ctypes.c_int), ("scale", ctypes.c_float),
-                ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int)]
+                ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int), ("commit_in_forward", ctypes.c_int)]
 
 
 class SwAttnError(RuntimeError):
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_forward.restype = i32
     L.sw_attn_forward_joint.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
     L.sw_attn_forward_joint.restype = i32
+    L.sw_attn_forward_commit.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.sw_attn_forward_commit.restype = i32
     L.sw_attn_forward_short_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward_short_noalloc.restype = i32
     L.sw_attn_selftest_timeout.argtypes = [vp, ctypes.c_int64, vp]

@@ -33,20 +33,24 @@ class SlidingWindowAttention:
 
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
-                 max_short_q: int = 0, schedule: str = "auto", device=None):
+                 max_short_q: int = 0, schedule: str = "auto", commit_in_forward: bool = False,
+                 device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
                              out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
                              scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
                              schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
-                                       "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule])
+                                       "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule],
+                             commit_in_forward=int(bool(commit_in_forward)))
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()
         N.check(self._lib.sw_attn_create_ex(ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
         self.B, self.H, self.d, self.T, self.W, self.n_cond, self.sink = B, H, d, T, W, n_cond, bool(sink)
+        # window slots of the ring: W, or W + 1 (a spare slot) with commit_in_forward
+        self.R = W + 1 if (commit_in_forward and W > 0) else W
         self.out_dtype = out_dtype
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         nbytes = int(self._lib.sw_attn_workspace_bytes(h))
@@ -100,6 +104,24 @@ class SlidingWindowAttention:
 
     __call__ = forward
 
+    def forward_commit(self, Q: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
+                       out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """The chunk's clean pass: forward of all T queries that also commits K_cur / V_cur to the
+        cache (sw_attn_forward_commit; the handle needs commit_in_forward)."""
+        shape = (self.B, self.T, self.H, self.d)
+        for name, t in (("Q", Q), ("K_cur", K_cur), ("V_cur", V_cur)):
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty(shape, dtype=self.out_dtype, device=Q.device)
+        elif tuple(out.shape) != shape or out.dtype != self.out_dtype:
+            raise ValueError("out must be [B, T, H, d] in the handle's out_dtype")
+        N.check(self._lib.sw_attn_forward_commit(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
+                                                 _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+                                                 _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                                 _dev_ptr(out, "out"), _stream_ptr(stream)))
+        return out
+
     def forward_joint(self, Q: torch.Tensor, Q_cond: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
                       out: torch.Tensor | None = None, out_cond: torch.Tensor | None = None,
                       stream=None) -> tuple[torch.Tensor, torch.Tensor]:
@@ -145,7 +167,7 @@ class SlidingWindowAttention:
 
     def cache_views(self):
         """(K_cache, V_cache) as [B, H, S, T, d] bf16 views of the workspace (for inspection)."""
-        S = self.W + (1 if self.sink else 0)
+        S = self.R + (1 if self.sink else 0)
         ko, vo = ctypes.c_size_t(0), ctypes.c_size_t(0)
         N.check(self._lib.sw_attn_cache_offsets(self._h, ctypes.byref(ko), ctypes.byref(vo)))
         n = 2 * self.B * self.H * S * self.T * self.d

@@ -127,6 +127,13 @@ __device__ __forceinline__ void load_table(SmemCtl* ctl, const int32_t* table, i
     }
 }
 
+// Segment of key tile j.
+__device__ __forceinline__ int tile_seg(const SmemCtl* ctl, int j) {
+    int s = 0;
+    while (s + 1 < ctl->n_seg && ctl->seg_tile0[s + 1] <= j) ++s;
+    return s;
+}
+
 // Which segment key tile j belongs to, its first key row, and how many of its rows are keys.
 __device__ __forceinline__ void tile_of(const SmemCtl* ctl, int j, int& seg, int& row0, int& valid) {
     int s = 0;
@@ -176,6 +183,57 @@ __device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl*
             tma_load_4d(d, kv ? &p.tm_vcur : &p.tm_kcur, bar, c * kBoxCols, h, row0, b);
     }
 }
+
+// Fused commit: the producer stores the active chunk's K_cur / V_cur tiles, which it has just
+// loaded into the K/V ring for the attention, from shared memory to the chunk's ring slot in
+// the cache.  A tile's store is issued kStages - 1 ring items after its load (by then the load
+// has landed, and the stage cannot have been refilled), and a stage is refilled only after
+// every issued store has finished reading shared memory.  The producer flushes the queue and
+// waits for the stores to complete before it finishes.
+template <int D, int kStages>
+struct CommitQueue {
+    static constexpr int kCap = 8;
+    int n = 0, head = 0;
+    uint32_t pending = 0;   // stages with a store that may still be reading them
+    uint32_t item[kCap];
+    int j[kCap], kv[kCap], h[kCap], b[kCap];
+
+    __device__ __forceinline__ void push(uint32_t it, int j_, int kv_, int h_, int b_) {
+        const int t = (head + n) % kCap;
+        item[t] = it; j[t] = j_; kv[t] = kv_; h[t] = h_; b[t] = b_;
+        ++n;
+    }
+    // Before stage s takes a new load: its last store (if any) must have read it.
+    __device__ __forceinline__ void before_refill(int s) {
+        if ((pending >> s) & 1u) {
+            bulk_wait_read_all();
+            pending = 0;
+        }
+    }
+    // Issue the stores of queued tiles loaded at least kStages - 1 items before item it_now
+    // (every queued tile with force).  Returns false if a wait gave up.
+    __device__ __forceinline__ bool issue(const AttnParams& p, const SmemCtl* ctl, const uint8_t* kv_smem,
+                                          int slot, uint32_t it_now, bool force, volatile int* abort_flag) {
+        while (n > 0 && (force || it_now - item[head] >= (uint32_t)(kStages - 1))) {
+            const uint32_t i = item[head];
+            const int s = (int)(i % kStages);
+            if (!wait_or_abort(smem_u32(&ctl->kv_full[s]), (i / kStages) & 1, abort_flag)) return false;
+            int seg, row0, valid;
+            tile_of(ctl, j[head], seg, row0, valid);
+            fence_proxy_async_smem();
+            const uint32_t src = smem_u32(kv_smem + (size_t)s * TileCfg<D>::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
+                tma_store_5d(kv[head] ? &p.tm_cache_v : &p.tm_cache_k, src + c * kBoxBytes, c * kBoxCols, row0,
+                             slot, h[head], b[head]);
+            bulk_commit_group();
+            pending |= 1u << s;
+            head = (head + 1) % kCap;
+            --n;
+        }
+        return true;
+    }
+};
 
 // S[tS] = Q(q_tile) K(k_tile)^T: M = 128 queries, N = 128 keys, K = D, bf16 -> fp32.
 template <int D>

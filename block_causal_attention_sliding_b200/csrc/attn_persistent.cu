@@ -76,6 +76,9 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             uint32_t it = 0;
             int pi = 0;
             bool ok = true;
+            // fused commit: the pieces of Q-tile pair 0 store the chunk's K_cur / V_cur tiles
+            const int cslot = p.commit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
+            CommitQueue<D, kStages> cq;
             while (ok && next_piece(sched, pit, pc)) {
                 const int b = pc.bh / p.H, h = pc.bh % p.H;
                 // the Q buffers are reused: wait until every S MMA of the previous piece is done
@@ -96,12 +99,20 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                             ok = false;
                             break;
                         }
+                        cq.before_refill(s);
                         const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
                         mbar_arrive_expect_tx(fbar, kTileBytes);
                         load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                        if (cslot >= 0 && pc.pair == 0 && ctl->seg_kind[tile_seg(ctl, j)] == 2) cq.push(it, j, kv, h, b);
+                        if (cq.n > 0 && !cq.issue(p, ctl, kv_smem, cslot, it, false, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                     }
                 }
             }
+            if (cq.n > 0 && ok) (void)cq.issue(p, ctl, kv_smem, cslot, it, true, abort_flag);
+            bulk_wait_all();
             for (int s = 0; s < kStages; ++s) {
                 if (it > (uint32_t)s) {
                     const uint32_t uses = (it - 1 - s) / kStages + 1;

@@ -10,20 +10,11 @@
 
 namespace swattn {
 
-// Ring slot of committed chunk c: the sink owns slot 0; window chunks rotate through the
-// remaining W slots, so chunk c lands where chunk c - W (the one leaving the window) was.
-__device__ __forceinline__ int ring_slot(int c, int W, int sink) {
-    if (sink) {
-        if (c == 0) return 0;
-        return W > 0 ? 1 + (c - 1) % W : -1;
-    }
-    return W > 0 ? c % W : -1;
-}
-
 // K1: advance the counter (after an append) and write the visibility table of the active
 // chunk k: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...], in the order
-// condition, sink, window ascending, current.  One thread: a few dozen integers.
-__global__ void table_build_kernel(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+// condition, sink, window ascending, current; slots of a ring with R window slots.  One
+// thread: a few dozen integers.
+__global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
                                    int reset) {
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
     int32_t* tab = state + kStateHeaderInts;
@@ -49,15 +40,15 @@ __global__ void table_build_kernel(int32_t* state, int W, int sink, int n_cond, 
     if (n_cond > 0) put(0, -1, -1, n_cond);
     const int first_win = k - W > 0 ? k - W : 0;
     if (sink && k >= 1 && first_win > 0) put(1, 0, 0, T);      // sink outside the window
-    for (int j = first_win; j < k; ++j) put(1, j, ring_slot(j, W, sink), T);
+    for (int j = first_win; j < k; ++j) put(1, j, ring_slot(j, R, sink), T);
     put(2, k, -1, T);
     tab[0] = k; tab[1] = nseg; tab[2] = nvis;
     for (int i = pos; i < cap; ++i) tab[i] = -1;
 }
 
-cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+cudaError_t launch_table_build(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
                                cudaStream_t stream) {
-    table_build_kernel<<<1, 32, 0, stream>>>(state, W, sink, n_cond, T, advance, 0);
+    table_build_kernel<<<1, 32, 0, stream>>>(state, W, R, sink, n_cond, T, advance, 0);
     return cudaGetLastError();
 }
 
@@ -66,9 +57,9 @@ __global__ void zero_kernel(int32_t* p, long long n) {
         p[i] = 0;
 }
 
-cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
+cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_cond, int T,
                                int32_t* counters, long long n_counters, cudaStream_t stream) {
-    table_build_kernel<<<1, 32, 0, stream>>>(state, W, sink, n_cond, T, 0, 1);
+    table_build_kernel<<<1, 32, 0, stream>>>(state, W, R, sink, n_cond, T, 0, 1);
     if (n_counters > 0) {
         const long long blocks = (n_counters + 255) / 256;
         zero_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(counters, n_counters);
@@ -89,10 +80,10 @@ __global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__
                                                        uint4* __restrict__ dstK,
                                                        uint4* __restrict__ dstV, int N, int H,
                                                        int vpr_log2, int rows_per_bh, int ring,
-                                                       int W, int sink, int S, int32_t* state) {
+                                                       int R, int sink, int S, int32_t* state) {
     int slot = 0;
     if (ring) {
-        slot = ring_slot(state[0], W, sink);
+        slot = ring_slot(state[0], R, sink);
         if (slot < 0) return;                 // W = 0: nothing is kept for this chunk
         if (slot >= S) {                      // cannot happen; recorded, never trapped
             if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
@@ -115,7 +106,7 @@ __global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__
 }
 
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
-                            int H, int d, int rows_per_bh, int ring, int W, int sink, int S,
+                            int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
                             int32_t* state, cudaStream_t stream) {
     const int vpr = d / 8;                          // 16-byte vectors per head row
     int vpr_log2 = 0;
@@ -129,7 +120,7 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
     dim3 grid((unsigned)rows, 2);
     relayout_kernel<<<grid, threads, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
-        static_cast<uint4*>(dstV), N, H, vpr_log2, rows_per_bh, ring, W, sink, S, state);
+        static_cast<uint4*>(dstV), N, H, vpr_log2, rows_per_bh, ring, R, sink, S, state);
     return cudaGetLastError();
 }
 

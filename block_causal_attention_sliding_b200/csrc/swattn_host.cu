@@ -26,6 +26,7 @@ struct sw_attn {
     size_t off_kcache = 0, off_vcache = 0, off_kcond = 0, off_vcond = 0, off_opart = 0, off_ml = 0;
     size_t off_sk_o = 0, off_sk_ml = 0, off_sk_cnt = 0;
     int sk_pairs = 0;
+    int R = 0;                 // window slots of the ring (W, or W + 1 with commit_in_forward)
     long long n_counters = 0;
     size_t total = 0;
     char* ws = nullptr;
@@ -107,7 +108,8 @@ int check_cfg(const sw_attn_config& c) {
     if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID && c.schedule != SW_SCHED_TRI &&
         c.schedule != SW_SCHED_AUTO)
         return fail(SW_EINVAL, "bad schedule");
-    const double elems = (double)c.B * c.H * (c.W + 1) * c.tokens_per_chunk * c.d;
+    if (c.commit_in_forward != 0 && c.commit_in_forward != 1) return fail(SW_EINVAL, "commit_in_forward must be 0 or 1");
+    const double elems = (double)c.B * c.H * (c.W + 2) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
         (double)c.n_cond * c.H * c.B > 2.0e9)
         return fail(SW_ESHAPE, "problem too large");
@@ -131,7 +133,9 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->cfg = *cfg;
     if (h->cfg.scale <= 0.f) h->cfg.scale = 1.0f / std::sqrt((float)cfg->d);
     h->short_q = cfg->max_short_q == 0 ? kMaxShortQ : (cfg->max_short_q < 0 ? 0 : cfg->max_short_q);
-    h->S = cfg->W + (cfg->sink ? 1 : 0);
+    // window slots: W, or W + 1 to keep a spare slot for commits during the chunk's own forward
+    h->R = cfg->commit_in_forward && cfg->W > 0 ? cfg->W + 1 : cfg->W;
+    h->S = h->R + (cfg->sink ? 1 : 0);
     h->table_ints = table_ints_for(cfg->W);
     const int bh = cfg->B * cfg->H;
     h->max_splits = std::max(1, std::min(kMaxSplits, (148 + bh - 1) / bh));   // B200: 148 SMs
@@ -162,6 +166,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     std::memset(&c, 0, sizeof c);
     c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
     c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_AUTO;
+    c.commit_in_forward = 0;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -204,7 +209,7 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, strides, box, "K cond"))) return rc;
         if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, strides, box, "V cond"))) return rc;
     }
-    e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, c.sink, c.n_cond, c.tokens_per_chunk,
+    e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk,
                            reinterpret_cast<int32_t*>(ws + h->off_sk_cnt), h->n_counters,
                            static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state reset launch");
@@ -221,7 +226,7 @@ int sw_attn_reset(sw_attn_t* h, void* stream) {
     if (!h) return fail(SW_EINVAL, "null handle");
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     const sw_attn_config& c = h->cfg;
-    cudaError_t e = launch_state_reset(reinterpret_cast<int32_t*>(h->ws), c.W, c.sink, c.n_cond,
+    cudaError_t e = launch_state_reset(reinterpret_cast<int32_t*>(h->ws), c.W, h->R, c.sink, c.n_cond,
                                        c.tokens_per_chunk, reinterpret_cast<int32_t*>(h->ws + h->off_sk_cnt),
                                        h->n_counters, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "state reset launch");
@@ -236,7 +241,7 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
     if (!K_cond || !V_cond) return fail(SW_EINVAL, "null condition tensor");
     if (!aligned16(K_cond) || !aligned16(V_cond)) return fail(SW_EALIGN, "condition tensors must be 16-byte aligned");
     cudaError_t e = launch_relayout(K_cond, V_cond, h->ws + h->off_kcond, h->ws + h->off_vcond, c.B, c.n_cond,
-                                    c.H, c.d, c.n_cond, 0, c.W, c.sink, h->S, reinterpret_cast<int32_t*>(h->ws),
+                                    c.H, c.d, c.n_cond, 0, h->R, c.sink, h->S, reinterpret_cast<int32_t*>(h->ws),
                                     static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "condition copy launch");
     h->cond_set = true;
@@ -255,10 +260,10 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     cudaError_t e;
     if (h->S > 0) {
         e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
-                            h->S * c.tokens_per_chunk, 1, c.W, c.sink, h->S, state, st);
+                            h->S * c.tokens_per_chunk, 1, h->R, c.sink, h->S, state, st);
         if (e != cudaSuccess) return cuda_fail(e, "append launch");
     }
-    e = launch_table_build(state, c.W, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
+    e = launch_table_build(state, c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
 }
 
@@ -305,6 +310,9 @@ static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const v
     p.H = c.H;
     p.n_q = n_q;
     p.n_qc = 0;
+    p.commit = 0;
+    p.ring_R = h->R;
+    p.sink = c.sink;
     p.out_f32 = c.out_dtype == SW_OUT_F32;
     p.scale_log2 = c.scale * 1.4426950408889634f;
     return SW_OK;
@@ -373,6 +381,41 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         return SW_OK;
     }
     return launch_full(h, p, st);
+}
+
+int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out,
+                           void* stream) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
+    const sw_attn_config& c = h->cfg;
+    if (!c.commit_in_forward) return fail(SW_ESTATE, "the handle was not created with commit_in_forward");
+    if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
+    if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
+        return fail(SW_EALIGN, "Q, K_cur, V_cur and out must be 16-byte aligned");
+    AttnParams p;
+    int rc;
+    if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, c.tokens_per_chunk))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long nqt = (c.tokens_per_chunk + kBlockM - 1) / kBlockM;
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    if (resolve_schedule_tiles(h, nqt) == SW_SCHED_TRI) {
+        // the three-buffer kernel does not store K/V: forward, then the copy into the same slot
+        if ((rc = launch_full(h, p, st))) return rc;
+        if (h->S > 0) {
+            cudaError_t e = launch_relayout(K_cur, V_cur, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B,
+                                            c.tokens_per_chunk, c.H, c.d, h->S * c.tokens_per_chunk, 1, h->R, c.sink,
+                                            h->S, state, st);
+            if (e != cudaSuccess) return cuda_fail(e, "append launch");
+        }
+    } else {
+        p.commit = h->S > 0 ? 1 : 0;
+        if ((rc = launch_full(h, p, st))) return rc;
+    }
+    cudaError_t e = launch_table_build(state, c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "table launch");
+    return SW_OK;
 }
 
 int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const void* K_cur, const void* V_cur,

@@ -19,6 +19,18 @@ constexpr int kMaxPersistentCtas = 160;   // >= SMs of a B200 (148)
 
 __host__ __device__ inline int table_ints_for(int W) { return 3 + 4 * (W + 3); }
 
+// Ring slot of committed chunk c with R window slots: the sink (if any) owns slot 0 and window
+// chunks rotate through the R slots after it, chunk c taking the slot of chunk c - R.  R = W
+// is the plain ring; R = W + 1 keeps one spare slot, so chunk k can be written into the cache
+// while its own forward still reads every visible chunk.  -1: the chunk is not kept (R = 0).
+__host__ __device__ inline int ring_slot(int c, int R, int sink) {
+    if (sink) {
+        if (c == 0) return 0;
+        return R > 0 ? 1 + (c - 1) % R : -1;
+    }
+    return R > 0 ? c % R : -1;
+}
+
 // Device-side state layout: int32 words at the start of the workspace.
 //   state[0] = chunks committed (= index k of the active chunk)
 //   state[1] = status bits (SW_STATUS_*)
@@ -43,6 +55,9 @@ struct alignas(64) AttnParams {
     int32_t* status;         // device status word
     int B, H, n_q;
     int n_qc;                // condition-stream query rows (0: none); their Q tiles follow the chunk's
+    int commit;              // 1: also store K_cur / V_cur into the ring slot of the active chunk
+    int ring_R;              // window slots of the ring (for the commit slot)
+    int sink;
     int out_f32;
     int splits;              // 0: full mode (normalised output); >= 1: split-K partials
     float scale_log2;        // softmax scale * log2(e)
@@ -54,14 +69,14 @@ struct alignas(64) AttnParams {
 };
 
 // kernel launchers (defined in the .cu files)
-cudaError_t launch_table_build(int32_t* state, int W, int sink, int n_cond, int T, int advance,
+cudaError_t launch_table_build(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
                                cudaStream_t stream);
-cudaError_t launch_state_reset(int32_t* state, int W, int sink, int n_cond, int T,
+cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_cond, int T,
                                int32_t* counters, long long n_counters, cudaStream_t stream);
 // Copy [B, N, H, d] bf16 K and V into [B][H][rows_per_bh][d] regions at row offset
 // slot * N (slot from the device counter when `ring` is set, else 0).
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
-                            int H, int d, int rows_per_bh, int ring, int W, int sink, int S,
+                            int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
                             int32_t* state, cudaStream_t stream);
 cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
                              cudaStream_t stream);

@@ -80,6 +80,9 @@ typedef struct {
                                 negative disables the split-K path */
     int   schedule;          /* full path: SW_SCHED_AUTO (default), SW_SCHED_PERSISTENT,
                                 SW_SCHED_GRID or SW_SCHED_TRI */
+    int   commit_in_forward; /* 1: keep one spare window slot (W + 1 in all) so that
+                                sw_attn_forward_commit can write the chunk's K/V into the cache
+                                while its own forward runs; 0 (default): W window slots */
 } sw_attn_config;
 
 /* schedules of the full path */
@@ -142,6 +145,22 @@ SW_API int sw_attn_append_chunk(sw_attn_t *h, const void *K, const void *V, void
  */
 SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const void *V_cur,
                     void *out, int n_q, void *stream);
+
+/*
+ * Forward of the chunk's last (clean) pass that also commits the chunk: the same result as
+ * sw_attn_forward(Q, K_cur, V_cur, out, T) followed by sw_attn_append_chunk(K_cur, V_cur), in
+ * one attention launch plus the table update.  The clean K/V of a finished chunk go straight
+ * into the cache (tutorial, section "软硬件协同部署"; neurohive review, section "Откуда берётся
+ * 30 FPS": the clean-KV cache build is its own 31 ms stage of a chunk).  On the persistent and
+ * grid schedules the attention kernel stores the K_cur / V_cur tiles it has already loaded
+ * into shared memory to the chunk's ring slot (TMA bulk stores): no second read of K_cur and
+ * V_cur from HBM and no separate copy launch.  The slot written is never one this forward
+ * reads, because the handle keeps a spare window slot (commit_in_forward = 1, required:
+ * SW_ESTATE otherwise).  On the three-buffer schedule the forward is followed by the copy.
+ * Q, K_cur, V_cur [B, T, H, d] bf16; out [B, T, H, d].
+ */
+SW_API int sw_attn_forward_commit(sw_attn_t *h, const void *Q, const void *K_cur, const void *V_cur,
+                                  void *out, void *stream);
 
 /*
  * Joint forward of the chunk's queries and the condition-stream queries, in one launch.

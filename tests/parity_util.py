@@ -35,11 +35,12 @@ def sample_rows(n_q: int, n: int, seed: int) -> np.ndarray:
 
 
 def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink=None, n_cond=None,
-                schedule="auto"):
+                schedule="auto", commit_in_forward=False):
     return SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W if W is None else W,
                                   n_cond=wl.n_cond if n_cond is None else n_cond,
                                   sink=wl.sink if sink is None else sink, out_dtype=out_dtype,
-                                  max_short_q=max_short_q, schedule=schedule, device=dev)
+                                  max_short_q=max_short_q, schedule=schedule,
+                                  commit_in_forward=commit_in_forward, device=dev)
 
 
 def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, n_q=None,
@@ -133,6 +134,85 @@ def stream_and_check_joint(wl, dev, *, chunks, check_at=None, n_rows=None, promp
         h.append_chunk(K.to(dev), V.to(dev))
         hist_K.append(K.cpu())
         hist_V.append(V.cpu())
+        if keep_last is not None:
+            for c in range(1, max(1, len(hist_K) - keep_last)):
+                hist_K[c] = None
+                hist_V[c] = None
+    torch.cuda.synchronize()
+    assert h.status() == 0, f"device status {h.status():#x}"
+    return results
+
+
+def check_cache_against_ring(h, ring, chunks):
+    """Every slot of the handle's cache holds, bit for bit, the chunk the oracle's ring model
+    puts there; slots the model leaves empty still hold the NaN poison."""
+    kc, vc = h.cache_views()
+    held = ring.slot_chunks()
+    assert len(held) == kc.shape[2]
+    for s, c in enumerate(held):
+        gk, gv = kc[:, :, s].cpu(), vc[:, :, s].cpu()          # [B, H, T, d]
+        if c < 0:
+            assert torch.isnan(gk.float()).all() and torch.isnan(gv.float()).all(), f"slot {s} written"
+        else:
+            ek, ev = chunks[c]
+            assert torch.equal(gk.view(torch.int16), ek.permute(0, 2, 1, 3).contiguous().view(torch.int16)), s
+            assert torch.equal(gv.view(torch.int16), ev.permute(0, 2, 1, 3).contiguous().view(torch.int16)), s
+
+
+def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, n_rows=None,
+                            check_cache=True, append_at=(), keep_last=None, gen_on_device=False,
+                            out_dtype=torch.float32, seed=0, tol=(MAX_ABS, MEAN_REL)):
+    """Stream through a handle created with commit_in_forward: per chunk, the first step's
+    forward, then the last step's forward_commit (its K_cur / V_cur become the chunk's cache
+    entry) -- or, at the chunks in `append_at`, a plain forward plus append_chunk.  After every
+    chunk the table is compared with the oracle's table for the ring with a spare slot and (with
+    check_cache) the cache with the oracle's ring model, bit for bit; at the chunks in
+    `check_at` (all if None) both outputs are compared with the oracle.
+    Returns a list of (k, step, max_abs, mean_rel)."""
+    h = make_handle(wl, dev, out_dtype=out_dtype, max_short_q=-1, schedule=schedule, commit_in_forward=True)
+    R = h.R
+    if check_cache:
+        kc, vc = h.cache_views()
+        kc.fill_(float("nan"))
+        vc.fill_(float("nan"))
+    gdev = dev if gen_on_device else "cpu"
+    Kc, Vc = synth.cond_inputs(wl, seed=seed, device=gdev)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    Kc, Vc = Kc.cpu(), Vc.cpu()
+    ring = oracle.Ring(B=wl.B, H=wl.H, d=wl.d, T=wl.T, n_cond=0, W=wl.W, sink=wl.sink, Kc=None, Vc=None, R=R) \
+        if check_cache else None
+    hist_K, hist_V, committed, results = [], [], {}, []
+    for k in range(chunks):
+        for step in range(wl.steps):
+            Q, K, V = synth.chunk_inputs(wl, k, step, seed=seed, device=gdev)
+            last = step == wl.steps - 1
+            if last and k not in append_at:
+                out = h.forward_commit(Q.to(dev), K.to(dev), V.to(dev))
+            else:
+                out = h.forward(Q.to(dev), K.to(dev), V.to(dev))
+            if check_at is None or k in check_at:
+                r = None if n_rows is None else sample_rows(wl.T, n_rows, seed=1000 * k + step)
+                ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
+                                       k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V, Q=Q.cpu(),
+                                       K_cur=K.cpu(), V_cur=V.cpu(), rows=r)
+                got = out.float().cpu().numpy()
+                if r is not None:
+                    got = got[:, r]
+                ma, mr = compare(got, ref, *tol)
+                results.append((k, step, ma, mr))
+        if k in append_at:
+            h.append_chunk(K.to(dev), V.to(dev))
+        Kh, Vh = K.cpu(), V.cpu()
+        hist_K.append(Kh)
+        hist_V.append(Vh)
+        torch.cuda.synchronize()
+        tab = h.table().cpu().numpy()
+        ref_tab = oracle.table(k + 1, wl.W, wl.sink, wl.n_cond, wl.T, R=R)
+        assert np.array_equal(tab[:len(ref_tab)], ref_tab), (k, tab, ref_tab)
+        if check_cache:
+            ring.append(Kh, Vh)
+            committed[k] = (Kh, Vh)
+            check_cache_against_ring(h, ring, committed)
         if keep_last is not None:
             for c in range(1, max(1, len(hist_K) - keep_last)):
                 hist_K[c] = None

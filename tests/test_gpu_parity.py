@@ -17,7 +17,8 @@ import oracle
 from block_causal_attention_sliding_b200 import synth
 from block_causal_attention_sliding_b200.configs import WORKLOADS, Workload
 
-from parity_util import compare, make_handle, stream_and_check, stream_and_check_joint
+from parity_util import (compare, make_handle, stream_and_check, stream_and_check_commit,
+                         stream_and_check_joint)
 
 pytestmark = pytest.mark.gpu
 
@@ -268,6 +269,43 @@ def test_joint_720p_sampled(dev):
     res = stream_and_check_joint(wl, dev, chunks=5, check_at={0, 4}, n_rows=40, prompts={4: 1},
                                  keep_last=wl.W + 1, gen_on_device=True)
     assert len(res) == 8
+
+
+# ------------------------------------------------------------------ fused clean-KV commit
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("W,sink", [(2, True), (1, False), (3, True), (0, True)])
+def test_commit_in_forward_stream(dev, W, sink, schedule):
+    """The clean pass commits its own K/V: tables and cache contents bit-exact against the
+    oracle's ring with a spare slot after every chunk, both outputs against the oracle."""
+    wl = dataclasses.replace(RAGGED, W=W, sink=sink, chunks=7)
+    res = stream_and_check_commit(wl, dev, chunks=wl.chunks, schedule=schedule)
+    assert len(res) == wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_commit_mixed_with_append(dev, schedule):
+    """Commits in the forward and plain appends interleaved on one handle: the same cache."""
+    wl = dataclasses.replace(RAGGED, d=64, chunks=8)
+    stream_and_check_commit(wl, dev, chunks=wl.chunks, schedule=schedule, append_at={1, 4, 5})
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+@pytest.mark.parametrize("H,T", [(1, 129), (5, 640)])
+def test_commit_split_shapes(dev, H, T, schedule):
+    """Shapes whose first Q-tile pair is cut between several CTAs: every K/V tile of the chunk
+    is stored exactly once."""
+    wl = Workload("split", B=1, H=H, d=128, T=T, n_cond=64, W=2, sink=True, chunks=5, steps=2)
+    stream_and_check_commit(wl, dev, chunks=wl.chunks, schedule=schedule)
+
+
+def test_commit_720p_sampled(dev):
+    """720p in the benchmark's launch configuration, clean pass committing: sampled rows at
+    chunks 0, W + 1 and the last, cache bit-exact after every chunk."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_commit(wl, dev, chunks=7, check_at={0, 4, 6}, n_rows=32, keep_last=wl.W + 1,
+                                  gen_on_device=True)
+    assert len(res) == 6
 
 
 def test_long_horizon_constant_memory(dev):
