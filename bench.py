@@ -321,6 +321,7 @@ def run_cuda(args, wl, world, rank, local):
             h.close()
             h = None
             paths["long_horizon"] = long_horizon(args, dev, stream, pool)
+            paths["commit"] = commit_path(args, dev, stream, pool)
             paths["workloads"] = other_workloads(args, dev, stream, peaks)
 
     if rank == 0:
@@ -452,6 +453,47 @@ def long_horizon(args, dev, stream, pool):
                 "status_interleaved": max(hx.status() for hx in hs)})
     for hx in hs:
         hx.close()
+    return res
+
+
+def commit_path(args, dev, stream, pool):
+    """The steady-state 720p chunk step with the clean pass committing its own K/V
+    (forward, forward_commit) against forward, forward, append_chunk, on one handle created with
+    commit_in_forward (the append path writes the same slots).  Chunks alternate between the two
+    forms so both see the same clock."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    wl = WORKLOADS["720p"]
+    h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                               out_dtype=torch.bfloat16, schedule=args.schedule, commit_in_forward=True,
+                               device=dev)
+    Kc, Vc = synth.cond_inputs(wl, seed=9, device=dev)
+    h.set_cond(Kc, Vc)
+    outs = [torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev) for _ in range(wl.steps)]
+    for c in range(wl.W + 2):
+        (Q0, K0, V0), (Q1, K1, V1) = pool[c % len(pool)]
+        h.forward(Q0, K0, V0, out=outs[0])
+        h.forward_commit(Q1, K1, V1, out=outs[1])
+    reps = 30
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * reps)]
+    torch.cuda.synchronize(dev)
+    for r in range(reps):
+        (Q0, K0, V0), (Q1, K1, V1) = pool[r % len(pool)]
+        ev[4 * r].record(stream)
+        h.forward(Q0, K0, V0, out=outs[0])
+        h.forward_commit(Q1, K1, V1, out=outs[1])
+        ev[4 * r + 1].record(stream)
+        ev[4 * r + 2].record(stream)
+        h.forward(Q0, K0, V0, out=outs[0])
+        h.forward(Q1, K1, V1, out=outs[1])
+        h.append_chunk(K1, V1)
+        ev[4 * r + 3].record(stream)
+    torch.cuda.synchronize(dev)
+    fused = statistics.median(ev[4 * r].elapsed_time(ev[4 * r + 1]) for r in range(reps))
+    plain = statistics.median(ev[4 * r + 2].elapsed_time(ev[4 * r + 3]) for r in range(reps))
+    res = {"chunk_ms_fused_commit": round(fused, 4), "chunk_ms_forward_append": round(plain, 4),
+           "saved_us": round((plain - fused) * 1e3, 1), "chunks_each": reps, "status": h.status(),
+           "schedule": h.schedule_for()}
+    h.close()
     return res
 
 

@@ -188,20 +188,22 @@ __device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl*
 // loaded into the K/V ring for the attention, from shared memory to the chunk's ring slot in
 // the cache.  A tile's store is issued kStages - 1 ring items after its load (by then the load
 // has landed, and the stage cannot have been refilled), and a stage is refilled only after
-// every issued store has finished reading shared memory.  The producer flushes the queue and
-// waits for the stores to complete before it finishes.
+// every issued store has finished reading shared memory.  The last kStages - 1 items are kept
+// in registers, one packed 64-bit word each (store it; j, head, stream, K or V), shifted once per item;
+// the producer flushes them and waits for the stores to complete before it finishes.  The
+// per-item work is kept out of line: inlined, it changed the register allocation of the whole
+// kernel and cost more (measured) than the stores themselves.
 template <int D, int kStages>
 struct CommitQueue {
-    static constexpr int kCap = 8;
-    int n = 0, head = 0;
-    uint32_t pending = 0;   // stages with a store that may still be reading them
-    uint32_t item[kCap];
-    int j[kCap], kv[kCap], h[kCap], b[kCap];
+    static constexpr int kLag = kStages - 1;
+    static_assert(kLag >= 1 && kLag <= 7, "commit history");
+    uint64_t hist[kLag] = {};   // hist[0]: oldest
+    uint32_t pending = 0;       // stages with a store that may still be reading them
 
-    __device__ __forceinline__ void push(uint32_t it, int j_, int kv_, int h_, int b_) {
-        const int t = (head + n) % kCap;
-        item[t] = it; j[t] = j_; kv[t] = kv_; h[t] = h_; b[t] = b_;
-        ++n;
+    // bit 63: store it; bits 32..62: key tile j; 16..31: head; 1..15: stream; 0: V (1) or K (0)
+    __device__ __forceinline__ static uint64_t pack(bool store, int j, int kv, int h, int b) {
+        return (store ? (1ull << 63) : 0ull) | ((uint64_t)(uint32_t)j << 32) | ((uint64_t)(h & 0xffff) << 16) |
+               ((uint64_t)(b & 0x7fff) << 1) | (uint64_t)(kv & 1);
     }
     // Before stage s takes a new load: its last store (if any) must have read it.
     __device__ __forceinline__ void before_refill(int s) {
@@ -210,26 +212,43 @@ struct CommitQueue {
             pending = 0;
         }
     }
-    // Issue the stores of queued tiles loaded at least kStages - 1 items before item it_now
-    // (every queued tile with force).  Returns false if a wait gave up.
-    __device__ __forceinline__ bool issue(const AttnParams& p, const SmemCtl* ctl, const uint8_t* kv_smem,
-                                          int slot, uint32_t it_now, bool force, volatile int* abort_flag) {
-        while (n > 0 && (force || it_now - item[head] >= (uint32_t)(kStages - 1))) {
-            const uint32_t i = item[head];
-            const int s = (int)(i % kStages);
-            if (!wait_or_abort(smem_u32(&ctl->kv_full[s]), (i / kStages) & 1, abort_flag)) return false;
-            int seg, row0, valid;
-            tile_of(ctl, j[head], seg, row0, valid);
-            fence_proxy_async_smem();
-            const uint32_t src = smem_u32(kv_smem + (size_t)s * TileCfg<D>::kTileBytes);
+    __device__ __noinline__ bool store_one(const AttnParams& p, const SmemCtl* ctl, const uint8_t* kv_smem,
+                                              int slot, uint32_t i, uint64_t w, volatile int* abort_flag) {
+        const int s = (int)(i % kStages);
+        if (!wait_or_abort(smem_u32(&ctl->kv_full[s]), (i / kStages) & 1, abort_flag)) return false;
+        const int j = (int)((w >> 32) & 0x7fffffffu), kv = (int)(w & 1u);
+        const int h = (int)((w >> 16) & 0xffffu), b = (int)((w >> 1) & 0x7fffu);
+        int seg, row0, valid;
+        tile_of(ctl, j, seg, row0, valid);
+        fence_proxy_async_smem();
+        const uint32_t src = smem_u32(kv_smem + (size_t)s * TileCfg<D>::kTileBytes);
 #pragma unroll
-            for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
-                tma_store_5d(kv[head] ? &p.tm_cache_v : &p.tm_cache_k, src + c * kBoxBytes, c * kBoxCols, row0,
-                             slot, h[head], b[head]);
-            bulk_commit_group();
-            pending |= 1u << s;
-            head = (head + 1) % kCap;
-            --n;
+        for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
+            tma_store_5d(kv ? &p.tm_cache_v : &p.tm_cache_k, src + c * kBoxBytes, c * kBoxCols, row0, slot, h, b);
+        bulk_commit_group();
+        pending |= 1u << s;
+        return true;
+    }
+    // Item it (just loaded) enters the history; the item kLag before it leaves and is stored if
+    // marked.  Returns false if a wait gave up.
+    __device__ __noinline__ bool step(const AttnParams& p, const SmemCtl* ctl, const uint8_t* kv_smem, int slot,
+                                         uint32_t it, uint64_t w, volatile int* abort_flag) {
+        const uint64_t out = hist[0];
+#pragma unroll
+        for (int q = 0; q + 1 < kLag; ++q) hist[q] = hist[q + 1];
+        hist[kLag - 1] = w;
+        if ((out >> 63) && it >= (uint32_t)kLag) return store_one(p, ctl, kv_smem, slot, it - kLag, out, abort_flag);
+        return true;
+    }
+    // Store every marked item still in the history (the last items of the launch).
+    __device__ __noinline__ bool flush(const AttnParams& p, const SmemCtl* ctl, const uint8_t* kv_smem, int slot,
+                                          uint32_t it_next, volatile int* abort_flag) {
+#pragma unroll
+        for (int q = 0; q < kLag; ++q) {
+            const uint32_t i = it_next - kLag + q;
+            if ((hist[q] >> 63) && it_next >= (uint32_t)(kLag - q) &&
+                !store_one(p, ctl, kv_smem, slot, i, hist[q], abort_flag))
+                return false;
         }
         return true;
     }

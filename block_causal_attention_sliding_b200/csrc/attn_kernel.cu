@@ -93,8 +93,9 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             }
             uint32_t it = 0;
             bool ok = true;
-            // fused commit: the CTA of the first Q-tile pair stores the chunk's K_cur / V_cur tiles
-            const int cslot = (p.commit && !split_mode && blockIdx.x == 0) ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
+            // fused commit: the chunk's K_cur / V_cur tile j is stored by the CTA of Q-tile pair
+            // j mod (pairs), so the stores spread over the CTAs of each head
+            const int cslot = (p.commit && !split_mode) ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
             CommitQueue<D, kStages> cq;
             for (int j = t0; j < t1 && ok; ++j) {
                 for (int kv = 0; kv < 2; ++kv, ++it) {
@@ -108,15 +109,20 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                     const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
                     mbar_arrive_expect_tx(fbar, kTileBytes);
                     load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
-                    if (cslot >= 0 && ctl->seg_kind[tile_seg(ctl, j)] == 2) cq.push(it, j, kv, h, b);
-                    if (cq.n > 0 && !cq.issue(p, ctl, kv_smem, cslot, it, false, abort_flag)) {
-                        ok = false;
-                        break;
+                    if (cslot >= 0) {
+                        const bool mine = (int)blockIdx.x == j % (int)gridDim.x && ctl->seg_kind[tile_seg(ctl, j)] == 2;
+                        if (!cq.step(p, ctl, kv_smem, cslot, it, CommitQueue<D, kStages>::pack(mine, j, kv, h, b),
+                                     abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                     }
                 }
             }
-            if (cq.n > 0 && ok) (void)cq.issue(p, ctl, kv_smem, cslot, it, true, abort_flag);
-            bulk_wait_all();
+            if (cslot >= 0) {
+                if (ok) (void)cq.flush(p, ctl, kv_smem, cslot, it, abort_flag);
+                bulk_wait_all();
+            }
             // never leave while copies are in flight: the last fill of every stage has landed
             for (int s = 0; s < kStages; ++s) {
                 if (it > (uint32_t)s) {

@@ -21,7 +21,9 @@
 
 namespace swattn {
 
-template <int D>
+// kCommit: the launch also stores the chunk's K_cur / V_cur into the cache (fused commit); a
+// separate instantiation, so the plain forward carries none of that code.
+template <int D, bool kCommit>
 __global__ void __launch_bounds__(AttnLayout<D, 2>::kThreads, 1)
 attn_persistent_kernel(const __grid_constant__ AttnParams p) {
     constexpr int NQ = 2;
@@ -76,8 +78,9 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             uint32_t it = 0;
             int pi = 0;
             bool ok = true;
-            // fused commit: the pieces of Q-tile pair 0 store the chunk's K_cur / V_cur tiles
-            const int cslot = p.commit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
+            // fused commit: the chunk's K_cur / V_cur tile j is stored by the piece of Q-tile pair
+            // j mod npairs that loads it, so the stores spread over the CTAs
+            const int cslot = kCommit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
             CommitQueue<D, kStages> cq;
             while (ok && next_piece(sched, pit, pc)) {
                 const int b = pc.bh / p.H, h = pc.bh % p.H;
@@ -99,20 +102,26 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                             ok = false;
                             break;
                         }
-                        cq.before_refill(s);
+                        if (kCommit) cq.before_refill(s);
                         const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
                         mbar_arrive_expect_tx(fbar, kTileBytes);
                         load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
-                        if (cslot >= 0 && pc.pair == 0 && ctl->seg_kind[tile_seg(ctl, j)] == 2) cq.push(it, j, kv, h, b);
-                        if (cq.n > 0 && !cq.issue(p, ctl, kv_smem, cslot, it, false, abort_flag)) {
-                            ok = false;
-                            break;
+                        if (kCommit) {
+                            const bool mine = cslot >= 0 && pc.pair == j % sched.npairs &&
+                                              ctl->seg_kind[tile_seg(ctl, j)] == 2;
+                            if (!cq.step(p, ctl, kv_smem, cslot, it, CommitQueue<D, kStages>::pack(mine, j, kv, h, b),
+                                         abort_flag)) {
+                                ok = false;
+                                break;
+                            }
                         }
                     }
                 }
             }
-            if (cq.n > 0 && ok) (void)cq.issue(p, ctl, kv_smem, cslot, it, true, abort_flag);
-            bulk_wait_all();
+            if (kCommit) {
+                if (ok) (void)cq.flush(p, ctl, kv_smem, cslot, it, abort_flag);
+                bulk_wait_all();
+            }
             for (int s = 0; s < kStages; ++s) {
                 if (it > (uint32_t)s) {
                     const uint32_t uses = (it - 1 - s) / kStages + 1;
@@ -345,7 +354,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 template <int D>
 static cudaError_t launch_persistent_d(const AttnParams& p, int ctas, cudaStream_t stream) {
     using L = AttnLayout<D, 2>;
-    auto kern = attn_persistent_kernel<D>;
+    auto kern = p.commit ? attn_persistent_kernel<D, true> : attn_persistent_kernel<D, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     kern<<<ctas, L::kThreads, L::kSmemBytes, stream>>>(p);

@@ -391,6 +391,7 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     const sw_attn_config& c = h->cfg;
     if (!c.commit_in_forward) return fail(SW_ESTATE, "the handle was not created with commit_in_forward");
+    if (c.B > 32767 || c.H > 65535) return fail(SW_ESHAPE, "a committing forward supports B <= 32767, H <= 65535");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
         return fail(SW_EALIGN, "Q, K_cur, V_cur and out must be 16-byte aligned");
