@@ -322,6 +322,7 @@ def run_cuda(args, wl, world, rank, local):
             h = None
             paths["long_horizon"] = long_horizon(args, dev, stream, pool)
             paths["commit"] = commit_path(args, dev, stream, pool)
+            paths["layers"] = layers_path(args, dev, stream)
             paths["workloads"] = other_workloads(args, dev, stream, peaks)
 
     if rank == 0:
@@ -495,6 +496,71 @@ def commit_path(args, dev, stream, pool):
            "schedule": h.schedule_for()}
     h.close()
     return res
+
+
+def layers_path(args, dev, stream, n_layers=8):
+    """A chunk step of an n-layer model at 480p: each layer (one handle, its own cache) runs its
+    two forwards, then every layer commits the chunk.  Timed with per-layer appends, with one
+    batched append for all layers, and with the whole step replayed from a CUDA graph."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention, append_chunk_batched
+    wl = WORKLOADS["480p"]
+    hs, ins, outs = [], [], []
+    for l in range(n_layers):
+        h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                   out_dtype=torch.bfloat16, schedule=args.schedule, device=dev)
+        Kc, Vc = synth.cond_inputs(wl, seed=20 + l, device=dev)
+        h.set_cond(Kc, Vc)
+        hs.append(h)
+        ins.append([synth.chunk_inputs(wl, 3, s, seed=20 + l, device=dev) for s in range(wl.steps)])
+        outs.append([torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev) for _ in range(wl.steps)])
+
+    def forwards():
+        for l in range(n_layers):
+            for s in range(wl.steps):
+                hs[l].forward(*ins[l][s], out=outs[l][s])
+
+    def step_each():
+        forwards()
+        for l in range(n_layers):
+            hs[l].append_chunk(ins[l][-1][1], ins[l][-1][2])
+
+    def step_batched():
+        forwards()
+        append_chunk_batched(hs, [x[-1][1] for x in ins], [x[-1][2] for x in ins])
+
+    for _ in range(wl.steady_k()):
+        step_batched()
+    reps = 20
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(torch.cuda.current_stream())
+        for _ in range(reps):
+            fn()
+        e1.record(torch.cuda.current_stream())
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    t_each = timed(step_each)
+    t_batched = timed(step_batched)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step_batched()
+    torch.cuda.current_stream().wait_stream(side)
+    t_graph = timed(graph.replay)
+    status = max(h.status() for h in hs)
+    del graph
+    for h in hs:
+        h.close()
+    return {"workload": wl.name, "layers": n_layers, "ms_per_chunk_appends_each": round(t_each, 4),
+            "ms_per_chunk_batched_append": round(t_batched, 4), "ms_per_chunk_graph": round(t_graph, 4),
+            "status": status}
 
 
 def other_workloads(args, dev, stream, peaks):

@@ -19,7 +19,7 @@ SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
 EXPORTS = (
     "sw_attn_create", "sw_attn_create_ex", "sw_attn_workspace_bytes", "sw_attn_bind_workspace",
     "sw_attn_set_cond", "sw_attn_append_chunk", "sw_attn_forward", "sw_attn_forward_joint",
-    "sw_attn_forward_commit",
+    "sw_attn_forward_commit", "sw_attn_append_chunk_batched",
     "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_forward_joint.restype = i32
     L.sw_attn_forward_commit.argtypes = [vp, vp, vp, vp, vp, vp]
     L.sw_attn_forward_commit.restype = i32
+    L.sw_attn_append_chunk_batched.argtypes = [vp, i32, vp, vp, vp]
+    L.sw_attn_append_chunk_batched.restype = i32
     L.sw_attn_forward_short_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.sw_attn_forward_short_noalloc.restype = i32
     L.sw_attn_selftest_timeout.argtypes = [vp, ctypes.c_int64, vp]

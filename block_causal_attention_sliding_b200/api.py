@@ -186,3 +186,21 @@ class SlidingWindowAttention:
             self.close()
         except Exception:
             pass
+
+
+def append_chunk_batched(handles, Ks, Vs, stream=None) -> None:
+    """Commit the finished chunk of several handles (e.g. every layer of a model) in one copy
+    launch and one table launch (sw_attn_append_chunk_batched).  Handles share B, H, d, T."""
+    n = len(handles)
+    if n < 1 or len(Ks) != n or len(Vs) != n:
+        raise ValueError("need one K and one V per handle")
+    for h, K, V in zip(handles, Ks, Vs):
+        shape = (h.B, h.T, h.H, h.d)
+        if tuple(K.shape) != shape or tuple(V.shape) != shape:
+            raise ValueError(f"K and V must have shape {shape}")
+    lib = handles[0]._lib
+    hp = (ctypes.c_void_p * n)(*[h._h.value for h in handles])
+    kp = (ctypes.c_void_p * n)(*[_dev_ptr(K, "K", torch.bfloat16) for K in Ks])
+    vp = (ctypes.c_void_p * n)(*[_dev_ptr(V, "V", torch.bfloat16) for V in Vs])
+    N.check(lib.sw_attn_append_chunk_batched(ctypes.cast(hp, ctypes.c_void_p), n, ctypes.cast(kp, ctypes.c_void_p),
+                                             ctypes.cast(vp, ctypes.c_void_p), _stream_ptr(stream)))

@@ -14,9 +14,7 @@ namespace swattn {
 // chunk k: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...], in the order
 // condition, sink, window ascending, current; slots of a ring with R window slots.  One
 // thread: a few dozen integers.
-__global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
-                                   int reset) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+__device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance, int reset) {
     int32_t* tab = state + kStateHeaderInts;
     if (reset) {
         state[0] = 0;
@@ -44,6 +42,12 @@ __global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n
     put(2, k, -1, T);
     tab[0] = k; tab[1] = nseg; tab[2] = nvis;
     for (int i = pos; i < cap; ++i) tab[i] = -1;
+}
+
+__global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
+                                   int reset) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    build_table(state, W, R, sink, n_cond, T, advance, reset);
 }
 
 cudaError_t launch_table_build(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
@@ -75,12 +79,10 @@ cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_con
 // vector k of the row (head k / vpr, vector k % vpr), looping when H * vpr exceeds the block,
 // so consecutive threads read consecutive bytes and write whole 16-byte pieces of 2d-byte
 // destination rows.  No division in the copy loop (vpr is a power of two).
-__global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__ srcK,
-                                                       const uint4* __restrict__ srcV,
-                                                       uint4* __restrict__ dstK,
-                                                       uint4* __restrict__ dstV, int N, int H,
-                                                       int vpr_log2, int rows_per_bh, int ring,
-                                                       int R, int sink, int S, int32_t* state) {
+__device__ __forceinline__ void relayout_row(const uint4* __restrict__ srcK, const uint4* __restrict__ srcV,
+                                             uint4* __restrict__ dstK, uint4* __restrict__ dstV, int N, int H,
+                                             int vpr_log2, int rows_per_bh, int ring, int R, int sink, int S,
+                                             int32_t* state) {
     int slot = 0;
     if (ring) {
         slot = ring_slot(state[0], R, sink);
@@ -103,6 +105,49 @@ __global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__
         const int h = k >> vpr_log2, v = k & (vpr - 1);
         dst[(drow0 + (size_t)h * rows_per_bh) * vpr + v] = __ldg(s_row + k);
     }
+}
+
+__global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__ srcK,
+                                                       const uint4* __restrict__ srcV,
+                                                       uint4* __restrict__ dstK,
+                                                       uint4* __restrict__ dstV, int N, int H,
+                                                       int vpr_log2, int rows_per_bh, int ring,
+                                                       int R, int sink, int S, int32_t* state) {
+    relayout_row(srcK, srcV, dstK, dstV, N, H, vpr_log2, rows_per_bh, ring, R, sink, S, state);
+}
+
+// Batched commit: blockIdx.z selects the handle; each copies into its own ring slot (from its
+// own counter), exactly as relayout_kernel does for one handle.
+__global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_constant__ AppendBatch a, int N, int H,
+                                                             int vpr_log2, int T) {
+    const int l = blockIdx.z;
+    relayout_row(static_cast<const uint4*>(a.K[l]), static_cast<const uint4*>(a.V[l]), static_cast<uint4*>(a.dstK[l]),
+                 static_cast<uint4*>(a.dstV[l]), N, H, vpr_log2, a.S[l] * T, 1, a.R[l], a.sink[l], a.S[l], a.state[l]);
+}
+
+// Batched table advance: block l advances handle l's counter and rebuilds its table.
+__global__ void table_build_batch_kernel(const __grid_constant__ AppendBatch a, int T) {
+    const int l = blockIdx.x;
+    if (threadIdx.x != 0 || l >= a.n) return;
+    build_table(a.state[l], a.W[l], a.R[l], a.sink[l], a.n_cond[l], T, 1, 0);
+}
+
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, cudaStream_t stream) {
+    if (a.n < 1 || a.n > kMaxBatch) return cudaErrorInvalidValue;
+    const int vpr = d / 8;
+    int vpr_log2 = 0;
+    while ((1 << vpr_log2) < vpr) ++vpr_log2;
+    if ((1 << vpr_log2) != vpr) return cudaErrorInvalidValue;
+    const long long rows = (long long)B * T;
+    if (rows < 1 || rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int per_row = H * vpr;
+    const int threads = per_row >= 512 ? 512 : ((per_row + 31) / 32) * 32;
+    // handles without a ring (S = 0) return at once inside the kernel (slot -1)
+    relayout_batch_kernel<<<dim3((unsigned)rows, 2, (unsigned)a.n), threads, 0, stream>>>(a, T, H, vpr_log2, T);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    table_build_batch_kernel<<<a.n, 32, 0, stream>>>(a, T);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,

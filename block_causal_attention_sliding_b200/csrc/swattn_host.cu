@@ -383,6 +383,50 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
     return launch_full(h, p, st);
 }
 
+int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const* K, const void* const* V,
+                                 void* stream) {
+    g_err.clear();
+    if (!hs || !K || !V || n < 1) return fail(SW_EINVAL, "null array or n < 1");
+    const sw_attn_t* h0 = hs[0];
+    if (!h0) return fail(SW_EINVAL, "null handle 0");
+    const sw_attn_config& c0 = h0->cfg;
+    for (int l = 0; l < n; ++l) {
+        const sw_attn_t* h = hs[l];
+        if (!h) return fail(SW_EINVAL, "null handle %d", l);
+        if (!h->ws) return fail(SW_ESTATE, "handle %d has no workspace bound", l);
+        if (h->device != h0->device) return fail(SW_ESTATE, "handle %d is on another device", l);
+        const sw_attn_config& c = h->cfg;
+        if (c.B != c0.B || c.H != c0.H || c.d != c0.d || c.tokens_per_chunk != c0.tokens_per_chunk)
+            return fail(SW_ESHAPE, "handle %d: B, H, d and T must match handle 0", l);
+        if (!K[l] || !V[l]) return fail(SW_EINVAL, "null K or V for handle %d", l);
+        if (!aligned16(K[l]) || !aligned16(V[l])) return fail(SW_EALIGN, "K and V of handle %d must be 16-byte aligned", l);
+        for (int m = 0; m < l; ++m)
+            if (hs[m] == h) return fail(SW_EINVAL, "handle %d appears twice", l);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int l0 = 0; l0 < n; l0 += kMaxBatch) {
+        AppendBatch a;
+        std::memset(&a, 0, sizeof a);
+        a.n = std::min(kMaxBatch, n - l0);
+        for (int q = 0; q < a.n; ++q) {
+            sw_attn_t* h = hs[l0 + q];
+            a.K[q] = K[l0 + q];
+            a.V[q] = V[l0 + q];
+            a.dstK[q] = h->ws + h->off_kcache;
+            a.dstV[q] = h->ws + h->off_vcache;
+            a.state[q] = reinterpret_cast<int32_t*>(h->ws);
+            a.R[q] = h->R;
+            a.S[q] = h->S;
+            a.W[q] = h->cfg.W;
+            a.sink[q] = h->cfg.sink;
+            a.n_cond[q] = h->cfg.n_cond;
+        }
+        cudaError_t e = launch_append_batch(a, c0.B, c0.tokens_per_chunk, c0.H, c0.d, st);
+        if (e != cudaSuccess) return cuda_fail(e, "batched append launch");
+    }
+    return SW_OK;
+}
+
 int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out,
                            void* stream) {
     g_err.clear();

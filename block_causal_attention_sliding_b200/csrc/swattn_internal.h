@@ -78,6 +78,20 @@ cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_con
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
                             int32_t* state, cudaStream_t stream);
+// One chunk commit for each of up to kMaxBatch handles (layers) of the same B, T, H, d, in one
+// copy launch and one table launch (the per-handle window, sink, slots and counter stay apart).
+constexpr int kMaxBatch = 32;
+struct AppendBatch {
+    const void* K[kMaxBatch];
+    const void* V[kMaxBatch];
+    void* dstK[kMaxBatch];       // the handle's K cache region [B][H][S * T][d]
+    void* dstV[kMaxBatch];
+    int32_t* state[kMaxBatch];   // the handle's device state (counter, status, table)
+    int R[kMaxBatch], S[kMaxBatch], W[kMaxBatch], sink[kMaxBatch], n_cond[kMaxBatch];
+    int n;                       // handles in this launch
+};
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, cudaStream_t stream);
+
 cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
                              cudaStream_t stream);
 cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream);

@@ -147,6 +147,20 @@ SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const
                     void *out, int n_q, void *stream);
 
 /*
+ * Commit the finished chunk of n handles at once -- typically the n layers of one model, each
+ * with its own cache: the same effect as sw_attn_append_chunk(handles[l], K[l], V[l]) for every
+ * l, in one copy launch and one table launch per 32 handles instead of two launches per handle
+ * (the clean-KV cache build of a chunk covers every layer: tutorial, section "软硬件协同部署";
+ * neurohive review, section "Откуда берётся 30 FPS").  All handles share B, H, d and T; window,
+ * sink, condition count and chunk counter are each handle's own.  K[l], V[l]: [B, T, H, d] bf16.
+ * A handle may appear only once (SW_EINVAL).  Forwards of different layers depend on one
+ * another through the model and stay separate launches; a whole chunk step (every layer's
+ * forwards and this call) can be captured into one CUDA graph, since no call synchronises.
+ */
+SW_API int sw_attn_append_chunk_batched(sw_attn_t *const *handles, int n, const void *const *K,
+                                        const void *const *V, void *stream);
+
+/*
  * Forward of the chunk's last (clean) pass that also commits the chunk: the same result as
  * sw_attn_forward(Q, K_cur, V_cur, out, T) followed by sw_attn_append_chunk(K_cur, V_cur), in
  * one attention launch plus the table update.  The clean K/V of a finished chunk go straight

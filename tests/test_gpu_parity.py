@@ -308,6 +308,112 @@ def test_commit_720p_sampled(dev):
     assert len(res) == 6
 
 
+# ------------------------------------------------------------------ several layers per chunk step
+
+LAYERS = [dict(W=2, sink=True, n_cond=40, commit_in_forward=False), dict(W=1, sink=False, n_cond=8, commit_in_forward=False),
+          dict(W=3, sink=True, n_cond=0, commit_in_forward=True), dict(W=0, sink=True, n_cond=40, commit_in_forward=False),
+          dict(W=2, sink=False, n_cond=130, commit_in_forward=True)]
+
+
+def test_append_batched_matches_ring(dev):
+    """Five layers with different windows, sinks, condition counts and slot counts, committed
+    together: every layer's table and cache equal its own oracle model, bit for bit."""
+    from block_causal_attention_sliding_b200.api import append_chunk_batched
+    from parity_util import check_cache_against_ring
+    B, H, d, T, chunks = 2, 3, 64, 40, 9
+    hs, rings, held = [], [], []
+    for cfg in LAYERS:
+        wl = Workload("l", B=B, H=H, d=d, T=T, n_cond=cfg["n_cond"], W=cfg["W"], sink=cfg["sink"], chunks=chunks, steps=1)
+        h = make_handle(wl, dev, commit_in_forward=cfg["commit_in_forward"])
+        kc, vc = h.cache_views()
+        kc.fill_(float("nan"))
+        vc.fill_(float("nan"))
+        hs.append(h)
+        rings.append(oracle.Ring(B=B, H=H, d=d, T=T, n_cond=0, W=cfg["W"], sink=cfg["sink"], Kc=None, Vc=None, R=h.R))
+        held.append({})
+    for c in range(chunks):
+        Ks = [synth.draw((B, T, H, d), 500 + 10 * c + 2 * l) for l in range(len(hs))]
+        Vs = [synth.draw((B, T, H, d), 501 + 10 * c + 2 * l) for l in range(len(hs))]
+        append_chunk_batched(hs, [K.to(dev) for K in Ks], [V.to(dev) for V in Vs])
+        torch.cuda.synchronize()
+        for l, (h, cfg) in enumerate(zip(hs, LAYERS)):
+            rings[l].append(Ks[l], Vs[l])
+            held[l][c] = (Ks[l], Vs[l])
+            check_cache_against_ring(h, rings[l], held[l])
+            ref = oracle.table(c + 1, cfg["W"], cfg["sink"], cfg["n_cond"], T, R=h.R)
+            assert np.array_equal(h.table().cpu().numpy()[:len(ref)], ref), (l, c)
+    for h in hs:
+        assert h.status() == 0
+
+
+def test_chunk_step_graph_capture(dev):
+    """A three-layer chunk step -- each layer's two forwards, then one batched commit -- captured
+    once into a CUDA graph and replayed chunk after chunk gives the same outputs, bit for bit,
+    as the same calls run eagerly, and both match the oracle at the checked chunks."""
+    from block_causal_attention_sliding_b200.api import append_chunk_batched
+    wl = dataclasses.replace(RAGGED, chunks=6)
+    L = 3
+    def layer_handles():
+        hs = []
+        for l in range(L):
+            h = make_handle(wl, dev, schedule="persistent" if l != 1 else "tri")
+            Kc, Vc = synth.cond_inputs(wl, seed=l)
+            h.set_cond(Kc.to(dev), Vc.to(dev))
+            hs.append(h)
+        return hs
+    def inputs(k):
+        return [[[t.to(dev) for t in synth.chunk_inputs(wl, k, s, seed=10 + l)] for s in range(wl.steps)] for l in range(L)]
+    # eager
+    eager_hs = layer_handles()
+    eager_out = []
+    for k in range(wl.chunks):
+        x = inputs(k)
+        outs = [[eager_hs[l].forward(*x[l][s]).clone() for s in range(wl.steps)] for l in range(L)]
+        append_chunk_batched(eager_hs, [x[l][-1][1] for l in range(L)], [x[l][-1][2] for l in range(L)])
+        eager_out.append(outs)
+    torch.cuda.synchronize()
+    # graph: static input and output buffers, one capture of a whole chunk step
+    g_hs = layer_handles()
+    static_in = inputs(0)
+    static_out = [[torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.float32, device=dev) for _ in range(wl.steps)]
+                  for _ in range(L)]
+
+    def step():
+        for l in range(L):
+            for s in range(wl.steps):
+                g_hs[l].forward(*static_in[l][s], out=static_out[l][s])
+        append_chunk_batched(g_hs, [static_in[l][-1][1] for l in range(L)], [static_in[l][-1][2] for l in range(L)])
+
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step()
+    torch.cuda.current_stream().wait_stream(side)
+    for k in range(wl.chunks):
+        x = inputs(k)
+        for l in range(L):
+            for s in range(wl.steps):
+                for dst, src in zip(static_in[l][s], x[l][s]):
+                    dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        for l in range(L):
+            for s in range(wl.steps):
+                assert torch.equal(static_out[l][s], eager_out[k][l][s]), (k, l, s)
+    for h in eager_hs + g_hs:
+        assert h.status() == 0
+    # spot check against the oracle: layer 0, last chunk, last step
+    k = wl.chunks - 1
+    Kc, Vc = synth.cond_inputs(wl, seed=0)
+    hist = [synth.chunk_inputs(wl, c, wl.steps - 1, seed=10) for c in range(k)]
+    Q, K, V = synth.chunk_inputs(wl, k, wl.steps - 1, seed=10)
+    ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink, k=k, Kc=Kc, Vc=Vc,
+                           hist_K=[t[1] for t in hist], hist_V=[t[2] for t in hist], Q=Q, K_cur=K, V_cur=V)
+    compare(eager_out[k][0][-1].cpu().numpy(), ref)
+
+
 def test_long_horizon_constant_memory(dev):
     """225 chunks: the device table stays exact, memory does not grow, the last chunk matches
     the oracle on sampled rows."""
