@@ -323,6 +323,7 @@ def run_cuda(args, wl, world, rank, local):
             paths["long_horizon"] = long_horizon(args, dev, stream, pool)
             paths["commit"] = commit_path(args, dev, stream, pool)
             paths["layers"] = layers_path(args, dev, stream)
+            paths["fp8_qk"] = fp8_path(args, dev, stream, peaks)
             paths["workloads"] = other_workloads(args, dev, stream, peaks)
 
     if rank == 0:
@@ -495,6 +496,41 @@ def commit_path(args, dev, stream, pool):
            "saved_us": round((plain - fused) * 1e3, 1), "chunks_each": reps, "status": h.status(),
            "schedule": h.schedule_for()}
     h.close()
+    return res
+
+
+def fp8_path(args, dev, stream, peaks):
+    """The 720p steady-state forward with e4m3 queries and keys (S on kind::f8f6f4, e4m3 K
+    cache) and bf16 V, against the bf16 forward of the same draws, both timed alone."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    wl = WORKLOADS["720p"]
+    sc = synth.FP8_SCALE
+    res = {}
+    for name, fp8 in (("bf16", False), ("e4m3_qk", True)):
+        h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                   out_dtype=torch.bfloat16, qk_fp8=fp8, q_scale=sc, k_scale=sc, device=dev)
+        Kc, Vc = (synth.cond_inputs_fp8 if fp8 else synth.cond_inputs)(wl, seed=11, device=dev)
+        h.set_cond(Kc, Vc)
+        Q, K, V = (synth.chunk_inputs_fp8 if fp8 else synth.chunk_inputs)(wl, 0, 0, seed=11, device=dev)
+        for _ in range(wl.steady_k()):
+            h.append_chunk(K, V)
+        out = torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            h.forward(Q, K, V, out=out)
+        torch.cuda.synchronize(dev)
+        reps = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(torch.cuda.current_stream())
+        for _ in range(reps):
+            h.forward(Q, K, V, out=out)
+        e1.record(torch.cuda.current_stream())
+        torch.cuda.synchronize(dev)
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        tf = wl.flops_forward(wl.steady_k()) / t / 1e12
+        res[name] = {"ms_per_forward": round(t * 1e3, 4), "TFLOP/s": round(tf, 2), "workspace_bytes": h.workspace_bytes(),
+                     "status": h.status()}
+        h.close()
+    res["note"] = "e4m3 Q/K with per-tensor scale 2^-4, bf16 V and P; FLOPs counted as for bf16"
     return res
 
 

@@ -31,7 +31,8 @@ class SwAttnConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("tokens_per_chunk", ctypes.c_int), ("W", ctypes.c_int), ("n_cond", ctypes.c_int),
                 ("sink", ctypes.c_int), ("out_dtype", ctypes.c_int), ("scale", ctypes.c_float),
-                ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int), ("commit_in_forward", ctypes.c_int)]
+                ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int), ("commit_in_forward", ctypes.c_int),
+                ("qk_fp8", ctypes.c_int), ("q_scale", ctypes.c_float), ("k_scale", ctypes.c_float)]
 
 
 class SwAttnError(RuntimeError):

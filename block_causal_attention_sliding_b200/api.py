@@ -34,7 +34,7 @@ class SlidingWindowAttention:
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
                  max_short_q: int = 0, schedule: str = "auto", commit_in_forward: bool = False,
-                 device=None):
+                 qk_fp8: bool = False, q_scale: float = 1.0, k_scale: float = 1.0, device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
@@ -42,7 +42,8 @@ class SlidingWindowAttention:
                              scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
                              schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
                                        "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule],
-                             commit_in_forward=int(bool(commit_in_forward)))
+                             commit_in_forward=int(bool(commit_in_forward)), qk_fp8=int(bool(qk_fp8)),
+                             q_scale=float(q_scale), k_scale=float(k_scale))
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()
@@ -51,6 +52,9 @@ class SlidingWindowAttention:
         self.B, self.H, self.d, self.T, self.W, self.n_cond, self.sink = B, H, d, T, W, n_cond, bool(sink)
         # window slots of the ring: W, or W + 1 (a spare slot) with commit_in_forward
         self.R = W + 1 if (commit_in_forward and W > 0) else W
+        # e4m3 queries and keys (FP8 handle), bf16 otherwise; V is always bf16
+        self.qk_fp8 = bool(qk_fp8)
+        self.qk_dtype = torch.float8_e4m3fn if self.qk_fp8 else torch.bfloat16
         self.out_dtype = out_dtype
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         nbytes = int(self._lib.sw_attn_workspace_bytes(h))
@@ -72,7 +76,7 @@ class SlidingWindowAttention:
         for name, t in (("K_cond", K_cond), ("V_cond", V_cond)):
             if tuple(t.shape) != shape:
                 raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
-        N.check(self._lib.sw_attn_set_cond(self._h, _dev_ptr(K_cond, "K_cond", torch.bfloat16),
+        N.check(self._lib.sw_attn_set_cond(self._h, _dev_ptr(K_cond, "K_cond", self.qk_dtype),
                                            _dev_ptr(V_cond, "V_cond", torch.bfloat16), _stream_ptr(stream)))
 
     def append_chunk(self, K: torch.Tensor, V: torch.Tensor, stream=None) -> None:
@@ -80,7 +84,7 @@ class SlidingWindowAttention:
         for name, t in (("K", K), ("V", V)):
             if tuple(t.shape) != shape:
                 raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
-        N.check(self._lib.sw_attn_append_chunk(self._h, _dev_ptr(K, "K", torch.bfloat16),
+        N.check(self._lib.sw_attn_append_chunk(self._h, _dev_ptr(K, "K", self.qk_dtype),
                                                _dev_ptr(V, "V", torch.bfloat16), _stream_ptr(stream)))
 
     def forward(self, Q: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
@@ -96,8 +100,8 @@ class SlidingWindowAttention:
             out = torch.empty((self.B, n_q, self.H, self.d), dtype=self.out_dtype, device=Q.device)
         elif tuple(out.shape) != tuple(Q.shape) or out.dtype != self.out_dtype:
             raise ValueError("out must match Q's shape and the handle's out_dtype")
-        N.check(self._lib.sw_attn_forward(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
-                                          _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+        N.check(self._lib.sw_attn_forward(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
+                                          _dev_ptr(K_cur, "K_cur", self.qk_dtype),
                                           _dev_ptr(V_cur, "V_cur", torch.bfloat16),
                                           _dev_ptr(out, "out"), n_q, _stream_ptr(stream)))
         return out
@@ -116,8 +120,8 @@ class SlidingWindowAttention:
             out = torch.empty(shape, dtype=self.out_dtype, device=Q.device)
         elif tuple(out.shape) != shape or out.dtype != self.out_dtype:
             raise ValueError("out must be [B, T, H, d] in the handle's out_dtype")
-        N.check(self._lib.sw_attn_forward_commit(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
-                                                 _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+        N.check(self._lib.sw_attn_forward_commit(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
+                                                 _dev_ptr(K_cur, "K_cur", self.qk_dtype),
                                                  _dev_ptr(V_cur, "V_cur", torch.bfloat16),
                                                  _dev_ptr(out, "out"), _stream_ptr(stream)))
         return out
@@ -140,9 +144,9 @@ class SlidingWindowAttention:
         for name, t, shp in (("out", out, q_shape), ("out_cond", out_cond, qc_shape)):
             if tuple(t.shape) != shp or t.dtype != self.out_dtype:
                 raise ValueError(f"{name} must be {shp} in the handle's out_dtype")
-        N.check(self._lib.sw_attn_forward_joint(self._h, _dev_ptr(Q, "Q", torch.bfloat16),
-                                                _dev_ptr(Q_cond, "Q_cond", torch.bfloat16),
-                                                _dev_ptr(K_cur, "K_cur", torch.bfloat16),
+        N.check(self._lib.sw_attn_forward_joint(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
+                                                _dev_ptr(Q_cond, "Q_cond", self.qk_dtype),
+                                                _dev_ptr(K_cur, "K_cur", self.qk_dtype),
                                                 _dev_ptr(V_cur, "V_cur", torch.bfloat16),
                                                 _dev_ptr(out, "out"), _dev_ptr(out_cond, "out_cond"),
                                                 _stream_ptr(stream)))
@@ -172,7 +176,8 @@ class SlidingWindowAttention:
         N.check(self._lib.sw_attn_cache_offsets(self._h, ctypes.byref(ko), ctypes.byref(vo)))
         n = 2 * self.B * self.H * S * self.T * self.d
         shape = (self.B, self.H, S, self.T, self.d)
-        kc = self.workspace[ko.value: ko.value + n].view(torch.bfloat16).view(shape)
+        nk = n // 2 if self.qk_fp8 else n
+        kc = self.workspace[ko.value: ko.value + nk].view(self.qk_dtype).view(shape)
         vc = self.workspace[vo.value: vo.value + n].view(torch.bfloat16).view(shape)
         return kc, vc
 
@@ -200,7 +205,7 @@ def append_chunk_batched(handles, Ks, Vs, stream=None) -> None:
             raise ValueError(f"K and V must have shape {shape}")
     lib = handles[0]._lib
     hp = (ctypes.c_void_p * n)(*[h._h.value for h in handles])
-    kp = (ctypes.c_void_p * n)(*[_dev_ptr(K, "K", torch.bfloat16) for K in Ks])
+    kp = (ctypes.c_void_p * n)(*[_dev_ptr(K, "K", h.qk_dtype) for h, K in zip(handles, Ks)])
     vp = (ctypes.c_void_p * n)(*[_dev_ptr(V, "V", torch.bfloat16) for V in Vs])
     N.check(lib.sw_attn_append_chunk_batched(ctypes.cast(hp, ctypes.c_void_p), n, ctypes.cast(kp, ctypes.c_void_p),
                                              ctypes.cast(vp, ctypes.c_void_p), _stream_ptr(stream)))

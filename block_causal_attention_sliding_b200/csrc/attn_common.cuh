@@ -165,15 +165,18 @@ __device__ __forceinline__ QSrc q_src(const AttnParams& p, int u) {
 
 // TMA loads of one 128-row K (kv = 0) or V (kv = 1) tile of key tile j of (b, h) into dst,
 // completing on bar: condition tokens, a ring slot, or the caller's current chunk.
-template <int D>
+template <int D, bool kQK8 = false>
 __device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl* ctl, int j, int kv,
                                              int h, int b, uint32_t dst, uint32_t bar) {
     int seg, row0, valid;
     tile_of(ctl, j, seg, row0, valid);
     const int kind = ctl->seg_kind[seg];
     const int slot = ctl->seg_slot[seg];
+    // an e4m3 K tile is one box of 128-byte rows; V (bf16) keeps its 64-column boxes
+    const int boxes = (kQK8 && kv == 0) ? 1 : TileCfg<D>::kBoxes;
 #pragma unroll
     for (int c = 0; c < TileCfg<D>::kBoxes; ++c) {
+        if (c >= boxes) break;
         const uint32_t d = dst + c * kBoxBytes;
         if (kind == 0)
             tma_load_4d(d, kv ? &p.tm_cond_v : &p.tm_cond_k, bar, c * kBoxCols, row0, h, b);
@@ -254,6 +257,24 @@ struct CommitQueue {
     }
 };
 
+// Bytes of one 128-row Q or K tile: bf16, or e4m3 (one 128-byte swizzle row per token, d = 128).
+template <int D, bool kQK8>
+struct QKTile {
+    static constexpr int kBytes = kQK8 ? kBlockM * D : TileCfg<D>::kTileBytes;
+    static constexpr int kBoxes = kQK8 ? 1 : TileCfg<D>::kBoxes;
+    static constexpr int kBoxCols = kQK8 ? D : swattn::kBoxCols;   // elements per box row
+    static_assert(!kQK8 || D == 128, "e4m3 Q/K tiles need d = 128");
+};
+
+// S = Q K^T with e4m3 Q and K tiles (d = 128, one 128-byte row per token): four K = 32 steps.
+__device__ __forceinline__ void issue_s_f8(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
+    constexpr uint32_t idesc = idesc_e4m3_f32(kBlockM, kBlockN);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+        mma_ss_f8(tS, smem_desc_sw128(q_tile + ks * 32, 16, 1024), smem_desc_sw128(k_tile + ks * 32, 16, 1024), idesc,
+                  ks > 0 ? 1u : 0u);
+}
+
 // S[tS] = Q(q_tile) K(k_tile)^T: M = 128 queries, N = 128 keys, K = D, bf16 -> fp32.
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
@@ -264,6 +285,13 @@ __device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_tile, uint32_t k
         mma_ss(tS, smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
                idesc, ks > 0 ? 1u : 0u);
     }
+}
+
+// S = Q K^T for either operand format.
+template <int D, bool kQK8>
+__device__ __forceinline__ void issue_s_qk(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
+    if constexpr (kQK8) issue_s_f8(tS, q_tile, k_tile);
+    else issue_s<D>(tS, q_tile, k_tile);
 }
 
 // O[tO] (+)= P[tP] V(v_tile): P (bf16 pairs in TMEM) is the A operand, V is MN-major in shared

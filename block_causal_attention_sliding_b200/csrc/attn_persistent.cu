@@ -23,7 +23,8 @@ namespace swattn {
 
 // kCommit: the launch also stores the chunk's K_cur / V_cur into the cache (fused commit); a
 // separate instantiation, so the plain forward carries none of that code.
-template <int D, bool kCommit>
+// kQK8: Q and K are e4m3 (d = 128), S = Q K^T on kind::f8f6f4; V, P and O as in the bf16 kernel.
+template <int D, bool kCommit, bool kQK8>
 __global__ void __launch_bounds__(AttnLayout<D, 2>::kThreads, 1)
 attn_persistent_kernel(const __grid_constant__ AttnParams p) {
     constexpr int NQ = 2;
@@ -86,12 +87,12 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 const int b = pc.bh / p.H, h = pc.bh % p.H;
                 // the Q buffers are reused: wait until every S MMA of the previous piece is done
                 if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(qbar, pc.live * kTileBytes);
+                mbar_arrive_expect_tx(qbar, pc.live * QKTile<D, kQK8>::kBytes);
                 for (int qt = 0; qt < pc.live; ++qt) {
                     const QSrc qs = q_src(p, pc.pair * NQ + qt);
-                    for (int c = 0; c < C::kBoxes; ++c)
+                    for (int c = 0; c < QKTile<D, kQK8>::kBoxes; ++c)
                         tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), qs.tm, qbar,
-                                    c * kBoxCols, h, qs.row0, b);
+                                    c * QKTile<D, kQK8>::kBoxCols, h, qs.row0, b);
                 }
                 ++pi;
                 for (int j = pc.j0; j < pc.j1 && ok; ++j) {
@@ -104,8 +105,8 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                         }
                         if (kCommit) cq.before_refill(s);
                         const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
-                        mbar_arrive_expect_tx(fbar, kTileBytes);
-                        load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                        mbar_arrive_expect_tx(fbar, kv == 0 ? QKTile<D, kQK8>::kBytes : kTileBytes);
+                        load_kv_tile<D, kQK8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
                         if (kCommit) {
                             const bool mine = cslot >= 0 && pc.pair == j % sched.npairs &&
                                               ctl->seg_kind[tile_seg(ctl, j)] == 2;
@@ -151,7 +152,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 if (!wait_or_abort(smem_u32(&ctl->kv_full[s0]), (it / kStages) & 1, abort_flag)) break;
                 tc_fence_after();
                 for (int qt = 0; qt < live; ++qt) {
-                    issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + s0 * kTileBytes);
+                    issue_s_qk<D, kQK8>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + s0 * kTileBytes);
                     mma_commit(smem_u32(&ctl->s_full[qt]));
                 }
                 if (n == 1) mma_commit(smem_u32(&ctl->q_empty));
@@ -200,7 +201,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                                 break;
                             }
                             // in issue order after the PV that reads P_q from the same columns
-                            issue_s<D>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
+                            issue_s_qk<D, kQK8>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
                             mma_commit(smem_u32(&ctl->s_full[qt]));
                         }
                     }
@@ -354,7 +355,10 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 template <int D>
 static cudaError_t launch_persistent_d(const AttnParams& p, int ctas, cudaStream_t stream) {
     using L = AttnLayout<D, 2>;
-    auto kern = p.commit ? attn_persistent_kernel<D, true> : attn_persistent_kernel<D, false>;
+    auto kern = p.commit ? attn_persistent_kernel<D, true, false> : attn_persistent_kernel<D, false, false>;
+    if constexpr (D == 128) {
+        if (p.qk_fp8) kern = attn_persistent_kernel<D, false, true>;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     kern<<<ctas, L::kThreads, L::kSmemBytes, stream>>>(p);

@@ -81,8 +81,8 @@ cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_con
 // destination rows.  No division in the copy loop (vpr is a power of two).
 __device__ __forceinline__ void relayout_row(const uint4* __restrict__ srcK, const uint4* __restrict__ srcV,
                                              uint4* __restrict__ dstK, uint4* __restrict__ dstV, int N, int H,
-                                             int vpr_log2, int rows_per_bh, int ring, int R, int sink, int S,
-                                             int32_t* state) {
+                                             int vpr_log2_k, int vpr_log2_v, int rows_per_bh, int ring, int R,
+                                             int sink, int S, int32_t* state) {
     int slot = 0;
     if (ring) {
         slot = ring_slot(state[0], R, sink);
@@ -95,6 +95,7 @@ __device__ __forceinline__ void relayout_row(const uint4* __restrict__ srcK, con
     }
     const uint4* __restrict__ src = blockIdx.y == 0 ? srcK : srcV;
     uint4* __restrict__ dst = blockIdx.y == 0 ? dstK : dstV;
+    const int vpr_log2 = blockIdx.y == 0 ? vpr_log2_k : vpr_log2_v;   // K may be e4m3 (half the bytes)
     const int row = blockIdx.x;                     // b * N + t
     const int b = row / N, t = row - b * N;
     const int vpr = 1 << vpr_log2;
@@ -111,18 +112,19 @@ __global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__
                                                        const uint4* __restrict__ srcV,
                                                        uint4* __restrict__ dstK,
                                                        uint4* __restrict__ dstV, int N, int H,
-                                                       int vpr_log2, int rows_per_bh, int ring,
+                                                       int vpr_log2_k, int vpr_log2_v, int rows_per_bh, int ring,
                                                        int R, int sink, int S, int32_t* state) {
-    relayout_row(srcK, srcV, dstK, dstV, N, H, vpr_log2, rows_per_bh, ring, R, sink, S, state);
+    relayout_row(srcK, srcV, dstK, dstV, N, H, vpr_log2_k, vpr_log2_v, rows_per_bh, ring, R, sink, S, state);
 }
 
 // Batched commit: blockIdx.z selects the handle; each copies into its own ring slot (from its
 // own counter), exactly as relayout_kernel does for one handle.
 __global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_constant__ AppendBatch a, int N, int H,
-                                                             int vpr_log2, int T) {
+                                                             int vpr_log2_k, int vpr_log2_v, int T) {
     const int l = blockIdx.z;
     relayout_row(static_cast<const uint4*>(a.K[l]), static_cast<const uint4*>(a.V[l]), static_cast<uint4*>(a.dstK[l]),
-                 static_cast<uint4*>(a.dstV[l]), N, H, vpr_log2, a.S[l] * T, 1, a.R[l], a.sink[l], a.S[l], a.state[l]);
+                 static_cast<uint4*>(a.dstV[l]), N, H, vpr_log2_k, vpr_log2_v, a.S[l] * T, 1, a.R[l], a.sink[l], a.S[l],
+                 a.state[l]);
 }
 
 // Batched table advance: block l advances handle l's counter and rebuilds its table.
@@ -132,18 +134,26 @@ __global__ void table_build_batch_kernel(const __grid_constant__ AppendBatch a, 
     build_table(a.state[l], a.W[l], a.R[l], a.sink[l], a.n_cond[l], T, 1, 0);
 }
 
-cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, cudaStream_t stream) {
+// 16-byte vectors per head row of d elements of esz bytes, as a power of two (-1: not one).
+static int vpr_log2_of(int d, int esz) {
+    const int vpr = d * esz / 16;
+    int l = 0;
+    while ((1 << l) < vpr) ++l;
+    return (vpr >= 1 && (1 << l) == vpr) ? l : -1;
+}
+
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, cudaStream_t stream) {
     if (a.n < 1 || a.n > kMaxBatch) return cudaErrorInvalidValue;
-    const int vpr = d / 8;
-    int vpr_log2 = 0;
-    while ((1 << vpr_log2) < vpr) ++vpr_log2;
-    if ((1 << vpr_log2) != vpr) return cudaErrorInvalidValue;
+    const int vpr_log2 = vpr_log2_of(d, 2), vpr_log2_k = vpr_log2_of(d, k_esz);
+    if (vpr_log2 < 0 || vpr_log2_k < 0) return cudaErrorInvalidValue;
+    const int vpr = 1 << vpr_log2;
     const long long rows = (long long)B * T;
     if (rows < 1 || rows > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int per_row = H * vpr;
     const int threads = per_row >= 512 ? 512 : ((per_row + 31) / 32) * 32;
     // handles without a ring (S = 0) return at once inside the kernel (slot -1)
-    relayout_batch_kernel<<<dim3((unsigned)rows, 2, (unsigned)a.n), threads, 0, stream>>>(a, T, H, vpr_log2, T);
+    relayout_batch_kernel<<<dim3((unsigned)rows, 2, (unsigned)a.n), threads, 0, stream>>>(a, T, H, vpr_log2_k, vpr_log2,
+                                                                                           T);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     table_build_batch_kernel<<<a.n, 32, 0, stream>>>(a, T);
@@ -152,11 +162,10 @@ cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d
 
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
-                            int32_t* state, cudaStream_t stream) {
-    const int vpr = d / 8;                          // 16-byte vectors per head row
-    int vpr_log2 = 0;
-    while ((1 << vpr_log2) < vpr) ++vpr_log2;
-    if ((1 << vpr_log2) != vpr) return cudaErrorInvalidValue;   // d is 64 or 128
+                            int32_t* state, cudaStream_t stream, int k_esz) {
+    const int vpr_log2 = vpr_log2_of(d, 2), vpr_log2_k = vpr_log2_of(d, k_esz);   // 16-byte vectors per row
+    if (vpr_log2 < 0 || vpr_log2_k < 0) return cudaErrorInvalidValue;              // d is 64 or 128
+    const int vpr = 1 << vpr_log2;
     const long long rows = (long long)B * N;
     if (rows < 1) return cudaSuccess;
     if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -165,7 +174,7 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
     dim3 grid((unsigned)rows, 2);
     relayout_kernel<<<grid, threads, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
-        static_cast<uint4*>(dstV), N, H, vpr_log2, rows_per_bh, ring, R, sink, S, state);
+        static_cast<uint4*>(dstV), N, H, vpr_log2_k, vpr_log2, rows_per_bh, ring, R, sink, S, state);
     return cudaGetLastError();
 }
 

@@ -72,13 +72,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// bf16 tiled map, 128-byte swizzle, boxes of 64 columns; out-of-range rows read as zero.
+// Tiled map with 128-byte swizzle and 128-byte box rows (64 bf16 or 128 e4m3 columns, esz = 2
+// or 1 bytes per element); out-of-range rows read as zero.
 int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-           const uint32_t* box, const char* what) {
+           const uint32_t* box, const char* what, int esz = 2) {
     auto fn = encode_fn();
     if (!fn) return fail(SW_ECUDA, "cuTensorMapEncodeTiled unavailable");
     uint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr),
+    CUresult r = fn(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                    const_cast<void*>(ptr),
                     reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides),
                     reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -87,12 +89,12 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, cons
     return SW_OK;
 }
 
-// user layout [B, N, H, d]: dims {d, H, N, B}; box 64 x 1 x 128 x 1 (128 rows of one head)
-int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, const char* what) {
+// user layout [B, N, H, d]: dims {d, H, N, B}; box (128 bytes) x 1 x 128 x 1 (128 rows of one head)
+int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, const char* what, int esz = 2) {
     const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)N, (uint64_t)B};
-    const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)N * H * d * 2};
-    const uint32_t box[4] = {64, 1, (uint32_t)kBlockN, 1};
-    return encode(m, ptr, 4, dims, strides, box, what);
+    const uint64_t strides[3] = {(uint64_t)d * esz, (uint64_t)H * d * esz, (uint64_t)N * H * d * esz};
+    const uint32_t box[4] = {(uint32_t)(128 / esz), 1, (uint32_t)kBlockN, 1};
+    return encode(m, ptr, 4, dims, strides, box, what, esz);
 }
 
 int check_cfg(const sw_attn_config& c) {
@@ -109,6 +111,10 @@ int check_cfg(const sw_attn_config& c) {
         c.schedule != SW_SCHED_AUTO)
         return fail(SW_EINVAL, "bad schedule");
     if (c.commit_in_forward != 0 && c.commit_in_forward != 1) return fail(SW_EINVAL, "commit_in_forward must be 0 or 1");
+    if (c.qk_fp8 != 0 && c.qk_fp8 != 1) return fail(SW_EINVAL, "qk_fp8 must be 0 or 1");
+    if (c.qk_fp8 && c.d != 128) return fail(SW_ESHAPE, "e4m3 Q/K need d = 128");
+    if (c.qk_fp8 && c.commit_in_forward) return fail(SW_ESHAPE, "commit_in_forward is not available with e4m3 Q/K");
+    if (!std::isfinite(c.q_scale) || !std::isfinite(c.k_scale)) return fail(SW_EINVAL, "scales must be finite");
     const double elems = (double)c.B * c.H * (c.W + 2) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
         (double)c.n_cond * c.H * c.B > 2.0e9)
@@ -133,6 +139,9 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->cfg = *cfg;
     if (h->cfg.scale <= 0.f) h->cfg.scale = 1.0f / std::sqrt((float)cfg->d);
     h->short_q = cfg->max_short_q == 0 ? kMaxShortQ : (cfg->max_short_q < 0 ? 0 : cfg->max_short_q);
+    if (cfg->qk_fp8) h->short_q = 0;   // e4m3 Q/K run on the persistent kernel only
+    if (h->cfg.q_scale <= 0.f) h->cfg.q_scale = 1.f;
+    if (h->cfg.k_scale <= 0.f) h->cfg.k_scale = 1.f;
     // window slots: W, or W + 1 to keep a spare slot for commits during the chunk's own forward
     h->R = cfg->commit_in_forward && cfg->W > 0 ? cfg->W + 1 : cfg->W;
     h->S = h->R + (cfg->sink ? 1 : 0);
@@ -141,9 +150,10 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->max_splits = std::max(1, std::min(kMaxSplits, (148 + bh - 1) / bh));   // B200: 148 SMs
     const size_t B = cfg->B, H = cfg->H, d = cfg->d, T = cfg->tokens_per_chunk;
     size_t off = align_up(sizeof(int32_t) * (kStateHeaderInts + h->table_ints), 1024);
-    h->off_kcache = off; off = align_up(off + B * H * h->S * T * d * 2, 1024);
+    const size_t ek = cfg->qk_fp8 ? 1 : 2;   // bytes per K element (e4m3 on an FP8 handle)
+    h->off_kcache = off; off = align_up(off + B * H * h->S * T * d * ek, 1024);
     h->off_vcache = off; off = align_up(off + B * H * h->S * T * d * 2, 1024);
-    h->off_kcond = off;  off = align_up(off + B * H * cfg->n_cond * d * 2, 1024);
+    h->off_kcond = off;  off = align_up(off + B * H * cfg->n_cond * d * ek, 1024);
     h->off_vcond = off;  off = align_up(off + B * H * cfg->n_cond * d * 2, 1024);
     h->off_opart = off;
     if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * d * 4, 1024);
@@ -167,6 +177,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
     c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_AUTO;
     c.commit_in_forward = 0;
+    c.qk_fp8 = 0; c.q_scale = 0.f; c.k_scale = 0.f;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -198,7 +209,12 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint64_t strides[4] = {row, row * c.tokens_per_chunk, row * c.tokens_per_chunk * h->S,
                                      row * c.tokens_per_chunk * h->S * c.H};
         const uint32_t box[5] = {64, (uint32_t)kBlockN, 1, 1, 1};
-        if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, strides, box, "K cache"))) return rc;
+        const int ek = c.qk_fp8 ? 1 : 2;   // K in e4m3 on an FP8 handle
+        const uint64_t rowk = (uint64_t)c.d * ek;
+        const uint64_t stridesk[4] = {rowk, rowk * c.tokens_per_chunk, rowk * c.tokens_per_chunk * h->S,
+                                      rowk * c.tokens_per_chunk * h->S * c.H};
+        const uint32_t boxk[5] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1, 1};
+        if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, stridesk, boxk, "K cache", ek))) return rc;
         if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, strides, box, "V cache"))) return rc;
     }
     if (c.n_cond > 0) {
@@ -206,7 +222,11 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint64_t row = (uint64_t)c.d * 2;
         const uint64_t strides[3] = {row, row * c.n_cond, row * c.n_cond * c.H};
         const uint32_t box[4] = {64, (uint32_t)kBlockN, 1, 1};
-        if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, strides, box, "K cond"))) return rc;
+        const int ek = c.qk_fp8 ? 1 : 2;
+        const uint64_t rowk = (uint64_t)c.d * ek;
+        const uint64_t stridesk[3] = {rowk, rowk * c.n_cond, rowk * c.n_cond * c.H};
+        const uint32_t boxk[4] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1};
+        if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, stridesk, boxk, "K cond", ek))) return rc;
         if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, strides, box, "V cond"))) return rc;
     }
     e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk,
@@ -242,7 +262,7 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
     if (!aligned16(K_cond) || !aligned16(V_cond)) return fail(SW_EALIGN, "condition tensors must be 16-byte aligned");
     cudaError_t e = launch_relayout(K_cond, V_cond, h->ws + h->off_kcond, h->ws + h->off_vcond, c.B, c.n_cond,
                                     c.H, c.d, c.n_cond, 0, h->R, c.sink, h->S, reinterpret_cast<int32_t*>(h->ws),
-                                    static_cast<cudaStream_t>(stream));
+                                    static_cast<cudaStream_t>(stream), c.qk_fp8 ? 1 : 2);
     if (e != cudaSuccess) return cuda_fail(e, "condition copy launch");
     h->cond_set = true;
     return SW_OK;
@@ -260,7 +280,7 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     cudaError_t e;
     if (h->S > 0) {
         e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
-                            h->S * c.tokens_per_chunk, 1, h->R, c.sink, h->S, state, st);
+                            h->S * c.tokens_per_chunk, 1, h->R, c.sink, h->S, state, st, c.qk_fp8 ? 1 : 2);
         if (e != cudaSuccess) return cuda_fail(e, "append launch");
     }
     e = launch_table_build(state, c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
@@ -271,6 +291,7 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
 // tiles than SMs, the three-buffer kernel (one tile per unit balances better); else persistent.
 static int resolve_schedule_tiles(const sw_attn_t* h, long long nqt) {
     const sw_attn_config& c = h->cfg;
+    if (c.qk_fp8) return SW_SCHED_PERSISTENT;   // the one kernel with an e4m3 Q/K form
     if (c.schedule != SW_SCHED_AUTO) return c.schedule;
     const long long pairs = (long long)c.B * c.H * ((nqt + 1) / 2);
     return pairs < h->num_sms ? SW_SCHED_TRI : SW_SCHED_PERSISTENT;
@@ -292,8 +313,9 @@ static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const v
     const sw_attn_config& c = h->cfg;
     std::memset(&p, 0, sizeof p);
     int rc;
-    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q"))) return rc;
-    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur"))) return rc;
+    const int eqk = c.qk_fp8 ? 1 : 2;
+    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q", eqk))) return rc;
+    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur", eqk))) return rc;
     if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
     // maps for regions this handle does not have are never read; fill them with a valid map
     p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
@@ -311,10 +333,12 @@ static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const v
     p.n_q = n_q;
     p.n_qc = 0;
     p.commit = 0;
+    p.qk_fp8 = c.qk_fp8;
     p.ring_R = h->R;
     p.sink = c.sink;
     p.out_f32 = c.out_dtype == SW_OUT_F32;
-    p.scale_log2 = c.scale * 1.4426950408889634f;
+    // e4m3 Q and K: S = (q * q_scale) . (k * k_scale), the scales folded into the softmax scale
+    p.scale_log2 = c.scale * 1.4426950408889634f * (c.qk_fp8 ? c.q_scale * c.k_scale : 1.f);
     return SW_OK;
 }
 
@@ -396,8 +420,9 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
         if (!h->ws) return fail(SW_ESTATE, "handle %d has no workspace bound", l);
         if (h->device != h0->device) return fail(SW_ESTATE, "handle %d is on another device", l);
         const sw_attn_config& c = h->cfg;
-        if (c.B != c0.B || c.H != c0.H || c.d != c0.d || c.tokens_per_chunk != c0.tokens_per_chunk)
-            return fail(SW_ESHAPE, "handle %d: B, H, d and T must match handle 0", l);
+        if (c.B != c0.B || c.H != c0.H || c.d != c0.d || c.tokens_per_chunk != c0.tokens_per_chunk ||
+            c.qk_fp8 != c0.qk_fp8)
+            return fail(SW_ESHAPE, "handle %d: B, H, d, T and the K format must match handle 0", l);
         if (!K[l] || !V[l]) return fail(SW_EINVAL, "null K or V for handle %d", l);
         if (!aligned16(K[l]) || !aligned16(V[l])) return fail(SW_EALIGN, "K and V of handle %d must be 16-byte aligned", l);
         for (int m = 0; m < l; ++m)
@@ -421,7 +446,7 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
             a.sink[q] = h->cfg.sink;
             a.n_cond[q] = h->cfg.n_cond;
         }
-        cudaError_t e = launch_append_batch(a, c0.B, c0.tokens_per_chunk, c0.H, c0.d, st);
+        cudaError_t e = launch_append_batch(a, c0.B, c0.tokens_per_chunk, c0.H, c0.d, c0.qk_fp8 ? 1 : 2, st);
         if (e != cudaSuccess) return cuda_fail(e, "batched append launch");
     }
     return SW_OK;
@@ -435,6 +460,7 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     const sw_attn_config& c = h->cfg;
     if (!c.commit_in_forward) return fail(SW_ESTATE, "the handle was not created with commit_in_forward");
+    if (c.qk_fp8) return fail(SW_ESTATE, "no committing forward with e4m3 Q/K");
     if (c.B > 32767 || c.H > 65535) return fail(SW_ESHAPE, "a committing forward supports B <= 32767, H <= 65535");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
@@ -478,7 +504,7 @@ int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const
     AttnParams p;
     int rc;
     if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, c.tokens_per_chunk))) return rc;
-    if ((rc = encode_user(&p.tm_qc, Q_cond, c.B, c.n_cond, c.H, c.d, "Q_cond"))) return rc;
+    if ((rc = encode_user(&p.tm_qc, Q_cond, c.B, c.n_cond, c.H, c.d, "Q_cond", c.qk_fp8 ? 1 : 2))) return rc;
     p.out_c = out_cond;
     p.n_qc = c.n_cond;
     return launch_full(h, p, static_cast<cudaStream_t>(stream));

@@ -56,6 +56,7 @@ struct alignas(64) AttnParams {
     int B, H, n_q;
     int n_qc;                // condition-stream query rows (0: none); their Q tiles follow the chunk's
     int commit;              // 1: also store K_cur / V_cur into the ring slot of the active chunk
+    int qk_fp8;              // 1: Q and K (current, cache, condition) are e4m3, scales folded into scale_log2
     int ring_R;              // window slots of the ring (for the commit slot)
     int sink;
     int out_f32;
@@ -77,7 +78,7 @@ cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_con
 // slot * N (slot from the device counter when `ring` is set, else 0).
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
-                            int32_t* state, cudaStream_t stream);
+                            int32_t* state, cudaStream_t stream, int k_esz = 2);
 // One chunk commit for each of up to kMaxBatch handles (layers) of the same B, T, H, d, in one
 // copy launch and one table launch (the per-handle window, sink, slots and counter stay apart).
 constexpr int kMaxBatch = 32;
@@ -90,7 +91,7 @@ struct AppendBatch {
     int R[kMaxBatch], S[kMaxBatch], W[kMaxBatch], sink[kMaxBatch], n_cond[kMaxBatch];
     int n;                       // handles in this launch
 };
-cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, cudaStream_t stream);
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, cudaStream_t stream);
 
 cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
                              cudaStream_t stream);

@@ -12,6 +12,9 @@ bf16 inputs.  Recipe (stated once, used everywhere):
     queries = 5; condition K/V use chunk 0, step 0 for the first prompt and chunk v, step 0 for
     prompt version v (a prompt changed mid-stream); condition queries use the (chunk, step) of
     the forward they belong to.
+  * FP8 inputs (queries and keys of an e4m3 handle): the same draws divided by a power-of-two
+    scale (FP8_SCALE, exact) and rounded to OCP e4m3 (float8_e4m3fn, round to nearest even);
+    the dequantised values x8 * FP8_SCALE are what the attention sees.
 The user layout is [B, N, H, d] contiguous.
 """
 from __future__ import annotations
@@ -63,3 +66,28 @@ def cond_inputs(wl, *, seed: int = 0, version: int = 0, device="cpu"):
 def cond_queries(wl, chunk: int, step: int, *, seed: int = 0, device="cpu"):
     """Condition-stream queries Q_cond [B, n_cond, H, d] for one (chunk, step)."""
     return draw((wl.B, wl.n_cond, wl.H, wl.d), stream_seed(seed, chunk, step, TID_QC), device=device)
+
+
+FP8_SCALE = 2.0 ** -4   # |x| / FP8_SCALE stays below the e4m3 limit (448) even for sigma-4 outlier keys
+
+
+def to_e4m3(x: torch.Tensor, scale: float = FP8_SCALE) -> torch.Tensor:
+    """x / scale rounded to e4m3 (scale a power of two, so the division is exact)."""
+    return (x.float() / scale).to(torch.float8_e4m3fn)
+
+
+def from_e4m3(x8: torch.Tensor, scale: float = FP8_SCALE) -> torch.Tensor:
+    """The dequantised values x8 * scale, exact in float32."""
+    return x8.float() * scale
+
+
+def chunk_inputs_fp8(wl, chunk: int, step: int, *, seed: int = 0, device="cpu"):
+    """Q and K_cur in e4m3, V_cur in bf16, for one (chunk, step) of an e4m3 handle."""
+    Q, K, V = chunk_inputs(wl, chunk, step, seed=seed, device=device)
+    return to_e4m3(Q), to_e4m3(K), V
+
+
+def cond_inputs_fp8(wl, *, seed: int = 0, version: int = 0, device="cpu"):
+    """Condition K in e4m3, V in bf16."""
+    Kc, Vc = cond_inputs(wl, seed=seed, version=version, device=device)
+    return to_e4m3(Kc), Vc

@@ -83,6 +83,14 @@ typedef struct {
     int   commit_in_forward; /* 1: keep one spare window slot (W + 1 in all) so that
                                 sw_attn_forward_commit can write the chunk's K/V into the cache
                                 while its own forward runs; 0 (default): W window slots */
+    int   qk_fp8;            /* 1: queries and keys are e4m3 (OCP FP8, 1 byte per element): Q,
+                                Q_cond, K_cur, the appended K and K_cond are e4m3 tensors of
+                                the same [B, N, H, d] shape, the K cache is kept in e4m3 (half
+                                the bytes) and S = Q K^T runs on kind::f8f6f4; V stays bf16.
+                                Requires d = 128; full path on the persistent schedule only
+                                (no split-K path, no commit_in_forward) */
+    float q_scale, k_scale;  /* dequantisation scales of the e4m3 Q and K (per tensor; <= 0
+                                selects 1): the attention uses q * q_scale and k * k_scale */
 } sw_attn_config;
 
 /* schedules of the full path */

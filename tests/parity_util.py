@@ -220,3 +220,53 @@ def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, 
     torch.cuda.synchronize()
     assert h.status() == 0, f"device status {h.status():#x}"
     return results
+
+
+def stream_and_check_fp8(wl, dev, *, chunks, check_at=None, n_rows=None, keep_last=None,
+                         gen_on_device=False, out_dtype=torch.float32, seed=0, joint=False,
+                         tol=(MAX_ABS, MEAN_REL)):
+    """Stream through a handle with e4m3 queries and keys (V bf16): 2 forwards then an append
+    per chunk, all Q/K in e4m3 with scale FP8_SCALE.  The oracle computes the same attention on
+    the dequantised values (exact in float32).  With joint, the forward also carries e4m3
+    condition queries.  Returns a list of (k, step, which, max_abs, mean_rel)."""
+    sc = synth.FP8_SCALE
+    h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                               out_dtype=out_dtype, qk_fp8=True, q_scale=sc, k_scale=sc, device=dev)
+    gdev = dev if gen_on_device else "cpu"
+    Kc8, Vc = synth.cond_inputs_fp8(wl, seed=seed, device=gdev)
+    h.set_cond(Kc8.to(dev), Vc.to(dev))
+    Kc = synth.from_e4m3(Kc8).cpu()
+    Vc = Vc.cpu()
+    hist_K, hist_V, results = [], [], []
+    for k in range(chunks):
+        for step in range(wl.steps):
+            Q8, K8, V = synth.chunk_inputs_fp8(wl, k, step, seed=seed, device=gdev)
+            if joint:
+                Qc8 = synth.to_e4m3(synth.cond_queries(wl, k, step, seed=seed, device=gdev))
+                out, out_c = h.forward_joint(Q8.to(dev), Qc8.to(dev), K8.to(dev), V.to(dev))
+                sets = (("chunk", Q8, out, wl.T), ("cond", Qc8, out_c, wl.n_cond))
+            else:
+                out = h.forward(Q8.to(dev), K8.to(dev), V.to(dev))
+                sets = (("chunk", Q8, out, wl.T),)
+            if check_at is None or k in check_at:
+                for which, q8, o, n in sets:
+                    r = None if n_rows is None else sample_rows(n, n_rows, seed=1000 * k + step)
+                    ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
+                                           k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V,
+                                           Q=synth.from_e4m3(q8).cpu(), K_cur=synth.from_e4m3(K8).cpu(),
+                                           V_cur=V.cpu(), rows=r)
+                    got = o.float().cpu().numpy()
+                    if r is not None:
+                        got = got[:, r]
+                    ma, mr = compare(got, ref, *tol)
+                    results.append((k, step, which, ma, mr))
+        h.append_chunk(K8.to(dev), V.to(dev))
+        hist_K.append(synth.from_e4m3(K8).cpu())
+        hist_V.append(V.cpu())
+        if keep_last is not None:
+            for c in range(1, max(1, len(hist_K) - keep_last)):
+                hist_K[c] = None
+                hist_V[c] = None
+    torch.cuda.synchronize()
+    assert h.status() == 0, f"device status {h.status():#x}"
+    return results

@@ -18,7 +18,7 @@ from block_causal_attention_sliding_b200 import synth
 from block_causal_attention_sliding_b200.configs import WORKLOADS, Workload
 
 from parity_util import (compare, make_handle, stream_and_check, stream_and_check_commit,
-                         stream_and_check_joint)
+                         stream_and_check_fp8, stream_and_check_joint)
 
 pytestmark = pytest.mark.gpu
 
@@ -412,6 +412,52 @@ def test_chunk_step_graph_capture(dev):
     ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink, k=k, Kc=Kc, Vc=Vc,
                            hist_K=[t[1] for t in hist], hist_V=[t[2] for t in hist], Q=Q, K_cur=K, V_cur=V)
     compare(eager_out[k][0][-1].cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------------ e4m3 queries and keys
+
+@pytest.mark.parametrize("W,sink,n_cond", [(2, True, 40), (1, False, 130), (0, True, 0)])
+def test_fp8_qk_ragged(dev, W, sink, n_cond):
+    """e4m3 Q and K (S on kind::f8f6f4, e4m3 K cache), bf16 V: every chunk and step, all rows,
+    against the oracle on the dequantised inputs."""
+    wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks)
+    assert len(res) == wl.chunks * wl.steps
+
+
+def test_fp8_qk_joint(dev):
+    """e4m3 chunk and condition queries in one joint launch."""
+    wl = dataclasses.replace(RAGGED, n_cond=130, chunks=4)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True)
+    assert len(res) == 2 * wl.chunks * wl.steps
+
+
+def test_fp8_qk_cache_bytes(dev):
+    """The e4m3 K cache holds exactly the appended e4m3 keys (bit for bit) at half the bytes."""
+    wl = dataclasses.replace(RAGGED, chunks=3)
+    sc = synth.FP8_SCALE
+    h = make_handle(wl, dev)
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    h8 = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                qk_fp8=True, q_scale=sc, k_scale=sc, device=dev)
+    assert h8.workspace_bytes() < h.workspace_bytes()
+    kc, vc = h8.cache_views()
+    for c in range(wl.chunks):
+        _, K8, V = synth.chunk_inputs_fp8(wl, c, 1)
+        h8.append_chunk(K8.to(dev), V.to(dev))
+        torch.cuda.synchronize()
+        s_ = oracle.slot(c, wl.W, wl.sink)
+        assert torch.equal(kc[:, :, s_].cpu().view(torch.uint8), K8.permute(0, 2, 1, 3).contiguous().view(torch.uint8))
+        assert torch.equal(vc[:, :, s_].cpu().view(torch.int16), V.permute(0, 2, 1, 3).contiguous().view(torch.int16))
+    assert h8.status() == 0
+
+
+def test_fp8_qk_720p_sampled(dev):
+    """720p with e4m3 Q and K: sampled rows at chunks 0, W + 1 and the last of 7."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_fp8(wl, dev, chunks=7, check_at={0, 4, 6}, n_rows=32, keep_last=wl.W + 1,
+                               gen_on_device=True)
+    assert len(res) == 6
 
 
 def test_long_horizon_constant_memory(dev):
