@@ -392,7 +392,12 @@ template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
                                                       const float* __restrict__ ml_part, void* out,
                                                       int B, int H, int n_q, int splits, int out_f32) {
+    // one warp per output row; each lane owns D / 32 consecutive columns.  The splits are read
+    // eight at a time with every load of a group issued before any is used (one memory round
+    // trip per group), and merged with a running max like the online softmax.
     constexpr int V = D / 32;
+    constexpr int G = 8;
+    static_assert(V == 4 || V == 2, "d = 128 or 64");
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int total = B * H * n_q;
@@ -401,22 +406,51 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     const int bh = warp / n_q;
     const int b = bh / H, h = bh % H;
     const size_t stride_split = (size_t)B * H * kBlockM;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s)
-        M = fmaxf(M, ml_part[((size_t)s * stride_split + (size_t)bh * kBlockM + row) * 2]);
+    const size_t row0 = (size_t)bh * kBlockM + row;
+    float M = -INFINITY, den = 0.f;
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-    float den = 0.f;
-    for (int s = 0; s < splits; ++s) {
-        const size_t prow = (size_t)s * stride_split + (size_t)bh * kBlockM + row;
-        const float ms = ml_part[prow * 2];
-        if (ms == -INFINITY) continue;            // empty slice
-        const float w = ex2_approx(ms - M);
-        den += w * ml_part[prow * 2 + 1];
-        const float* src = o_part + prow * D + lane * V;
+    for (int s0 = 0; s0 < splits; s0 += G) {
+        float2 ml[G];
+        float o[G][V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] += w * src[i];
+        for (int g = 0; g < G; ++g) {
+            const int s = s0 + g;
+            if (s < splits) {
+                const size_t prow = (size_t)s * stride_split + row0;
+                ml[g] = __ldg(reinterpret_cast<const float2*>(ml_part) + prow);
+                const float* src = o_part + prow * D + lane * V;
+                if (V == 4) {
+                    const float4 t = __ldg(reinterpret_cast<const float4*>(src));
+                    o[g][0] = t.x; o[g][1] = t.y; o[g][V > 2 ? 2 : 0] = t.z; o[g][V > 3 ? 3 : 0] = t.w;
+                } else {
+                    const float2 t = __ldg(reinterpret_cast<const float2*>(src));
+                    o[g][0] = t.x; o[g][1] = t.y;
+                }
+            } else {
+                ml[g] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int i = 0; i < V; ++i) o[g][i] = 0.f;
+            }
+        }
+        float Mg = M;
+#pragma unroll
+        for (int g = 0; g < G; ++g) Mg = fmaxf(Mg, ml[g].x);
+        if (Mg == -INFINITY) continue;                 // every slice so far is empty
+        const float f = ex2_approx(M - Mg);            // 0 while nothing has been merged
+        den *= f;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] *= f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            if (ml[g].x == -INFINITY) continue;        // empty slice (or past the last split)
+            const float w = ex2_approx(ml[g].x - Mg);
+            den += w * ml[g].y;
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[i] += w * o[g][i];
+        }
+        M = Mg;
     }
     const float inv = 1.f / den;
     const size_t orow = ((size_t)b * n_q + row) * H + h;
