@@ -327,9 +327,14 @@ __device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t
 // (the PV of those keys may then start) and the caller arrives on p_full after the return.
 // A warp that must rescale O first publishes nothing early: its O rescale has to land before
 // any PV of this tile.  The caller has waited for S.
-template <int D>
+// kWaitO: S was computed ahead of the previous tile's PV (double-buffered S), so before an O
+// rescale the warp waits for that PV on o_bar (phase parity o_parity).  Without it, the
+// previous PV is known complete (it was issued before this tile's S).
+template <int D, bool kWaitO = false>
 __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
-                                             uint32_t p_half_bar, float sl2, float& m_ref, float& l) {
+                                             uint32_t p_half_bar, float sl2, float& m_ref, float& l,
+                                             uint32_t o_bar = 0, uint32_t o_parity = 0,
+                                             volatile int* flag = nullptr) {
     uint32_t sr[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
@@ -420,7 +425,9 @@ __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid
         // done once the S row is dead (low register pressure); it must land before this
         // tile's PV, which waits for p_half (arrived below) and p_full.  The previous PV into
         // O has completed: it was issued before this tile's S, whose completion the caller
-        // has waited for, and the tensor pipe completes one thread's MMAs in issue order.
+        // has waited for, and the tensor pipe completes one thread's MMAs in issue order --
+        // or, with kWaitO, the wait below has seen it complete.
+        if constexpr (kWaitO) (void)warp_wait(o_bar, o_parity, flag);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];

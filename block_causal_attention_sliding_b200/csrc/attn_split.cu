@@ -1,0 +1,277 @@
+// attn_split.cu -- split-K attention for short query sets (n_q <= 128 queries of the active
+// chunk over the whole visible key set), sm_100a.
+//
+// The same result as the chunk forward -- softmax(scale * Q K^T) V over the keys the
+// visibility table lists (condition tokens, sink, window chunks, current chunk; agifrontier
+// tutorial "JoyAI-Video-Edit：单卡720p 30帧，两步蒸馏攻克流式视频编辑", section
+// "从双向编辑到分块因果架构的蜕变") -- for a query set too small to fill the GPU with query
+// tiles.  The key tiles of each (b, h) are cut into `splits` contiguous slices, one CTA per
+// slice; each CTA writes the unnormalised partial (O, m, l) of its slice and the combine kernel
+// merges the slices with a log-sum-exp weighting.
+//
+// One CTA = one 128-row Q tile (rows past n_q are TMA zero-fill) and one slice of key tiles:
+//   warp 0      TMA producer: Q once, then K and V tiles of the slice through a ring of kStages
+//               shared-memory stages (deeper than the chunk kernels': the slice is read from
+//               HBM once and nothing else hides its latency).
+//   warp 1      MMA issuer (one thread).  S is double-buffered in TMEM: S_{j+1} = Q K_{j+1}^T is
+//               issued as soon as K_{j+1} lands, before the PV of tile j, so the tensor core
+//               computes the next scores while the softmax warps work on this tile.  O += P_j V_j
+//               follows P_j in two halves.
+//   warps 2..5  softmax, thread = query row = TMEM lane.  Only warps whose 32 rows hold a query
+//               take part; the others idle until the teardown.
+// TMEM: S0 | S1 | O (128 + 128 + d columns of 512).  An O rescale (rare: the reference max grew
+// by more than 2^8) first waits for the previous tile's PV, which may still be in flight.
+//
+// The split-K pattern itself (partials plus a log-sum-exp merge) is the standard way to spread
+// a short query set over all SMs; the pages have no decode step of their own.
+#include "attn_common.cuh"
+
+namespace swattn {
+
+struct SplitCtl {
+    SmemCtl c;           // stage barriers, table copy, S/P/O barriers (index = S buffer)
+    uint64_t pv_done;    // one phase per key tile: O += P_j V_j has completed
+};
+
+template <int D>
+struct SplitLayout {
+    using C = TileCfg<D>;
+    static constexpr int kStages = D == 128 ? 6 : 8;   // 192 KB / 128 KB of K/V stages
+    static constexpr int kTileBytes = C::kTileBytes;
+    static constexpr int kQBytes = kTileBytes;
+    static constexpr int kCtlOffset = kQBytes + kStages * kTileBytes;
+    static constexpr int kNeed = kCtlOffset + (int)sizeof(SplitCtl) + 1024;   // + align slack
+    // at least 120 KB, so that one CTA fills an SM and never waits on another's TMEM columns
+    static constexpr int kSmemBytes = kNeed > 120 * 1024 ? kNeed : 120 * 1024;
+    static constexpr int kThreads = 192;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColO = 2 * kBlockN;
+    static_assert(kColO + D <= kTmemCols, "S0 | S1 | O must fit");
+    static_assert(kStages <= 8, "stage barriers");
+    static_assert(kNeed <= 227 * 1024, "shared memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(SplitLayout<D>::kThreads, 1)
+attn_split_kernel(const __grid_constant__ AttnParams p) {
+    using L = SplitLayout<D>;
+    constexpr int kStages = L::kStages;
+    constexpr int kTileBytes = L::kTileBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* q_smem = base;
+    uint8_t* kv_smem = base + L::kQBytes;
+    SplitCtl* x = reinterpret_cast<SplitCtl*>(base + L::kCtlOffset);
+    SmemCtl* ctl = &x->c;
+    volatile int* abort_flag = &ctl->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int n_rows = p.n_q < kBlockM ? p.n_q : kBlockM;   // query rows of the tile
+    const int n_warps = (n_rows + 31) >> 5;                  // softmax warps with a query row
+
+    // ---------------------------------------------------------------- set-up
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_init(smem_u32(&ctl->q_full), 1);
+            for (int s = 0; s < kStages; ++s) {
+                mbar_init(smem_u32(&ctl->kv_full[s]), 1);
+                mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+            }
+            for (int q = 0; q < 2; ++q) {
+                mbar_init(smem_u32(&ctl->s_full[q]), 1);
+                mbar_init(smem_u32(&ctl->p_half[q]), n_warps);
+                mbar_init(smem_u32(&ctl->p_full[q]), n_warps);
+            }
+            mbar_init(smem_u32(&ctl->o_full[0]), 1);
+            mbar_init(smem_u32(&x->pv_done), 1);
+            mbar_init(smem_u32(&ctl->drain), 1);
+            ctl->abort_flag = 0;
+            fence_mbar_init();
+        }
+        __syncwarp();
+        tmem_alloc(smem_u32(&ctl->tmem_base), L::kTmemCols);
+        tmem_relinquish();
+    } else if (warp == 2 && lane == 0) {
+        load_table(ctl, p.table, p.status);
+    } else if (warp == 1 && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_kcur);
+        tma_prefetch_desc(&p.tm_vcur);
+        tma_prefetch_desc(&p.tm_cache_k);
+        tma_prefetch_desc(&p.tm_cache_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = ctl->tmem_base;
+    const int n_tiles = ctl->n_tiles;
+    const int t0 = (int)((long long)blockIdx.x * n_tiles / p.splits);
+    const int t1 = (int)((long long)(blockIdx.x + 1) * n_tiles / p.splits);
+    const int n = t1 - t0;   // key tiles of this slice
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && n > 0) {
+            const uint32_t qbar = smem_u32(&ctl->q_full);
+            mbar_arrive_expect_tx(qbar, kTileBytes);
+            for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
+                tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * kBoxCols, h, 0, b);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int j = t0; j < t1 && ok; ++j) {
+                for (int kv = 0; kv < 2; ++kv, ++it) {
+                    const int s = it % kStages;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_empty[s]), ((it / kStages) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
+                    mbar_arrive_expect_tx(fbar, kTileBytes);
+                    load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                }
+            }
+            // never leave while copies are in flight: the last fill of every stage has landed
+            for (int s = 0; s < kStages; ++s) {
+                if (it > (uint32_t)s) {
+                    const uint32_t uses = (it - 1 - s) / kStages + 1;
+                    wait_drain(smem_u32(&ctl->kv_full[s]), (uses - 1) & 1);
+                }
+            }
+            wait_drain(qbar, 0);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n > 0) {
+            const uint32_t q_base = smem_u32(q_smem);
+            const uint32_t kv_base = smem_u32(kv_smem);
+            const uint32_t tO = tmem + L::kColO;
+            bool ok = wait_or_abort(smem_u32(&ctl->q_full), 0, abort_flag);
+            if (ok) ok = wait_or_abort(smem_u32(&ctl->kv_full[0]), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_s<D>(tmem, q_base, kv_base);   // S_0 into buffer 0
+                mma_commit(smem_u32(&ctl->s_full[0]));
+                mma_commit(smem_u32(&ctl->kv_empty[0]));
+            }
+            for (int jj = 0; jj < n && ok; ++jj) {
+                if (jj + 1 < n) {
+                    // S_{jj+1} into the other buffer: it held P_{jj-1}, whose PV was issued in
+                    // the previous iteration, and one thread's MMAs run in issue order
+                    const uint32_t itK = 2 * jj + 2;
+                    const int sK = itK % kStages;
+                    if (!wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const int nb = (jj + 1) & 1;
+                    issue_s<D>(tmem + nb * kBlockN, q_base, kv_base + sK * kTileBytes);
+                    mma_commit(smem_u32(&ctl->s_full[nb]));
+                    mma_commit(smem_u32(&ctl->kv_empty[sK]));
+                }
+                const uint32_t itV = 2 * jj + 1;
+                const int sV = itV % kStages;
+                const int buf = jj & 1;
+                const uint32_t ph = (jj >> 1) & 1;
+                const uint32_t tP = tmem + buf * kBlockN;
+                if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) break;
+                if (!wait_or_abort(smem_u32(&ctl->p_half[buf]), ph, abort_flag)) break;
+                tc_fence_after();
+                issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                if (!wait_or_abort(smem_u32(&ctl->p_full[buf]), ph, abort_flag)) break;
+                tc_fence_after();
+                issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                mma_commit(smem_u32(&x->pv_done));
+                mma_commit(smem_u32(&ctl->kv_empty[sV]));
+                if (jj + 1 == n) mma_commit(smem_u32(&ctl->o_full[0]));   // O complete: epilogue
+            }
+            // every MMA issued has completed before the CTA can release TMEM
+            mma_commit(smem_u32(&ctl->drain));
+            wait_drain(smem_u32(&ctl->drain), 0);
+        }
+    } else if ((warp & 3) < n_warps) {
+        // ------------------------------------------------------------ softmax warps
+        // warp w may only touch TMEM lane quarter w % 4
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;   // query row inside the tile
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t tO = lane_base + L::kColO;
+        float m_ref = -INFINITY;   // reference max, log2-scaled
+        float l = 0.f;             // row sum of the bf16-rounded exp2(s*sl2 - m_ref)
+        bool ok = true;
+        for (int jj = 0; jj < n; ++jj) {
+            int seg, row0, valid;
+            tile_of(ctl, t0 + jj, seg, row0, valid);
+            const int buf = jj & 1;
+            ok = warp_wait(smem_u32(&ctl->s_full[buf]), (jj >> 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            softmax_step<D, true>(lane_base + buf * kBlockN, tO, valid, jj == 0, smem_u32(&ctl->p_half[buf]),
+                                  p.scale_log2, m_ref, l, smem_u32(&x->pv_done), (uint32_t)((jj - 1) & 1),
+                                  abort_flag);
+            warp_arrive(smem_u32(&ctl->p_full[buf]));
+        }
+        // ------------------------------------------------------------ partials of the slice
+        const size_t prow = ((size_t)blockIdx.x * p.B * p.H + bh) * kBlockM + row;
+        if (n == 0) {
+            if (row < n_rows) {   // empty slice: neutral partials
+                float4* o4 = reinterpret_cast<float4*>(p.o_part + prow * D);
+                for (int c = 0; c < D / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                p.ml_part[prow * 2 + 0] = -INFINITY;
+                p.ml_part[prow * 2 + 1] = 0.f;
+            }
+        } else if (ok && warp_wait(smem_u32(&ctl->o_full[0]), 0, abort_flag)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld_dep(o);
+                if (row < n_rows) {
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                }
+            }
+            if (row < n_rows) {
+                p.ml_part[prow * 2 + 0] = m_ref;
+                p.ml_part[prow * 2 + 1] = l;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+    if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
+}
+
+template <int D>
+static cudaError_t launch_split_d(const AttnParams& p, int splits, cudaStream_t stream) {
+    using L = SplitLayout<D>;
+    auto kern = attn_split_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(splits, p.H, p.B);
+    kern<<<grid, L::kThreads, L::kSmemBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream) {
+    if (p.n_q < 1 || p.n_q > kBlockM || splits < 1) return cudaErrorInvalidValue;
+    if (d == 128) return launch_split_d<128>(p, splits, stream);
+    if (d == 64) return launch_split_d<64>(p, splits, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace swattn

@@ -73,16 +73,20 @@ cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_con
 
 // K2: copy K and V of one chunk from the user layout [B, N, H, d] into the head-major cache
 // layout [B][H][rows_per_bh][d] at row offset slot * N.
-// One block per token row (b, t) of K or V (blockIdx.y = 0 / 1): the row's H x d bf16 values are
-// contiguous in the caller's [B, N, H, d] layout, and head h's d values go to row
-// slot * N + t of the (b, h) panel of the destination.  Thread k of the block moves 16-byte
-// vector k of the row (head k / vpr, vector k % vpr), looping when H * vpr exceeds the block,
-// so consecutive threads read consecutive bytes and write whole 16-byte pieces of 2d-byte
-// destination rows.  No division in the copy loop (vpr is a power of two).
-__device__ __forceinline__ void relayout_row(const uint4* __restrict__ srcK, const uint4* __restrict__ srcV,
-                                             uint4* __restrict__ dstK, uint4* __restrict__ dstV, int N, int H,
-                                             int vpr_log2_k, int vpr_log2_v, int rows_per_bh, int ring, int R,
-                                             int sink, int S, int32_t* state) {
+// One block per kRelayoutRows consecutive token rows (b, t) of K or V (blockIdx.y = 0 / 1): a
+// row's H x d values are contiguous in the caller's [B, N, H, d] layout, and head h's d values
+// go to row slot * N + t of the (b, h) panel of the destination.  Thread k of the block moves
+// 16-byte vector k of every row of its group (head k / vpr, vector k % vpr), looping when H * vpr
+// exceeds the block; the group's loads are all issued before the first store, so each thread
+// keeps kRelayoutRows reads in flight.  Consecutive threads read consecutive bytes and write
+// whole 16-byte pieces of 2d-byte destination rows.  No division in the copy loop (vpr is a
+// power of two).
+constexpr int kRelayoutRows = 4;
+
+__device__ __forceinline__ void relayout_rows(const uint4* __restrict__ srcK, const uint4* __restrict__ srcV,
+                                              uint4* __restrict__ dstK, uint4* __restrict__ dstV, int N,
+                                              long long rows, int H, int vpr_log2_k, int vpr_log2_v, int rows_per_bh,
+                                              int ring, int R, int sink, int S, int32_t* state) {
     int slot = 0;
     if (ring) {
         slot = ring_slot(state[0], R, sink);
@@ -96,35 +100,48 @@ __device__ __forceinline__ void relayout_row(const uint4* __restrict__ srcK, con
     const uint4* __restrict__ src = blockIdx.y == 0 ? srcK : srcV;
     uint4* __restrict__ dst = blockIdx.y == 0 ? dstK : dstV;
     const int vpr_log2 = blockIdx.y == 0 ? vpr_log2_k : vpr_log2_v;   // K may be e4m3 (half the bytes)
-    const int row = blockIdx.x;                     // b * N + t
-    const int b = row / N, t = row - b * N;
     const int vpr = 1 << vpr_log2;
     const int per_row = H << vpr_log2;
-    const uint4* s_row = src + (size_t)row * per_row;
-    const size_t drow0 = (size_t)b * H * rows_per_bh + (size_t)slot * N + t;   // head 0's row
+    const long long row_first = (long long)blockIdx.x * kRelayoutRows;   // b * N + t of the group's first row
+    size_t drow0[kRelayoutRows];   // destination row of head 0, per row of the group
+    bool live[kRelayoutRows];
+#pragma unroll
+    for (int r = 0; r < kRelayoutRows; ++r) {
+        const long long row = row_first + r;
+        live[r] = row < rows;
+        const int b = (int)(row / N), t = (int)(row - (long long)b * N);
+        drow0[r] = (size_t)b * H * rows_per_bh + (size_t)slot * N + t;
+    }
     for (int k = threadIdx.x; k < per_row; k += blockDim.x) {
         const int h = k >> vpr_log2, v = k & (vpr - 1);
-        dst[(drow0 + (size_t)h * rows_per_bh) * vpr + v] = __ldg(s_row + k);
+        uint4 x[kRelayoutRows];
+#pragma unroll
+        for (int r = 0; r < kRelayoutRows; ++r)
+            if (live[r]) x[r] = __ldg(src + (size_t)(row_first + r) * per_row + k);
+#pragma unroll
+        for (int r = 0; r < kRelayoutRows; ++r)
+            if (live[r]) dst[(drow0[r] + (size_t)h * rows_per_bh) * vpr + v] = x[r];
     }
 }
 
 __global__ void __launch_bounds__(512) relayout_kernel(const uint4* __restrict__ srcK,
                                                        const uint4* __restrict__ srcV,
                                                        uint4* __restrict__ dstK,
-                                                       uint4* __restrict__ dstV, int N, int H,
+                                                       uint4* __restrict__ dstV, int N, long long rows, int H,
                                                        int vpr_log2_k, int vpr_log2_v, int rows_per_bh, int ring,
                                                        int R, int sink, int S, int32_t* state) {
-    relayout_row(srcK, srcV, dstK, dstV, N, H, vpr_log2_k, vpr_log2_v, rows_per_bh, ring, R, sink, S, state);
+    relayout_rows(srcK, srcV, dstK, dstV, N, rows, H, vpr_log2_k, vpr_log2_v, rows_per_bh, ring, R, sink, S, state);
 }
 
 // Batched commit: blockIdx.z selects the handle; each copies into its own ring slot (from its
 // own counter), exactly as relayout_kernel does for one handle.
-__global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_constant__ AppendBatch a, int N, int H,
-                                                             int vpr_log2_k, int vpr_log2_v, int T) {
+__global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_constant__ AppendBatch a, int N,
+                                                             long long rows, int H, int vpr_log2_k, int vpr_log2_v,
+                                                             int T) {
     const int l = blockIdx.z;
-    relayout_row(static_cast<const uint4*>(a.K[l]), static_cast<const uint4*>(a.V[l]), static_cast<uint4*>(a.dstK[l]),
-                 static_cast<uint4*>(a.dstV[l]), N, H, vpr_log2_k, vpr_log2_v, a.S[l] * T, 1, a.R[l], a.sink[l], a.S[l],
-                 a.state[l]);
+    relayout_rows(static_cast<const uint4*>(a.K[l]), static_cast<const uint4*>(a.V[l]), static_cast<uint4*>(a.dstK[l]),
+                  static_cast<uint4*>(a.dstV[l]), N, rows, H, vpr_log2_k, vpr_log2_v, a.S[l] * T, 1, a.R[l], a.sink[l],
+                  a.S[l], a.state[l]);
 }
 
 // Batched table advance: block l advances handle l's counter and rebuilds its table.
@@ -152,8 +169,9 @@ cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d
     const int per_row = H * vpr;
     const int threads = per_row >= 512 ? 512 : ((per_row + 31) / 32) * 32;
     // handles without a ring (S = 0) return at once inside the kernel (slot -1)
-    relayout_batch_kernel<<<dim3((unsigned)rows, 2, (unsigned)a.n), threads, 0, stream>>>(a, T, H, vpr_log2_k, vpr_log2,
-                                                                                           T);
+    const long long groups = (rows + kRelayoutRows - 1) / kRelayoutRows;
+    relayout_batch_kernel<<<dim3((unsigned)groups, 2, (unsigned)a.n), threads, 0, stream>>>(a, T, rows, H, vpr_log2_k,
+                                                                                            vpr_log2, T);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     table_build_batch_kernel<<<a.n, 32, 0, stream>>>(a, T);
@@ -171,10 +189,10 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
     if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int per_row = H * vpr;
     const int threads = per_row >= 512 ? 512 : ((per_row + 31) / 32) * 32;
-    dim3 grid((unsigned)rows, 2);
+    dim3 grid((unsigned)((rows + kRelayoutRows - 1) / kRelayoutRows), 2);
     relayout_kernel<<<grid, threads, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
-        static_cast<uint4*>(dstV), N, H, vpr_log2_k, vpr_log2, rows_per_bh, ring, R, sink, S, state);
+        static_cast<uint4*>(dstV), N, rows, H, vpr_log2_k, vpr_log2, rows_per_bh, ring, R, sink, S, state);
     return cudaGetLastError();
 }
 

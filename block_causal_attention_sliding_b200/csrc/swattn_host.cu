@@ -398,7 +398,7 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         p.splits = splits;
         p.o_part = reinterpret_cast<float*>(h->ws + h->off_opart);
         p.ml_part = reinterpret_cast<float*>(h->ws + h->off_ml);
-        cudaError_t e = launch_attention(p, c.d, 1, splits, st);
+        cudaError_t e = launch_split(p, c.d, splits, st);
         if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
         e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
         if (e != cudaSuccess) return cuda_fail(e, "combine launch");
@@ -572,6 +572,7 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
     const sw_attn_config& c = h->cfg;
+    if (c.qk_fp8) return fail(SW_ESTATE, "the split-K path has no e4m3 Q/K form");
     if (n_q < 1 || n_q > kMaxShortQ || n_q > c.tokens_per_chunk)
         return fail(SW_ESHAPE, "n_q must be in [1, min(%d, T)] (n_q=%d)", kMaxShortQ, n_q);
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
@@ -607,7 +608,7 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
     p.o_part = scratch;
     p.ml_part = scratch + (size_t)splits * bh * kBlockM * c.d;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    e = launch_attention(p, c.d, 1, (int)splits, st);
+    e = launch_split(p, c.d, (int)splits, st);
     if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
     e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, (int)splits, p.out_f32, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");

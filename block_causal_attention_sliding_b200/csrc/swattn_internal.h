@@ -97,6 +97,7 @@ cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, in
                              cudaStream_t stream);
 cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream);
 cudaError_t launch_tri(const AttnParams& p, int d, int ctas, cudaStream_t stream);
+cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
                            int n_q, int d, int splits, int out_f32, cudaStream_t stream);

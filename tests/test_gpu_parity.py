@@ -230,6 +230,43 @@ def test_short_queries_720p(dev, n_q):
     stream_and_check(wl, dev, chunks=6, check_at={0, 5}, n_q=n_q, keep_last=wl.W + 1, gen_on_device=True)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("H", [3, 24])
+@pytest.mark.parametrize("n_q", [1, 33, 100, 128])
+def test_short_queries_ragged(dev, d, H, n_q):
+    """Split-K path on ragged shapes, all rows of every chunk: query counts that fill one to four
+    32-row quarters of the tile, partly; H = 3 leaves most slices empty or one tile long, H = 24
+    gives slices of four and five tiles (both S buffers, odd and even counts)."""
+    wl = dataclasses.replace(RAGGED, d=d, H=H)
+    res = stream_and_check(wl, dev, chunks=wl.chunks, n_q=n_q, max_short_q=0)
+    assert len(res) == wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_short_queries_rescale(dev, d):
+    """Split-K path with all key tiles of a head in one slice (B*H above the SM count) and the
+    last chunk's keys scaled by 8, so that the row max jumps on the final tiles: the O rescale
+    then runs while the next tile's scores are already in the other S buffer."""
+    wl = Workload("rescale", B=1, H=150, d=d, T=300, n_cond=40, W=2, sink=True, chunks=4, steps=1)
+    h = make_handle(wl, dev, max_short_q=0)
+    Kc, Vc = synth.cond_inputs(wl)
+    h.set_cond(Kc.to(dev), Vc.to(dev))
+    hist_K, hist_V = [], []
+    for k in range(wl.chunks):
+        Q, K, V = synth.chunk_inputs(wl, k, 0, n_q=40)
+        if k == wl.chunks - 1:
+            K = K * 8   # exact in bf16
+        out = h.forward(Q.to(dev), K.to(dev), V.to(dev))
+        ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink, k=k, Kc=Kc, Vc=Vc,
+                               hist_K=hist_K, hist_V=hist_V, Q=Q, K_cur=K, V_cur=V)
+        compare(out.float().cpu().numpy(), ref)
+        h.append_chunk(K.to(dev), V.to(dev))
+        hist_K.append(K)
+        hist_V.append(V)
+    torch.cuda.synchronize()
+    assert h.status() == 0
+
+
 # ------------------------------------------------------------------ condition-stream queries
 
 @pytest.mark.parametrize("schedule", ["auto", "persistent", "grid", "tri"])
