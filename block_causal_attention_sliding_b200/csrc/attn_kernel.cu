@@ -1,6 +1,5 @@
-// attn_kernel.cu -- fused attention of the active chunk over the bounded cache (sm_100a):
-// the one-work-item-per-CTA kernel (grid over query blocks, heads and streams), its split-K
-// mode for short query sets, and the split-K combine.
+// attn_kernel.cu -- fused attention of the active chunk over the bounded cache (sm_100a): the
+// one-work-item-per-CTA kernel (grid over query-tile pairs, heads and streams).
 //
 // out = softmax(scale * Q K^T) V over the keys the visibility table lists: condition tokens,
 // the sink, the window chunks and the current chunk (block-causal: bidirectional inside the
@@ -18,8 +17,7 @@
 //               fp32 registers -- row max, lazy rescale of O only when the max grows by more
 //               than 2^8, exp2, row sum -- writes P as bf16 into the S columns.
 // The two Q tiles share every K/V tile, and while one warpgroup runs its softmax the tensor
-// core works on the other tile.  In split mode (short query sets) a CTA takes one Q tile and
-// a slice of the key tiles, and writes unnormalised partials that a combine kernel merges.
+// core works on the other tile.
 #include "attn_common.cuh"
 
 namespace swattn {
@@ -44,8 +42,6 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
-    const int bh = b * p.H + h;
-    const bool split_mode = p.splits > 0;
 
     // ---------------------------------------------------------------- set-up
     if (warp == 0) {
@@ -68,14 +64,8 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
     tc_fence_after();
 
     const uint32_t tmem = ctl->tmem_base;
-    const int n_tiles = ctl->n_tiles;
-    int t0 = 0, t1 = n_tiles;
-    if (split_mode) {
-        t0 = (int)((long long)blockIdx.x * n_tiles / p.splits);
-        t1 = (int)((long long)(blockIdx.x + 1) * n_tiles / p.splits);
-    }
-    const int n = t1 - t0;                          // key tiles this CTA processes
-    const int u0 = split_mode ? 0 : blockIdx.x * NQ;   // first Q tile of this CTA
+    const int n = ctl->n_tiles;                     // key tiles: every visible one
+    const int u0 = blockIdx.x * NQ;                 // first Q tile of this CTA
     // Q tiles of this CTA that hold at least one query row (the last CTA of a head may own
     // a single tile); tiles past n_q are neither loaded nor computed
     const int live = min(NQ, q_tiles(p) - u0);
@@ -95,9 +85,9 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
             bool ok = true;
             // fused commit: the chunk's K_cur / V_cur tile j is stored by the CTA of Q-tile pair
             // j mod (pairs), so the stores spread over the CTAs of each head
-            const int cslot = (p.commit && !split_mode) ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
+            const int cslot = p.commit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
             CommitQueue<D, kStages> cq;
-            for (int j = t0; j < t1 && ok; ++j) {
+            for (int j = 0; j < n && ok; ++j) {
                 for (int kv = 0; kv < 2; ++kv, ++it) {
                     const int s = it % kStages;
                     const uint32_t r = it / kStages;
@@ -284,7 +274,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
         bool ok = true;
         for (int jj = 0; jj < n; ++jj) {
             int seg, row0, valid;
-            tile_of(ctl, t0 + jj, seg, row0, valid);
+            tile_of(ctl, jj, seg, row0, valid);
             ok = warp_wait(smem_u32(&ctl->s_full[qt]), jj & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -294,16 +284,7 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
         // ------------------------------------------------------------ epilogue
         const QSrc qs = q_src(p, u0 + qt);
         const int m_row = qs.row0 + row;
-        if (n == 0) {
-            // split mode with an empty slice: neutral partials
-            if (split_mode) {
-                const size_t prow = ((size_t)blockIdx.x * p.B * p.H + bh) * kBlockM + row;
-                float4* o4 = reinterpret_cast<float4*>(p.o_part + prow * D);
-                for (int c = 0; c < D / 4; ++c) o4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                p.ml_part[prow * 2 + 0] = -INFINITY;
-                p.ml_part[prow * 2 + 1] = 0.f;
-            }
-        } else if (ok && warp_wait(o_bar, 0, abort_flag)) {   // o_full completes once, after the last PV
+        if (n > 0 && ok && warp_wait(o_bar, 0, abort_flag)) {   // o_full completes once, after the last PV
             tc_fence_after();
             const float inv = 1.f / l;
 #pragma unroll 1
@@ -311,20 +292,8 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
                 uint32_t o[32];
                 tmem_ld32(tO + c * 32, o);
                 tmem_wait_ld_dep(o);
-                if (split_mode) {
-                    const size_t prow = ((size_t)blockIdx.x * p.B * p.H + bh) * kBlockM + row;
-                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + c * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
-                    if (c == 0) {
-                        p.ml_part[prow * 2 + 0] = m_ref;
-                        p.ml_part[prow * 2 + 1] = l;
-                    }
-                } else if (m_row < qs.rows) {
+                if (m_row < qs.rows)
                     store_row_chunk<D>(qs.out, p.out_f32, ((size_t)b * qs.rows + m_row) * p.H + h, c, o, inv);
-                }
             }
         }
     }
@@ -339,10 +308,10 @@ attn_fwd_kernel(const __grid_constant__ AttnParams p) {
     if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
 }
 
-template <int D, int NQ>
+template <int D>
 static cudaError_t launch_one(const AttnParams& p, int grid_x, cudaStream_t stream) {
-    using L = AttnLayout<D, NQ>;
-    auto kern = attn_fwd_kernel<D, NQ>;
+    using L = AttnLayout<D, 2>;
+    auto kern = attn_fwd_kernel<D, 2>;
     // per device and cheap; set on every launch so any current device is covered
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kSmemBytes);
@@ -352,16 +321,9 @@ static cudaError_t launch_one(const AttnParams& p, int grid_x, cudaStream_t stre
     return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
-                             cudaStream_t stream) {
-    if (d == 128) {
-        return q_tiles_per_cta == 2 ? launch_one<128, 2>(p, grid_x, stream)
-                                    : launch_one<128, 1>(p, grid_x, stream);
-    }
-    if (d == 64) {
-        return q_tiles_per_cta == 2 ? launch_one<64, 2>(p, grid_x, stream)
-                                    : launch_one<64, 1>(p, grid_x, stream);
-    }
+cudaError_t launch_attention(const AttnParams& p, int d, int grid_x, cudaStream_t stream) {
+    if (d == 128) return launch_one<128>(p, grid_x, stream);
+    if (d == 64) return launch_one<64>(p, grid_x, stream);
     return cudaErrorInvalidValue;
 }
 
@@ -382,99 +344,6 @@ __global__ void selftest_timeout_kernel(int32_t* status, uint64_t limit_ns) {
 
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream) {
     selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
-    return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------ split-K combine (K4)
-// out[row] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (log-sum-exp merge).
-// One warp per (b, h, row); each lane owns d/32 consecutive columns.
-template <int D>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
-                                                      const float* __restrict__ ml_part, void* out,
-                                                      int B, int H, int n_q, int splits, int out_f32) {
-    // one warp per output row; each lane owns D / 32 consecutive columns.  The splits are read
-    // eight at a time with every load of a group issued before any is used (one memory round
-    // trip per group), and merged with a running max like the online softmax.
-    constexpr int V = D / 32;
-    constexpr int G = 8;
-    static_assert(V == 4 || V == 2, "d = 128 or 64");
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int total = B * H * n_q;
-    if (warp >= total) return;
-    const int row = warp % n_q;
-    const int bh = warp / n_q;
-    const int b = bh / H, h = bh % H;
-    const size_t stride_split = (size_t)B * H * kBlockM;
-    const size_t row0 = (size_t)bh * kBlockM + row;
-    float M = -INFINITY, den = 0.f;
-    float acc[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.f;
-    for (int s0 = 0; s0 < splits; s0 += G) {
-        float2 ml[G];
-        float o[G][V];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const int s = s0 + g;
-            if (s < splits) {
-                const size_t prow = (size_t)s * stride_split + row0;
-                ml[g] = __ldg(reinterpret_cast<const float2*>(ml_part) + prow);
-                const float* src = o_part + prow * D + lane * V;
-                if (V == 4) {
-                    const float4 t = __ldg(reinterpret_cast<const float4*>(src));
-                    o[g][0] = t.x; o[g][1] = t.y; o[g][V > 2 ? 2 : 0] = t.z; o[g][V > 3 ? 3 : 0] = t.w;
-                } else {
-                    const float2 t = __ldg(reinterpret_cast<const float2*>(src));
-                    o[g][0] = t.x; o[g][1] = t.y;
-                }
-            } else {
-                ml[g] = make_float2(-INFINITY, 0.f);
-#pragma unroll
-                for (int i = 0; i < V; ++i) o[g][i] = 0.f;
-            }
-        }
-        float Mg = M;
-#pragma unroll
-        for (int g = 0; g < G; ++g) Mg = fmaxf(Mg, ml[g].x);
-        if (Mg == -INFINITY) continue;                 // every slice so far is empty
-        const float f = ex2_approx(M - Mg);            // 0 while nothing has been merged
-        den *= f;
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] *= f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            if (ml[g].x == -INFINITY) continue;        // empty slice (or past the last split)
-            const float w = ex2_approx(ml[g].x - Mg);
-            den += w * ml[g].y;
-#pragma unroll
-            for (int i = 0; i < V; ++i) acc[i] += w * o[g][i];
-        }
-        M = Mg;
-    }
-    const float inv = 1.f / den;
-    const size_t orow = ((size_t)b * n_q + row) * H + h;
-    if (out_f32) {
-        float* dst = static_cast<float*>(out) + orow * D + lane * V;
-#pragma unroll
-        for (int i = 0; i < V; ++i) dst[i] = acc[i] * inv;
-    } else {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(out) + orow * D + lane * V);
-#pragma unroll
-        for (int i = 0; i < V; i += 2) dst[i / 2] = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-    }
-}
-
-cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
-                           int n_q, int d, int splits, int out_f32, cudaStream_t stream) {
-    const long long warps = (long long)B * H * n_q;
-    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
-    if (d == 128)
-        combine_kernel<128><<<blocks, 256, 0, stream>>>(o_part, ml_part, out, B, H, n_q, splits, out_f32);
-    else if (d == 64)
-        combine_kernel<64><<<blocks, 256, 0, stream>>>(o_part, ml_part, out, B, H, n_q, splits, out_f32);
-    else
-        return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
 

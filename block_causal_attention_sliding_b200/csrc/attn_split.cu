@@ -7,7 +7,7 @@
 // "从双向编辑到分块因果架构的蜕变") -- for a query set too small to fill the GPU with query
 // tiles.  The key tiles of each (b, h) are cut into `splits` contiguous slices, one CTA per
 // slice; each CTA writes the unnormalised partial (O, m, l) of its slice and the combine kernel
-// merges the slices with a log-sum-exp weighting.
+// (below; a programmatic dependent launch) merges the slices with a log-sum-exp weighting.
 //
 // One CTA = one 128-row Q tile (rows past n_q are TMA zero-fill) and one slice of key tiles:
 //   warp 0      TMA producer: Q once, then K and V tiles of the slice through a ring of kStages
@@ -109,6 +109,8 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the combine that follows may be scheduled now; it waits for this grid's completion itself
+    grid_dependents_launch();
 
     const uint32_t tmem = ctl->tmem_base;
     const int n_tiles = ctl->n_tiles;
@@ -271,6 +273,112 @@ cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t st
     if (p.n_q < 1 || p.n_q > kBlockM || splits < 1) return cudaErrorInvalidValue;
     if (d == 128) return launch_split_d<128>(p, splits, stream);
     if (d == 64) return launch_split_d<64>(p, splits, stream);
+    return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ split-K combine (K4)
+// out[row] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (log-sum-exp merge).
+// One warp per (b, h, row); each lane owns d/32 consecutive columns.
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
+                                                      const float* __restrict__ ml_part, void* out,
+                                                      int B, int H, int n_q, int splits, int out_f32) {
+    // one warp per output row; each lane owns D / 32 consecutive columns.  The splits are read
+    // eight at a time with every load of a group issued before any is used (one memory round
+    // trip per group), and merged with a running max like the online softmax.
+    constexpr int V = D / 32;
+    constexpr int G = 8;
+    static_assert(V == 4 || V == 2, "d = 128 or 64");
+    // launched as a programmatic dependent of the split kernel: wait until that grid has
+    // completed and its partials are visible (returns at once for a plain launch)
+    grid_dependency_wait();
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int total = B * H * n_q;
+    if (warp >= total) return;
+    const int row = warp % n_q;
+    const int bh = warp / n_q;
+    const int b = bh / H, h = bh % H;
+    const size_t stride_split = (size_t)B * H * kBlockM;
+    const size_t row0 = (size_t)bh * kBlockM + row;
+    float M = -INFINITY, den = 0.f;
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    for (int s0 = 0; s0 < splits; s0 += G) {
+        float2 ml[G];
+        float o[G][V];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int s = s0 + g;
+            if (s < splits) {
+                const size_t prow = (size_t)s * stride_split + row0;
+                ml[g] = __ldg(reinterpret_cast<const float2*>(ml_part) + prow);
+                const float* src = o_part + prow * D + lane * V;
+                if (V == 4) {
+                    const float4 t = __ldg(reinterpret_cast<const float4*>(src));
+                    o[g][0] = t.x; o[g][1] = t.y; o[g][V > 2 ? 2 : 0] = t.z; o[g][V > 3 ? 3 : 0] = t.w;
+                } else {
+                    const float2 t = __ldg(reinterpret_cast<const float2*>(src));
+                    o[g][0] = t.x; o[g][1] = t.y;
+                }
+            } else {
+                ml[g] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int i = 0; i < V; ++i) o[g][i] = 0.f;
+            }
+        }
+        float Mg = M;
+#pragma unroll
+        for (int g = 0; g < G; ++g) Mg = fmaxf(Mg, ml[g].x);
+        if (Mg == -INFINITY) continue;                 // every slice so far is empty
+        const float f = ex2_approx(M - Mg);            // 0 while nothing has been merged
+        den *= f;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] *= f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            if (ml[g].x == -INFINITY) continue;        // empty slice (or past the last split)
+            const float w = ex2_approx(ml[g].x - Mg);
+            den += w * ml[g].y;
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[i] += w * o[g][i];
+        }
+        M = Mg;
+    }
+    const float inv = 1.f / den;
+    const size_t orow = ((size_t)b * n_q + row) * H + h;
+    if (out_f32) {
+        float* dst = static_cast<float*>(out) + orow * D + lane * V;
+#pragma unroll
+        for (int i = 0; i < V; ++i) dst[i] = acc[i] * inv;
+    } else {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(out) + orow * D + lane * V);
+#pragma unroll
+        for (int i = 0; i < V; i += 2) dst[i / 2] = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+    }
+}
+
+cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
+                           int n_q, int d, int splits, int out_f32, cudaStream_t stream) {
+    const long long warps = (long long)B * H * n_q;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+    // programmatic dependent launch: the combine's blocks are scheduled while the split kernel
+    // finishes, and wait on the device (griddepcontrol.wait) instead of behind a launch gap
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (d == 128)
+        return cudaLaunchKernelEx(&cfg, combine_kernel<128>, o_part, ml_part, out, B, H, n_q, splits, out_f32);
+    if (d == 64)
+        return cudaLaunchKernelEx(&cfg, combine_kernel<64>, o_part, ml_part, out, B, H, n_q, splits, out_f32);
     return cudaErrorInvalidValue;
 }
 

@@ -337,4 +337,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Programmatic dependent launch: let the next kernel in the stream be scheduled early, and (in
+// that kernel) wait until the previous grid has completed with its memory visible.  Both are
+// no-ops unless the dependent was launched with programmatic stream serialization.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace swattn

@@ -252,6 +252,12 @@ int sw_attn_reset(sw_attn_t* h, void* stream) {
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "state reset launch");
 }
 
+// The table parameters of a handle, for launches that rebuild its table.
+static TableAdvance table_advance(const sw_attn_t* h) {
+    const sw_attn_config& c = h->cfg;
+    return TableAdvance{c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk};
+}
+
 int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void* stream) {
     g_err.clear();
     if (!h) return fail(SW_EINVAL, "null handle");
@@ -261,8 +267,8 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
     if (!K_cond || !V_cond) return fail(SW_EINVAL, "null condition tensor");
     if (!aligned16(K_cond) || !aligned16(V_cond)) return fail(SW_EALIGN, "condition tensors must be 16-byte aligned");
     cudaError_t e = launch_relayout(K_cond, V_cond, h->ws + h->off_kcond, h->ws + h->off_vcond, c.B, c.n_cond,
-                                    c.H, c.d, c.n_cond, 0, h->R, c.sink, h->S, reinterpret_cast<int32_t*>(h->ws),
-                                    static_cast<cudaStream_t>(stream), c.qk_fp8 ? 1 : 2);
+                                    c.H, c.d, c.n_cond, 0, h->S, reinterpret_cast<int32_t*>(h->ws), table_advance(h),
+                                    0, static_cast<cudaStream_t>(stream), c.qk_fp8 ? 1 : 2);
     if (e != cudaSuccess) return cuda_fail(e, "condition copy launch");
     h->cond_set = true;
     return SW_OK;
@@ -279,9 +285,10 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     int32_t* state = reinterpret_cast<int32_t*>(h->ws);
     cudaError_t e;
     if (h->S > 0) {
+        // the copy's last block advances the counter and rebuilds the table: one launch
         e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
-                            h->S * c.tokens_per_chunk, 1, h->R, c.sink, h->S, state, st, c.qk_fp8 ? 1 : 2);
-        if (e != cudaSuccess) return cuda_fail(e, "append launch");
+                            h->S * c.tokens_per_chunk, 1, h->S, state, table_advance(h), 1, st, c.qk_fp8 ? 1 : 2);
+        return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
     }
     e = launch_table_build(state, c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
@@ -351,7 +358,7 @@ static int launch_full(sw_attn_t* h, AttnParams& p, cudaStream_t st) {
     cudaError_t e;
     p.splits = 0;
     if (sched == SW_SCHED_GRID) {
-        e = launch_attention(p, c.d, 2, (int)((nqt + 1) / 2), st);
+        e = launch_attention(p, c.d, (int)((nqt + 1) / 2), st);
         if (e != cudaSuccess) return cuda_fail(e, "attention launch");
         return SW_OK;
     }
@@ -474,11 +481,11 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     if (resolve_schedule_tiles(h, nqt) == SW_SCHED_TRI) {
         // the three-buffer kernel does not store K/V: forward, then the copy into the same slot
         if ((rc = launch_full(h, p, st))) return rc;
-        if (h->S > 0) {
+        if (h->S > 0) {   // the copy launch also advances the table
             cudaError_t e = launch_relayout(K_cur, V_cur, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B,
-                                            c.tokens_per_chunk, c.H, c.d, h->S * c.tokens_per_chunk, 1, h->R, c.sink,
-                                            h->S, state, st);
-            if (e != cudaSuccess) return cuda_fail(e, "append launch");
+                                            c.tokens_per_chunk, c.H, c.d, h->S * c.tokens_per_chunk, 1, h->S, state,
+                                            table_advance(h), 1, st);
+            return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
         }
     } else {
         p.commit = h->S > 0 ? 1 : 0;

@@ -12,7 +12,7 @@ namespace swattn {
 constexpr int kBlockM = 128;       // query rows per Q tile (MMA M)
 constexpr int kBlockN = 128;       // keys per K/V tile (MMA N of QK^T, K of PV)
 constexpr int kMaxW = 64;          // largest window supported
-constexpr int kStateHeaderInts = 16;   // [0] chunks committed, [1] status bits, rest reserved
+constexpr int kStateHeaderInts = 16;   // [0] chunks committed, [1] status bits, [2] commit blocks done
 constexpr int kMaxShortQ = 128;    // split-K path handles one Q tile per (b, h)
 constexpr int kMaxSplits = 64;
 constexpr int kMaxPersistentCtas = 160;   // >= SMs of a B200 (148)
@@ -34,6 +34,7 @@ __host__ __device__ inline int ring_slot(int c, int R, int sink) {
 // Device-side state layout: int32 words at the start of the workspace.
 //   state[0] = chunks committed (= index k of the active chunk)
 //   state[1] = status bits (SW_STATUS_*)
+//   state[2] = blocks of a running chunk-commit copy that have finished (0 between launches)
 //   state[kStateHeaderInts ...] = visibility table (table_ints_for(W) entries)
 
 // Everything a launch of the attention kernel needs.  Passed by value as a __grid_constant__
@@ -74,11 +75,16 @@ cudaError_t launch_table_build(int32_t* state, int W, int R, int sink, int n_con
                                cudaStream_t stream);
 cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_cond, int T,
                                int32_t* counters, long long n_counters, cudaStream_t stream);
+// What a table rebuild needs: window, ring slots, sink flag, condition tokens, chunk tokens.
+struct TableAdvance {
+    int W, R, sink, n_cond, T;
+};
 // Copy [B, N, H, d] bf16 K and V into [B][H][rows_per_bh][d] regions at row offset
-// slot * N (slot from the device counter when `ring` is set, else 0).
+// slot * N (slot from the device counter when `ring` is set, else 0).  With `advance` (ring
+// only) the same launch then advances the counter and rebuilds the table (a chunk commit).
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
-                            int H, int d, int rows_per_bh, int ring, int R, int sink, int S,
-                            int32_t* state, cudaStream_t stream, int k_esz = 2);
+                            int H, int d, int rows_per_bh, int ring, int S, int32_t* state, const TableAdvance& ta,
+                            int advance, cudaStream_t stream, int k_esz = 2);
 // One chunk commit for each of up to kMaxBatch handles (layers) of the same B, T, H, d, in one
 // copy launch and one table launch (the per-handle window, sink, slots and counter stay apart).
 constexpr int kMaxBatch = 32;
@@ -93,8 +99,7 @@ struct AppendBatch {
 };
 cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, cudaStream_t stream);
 
-cudaError_t launch_attention(const AttnParams& p, int d, int q_tiles_per_cta, int grid_x,
-                             cudaStream_t stream);
+cudaError_t launch_attention(const AttnParams& p, int d, int grid_x, cudaStream_t stream);
 cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream);
 cudaError_t launch_tri(const AttnParams& p, int d, int ctas, cudaStream_t stream);
 cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream);

@@ -383,6 +383,57 @@ def test_append_batched_matches_ring(dev):
         assert h.status() == 0
 
 
+def test_decode_step_graph_capture(dev):
+    """Short-query forwards (the split-K kernel, then its combine as a programmatic dependent
+    launch) and a single-handle commit (copy and table advance in one launch), captured once into
+    a CUDA graph and replayed chunk after chunk, give the eager calls' outputs bit for bit."""
+    wl = dataclasses.replace(RAGGED, H=24, chunks=6)
+    n_q = 40
+
+    def handle():
+        h = make_handle(wl, dev, max_short_q=0)
+        Kc, Vc = synth.cond_inputs(wl)
+        h.set_cond(Kc.to(dev), Vc.to(dev))
+        return h
+
+    def inputs(k):
+        return [[t.to(dev) for t in synth.chunk_inputs(wl, k, s, n_q=n_q)] for s in range(wl.steps)]
+
+    eager = handle()
+    eager_out = []
+    for k in range(wl.chunks):
+        x = inputs(k)
+        eager_out.append([eager.forward(*x[s]).clone() for s in range(wl.steps)])
+        eager.append_chunk(x[-1][1], x[-1][2])
+    torch.cuda.synchronize()
+    g = handle()
+    static_in = inputs(0)
+    static_out = [torch.empty((wl.B, n_q, wl.H, wl.d), dtype=torch.float32, device=dev) for _ in range(wl.steps)]
+
+    def step():
+        for s in range(wl.steps):
+            g.forward(*static_in[s], out=static_out[s])
+        g.append_chunk(static_in[-1][1], static_in[-1][2])
+
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step()
+    torch.cuda.current_stream().wait_stream(side)
+    for k in range(wl.chunks):
+        for dst_s, src_s in zip(static_in, inputs(k)):
+            for dst, src in zip(dst_s, src_s):
+                dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        for s in range(wl.steps):
+            assert torch.equal(static_out[s], eager_out[k][s]), (k, s)
+    assert np.array_equal(g.table().cpu().numpy(), eager.table().cpu().numpy())
+    assert eager.status() == 0 and g.status() == 0
+
+
 def test_chunk_step_graph_capture(dev):
     """A three-layer chunk step -- each layer's two forwards, then one batched commit -- captured
     once into a CUDA graph and replayed chunk after chunk gives the same outputs, bit for bit,
