@@ -157,7 +157,7 @@ SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const
 /*
  * Commit the finished chunk of n handles at once -- typically the n layers of one model, each
  * with its own cache: the same effect as sw_attn_append_chunk(handles[l], K[l], V[l]) for every
- * l, in one copy launch and one table launch per 32 handles instead of two launches per handle
+ * l, in one launch per 32 handles (each handle's copy, then its counter and table) instead of one per handle
  * (the clean-KV cache build of a chunk covers every layer: tutorial, section "软硬件协同部署";
  * neurohive review, section "Откуда берётся 30 FPS").  All handles share B, H, d and T; window,
  * sink, condition count and chunk counter are each handle's own.  K[l], V[l]: [B, T, H, d] bf16.
@@ -226,6 +226,7 @@ SW_API int sw_attn_forward_joint(sw_attn_t *h, const void *Q, const void *Q_cond
  *     current); make that first call before any stream capture.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.  Same argument rules as
  *     sw_attn_forward; the caller's current device must be the workspace's device.
+ *   - Handles with e4m3 Q/K (qk_fp8) have no split-K form: SW_ESTATE.
  */
 SW_API int sw_attn_forward_short_noalloc(sw_attn_t *h, const void *Q, const void *K_cur,
                                          const void *V_cur, void *out, int n_q, void *stream);
