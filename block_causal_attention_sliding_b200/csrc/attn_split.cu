@@ -97,8 +97,6 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
         __syncwarp();
         tmem_alloc(smem_u32(&ctl->tmem_base), L::kTmemCols);
         tmem_relinquish();
-    } else if (warp == 2 && lane == 0) {
-        load_table(ctl, p.table, p.status);
     } else if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_kcur);
@@ -106,6 +104,11 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
         tma_prefetch_desc(&p.tm_cache_k);
         tma_prefetch_desc(&p.tm_cache_v);
     }
+    // launched as a programmatic dependent: the set-up above overlaps the previous kernel's
+    // tail; nothing the previous kernel may have written (table, Q, K/V, partials) is read or
+    // written before it has completed
+    grid_dependency_wait();
+    if (warp == 2 && lane == 0) load_table(ctl, p.table, p.status);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -258,15 +261,32 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
     if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
 }
 
+// A launch that may begin while the stream's previous kernel finishes (programmatic stream
+// serialization); the kernel itself waits for that kernel's completion (griddepcontrol.wait)
+// before it touches memory the previous kernel may write.
+template <typename... Params, typename... Args>
+static cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int D>
 static cudaError_t launch_split_d(const AttnParams& p, int splits, cudaStream_t stream) {
     using L = SplitLayout<D>;
     auto kern = attn_split_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(splits, p.H, p.B);
-    kern<<<grid, L::kThreads, L::kSmemBytes, stream>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(splits, p.H, p.B), dim3(L::kThreads), L::kSmemBytes, stream, p);
 }
 
 cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream) {
@@ -289,6 +309,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     constexpr int V = D / 32;
     constexpr int G = 8;
     static_assert(V == 4 || V == 2, "d = 128 or 64");
+    // the next kernel in the stream (the next split-K forward, say) may start its set-up now;
+    // it waits for this grid's completion before it reads or writes anything
+    grid_dependents_launch();
     // launched as a programmatic dependent of the split kernel: wait until that grid has
     // completed and its partials are visible (returns at once for a plain launch)
     grid_dependency_wait();
@@ -365,20 +388,12 @@ cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out,
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     // programmatic dependent launch: the combine's blocks are scheduled while the split kernel
     // finishes, and wait on the device (griddepcontrol.wait) instead of behind a launch gap
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if (d == 128)
-        return cudaLaunchKernelEx(&cfg, combine_kernel<128>, o_part, ml_part, out, B, H, n_q, splits, out_f32);
+        return launch_dependent(combine_kernel<128>, dim3(blocks), dim3(256), 0, stream, o_part, ml_part, out, B, H,
+                                n_q, splits, out_f32);
     if (d == 64)
-        return cudaLaunchKernelEx(&cfg, combine_kernel<64>, o_part, ml_part, out, B, H, n_q, splits, out_f32);
+        return launch_dependent(combine_kernel<64>, dim3(blocks), dim3(256), 0, stream, o_part, ml_part, out, B, H,
+                                n_q, splits, out_f32);
     return cudaErrorInvalidValue;
 }
 
