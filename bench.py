@@ -681,7 +681,7 @@ def side_paths(h, wl, pool, dev, stream, peaks):
     out["append"] = {"us": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
                      "frac_hbm": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 3), "bytes": nbytes,
                      "sources": f"{len(kv)} (K, V) inputs cycled, {len(kv) * 2 * K.numel() * K.element_size() >> 20} MiB",
-                     "note": "one launch: the copy's last block advances the counter and the table"}
+                     "note": f"one launch ({h.commit_kind()} commit): the copy, then the counter and table advance"}
     k = wl.steady_k()
     nvis = wl.n_vis(k)
     dec = {}

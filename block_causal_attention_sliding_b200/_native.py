@@ -23,7 +23,7 @@ EXPORTS = (
     "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
-    "sw_attn_selftest_timeout", "sw_attn_schedule_for",
+    "sw_attn_selftest_timeout", "sw_attn_schedule_for", "sw_attn_commit_kind",
 )
 
 
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_selftest_timeout.restype = i32
     L.sw_attn_schedule_for.argtypes = [vp, i32]
     L.sw_attn_schedule_for.restype = i32
+    L.sw_attn_commit_kind.argtypes = [vp]
+    L.sw_attn_commit_kind.restype = i32
     L.sw_attn_table_ints.argtypes = [vp]
     L.sw_attn_table_ints.restype = i32
     L.sw_attn_get_table.argtypes = [vp, vp, vp]

@@ -63,6 +63,13 @@ class SlidingWindowAttention:
             N.check(self._lib.sw_attn_bind_workspace(h, self.workspace.data_ptr(), nbytes, _stream_ptr()))
         self.table_ints = int(self._lib.sw_attn_table_ints(h))
 
+    def commit_kind(self) -> str:
+        """How chunk commits move K and V into the ring: "tma" (bulk copies) or "copy" (kernel)."""
+        r = int(self._lib.sw_attn_commit_kind(self._h))
+        if r < 0:
+            N.check(r)
+        return "tma" if r == 1 else "copy"
+
     def schedule_for(self, n_q: int | None = None) -> str:
         """The schedule a full-path forward of n_q queries (default T) runs with."""
         r = int(self._lib.sw_attn_schedule_for(self._h, self.T if n_q is None else n_q))

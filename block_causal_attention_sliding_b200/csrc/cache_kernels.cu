@@ -6,7 +6,8 @@
 // completes, so memory and per-chunk work stay constant (agifrontier tutorial "JoyAI-Video-
 // Edit：单卡720p 30帧，两步蒸馏攻克流式视频编辑", sections "从双向编辑到分块因果架构的蜕变" and
 // "软硬件协同部署"; neurohive review "JoyAI-Video-Edit", section "Чанки и борьба с дрейфом").
-#include "swattn_internal.h"
+#include "commit_copy.h"
+#include "ptx.cuh"
 
 namespace swattn {
 
@@ -179,6 +180,99 @@ __global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_consta
     advance_after_commit(a.state[l], ta);
 }
 
+// K2 with the tensor-memory accelerator: a chunk commit as TMA bulk copies.  The source map
+// reads the caller's [B, T, H, d] K (or V) with its dimensions ordered {d, t, h, b}, so one box
+// of kCommitRows token rows x h_box heads x 128 bytes of d lands in shared memory as
+// [head][row][128 B] -- exactly the layout of the same box of the head-major cache map
+// {d, T, S, H, B}.  Each item (K or V, stream, row group, head group, 128-byte column block) is
+// one TMA load and one TMA store from the same buffer; rows and heads past the ends read as
+// zero and are not stored.  One thread per CTA (one CTA per SM) streams its contiguous share of
+// the items through kCommitBufs buffers, refilling a buffer once the store issued from it one
+// item earlier has read it, so the other loads stay in flight.  Every wait is bounded; on a
+// timeout the status word records it and the thread still drains what it issued.
+constexpr int kCommitBufs = 8;     // buffers of up to 128 B x 8 rows x 24 heads = 24 KB
+
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+struct CommitItems {
+    int B, T, H, nt, nh, cbk, cbv;   // streams, rows, heads, row groups, head groups, column blocks of K and V
+    int colk, colv;                  // elements per 128-byte column block of K and V
+    __device__ long long per_k() const { return (long long)B * nt * nh * cbk; }
+    __device__ long long total() const { return per_k() + (long long)B * nt * nh * cbv; }
+    // item -> (K or V, stream, first row, first head, first column)
+    __device__ void decode(long long i, int& kv, int& b, int& t0, int& h0, int& c0) const {
+        kv = i >= per_k();
+        if (kv) i -= per_k();
+        const int cb = kv ? cbv : cbk;
+        const int c = (int)(i % cb);
+        i /= cb;
+        const int hg = (int)(i % nh);
+        i /= nh;
+        const int tg = (int)(i % nt);
+        b = (int)(i / nt);
+        t0 = tg * kCommitRows;
+        h0 = hg * kCommitHeads;
+        c0 = c * (kv ? colv : colk);
+    }
+};
+
+__global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant__ CommitMaps m, CommitItems it,
+                                                           int box_bytes, int32_t* state, TableAdvance ta, int S) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[kCommitBufs];
+    if (threadIdx.x == 0) {
+        const int slot = commit_slot(state, ta.R, ta.sink, S);
+        const long long total = it.total();
+        const long long i0 = slot >= 0 ? (long long)blockIdx.x * total / gridDim.x : 0;
+        const long long i1 = slot >= 0 ? (long long)(blockIdx.x + 1) * total / gridDim.x : 0;
+        for (int q = 0; q < kCommitBufs; ++q) mbar_init(smem_u32(&full[q]), 1);
+        fence_mbar_init();
+        auto load = [&](long long i) {
+            int kv, b, t0, h0, c0;
+            it.decode(i, kv, b, t0, h0, c0);
+            const int q = (int)((i - i0) % kCommitBufs);
+            const uint32_t bar = smem_u32(&full[q]);
+            mbar_arrive_expect_tx(bar, box_bytes);
+            tma_load_4d(smem_u32(base + (size_t)q * box_bytes), kv ? &m.src_v : &m.src_k, bar, c0, t0, h0, b);
+        };
+        for (long long i = i0; i < i1 && i < i0 + kCommitBufs; ++i) load(i);
+        int never = 0;
+        long long done = i0;   // items whose load has been waited for
+        for (long long i = i0; i < i1; ++i, ++done) {
+            const long long k = i - i0;
+            if (!mbar_wait(smem_u32(&full[k % kCommitBufs]), (uint32_t)((k / kCommitBufs) & 1), &never,
+                           1000000000ull)) {
+                atomicOr(state + 1, SW_STATUS_TIMEOUT);
+                break;
+            }
+            int kv, b, t0, h0, c0;
+            it.decode(i, kv, b, t0, h0, c0);
+            fence_proxy_async_smem();
+            tma_store_5d(kv ? &m.dst_v : &m.dst_k, smem_u32(base + (size_t)(k % kCommitBufs) * box_bytes), c0, t0, slot,
+                         h0, b);
+            bulk_commit_group();
+            // the buffer of item i - 1 takes item i - 1 + kCommitBufs once that item's store has
+            // read it (the store just issued may still be reading its own buffer)
+            if (k >= 1 && i - 1 + kCommitBufs < i1) {
+                bulk_wait_read_1();
+                load(i - 1 + kCommitBufs);
+            }
+        }
+        // loads issued but not waited for (only after a timeout): let them land, boundedly
+        // (the prologue issued items i0 .. i0 + kCommitBufs - 1; iteration i, once done, issued item
+        // i - 1 + kCommitBufs)
+        long long issued = done == i0 ? i0 + kCommitBufs : done + kCommitBufs - 1;
+        if (issued > i1) issued = i1;
+        for (long long i = done; i < issued; ++i) {
+            const long long k = i - i0;
+            (void)mbar_wait(smem_u32(&full[k % kCommitBufs]), (uint32_t)((k / kCommitBufs) & 1), &never, 1000000000ull);
+        }
+        bulk_wait_all();   // every store complete before the buffers go away
+    }
+    advance_after_commit(state, ta);
+}
+
 // 16-byte vectors per head row of d elements of esz bytes, as a power of two (-1: not one).
 static int vpr_log2_of(int d, int esz) {
     const int vpr = d * esz / 16;
@@ -217,6 +311,28 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
     relayout_kernel<<<grid, threads, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
         static_cast<uint4*>(dstV), N, rows, H, vpr_log2_k, vpr_log2, rows_per_bh, ring, S, state, ta, advance);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int32_t* state,
+                              const TableAdvance& ta, int S, int ctas, cudaStream_t stream) {
+    if (B < 1 || T < 1 || H < 1 || ctas < 1 || (d * 2) % 128 != 0 || (d * k_esz) % 128 != 0) return cudaErrorInvalidValue;
+    CommitItems it;
+    it.B = B;
+    it.T = T;
+    it.H = H;
+    it.nt = (T + kCommitRows - 1) / kCommitRows;
+    it.nh = (H + kCommitHeads - 1) / kCommitHeads;
+    it.cbk = d * k_esz / 128;
+    it.cbv = d * 2 / 128;
+    it.colk = 128 / k_esz;
+    it.colv = 64;
+    const int h_box = H < kCommitHeads ? H : kCommitHeads;
+    const int box_bytes = 128 * kCommitRows * h_box;
+    const int smem = kCommitBufs * box_bytes + 1024;
+    cudaError_t e = cudaFuncSetAttribute(commit_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    commit_tma_kernel<<<ctas, 32, smem, stream>>>(maps, it, box_bytes, state, ta, S);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,22 @@
+// commit_copy.h -- the TMA form of the chunk commit (append/evict): declarations shared by the
+// kernel (cache_kernels.cu) and the host code (swattn_host.cu).
+#pragma once
+#include "swattn_internal.h"
+
+namespace swattn {
+
+// src maps over the caller's K and V ([B, T, H, d], dimensions ordered {d, t, h, b}); dst maps
+// over the ring ({d, T, S, H, B}); boxes of 128 bytes x kCommitRows rows x min(H, kCommitHeads)
+// heads, 128-byte swizzle on both sides, so a loaded box is stored as it lies.
+struct CommitMaps {
+    CUtensorMap src_k, src_v, dst_k, dst_v;
+};
+constexpr int kCommitRows = 8;
+constexpr int kCommitHeads = 24;
+
+// Copy the finished chunk into the ring slot the device counter names, then (last CTA) advance
+// the counter and rebuild the table.  ctas: one per SM.  k_esz: bytes per K element (1: e4m3).
+cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int32_t* state,
+                              const TableAdvance& ta, int S, int ctas, cudaStream_t stream);
+
+}  // namespace swattn

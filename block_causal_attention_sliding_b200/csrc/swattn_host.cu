@@ -13,6 +13,7 @@
 
 #include <cudaTypedefs.h>
 
+#include "commit_copy.h"
 #include "swattn_internal.h"
 
 using namespace swattn;
@@ -35,6 +36,8 @@ struct sw_attn {
     int num_sms = 148;
     bool cond_set = false;
     CUtensorMap tm_cache_k, tm_cache_v, tm_cond_k, tm_cond_v;
+    CUtensorMap tm_commit_k, tm_commit_v;   // the ring with the TMA commit's box
+    bool commit_tma = false;                // chunk commits by TMA bulk copies (else the copy kernel)
 };
 
 namespace {
@@ -94,6 +97,16 @@ int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, con
     const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)N, (uint64_t)B};
     const uint64_t strides[3] = {(uint64_t)d * esz, (uint64_t)H * d * esz, (uint64_t)N * H * d * esz};
     const uint32_t box[4] = {(uint32_t)(128 / esz), 1, (uint32_t)kBlockN, 1};
+    return encode(m, ptr, 4, dims, strides, box, what, esz);
+}
+
+// The caller's [B, T, H, d] K or V for a TMA chunk commit: dims ordered {d, t, h, b} (strides
+// T: H*d, h: d, b: T*H*d elements), box 128 bytes x kCommitRows rows x min(H, kCommitHeads) heads.
+int encode_commit_src(CUtensorMap* m, const void* ptr, int B, int T, int H, int d, const char* what, int esz) {
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)T, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)H * d * esz, (uint64_t)d * esz, (uint64_t)T * H * d * esz};
+    const uint32_t box[4] = {(uint32_t)(128 / esz), (uint32_t)kCommitRows,
+                             (uint32_t)(H < kCommitHeads ? H : kCommitHeads), 1};
     return encode(m, ptr, 4, dims, strides, box, what, esz);
 }
 
@@ -216,6 +229,19 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint32_t boxk[5] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1, 1};
         if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, stridesk, boxk, "K cache", ek))) return rc;
         if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, strides, box, "V cache"))) return rc;
+        // chunk commits by TMA: the ring with a box of 128 bytes x kCommitRows rows x up to
+        // kCommitHeads heads, and a trial map of the caller side (permuted strides); where the
+        // driver declines either, commits use the copy kernel
+        const uint32_t hb = (uint32_t)(c.H < kCommitHeads ? c.H : kCommitHeads);
+        const uint32_t cboxk[5] = {(uint32_t)(128 / ek), (uint32_t)kCommitRows, 1, hb, 1};
+        const uint32_t cbox[5] = {64, (uint32_t)kCommitRows, 1, hb, 1};
+        CUtensorMap trial;
+        h->commit_tma = (c.d * ek) % 128 == 0 && (c.d * 2) % 128 == 0 &&
+                        encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cboxk, "K cache", ek) == SW_OK &&
+                        encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, strides, cbox, "V cache") == SW_OK &&
+                        encode_commit_src(&trial, ws + h->off_kcache, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek) ==
+                            SW_OK;
+        g_err.clear();
     }
     if (c.n_cond > 0) {
         const uint64_t dims[4] = {(uint64_t)c.d, (uint64_t)c.n_cond, (uint64_t)c.H, (uint64_t)c.B};
@@ -274,6 +300,29 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
     return SW_OK;
 }
 
+// One chunk commit of K and V ([B, T, H, d]) into the ring slot the device counter names, with
+// the counter advance and table rebuild in the same launch: TMA bulk copies (one CTA per SM),
+// or the copy kernel where the handle's maps could not be made.
+static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_t st) {
+    const sw_attn_config& c = h->cfg;
+    const int ek = c.qk_fp8 ? 1 : 2;
+    int32_t* state = reinterpret_cast<int32_t*>(h->ws);
+    cudaError_t e;
+    if (h->commit_tma) {
+        CommitMaps m;
+        int rc;
+        if ((rc = encode_commit_src(&m.src_k, K, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek))) return rc;
+        if ((rc = encode_commit_src(&m.src_v, V, c.B, c.tokens_per_chunk, c.H, c.d, "V", 2))) return rc;
+        m.dst_k = h->tm_commit_k;
+        m.dst_v = h->tm_commit_v;
+        e = launch_commit_tma(m, c.B, c.tokens_per_chunk, c.H, c.d, ek, state, table_advance(h), h->S, h->num_sms, st);
+    } else {
+        e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
+                            h->S * c.tokens_per_chunk, 1, h->S, state, table_advance(h), 1, st, ek);
+    }
+    return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
+}
+
 int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* stream) {
     g_err.clear();
     if (!h) return fail(SW_EINVAL, "null handle");
@@ -284,12 +333,7 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t* state = reinterpret_cast<int32_t*>(h->ws);
     cudaError_t e;
-    if (h->S > 0) {
-        // the copy's last block advances the counter and rebuilds the table: one launch
-        e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
-                            h->S * c.tokens_per_chunk, 1, h->S, state, table_advance(h), 1, st, c.qk_fp8 ? 1 : 2);
-        return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
-    }
+    if (h->S > 0) return launch_commit(h, K, V, st);
     e = launch_table_build(state, c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk, 1, st);
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "table build launch");
 }
@@ -312,6 +356,13 @@ int sw_attn_schedule_for(const sw_attn_t* h, int n_q) {
     g_err.clear();
     if (!h || n_q < 1) return fail(SW_EINVAL, "null handle or n_q < 1");
     return resolve_schedule(h, n_q);
+}
+
+int sw_attn_commit_kind(const sw_attn_t* h) {
+    g_err.clear();
+    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
+    return h->commit_tma ? SW_COMMIT_TMA : SW_COMMIT_COPY;
 }
 
 // Tensor maps, pointers and scalars every forward shares (the chunk's own n_q queries).
@@ -481,12 +532,7 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     if (resolve_schedule_tiles(h, nqt) == SW_SCHED_TRI) {
         // the three-buffer kernel does not store K/V: forward, then the copy into the same slot
         if ((rc = launch_full(h, p, st))) return rc;
-        if (h->S > 0) {   // the copy launch also advances the table
-            cudaError_t e = launch_relayout(K_cur, V_cur, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B,
-                                            c.tokens_per_chunk, c.H, c.d, h->S * c.tokens_per_chunk, 1, h->S, state,
-                                            table_advance(h), 1, st);
-            return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
-        }
+        if (h->S > 0) return launch_commit(h, K_cur, V_cur, st);   // the copy launch also advances the table
     } else {
         p.commit = h->S > 0 ? 1 : 0;
         if ((rc = launch_full(h, p, st))) return rc;

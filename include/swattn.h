@@ -264,6 +264,17 @@ SW_API int sw_attn_selftest_timeout(sw_attn_t *h, int64_t limit_ns, void *stream
  */
 SW_API int sw_attn_schedule_for(const sw_attn_t* h, int n_q);
 
+/*
+ * How this handle's chunk commits (sw_attn_append_chunk, and the copy after a committing forward
+ * on the three-buffer schedule) move K and V into the ring: SW_COMMIT_TMA (TMA bulk copies, one
+ * CTA per SM) or SW_COMMIT_COPY (the copy kernel, used where the driver declines the TMA maps or
+ * the handle has no ring).  Fixed at sw_attn_bind_workspace.  Host only, no CUDA call.  Returns
+ * the kind, SW_EINVAL for a null handle, or SW_ESTATE before a workspace is bound.
+ */
+#define SW_COMMIT_COPY 0
+#define SW_COMMIT_TMA 1
+SW_API int sw_attn_commit_kind(const sw_attn_t* h);
+
 /* Synchronise the device, then read the device status bits into *host_status. */
 SW_API int sw_attn_get_status(sw_attn_t *h, int32_t *host_status);
 

@@ -105,6 +105,36 @@ def test_cache_contents_match_ring_model(dev, W, sink):
     assert h.status() == 0
 
 
+@pytest.mark.parametrize("B,H,d,T", [(1, 24, 128, 300), (2, 3, 64, 17), (1, 32, 128, 130), (2, 50, 64, 9),
+                                     (1, 24, 128, 3180)])
+def test_commit_tma_matches_ring_model(dev, B, H, d, T):
+    """Chunk commits by TMA bulk copies (the kind a B200 handle resolves to): every slot bit-exact
+    against the oracle's ring model after every commit, empty slots untouched, tables advanced.
+    Shapes: one full head box and ragged row groups, fewer heads than a box, two head boxes (the
+    second partly past H), d = 64 (one column block) and the 720p chunk."""
+    from parity_util import check_cache_against_ring
+    W, chunks = 2, 6
+    wl = Workload("ct", B=B, H=H, d=d, T=T, n_cond=0, W=W, sink=True, chunks=chunks, steps=1)
+    h = make_handle(wl, dev)
+    assert h.commit_kind() == "tma"
+    kc, vc = h.cache_views()
+    kc.fill_(float("nan"))
+    vc.fill_(float("nan"))
+    ring = oracle.Ring(B=B, H=H, d=d, T=T, n_cond=0, W=W, sink=True, Kc=None, Vc=None)
+    held = {}
+    for c in range(chunks):
+        K = synth.draw((B, T, H, d), 900 + 2 * c)
+        V = synth.draw((B, T, H, d), 901 + 2 * c)
+        h.append_chunk(K.to(dev), V.to(dev))
+        ring.append(K, V)
+        held[c] = (K, V)
+        torch.cuda.synchronize()
+        check_cache_against_ring(h, ring, held)
+        ref = oracle.table(c + 1, W, True, 0, T)
+        assert np.array_equal(h.table().cpu().numpy()[:len(ref)], ref), c
+    assert h.status() == 0
+
+
 # ------------------------------------------------------------------ K3 / K4 attention
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
