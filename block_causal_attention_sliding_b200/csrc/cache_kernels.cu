@@ -182,42 +182,38 @@ __global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_consta
 
 // K2 with the tensor-memory accelerator: a chunk commit as TMA bulk copies.  The source map
 // reads the caller's [B, T, H, d] K (or V) with its dimensions ordered {d, t, h, b}, so one box
-// of kCommitRows token rows x h_box heads x 128 bytes of d lands in shared memory as
-// [head][row][128 B] -- exactly the layout of the same box of the head-major cache map
-// {d, T, S, H, B}.  Each item (K or V, stream, row group, head group, 128-byte column block) is
-// one TMA load and one TMA store from the same buffer; rows and heads past the ends read as
-// zero and are not stored.  One thread per CTA (one CTA per SM) streams its contiguous share of
+// of kCommitRows token rows x h_box heads x d lands in shared memory as [head][row][d] --
+// exactly the layout of the same box of the head-major cache map {d, T, S, H, B}.  Each item
+// (K or V, stream, row group, head group) is one TMA load and one TMA store from the same
+// buffer; rows and heads past the ends read as zero and are not stored.  One thread per CTA (one CTA per SM) streams its contiguous share of
 // the items through kCommitBufs buffers, refilling a buffer once the store issued from it one
 // item earlier has read it, so the other loads stay in flight.  Every wait is bounded; on a
 // timeout the status word records it and the thread still drains what it issued.
-constexpr int kCommitBufs = 8;     // buffers of up to 128 B x 8 rows x 24 heads = 24 KB
+constexpr int kCommitBufs = 8;     // buffers of up to 256 B x 4 rows x 24 heads = 24 KB
 
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
 struct CommitItems {
-    int B, T, H, nt, nh, cbk, cbv;   // streams, rows, heads, row groups, head groups, column blocks of K and V
-    int colk, colv;                  // elements per 128-byte column block of K and V
-    __device__ long long per_k() const { return (long long)B * nt * nh * cbk; }
-    __device__ long long total() const { return per_k() + (long long)B * nt * nh * cbv; }
-    // item -> (K or V, stream, first row, first head, first column)
-    __device__ void decode(long long i, int& kv, int& b, int& t0, int& h0, int& c0) const {
-        kv = i >= per_k();
-        if (kv) i -= per_k();
-        const int cb = kv ? cbv : cbk;
-        const int c = (int)(i % cb);
-        i /= cb;
+    int B, T, H, nt, nh;   // streams, rows, heads, row groups, head groups
+    __device__ long long per_kv() const { return (long long)B * nt * nh; }
+    __device__ long long total() const { return 2 * per_kv(); }
+    // item -> (K or V, stream, first row, first head)
+    __device__ void decode(long long i, int& kv, int& b, int& t0, int& h0) const {
+        kv = i >= per_kv();
+        if (kv) i -= per_kv();
         const int hg = (int)(i % nh);
         i /= nh;
         const int tg = (int)(i % nt);
         b = (int)(i / nt);
         t0 = tg * kCommitRows;
         h0 = hg * kCommitHeads;
-        c0 = c * (kv ? colv : colk);
     }
 };
 
 __global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant__ CommitMaps m, CommitItems it,
-                                                           int box_bytes, int32_t* state, TableAdvance ta, int S) {
+                                                           int box_k, int box_v, int32_t* state, TableAdvance ta,
+                                                           int S) {
+    const int box_bytes = box_k > box_v ? box_k : box_v;   // buffer stride (K may be e4m3)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kCommitBufs];
@@ -229,12 +225,12 @@ __global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant
         for (int q = 0; q < kCommitBufs; ++q) mbar_init(smem_u32(&full[q]), 1);
         fence_mbar_init();
         auto load = [&](long long i) {
-            int kv, b, t0, h0, c0;
-            it.decode(i, kv, b, t0, h0, c0);
+            int kv, b, t0, h0;
+            it.decode(i, kv, b, t0, h0);
             const int q = (int)((i - i0) % kCommitBufs);
             const uint32_t bar = smem_u32(&full[q]);
-            mbar_arrive_expect_tx(bar, box_bytes);
-            tma_load_4d(smem_u32(base + (size_t)q * box_bytes), kv ? &m.src_v : &m.src_k, bar, c0, t0, h0, b);
+            mbar_arrive_expect_tx(bar, kv ? box_v : box_k);
+            tma_load_4d(smem_u32(base + (size_t)q * box_bytes), kv ? &m.src_v : &m.src_k, bar, 0, t0, h0, b);
         };
         for (long long i = i0; i < i1 && i < i0 + kCommitBufs; ++i) load(i);
         int never = 0;
@@ -246,10 +242,10 @@ __global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant
                 atomicOr(state + 1, SW_STATUS_TIMEOUT);
                 break;
             }
-            int kv, b, t0, h0, c0;
-            it.decode(i, kv, b, t0, h0, c0);
+            int kv, b, t0, h0;
+            it.decode(i, kv, b, t0, h0);
             fence_proxy_async_smem();
-            tma_store_5d(kv ? &m.dst_v : &m.dst_k, smem_u32(base + (size_t)(k % kCommitBufs) * box_bytes), c0, t0, slot,
+            tma_store_5d(kv ? &m.dst_v : &m.dst_k, smem_u32(base + (size_t)(k % kCommitBufs) * box_bytes), 0, t0, slot,
                          h0, b);
             bulk_commit_group();
             // the buffer of item i - 1 takes item i - 1 + kCommitBufs once that item's store has
@@ -316,23 +312,19 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
 
 cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int32_t* state,
                               const TableAdvance& ta, int S, int ctas, cudaStream_t stream) {
-    if (B < 1 || T < 1 || H < 1 || ctas < 1 || (d * 2) % 128 != 0 || (d * k_esz) % 128 != 0) return cudaErrorInvalidValue;
+    if (B < 1 || T < 1 || H < 1 || ctas < 1 || (d * k_esz) % 16 != 0 || d * 2 > 256) return cudaErrorInvalidValue;
     CommitItems it;
     it.B = B;
     it.T = T;
     it.H = H;
     it.nt = (T + kCommitRows - 1) / kCommitRows;
     it.nh = (H + kCommitHeads - 1) / kCommitHeads;
-    it.cbk = d * k_esz / 128;
-    it.cbv = d * 2 / 128;
-    it.colk = 128 / k_esz;
-    it.colv = 64;
     const int h_box = H < kCommitHeads ? H : kCommitHeads;
-    const int box_bytes = 128 * kCommitRows * h_box;
-    const int smem = kCommitBufs * box_bytes + 1024;
+    const int box_k = d * k_esz * kCommitRows * h_box, box_v = d * 2 * kCommitRows * h_box;
+    const int smem = kCommitBufs * (box_k > box_v ? box_k : box_v) + 1024;
     cudaError_t e = cudaFuncSetAttribute(commit_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    commit_tma_kernel<<<ctas, 32, smem, stream>>>(maps, it, box_bytes, state, ta, S);
+    commit_tma_kernel<<<ctas, 32, smem, stream>>>(maps, it, box_k, box_v, state, ta, S);
     return cudaGetLastError();
 }
 

@@ -6,12 +6,13 @@
 namespace swattn {
 
 // src maps over the caller's K and V ([B, T, H, d], dimensions ordered {d, t, h, b}); dst maps
-// over the ring ({d, T, S, H, B}); boxes of 128 bytes x kCommitRows rows x min(H, kCommitHeads)
-// heads, 128-byte swizzle on both sides, so a loaded box is stored as it lies.
+// over the ring ({d, T, S, H, B}); boxes of whole d rows x kCommitRows rows x min(H, kCommitHeads)
+// heads, unswizzled on both sides (no thread reads the buffers), so a loaded box is stored as it
+// lies.  With H <= kCommitHeads a source box is kCommitRows whole token rows, contiguous.
 struct CommitMaps {
     CUtensorMap src_k, src_v, dst_k, dst_v;
 };
-constexpr int kCommitRows = 8;
+constexpr int kCommitRows = 4;
 constexpr int kCommitHeads = 24;
 
 // Copy the finished chunk into the ring slot the device counter names, then (last CTA) advance

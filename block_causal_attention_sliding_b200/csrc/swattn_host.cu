@@ -75,10 +75,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Tiled map with 128-byte swizzle and 128-byte box rows (64 bf16 or 128 e4m3 columns, esz = 2
-// or 1 bytes per element); out-of-range rows read as zero.
+// Tiled map, by default with 128-byte swizzle and 128-byte box rows (64 bf16 or 128 e4m3 columns,
+// esz = 2 or 1 bytes per element); out-of-range rows read as zero.
 int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-           const uint32_t* box, const char* what, int esz = 2) {
+           const uint32_t* box, const char* what, int esz = 2,
+           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto fn = encode_fn();
     if (!fn) return fail(SW_ECUDA, "cuTensorMapEncodeTiled unavailable");
     uint32_t estr[5] = {1, 1, 1, 1, 1};
@@ -86,7 +87,7 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, cons
                     const_cast<void*>(ptr),
                     reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides),
                     reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(SW_ECUDA, "tensor map for %s: CUresult %d", what, (int)r);
     return SW_OK;
@@ -101,13 +102,13 @@ int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, con
 }
 
 // The caller's [B, T, H, d] K or V for a TMA chunk commit: dims ordered {d, t, h, b} (strides
-// T: H*d, h: d, b: T*H*d elements), box 128 bytes x kCommitRows rows x min(H, kCommitHeads) heads.
+// T: H*d, h: d, b: T*H*d elements), box d x kCommitRows rows x min(H, kCommitHeads) heads,
+// unswizzled.
 int encode_commit_src(CUtensorMap* m, const void* ptr, int B, int T, int H, int d, const char* what, int esz) {
     const uint64_t dims[4] = {(uint64_t)d, (uint64_t)T, (uint64_t)H, (uint64_t)B};
     const uint64_t strides[3] = {(uint64_t)H * d * esz, (uint64_t)d * esz, (uint64_t)T * H * d * esz};
-    const uint32_t box[4] = {(uint32_t)(128 / esz), (uint32_t)kCommitRows,
-                             (uint32_t)(H < kCommitHeads ? H : kCommitHeads), 1};
-    return encode(m, ptr, 4, dims, strides, box, what, esz);
+    const uint32_t box[4] = {(uint32_t)d, (uint32_t)kCommitRows, (uint32_t)(H < kCommitHeads ? H : kCommitHeads), 1};
+    return encode(m, ptr, 4, dims, strides, box, what, esz, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 int check_cfg(const sw_attn_config& c) {
@@ -229,18 +230,18 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint32_t boxk[5] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1, 1};
         if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, stridesk, boxk, "K cache", ek))) return rc;
         if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, strides, box, "V cache"))) return rc;
-        // chunk commits by TMA: the ring with a box of 128 bytes x kCommitRows rows x up to
-        // kCommitHeads heads, and a trial map of the caller side (permuted strides); where the
+        // chunk commits by TMA: the ring with a box of d x kCommitRows rows x up to kCommitHeads
+        // heads (unswizzled), and a trial map of the caller side (permuted strides); where the
         // driver declines either, commits use the copy kernel
         const uint32_t hb = (uint32_t)(c.H < kCommitHeads ? c.H : kCommitHeads);
-        const uint32_t cboxk[5] = {(uint32_t)(128 / ek), (uint32_t)kCommitRows, 1, hb, 1};
-        const uint32_t cbox[5] = {64, (uint32_t)kCommitRows, 1, hb, 1};
+        const uint32_t cbox[5] = {(uint32_t)c.d, (uint32_t)kCommitRows, 1, hb, 1};
         CUtensorMap trial;
-        h->commit_tma = (c.d * ek) % 128 == 0 && (c.d * 2) % 128 == 0 &&
-                        encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cboxk, "K cache", ek) == SW_OK &&
-                        encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, strides, cbox, "V cache") == SW_OK &&
-                        encode_commit_src(&trial, ws + h->off_kcache, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek) ==
-                            SW_OK;
+        h->commit_tma =
+            encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cbox, "K cache", ek,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
+            encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, strides, cbox, "V cache", 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
+            encode_commit_src(&trial, ws + h->off_kcache, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek) == SW_OK;
         g_err.clear();
     }
     if (c.n_cond > 0) {
