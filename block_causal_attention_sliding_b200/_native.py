@@ -14,6 +14,7 @@ SW_OK, SW_EINVAL, SW_ESHAPE, SW_EALIGN, SW_ESTATE, SW_ECUDA = 0, -1, -2, -3, -4,
 SW_STATUS_TIMEOUT, SW_STATUS_BAD_SLOT, SW_STATUS_OVERFLOW = 0x1, 0x2, 0x4
 SW_OUT_BF16, SW_OUT_F32 = 0, 1
 SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
+SW_COMMIT_AUTO, SW_COMMIT_COPY, SW_COMMIT_TMA = 0, 1, 2
 
 # every symbol include/swattn.h declares
 EXPORTS = (
@@ -32,7 +33,8 @@ class SwAttnConfig(ctypes.Structure):
                 ("tokens_per_chunk", ctypes.c_int), ("W", ctypes.c_int), ("n_cond", ctypes.c_int),
                 ("sink", ctypes.c_int), ("out_dtype", ctypes.c_int), ("scale", ctypes.c_float),
                 ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int), ("commit_in_forward", ctypes.c_int),
-                ("qk_fp8", ctypes.c_int), ("q_scale", ctypes.c_float), ("k_scale", ctypes.c_float)]
+                ("qk_fp8", ctypes.c_int), ("q_scale", ctypes.c_float), ("k_scale", ctypes.c_float),
+                ("commit_path", ctypes.c_int)]
 
 
 class SwAttnError(RuntimeError):

@@ -34,7 +34,8 @@ class SlidingWindowAttention:
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
                  max_short_q: int = 0, schedule: str = "auto", commit_in_forward: bool = False,
-                 qk_fp8: bool = False, q_scale: float = 1.0, k_scale: float = 1.0, device=None):
+                 qk_fp8: bool = False, q_scale: float = 1.0, k_scale: float = 1.0, commit_path: str = "auto",
+                 device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
@@ -43,7 +44,9 @@ class SlidingWindowAttention:
                              schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
                                        "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule],
                              commit_in_forward=int(bool(commit_in_forward)), qk_fp8=int(bool(qk_fp8)),
-                             q_scale=float(q_scale), k_scale=float(k_scale))
+                             q_scale=float(q_scale), k_scale=float(k_scale),
+                             commit_path={"auto": N.SW_COMMIT_AUTO, "copy": N.SW_COMMIT_COPY,
+                                          "tma": N.SW_COMMIT_TMA}[commit_path])
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()
@@ -68,7 +71,7 @@ class SlidingWindowAttention:
         r = int(self._lib.sw_attn_commit_kind(self._h))
         if r < 0:
             N.check(r)
-        return "tma" if r == 1 else "copy"
+        return "tma" if r == N.SW_COMMIT_TMA else "copy"
 
     def schedule_for(self, n_q: int | None = None) -> str:
         """The schedule a full-path forward of n_q queries (default T) runs with."""

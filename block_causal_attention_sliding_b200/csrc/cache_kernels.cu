@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_consta
 // the items through kCommitBufs buffers, refilling a buffer once the store issued from it one
 // item earlier has read it, so the other loads stay in flight.  Every wait is bounded; on a
 // timeout the status word records it and the thread still drains what it issued.
-constexpr int kCommitBufs = 8;     // buffers of up to 256 B x 4 rows x 24 heads = 24 KB
+// kCommitBufs buffers of up to 256 B x 4 rows x 24 heads = 24 KB
 
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 

@@ -14,6 +14,7 @@ struct CommitMaps {
 };
 constexpr int kCommitRows = 4;
 constexpr int kCommitHeads = 24;
+constexpr int kCommitBufs = 8;   // buffers per CTA (one CTA per SM)
 
 // Copy the finished chunk into the ring slot the device counter names, then (last CTA) advance
 // the counter and rebuild the table.  ctas: one per SM.  k_esz: bytes per K element (1: e4m3).

@@ -129,6 +129,8 @@ int check_cfg(const sw_attn_config& c) {
     if (c.qk_fp8 && c.d != 128) return fail(SW_ESHAPE, "e4m3 Q/K need d = 128");
     if (c.qk_fp8 && c.commit_in_forward) return fail(SW_ESHAPE, "commit_in_forward is not available with e4m3 Q/K");
     if (!std::isfinite(c.q_scale) || !std::isfinite(c.k_scale)) return fail(SW_EINVAL, "scales must be finite");
+    if (c.commit_path != SW_COMMIT_AUTO && c.commit_path != SW_COMMIT_COPY && c.commit_path != SW_COMMIT_TMA)
+        return fail(SW_EINVAL, "bad commit_path");
     const double elems = (double)c.B * c.H * (c.W + 2) * c.tokens_per_chunk * c.d;
     if (elems > 4.0e12 || (double)c.tokens_per_chunk * c.H * c.B > 2.0e9 ||
         (double)c.n_cond * c.H * c.B > 2.0e9)
@@ -191,7 +193,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     c.B = 1; c.H = H; c.d = d; c.tokens_per_chunk = tokens_per_chunk; c.W = W; c.n_cond = n_cond;
     c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_AUTO;
     c.commit_in_forward = 0;
-    c.qk_fp8 = 0; c.q_scale = 0.f; c.k_scale = 0.f;
+    c.qk_fp8 = 0; c.q_scale = 0.f; c.k_scale = 0.f; c.commit_path = SW_COMMIT_AUTO;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -236,7 +238,12 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint32_t hb = (uint32_t)(c.H < kCommitHeads ? c.H : kCommitHeads);
         const uint32_t cbox[5] = {(uint32_t)c.d, (uint32_t)kCommitRows, 1, hb, 1};
         CUtensorMap trial;
-        h->commit_tma =
+        // auto: TMA only when every SM gets at least a full ring of items
+        const long long items = 2LL * c.B * ((c.tokens_per_chunk + kCommitRows - 1) / kCommitRows) *
+                                ((c.H + kCommitHeads - 1) / kCommitHeads);
+        const bool want = c.commit_path == SW_COMMIT_TMA ||
+                          (c.commit_path == SW_COMMIT_AUTO && items >= (long long)kCommitBufs * sms);
+        h->commit_tma = want &&
             encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cbox, "K cache", ek,
                    CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
             encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, strides, cbox, "V cache", 2,

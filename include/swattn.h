@@ -91,6 +91,9 @@ typedef struct {
                                 (no split-K path, no commit_in_forward) */
     float q_scale, k_scale;  /* dequantisation scales of the e4m3 Q and K (per tensor; <= 0
                                 selects 1): the attention uses q * q_scale and k * k_scale */
+    int   commit_path;       /* chunk commits: SW_COMMIT_AUTO (default; TMA bulk copies when
+                                the commit gives every SM at least a full ring of 8 items, else
+                                the copy kernel), SW_COMMIT_TMA or SW_COMMIT_COPY */
 } sw_attn_config;
 
 /* schedules of the full path */
@@ -267,12 +270,15 @@ SW_API int sw_attn_schedule_for(const sw_attn_t* h, int n_q);
 /*
  * How this handle's chunk commits (sw_attn_append_chunk, and the copy after a committing forward
  * on the three-buffer schedule) move K and V into the ring: SW_COMMIT_TMA (TMA bulk copies, one
- * CTA per SM) or SW_COMMIT_COPY (the copy kernel, used where the driver declines the TMA maps or
- * the handle has no ring).  Fixed at sw_attn_bind_workspace.  Host only, no CUDA call.  Returns
+ * CTA per SM) or SW_COMMIT_COPY (the copy kernel).  Chosen at sw_attn_bind_workspace from the
+ * config's commit_path: the copy kernel where the driver declines the TMA maps or the handle has
+ * no ring, and under SW_COMMIT_AUTO also for commits too small to fill every SM's ring of 8
+ * items (at 480p the copy kernel is faster; at 720p TMA is).  Host only, no CUDA call.  Returns
  * the kind, SW_EINVAL for a null handle, or SW_ESTATE before a workspace is bound.
  */
-#define SW_COMMIT_COPY 0
-#define SW_COMMIT_TMA 1
+#define SW_COMMIT_AUTO 0
+#define SW_COMMIT_COPY 1
+#define SW_COMMIT_TMA 2
 SW_API int sw_attn_commit_kind(const sw_attn_t* h);
 
 /* Synchronise the device, then read the device status bits into *host_status. */

@@ -35,12 +35,12 @@ def sample_rows(n_q: int, n: int, seed: int) -> np.ndarray:
 
 
 def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink=None, n_cond=None,
-                schedule="auto", commit_in_forward=False):
+                schedule="auto", commit_in_forward=False, commit_path="auto"):
     return SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W if W is None else W,
                                   n_cond=wl.n_cond if n_cond is None else n_cond,
                                   sink=wl.sink if sink is None else sink, out_dtype=out_dtype,
                                   max_short_q=max_short_q, schedule=schedule,
-                                  commit_in_forward=commit_in_forward, device=dev)
+                                  commit_in_forward=commit_in_forward, commit_path=commit_path, device=dev)
 
 
 def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, n_q=None,

@@ -108,14 +108,14 @@ def test_cache_contents_match_ring_model(dev, W, sink):
 @pytest.mark.parametrize("B,H,d,T", [(1, 24, 128, 300), (2, 3, 64, 17), (1, 32, 128, 130), (2, 50, 64, 9),
                                      (1, 24, 128, 3180)])
 def test_commit_tma_matches_ring_model(dev, B, H, d, T):
-    """Chunk commits by TMA bulk copies (the kind a B200 handle resolves to): every slot bit-exact
-    against the oracle's ring model after every commit, empty slots untouched, tables advanced.
-    Shapes: one full head box and ragged row groups, fewer heads than a box, two head boxes (the
-    second partly past H), d = 64 (one column block) and the 720p chunk."""
+    """Chunk commits by TMA bulk copies (forced where the automatic choice would take the copy
+    kernel): every slot bit-exact against the oracle's ring model after every commit, empty slots
+    untouched, tables advanced.  Shapes: one full head box and ragged row groups, fewer heads than
+    a box, two head boxes (the second partly past H), d = 64 and the 720p chunk."""
     from parity_util import check_cache_against_ring
     W, chunks = 2, 6
     wl = Workload("ct", B=B, H=H, d=d, T=T, n_cond=0, W=W, sink=True, chunks=chunks, steps=1)
-    h = make_handle(wl, dev)
+    h = make_handle(wl, dev, commit_path="tma")
     assert h.commit_kind() == "tma"
     kc, vc = h.cache_views()
     kc.fill_(float("nan"))
@@ -133,6 +133,22 @@ def test_commit_tma_matches_ring_model(dev, B, H, d, T):
         ref = oracle.table(c + 1, W, True, 0, T)
         assert np.array_equal(h.table().cpu().numpy()[:len(ref)], ref), c
     assert h.status() == 0
+
+
+def test_commit_path_choice(dev):
+    """The automatic commit path: TMA where every SM gets a full ring of items (720p, stress),
+    the copy kernel for smaller commits (480p, tiny); either can be forced."""
+    kinds = {}
+    for name in ("tiny", "480p", "720p", "stress"):
+        wl = WORKLOADS[name]
+        h = make_handle(wl, dev)
+        kinds[name] = h.commit_kind()
+        h.close()
+    assert kinds == {"tiny": "copy", "480p": "copy", "720p": "tma", "stress": "tma"}, kinds
+    wl = WORKLOADS["720p"]
+    h = make_handle(wl, dev, commit_path="copy")
+    assert h.commit_kind() == "copy"
+    h.close()
 
 
 # ------------------------------------------------------------------ K3 / K4 attention
