@@ -185,11 +185,12 @@ __global__ void __launch_bounds__(512) relayout_batch_kernel(const __grid_consta
 // of kCommitRows token rows x h_box heads x d lands in shared memory as [head][row][d] --
 // exactly the layout of the same box of the head-major cache map {d, T, S, H, B}.  Each item
 // (K or V, stream, row group, head group) is one TMA load and one TMA store from the same
-// buffer; rows and heads past the ends read as zero and are not stored.  One thread per CTA (one CTA per SM) streams its contiguous share of
-// the items through kCommitBufs buffers, refilling a buffer once the store issued from it one
-// item earlier has read it, so the other loads stay in flight.  Every wait is bounded; on a
-// timeout the status word records it and the thread still drains what it issued.
-// kCommitBufs buffers of up to 256 B x 4 rows x 24 heads = 24 KB
+// buffer; rows and heads past the ends read as zero and are not stored.  Both maps are
+// unswizzled (no thread reads the buffers).  One thread per CTA (one CTA per SM) streams its
+// contiguous share of the items through kCommitBufs buffers (up to 256 B x 4 rows x 24 heads =
+// 24 KB each), refilling a buffer once the store issued from it one item earlier has read it, so
+// the other loads stay in flight.  Every wait is bounded; on a timeout the status word records
+// it and the thread still drains what it issued.
 
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
