@@ -566,14 +566,17 @@ def test_fp8_qk_joint(dev):
     assert len(res) == 2 * wl.chunks * wl.steps
 
 
-def test_fp8_qk_cache_bytes(dev):
-    """The e4m3 K cache holds exactly the appended e4m3 keys (bit for bit) at half the bytes."""
+@pytest.mark.parametrize("commit_path", ["copy", "tma"])
+def test_fp8_qk_cache_bytes(dev, commit_path):
+    """The e4m3 K cache holds exactly the appended e4m3 keys (bit for bit) at half the bytes, with
+    either commit path (the TMA one moves K in boxes of 128-byte rows, V in 256-byte rows)."""
     wl = dataclasses.replace(RAGGED, chunks=3)
     sc = synth.FP8_SCALE
     h = make_handle(wl, dev)
     from block_causal_attention_sliding_b200.api import SlidingWindowAttention
     h8 = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
-                                qk_fp8=True, q_scale=sc, k_scale=sc, device=dev)
+                                qk_fp8=True, q_scale=sc, k_scale=sc, commit_path=commit_path, device=dev)
+    assert h8.commit_kind() == commit_path
     assert h8.workspace_bytes() < h.workspace_bytes()
     kc, vc = h8.cache_views()
     for c in range(wl.chunks):
