@@ -5,7 +5,7 @@
 // visibility table lists (condition tokens, sink, window chunks, current chunk; agifrontier
 // tutorial "JoyAI-Video-Edit：单卡720p 30帧，两步蒸馏攻克流式视频编辑", section
 // "从双向编辑到分块因果架构的蜕变") -- for a query set too small to fill the GPU with query
-// tiles.  The key tiles of each (b, h) are cut into `splits` contiguous slices, one CTA per
+// tiles.  The key tiles of each (b, h) are dealt round-robin to `splits` slices, one CTA per
 // slice; each CTA writes the unnormalised partial (O, m, l) of its slice and the combine kernel
 // (below; a programmatic dependent launch) merges the slices with a log-sum-exp weighting.
 //
@@ -117,9 +117,11 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
 
     const uint32_t tmem = ctl->tmem_base;
     const int n_tiles = ctl->n_tiles;
-    const int t0 = (int)((long long)blockIdx.x * n_tiles / p.splits);
-    const int t1 = (int)((long long)(blockIdx.x + 1) * n_tiles / p.splits);
-    const int n = t1 - t0;   // key tiles of this slice
+    // slice s takes key tiles s, s + splits, s + 2 splits, ...: every slice gets the same mix of
+    // contiguous cache tiles and current-chunk tiles (read from the caller's [B, T, H, d] layout,
+    // 128 separate rows each), so the slices finish together
+    const int sl = blockIdx.x, ns = p.splits;
+    const int n = sl < n_tiles ? (n_tiles - sl + ns - 1) / ns : 0;   // key tiles of this slice
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -130,7 +132,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
                 tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * kBoxCols, h, 0, b);
             uint32_t it = 0;
             bool ok = true;
-            for (int j = t0; j < t1 && ok; ++j) {
+            for (int jj = 0, j = sl; jj < n && ok; ++jj, j += ns) {
                 for (int kv = 0; kv < 2; ++kv, ++it) {
                     const int s = it % kStages;
                     if (!wait_or_abort(smem_u32(&ctl->kv_empty[s]), ((it / kStages) & 1) ^ 1, abort_flag)) {
@@ -210,7 +212,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
         bool ok = true;
         for (int jj = 0; jj < n; ++jj) {
             int seg, row0, valid;
-            tile_of(ctl, t0 + jj, seg, row0, valid);
+            tile_of(ctl, sl + jj * ns, seg, row0, valid);
             const int buf = jj & 1;
             ok = warp_wait(smem_u32(&ctl->s_full[buf]), (jj >> 1) & 1, abort_flag);
             if (!ok) break;
