@@ -60,6 +60,8 @@ def _load():
     lib.swo_slot_r.restype = i32
     lib.swo_table_r.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32]
     lib.swo_table_r.restype = i32
+    lib.swo_vis_row.argtypes = [i32, i32, i32, vp, i32]
+    lib.swo_vis_row.restype = i32
     lib.swo_ring_create_r.argtypes = [i32] * 8 + [vp, vp]
     lib.swo_ring_create_r.restype = vp
     lib.swo_attention.argtypes = [i32] * 8 + [vp, vp, vp, vp, vp, i32, vp, vp, dbl, vp, i32, vp]
@@ -117,6 +119,16 @@ def table(k: int, W: int, sink: bool, n_cond: int, T: int, R: int | None = None)
     n = _load().swo_table_r(k, W, W if R is None else R, int(sink), n_cond, T, out.ctypes.data, cap)
     if n < 0:
         raise RuntimeError("swo_table: capacity")
+    return out[:n].copy()
+
+
+def vis_row(k: int, W: int, sink: bool) -> np.ndarray:
+    """Chunk bitmap row of the visibility table: uint8 [k], entry j = 1 iff history chunk j is
+    visible to active chunk k (the current chunk itself is not part of the row)."""
+    out = np.zeros(max(k, 1), dtype=np.uint8)
+    n = _load().swo_vis_row(k, W, int(sink), out.ctypes.data, out.shape[0])
+    if n < 0:
+        raise RuntimeError("swo_vis_row: bad arguments")
     return out[:n].copy()
 
 

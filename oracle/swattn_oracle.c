@@ -129,6 +129,20 @@ int swo_table(int k, int W, int sink, int n_cond, int T, int32_t *out, int cap)
     return swo_table_r(k, W, W, sink, n_cond, T, out, cap);
 }
 
+/*
+ * The chunk-level bitmap row of the visibility table for active chunk k: row[j] = 1 iff
+ * history chunk j is in Hist(k), for every j < k (chunk k itself, the current chunk, is always
+ * visible and is not part of the row).  This is the dense mask of the definition above taken
+ * at chunk granularity ([TUT] §从双向编辑到分块因果架构的蜕变: recent window plus the first chunk;
+ * [NH] §Чанки и борьба с дрейфом).  Writes k bytes; returns k, or -1 if cap < k.
+ */
+int swo_vis_row(int k, int W, int sink, unsigned char *row, int cap)
+{
+    if (k < 0 || cap < k) return -1;
+    for (int j = 0; j < k; j++) row[j] = (unsigned char)swo_visible(k, W, sink, j);
+    return k;
+}
+
 /* ---------------------------------------------------------------- dense oracle */
 
 static double dot_f(const float *a, const float *b, int d)

@@ -160,6 +160,9 @@ def test_golden_visibility_rule(oracle_mod, W, sink, k, vis, slots):
     segs = tab[3:].reshape(-1, 4)
     cache = segs[segs[:, 0] == 1]
     assert list(cache[:, 1]) == vis and list(cache[:, 2]) == slots
+    # and the chunk bitmap row marks exactly those chunks
+    row = oracle_mod.vis_row(k, W, sink)
+    assert row.shape == (k,) and list(np.flatnonzero(row)) == vis
 
 
 def test_golden_visible_keys(oracle_mod):
@@ -191,6 +194,10 @@ def test_tables_brute_force(oracle_mod, W, sink):
         assert list(segs[1:-1, 2]) == [where[j] for j in vis]
         assert tuple(segs[-1]) == (2, k, -1, 11)
         assert tab[2] == 3 + 11 * (len(vis) + 1)
+        # the chunk bitmap row: vis[k][j] = [j in Hist(k)] for every j < k, 0/1 only
+        row = oracle_mod.vis_row(k, W, sink)
+        assert row.shape == (k,) and set(np.unique(row)) <= {0, 1}
+        assert list(np.flatnonzero(row)) == vis
         # |Hist(k)| = min(k, W+1) with the sink, min(k, W) without
         assert len(vis) == (min(k, W + 1) if sink else min(k, W))
         if sink and k >= 1:
