@@ -13,8 +13,8 @@ namespace swattn {
 
 // K1: advance the counter (after an append) and write the visibility table of the active
 // chunk k: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...], in the order
-// condition, sink, window ascending, current; slots of a ring with R window slots.  One
-// thread: a few dozen integers.
+// condition, sink, window ascending, current; slots of a ring with R window slots; then the
+// chunk bitmap row (see table_vis_offset).  One thread: a few dozen integers.
 __device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance, int reset) {
     int32_t* tab = state + kStateHeaderInts;
     if (reset) {
@@ -31,7 +31,7 @@ __device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, 
             state[0] = k;
         }
     }
-    const int cap = table_ints_for(W);
+    const int cap = table_vis_offset(W);
     int pos = 3, nseg = 0, nvis = 0;
     auto put = [&](int kind, int chunk, int slot, int n) {
         tab[pos++] = kind; tab[pos++] = chunk; tab[pos++] = slot; tab[pos++] = n;
@@ -44,6 +44,15 @@ __device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, 
     put(2, k, -1, T);
     tab[0] = k; tab[1] = nseg; tab[2] = nvis;
     for (int i = pos; i < cap; ++i) tab[i] = -1;
+    // the chunk bitmap row vis[k][j] = [j in Hist(k)], j < k, in its constant-size form
+    uint32_t w[2] = {0u, 0u};
+    for (int i = 0; i < kVisSpan; ++i) {
+        const int j = k - kVisSpan + i;
+        if (j >= 0 && (j >= first_win || (sink && j == 0))) w[i >> 5] |= 1u << (i & 31);
+    }
+    tab[cap + 0] = (k >= 1 && (sink || first_win == 0)) ? 1 : 0;
+    tab[cap + 1] = (int32_t)w[0];
+    tab[cap + 2] = (int32_t)w[1];
 }
 
 __global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,

@@ -664,6 +664,8 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
     if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, n_q))) return rc;
     const int bh = c.B * c.H;
     long long splits = h->num_sms / bh;
+    // the same split count as sw_attn_forward; the clamp to what fits the array only binds on a
+    // GPU with more SMs than a B200 (there fit >= 148 / (B*H) for every accepted shape)
     splits = std::max<long long>(1, std::min<long long>(splits, std::min<long long>((long long)fit, kMaxSplits)));
     p.splits = (int)splits;
     p.o_part = scratch;

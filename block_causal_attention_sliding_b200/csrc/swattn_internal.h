@@ -17,7 +17,16 @@ constexpr int kMaxShortQ = 128;    // split-K path handles one Q tile per (b, h)
 constexpr int kMaxSplits = 64;
 constexpr int kMaxPersistentCtas = 160;   // >= SMs of a B200 (148)
 
-__host__ __device__ inline int table_ints_for(int W) { return 3 + 4 * (W + 3); }
+// The visibility table: [k, n_segments, N_vis], then 4 ints per segment for up to W + 3
+// segments (unused ones -1), then the chunk bitmap row in 3 ints (table_vis_offset):
+//   [vis_sink, vis_lo, vis_hi]: vis_sink = 1 iff chunk 0 is visible; bit i of the 64-bit word
+//   vis_hi:vis_lo = 1 iff chunk k - 64 + i is visible (bits of chunks before 0 are 0).
+// Every visible history chunk is the sink or one of the W <= 64 most recent chunks, so these
+// three words fix the whole row vis[k][j], j < k, in constant space however long the stream.
+constexpr int kVisWords = 3;
+constexpr int kVisSpan = 64;   // chunks covered by the bitmap row's window word
+__host__ __device__ inline int table_vis_offset(int W) { return 3 + 4 * (W + 3); }
+__host__ __device__ inline int table_ints_for(int W) { return table_vis_offset(W) + kVisWords; }
 
 // Ring slot of committed chunk c with R window slots: the sink (if any) owns slot 0 and window
 // chunks rotate through the R slots after it, chunk c taking the slot of chunk c - R.  R = W

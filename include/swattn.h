@@ -218,15 +218,20 @@ SW_API int sw_attn_forward_joint(sw_attn_t *h, const void *Q, const void *Q_cond
  * paper has no counterpart: this is an interface convenience of this library.
  *
  * Limits and behaviour:
- *   - The fixed array holds 4 Mi floats (16 MiB).  Each key split needs B*H*128*(d+2) floats;
- *     the call uses as many splits as fit (up to one per SM per (b, h)) and rejects with
- *     SW_ESHAPE a shape where not even one split fits (B*H > 252 at d = 128, > 496 at d = 64).
+ *   - The fixed array holds 4 Mi floats (16 MiB).  The call uses the same split count as
+ *     sw_attn_forward (one key split per SM per (b, h)), so its output equals that call's bit
+ *     for bit; the array only limits which shapes are accepted: each split needs
+ *     B*H*128*(d+2) floats, and a shape whose splits do not fit is rejected with SW_ESHAPE
+ *     (B*H > 252 at d = 128, > 496 at d = 64).  The clamp of the split count to what fits is
+ *     a guard for GPUs with more SMs; on a 148-SM B200 it never binds.
  *   - Every GPU that loads the library holds the 16 MiB until the process exits.
  *   - The array is shared by every call in the process and keeps the last call's contents;
  *     every split writes its own partials before the merge reads them, so nothing needs
  *     clearing, but calls that overlap on the GPU (two streams, two threads) race on it.
  *   - The first call on each device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current) and keeps it for the life of the process; make that first call before any
+ *     stream capture.  A device reset (cudaDeviceReset) invalidates the kept address: no call
+ *     may follow a reset of the device in the same process.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.  Same argument rules as
  *     sw_attn_forward; the caller's current device must be the workspace's device.
  *   - Handles with e4m3 Q/K (qk_fp8) have no split-K form: SW_ESTATE.
@@ -234,14 +239,21 @@ SW_API int sw_attn_forward_joint(sw_attn_t *h, const void *Q, const void *Q_cond
 SW_API int sw_attn_forward_short_noalloc(sw_attn_t *h, const void *Q, const void *K_cur,
                                          const void *V_cur, void *out, int n_q, void *stream);
 
-/* Number of int32 entries of the visibility table (3 + 4 * (W + 3)). */
+/* Number of int32 entries of the visibility table (3 + 4 * (W + 3) + 3). */
 SW_API int sw_attn_table_ints(const sw_attn_t *h);
 
 /*
  * Copy the device visibility table for the active chunk into dev_table (device memory,
- * sw_attn_table_ints entries): [k, n_segments, N_vis, then per segment (kind, chunk_id,
- * slot, n_tokens)], kind 0 = condition, 1 = cached chunk, 2 = current chunk; order:
- * condition, sink, window chunks ascending, current; unused entries are -1.
+ * sw_attn_table_ints entries):
+ *   [0..2]  k, n_segments, N_vis;
+ *   [3 .. 3 + 4 (W + 3))  per segment (kind, chunk_id, slot, n_tokens), kind 0 = condition,
+ *           1 = cached chunk, 2 = current chunk; order: condition, sink, window chunks
+ *           ascending, current; unused entries are -1;
+ *   [3 + 4 (W + 3) .. + 3)  the chunk bitmap row vis[k][j] = [chunk j is visible], j < k, in
+ *           constant size: vis_sink (1 iff chunk 0 is visible), then vis_lo, vis_hi, where bit
+ *           i of the 64-bit word vis_hi:vis_lo is vis[k][k - 64 + i] (0 for chunks before 0).
+ *           Every other entry of the row is 0: a visible history chunk is the sink or one of
+ *           the W <= 64 most recent (tutorial, section "从双向编辑到分块因果架构的蜕变").
  */
 SW_API int sw_attn_get_table(const sw_attn_t *h, int32_t *dev_table, void *stream);
 

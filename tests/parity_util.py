@@ -2,6 +2,9 @@
 FP64 oracle on the same seeded inputs, and compare."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -13,25 +16,100 @@ MAX_ABS = 1e-2      # tolerances on fp32 output, against the FP64 oracle
 MEAN_REL = 2e-3     # mean-relative = sum |got - ref| / sum |ref|
 
 
+BF16_U = 2.0 ** -8   # unit roundoff of bf16 (8 significant bits, round to nearest even)
+
+
+def bf16_out_tol(ref: np.ndarray, max_abs: float = MAX_ABS, mean_rel: float = MEAN_REL):
+    """Tolerance for bf16 output, derived from the fp32 one.  The kernel computes the output
+    in fp32 and rounds it once to bf16, which moves each value by at most BF16_U of itself:
+    |got - ref| <= |fp32 - ref| + BF16_U (|ref| + |fp32 - ref|).  So max-abs grows by
+    BF16_U (max|ref| + max_abs) and mean-relative by BF16_U (1 + mean_rel)."""
+    top = float(np.abs(ref).max()) if ref.size else 0.0
+    return max_abs + BF16_U * (top + max_abs), mean_rel + BF16_U * (1.0 + mean_rel)
+
+
+def _log_errors(ma: float, mr: float, n: int, tol) -> None:
+    """Append the observed errors to the file named by SWATTN_PARITY_LOG (one JSON line per
+    comparison, tagged with the running test), when that variable is set."""
+    path = os.environ.get("SWATTN_PARITY_LOG")
+    if not path:
+        return
+    rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], "max_abs": ma, "mean_rel": mr,
+           "values": n, "tol": [float(tol[0]), float(tol[1])]}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def compare(got: np.ndarray, ref: np.ndarray, max_abs: float = MAX_ABS, mean_rel: float = MEAN_REL):
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.isfinite(got).all(), "non-finite output"
     d = np.abs(got.astype(np.float64) - ref)
     ma = float(d.max())
     mr = float(d.sum() / max(np.abs(ref).sum(), 1e-300))
+    _log_errors(ma, mr, int(d.size), (max_abs, mean_rel))
     assert ma <= max_abs and mr <= mean_rel, f"max-abs {ma:.3e} (<= {max_abs}), mean-rel {mr:.3e} (<= {mean_rel})"
     return ma, mr
 
 
+VIS_SPAN = 64      # chunks covered by the window word of the device's bitmap row
+
+
+def vis_offset(W: int) -> int:
+    """Index of the bitmap row in the device table (after 3 + 4 (W + 3) segment ints)."""
+    return 3 + 4 * (W + 3)
+
+
+def expand_vis_row(words, k: int) -> np.ndarray:
+    """The device's constant-size bitmap row [vis_sink, vis_lo, vis_hi] expanded to the full row
+    vis[k][j], j < k (uint8).  Bit i of vis_hi:vis_lo is chunk k - 64 + i; vis_sink is chunk 0.
+    Asserts that no bit names a chunk before 0 and that the two encodings of chunk 0 agree."""
+    vis_sink, lo, hi = (int(x) & 0xffffffff for x in words)
+    assert vis_sink in (0, 1), vis_sink
+    word = lo | (hi << 32)
+    row = np.zeros(k, dtype=np.uint8)
+    for i in range(VIS_SPAN):
+        j = k - VIS_SPAN + i
+        bit = (word >> i) & 1
+        if j < 0:
+            assert bit == 0, (k, i)
+        elif bit:
+            row[j] = 1
+    if k >= 1:
+        if k <= VIS_SPAN:
+            assert row[0] == vis_sink, (k, row[0], vis_sink)
+        row[0] |= vis_sink
+    else:
+        assert vis_sink == 0
+    return row
+
+
+def check_table(got: np.ndarray, k: int, W: int, sink: bool, n_cond: int, T: int, R=None) -> None:
+    """The device table for active chunk k, bit for bit against the oracle: the segment list
+    (unused entries -1) and the chunk bitmap row."""
+    off = vis_offset(W)
+    assert got.shape[0] == off + 3, got.shape
+    ref = oracle.table(k, W, sink, n_cond, T, R=R)
+    np.testing.assert_array_equal(got[: len(ref)], ref)
+    assert (got[len(ref):off] == -1).all()
+    np.testing.assert_array_equal(expand_vis_row(got[off:off + 3], k), oracle.vis_row(k, W, sink))
+
+
 def sample_rows(n_q: int, n: int, seed: int) -> np.ndarray:
-    """Rows that always include both ends and the 128-row tile edges, plus random ones."""
+    """Query rows checked on the large workloads:
+      - both ends and both sides of every 128-row tile edge;
+      - one random row in every 32-row quarter of every tile, so that every softmax warp (a
+        warp owns one 32-lane quarter of a tile's rows) is compared in every tile;
+      - n random rows on top of those (distinct from them)."""
     fixed = {0, 1, n_q - 1, n_q - 2}
     for e in range(128, n_q, 128):
         fixed.update({e - 1, e})
-    fixed = sorted(r for r in fixed if 0 <= r < n_q)
     rng = np.random.default_rng(seed)
-    extra = rng.choice(n_q, size=min(n_q, max(0, n - len(fixed))), replace=False)
-    return np.array(sorted(set(fixed) | set(int(x) for x in extra)), dtype=np.int32)
+    for q0 in range(0, n_q, 32):
+        fixed.add(int(rng.integers(q0, min(q0 + 32, n_q))))
+    fixed = {r for r in fixed if 0 <= r < n_q}
+    rest = np.array(sorted(set(range(n_q)) - fixed), dtype=np.int64)
+    extra = rng.choice(rest, size=min(len(rest), max(0, n)), replace=False) if len(rest) else []
+    return np.array(sorted(fixed | set(int(x) for x in extra)), dtype=np.int32)
 
 
 def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink=None, n_cond=None,
@@ -43,9 +121,17 @@ def make_handle(wl, dev, *, out_dtype=torch.float32, max_short_q=0, W=None, sink
                                   commit_in_forward=commit_in_forward, commit_path=commit_path, device=dev)
 
 
+def tol_for(out_dtype, ref, tol=None):
+    """The tolerance of one comparison: the one given, else the parity tolerance for fp32 output
+    and the derived one (bf16_out_tol) for bf16 output."""
+    if tol is not None:
+        return tol
+    return bf16_out_tol(ref) if out_dtype == torch.bfloat16 else (MAX_ABS, MEAN_REL)
+
+
 def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, n_q=None,
                      out_dtype=torch.float32, max_short_q=0, poison=False, seed=0,
-                     tol=(MAX_ABS, MEAN_REL), keep_last=None, gen_on_device=False, schedule="auto"):
+                     tol=None, keep_last=None, gen_on_device=False, schedule="auto"):
     """Stream `chunks` chunks (2 forwards then an append each).  At the chunks in `check_at`
     (all if None) compare the CUDA output with the oracle, on all rows or on sampled rows.
     With gen_on_device the seeded draws use the GPU generator (faster for big shapes); the
@@ -78,7 +164,7 @@ def stream_and_check(wl, dev, *, chunks, check_at=None, rows=None, n_rows=None, 
                 got = out.float().cpu().numpy()
                 if r is not None:
                     got = got[:, r]
-                ma, mr = compare(got, ref, *tol)
+                ma, mr = compare(got, ref, *tol_for(out_dtype, ref, tol))
                 results.append((k, step, ma, mr))
         h.append_chunk(K.to(dev), V.to(dev))
         hist_K.append(K.cpu())
@@ -206,9 +292,7 @@ def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, 
         hist_K.append(Kh)
         hist_V.append(Vh)
         torch.cuda.synchronize()
-        tab = h.table().cpu().numpy()
-        ref_tab = oracle.table(k + 1, wl.W, wl.sink, wl.n_cond, wl.T, R=R)
-        assert np.array_equal(tab[:len(ref_tab)], ref_tab), (k, tab, ref_tab)
+        check_table(h.table().cpu().numpy(), k + 1, wl.W, wl.sink, wl.n_cond, wl.T, R=R)
         if check_cache:
             ring.append(Kh, Vh)
             committed[k] = (Kh, Vh)

@@ -59,7 +59,7 @@ def test_create_and_workspace_bytes(native):
     cond = 2 * 24 * 256 * 128 * 2
     # plus split-K partials and the persistent schedule's merge scratch (tens of MB)
     assert ring + cond <= ws <= ring + cond + 64 * 2 ** 20
-    assert L.sw_attn_table_ints(h) == 3 + 4 * (3 + 3)
+    assert L.sw_attn_table_ints(h) == 3 + 4 * (3 + 3) + 3
     ko, vo = ctypes.c_size_t(), ctypes.c_size_t()
     assert L.sw_attn_cache_offsets(h, ctypes.byref(ko), ctypes.byref(vo)) == 0
     assert ko.value % 1024 == 0 and vo.value - ko.value >= ring // 2

@@ -2,17 +2,17 @@
 
 sw_attn_forward_short_noalloc serves callers that cannot allocate device memory when they
 call (a host framework's fixed pool, a fixed-footprint server): its split-K partials live in
-a fixed array inside the library instead of the handle's workspace.  Its output must match
-the ordinary entry point's within the parity tolerance, on two calls in a row (the second
-call reuses the array the first one left behind).  Kept in a file of its own so a run that
-stops at the first failure has already run everything else; it must pass both alone and
-after the other tests.
+a fixed array inside the library instead of the handle's workspace.  On two calls in a row
+(the second reuses the array the first one left behind) its output must equal the ordinary
+entry point's bit for bit -- both run the same split kernel and combine with the same split
+count -- and match the FP64 oracle within the parity tolerance.  Kept in a file of its own so
+a run that stops at the first failure has already run everything else; it must pass both alone
+and after the other tests.
 """
 from __future__ import annotations
 
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -31,24 +31,33 @@ def test_noalloc_matches_forward_two_calls():
     B.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    import oracle
+    oracle.build()
     wl = Workload("noalloc", B=2, H=3, d=128, T=300, n_cond=40, W=2, sink=True, chunks=4, steps=1)
     h = make_handle(wl, dev)   # fp32 output
     Kc, Vc = synth.cond_inputs(wl)
     h.set_cond(Kc.to(dev), Vc.to(dev))
+    hist_K, hist_V = [], []
     for k in range(3):
         _, K, V = synth.chunk_inputs(wl, k, 0)
         h.append_chunk(K.to(dev), V.to(dev))
+        hist_K.append(K)
+        hist_V.append(V)
     lib = _native.lib()
     stream = torch.cuda.current_stream().cuda_stream
     for call, n_q in enumerate((64, 17)):
-        Q, K, V = (t.to(dev) for t in synth.chunk_inputs(wl, 3, call, n_q=n_q))
+        Qh, Kh, Vh = synth.chunk_inputs(wl, 3, call, n_q=n_q)
+        Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
         ref = h.forward(Q, K, V)                      # existing entry point (workspace scratch)
         out = torch.full_like(ref, float("nan"))
         rc = lib.sw_attn_forward_short_noalloc(h._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                                out.data_ptr(), n_q, ctypes.c_void_p(stream))
         assert rc == 0, lib.sw_attn_last_error().decode()
         torch.cuda.synchronize()
-        compare(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), MAX_ABS, MEAN_REL)
+        assert torch.equal(out, ref), f"call {call}: differs from sw_attn_forward"
+        exact = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink, k=3, Kc=Kc, Vc=Vc,
+                                 hist_K=hist_K, hist_V=hist_V, Q=Qh, K_cur=Kh, V_cur=Vh)
+        compare(out.cpu().numpy(), exact, MAX_ABS, MEAN_REL)
     assert h.status() == 0
     # a shape that cannot fit even one split in the fixed array is refused, not truncated
     big = make_handle(Workload("big", B=1, H=256, d=128, T=8, n_cond=0, W=0, sink=False, chunks=1, steps=1), dev)
