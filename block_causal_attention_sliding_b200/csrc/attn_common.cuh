@@ -266,55 +266,80 @@ struct QKTile {
     static_assert(!kQK8 || D == 128, "e4m3 Q/K tiles need d = 128");
 };
 
+// The MMA issue helpers below come in two forms: kWarp = false for one issuing thread, kWarp =
+// true for a converged warp in which one lane (elect.sync) issues and every lane computes the
+// operands.
+template <bool kWarp>
+__device__ __forceinline__ void mma_ss_any(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if constexpr (kWarp) mma_ss_warp(d, a, b, idesc, acc);
+    else mma_ss(d, a, b, idesc, acc);
+}
+template <bool kWarp>
+__device__ __forceinline__ void mma_ss_f8_any(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if constexpr (kWarp) mma_ss_f8_warp(d, a, b, idesc, acc);
+    else mma_ss_f8(d, a, b, idesc, acc);
+}
+template <bool kWarp>
+__device__ __forceinline__ void mma_ts_any(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if constexpr (kWarp) mma_ts_warp(d, a, b, idesc, acc);
+    else mma_ts(d, a, b, idesc, acc);
+}
+template <bool kWarp>
+__device__ __forceinline__ void mma_commit_any(uint32_t bar) {
+    if constexpr (kWarp) mma_commit_warp(bar);
+    else mma_commit(bar);
+}
+
 // S = Q K^T with e4m3 Q and K tiles (d = 128, one 128-byte row per token): four K = 32 steps.
+template <bool kWarp = false>
 __device__ __forceinline__ void issue_s_f8(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
     constexpr uint32_t idesc = idesc_e4m3_f32(kBlockM, kBlockN);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
-        mma_ss_f8(tS, smem_desc_sw128(q_tile + ks * 32, 16, 1024), smem_desc_sw128(k_tile + ks * 32, 16, 1024), idesc,
-                  ks > 0 ? 1u : 0u);
+        mma_ss_f8_any<kWarp>(tS, smem_desc_sw128(q_tile + ks * 32, 16, 1024), smem_desc_sw128(k_tile + ks * 32, 16, 1024),
+                             idesc, ks > 0 ? 1u : 0u);
 }
 
 // S[tS] = Q(q_tile) K(k_tile)^T: M = 128 queries, N = 128 keys, K = D, bf16 -> fp32.
-template <int D>
+template <int D, bool kWarp = false>
 __device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;   // 16 columns = 32 bytes
-        mma_ss(tS, smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
-               idesc, ks > 0 ? 1u : 0u);
+        mma_ss_any<kWarp>(tS, smem_desc_sw128(q_tile + off, 16, 1024), smem_desc_sw128(k_tile + off, 16, 1024),
+                          idesc, ks > 0 ? 1u : 0u);
     }
 }
 
 // S = Q K^T for either operand format.
-template <int D, bool kQK8>
+template <int D, bool kQK8, bool kWarp = false>
 __device__ __forceinline__ void issue_s_qk(uint32_t tS, uint32_t q_tile, uint32_t k_tile) {
-    if constexpr (kQK8) issue_s_f8(tS, q_tile, k_tile);
-    else issue_s<D>(tS, q_tile, k_tile);
+    if constexpr (kQK8) issue_s_f8<kWarp>(tS, q_tile, k_tile);
+    else issue_s<D, kWarp>(tS, q_tile, k_tile);
 }
 
 // O[tO] (+)= P[tP] V(v_tile): P (bf16 pairs in TMEM) is the A operand, V is MN-major in shared
 // memory (16 key rows per step = 2 KB; the two 64-column boxes are 16 KB apart).
-template <int D>
+template <int D, bool kWarp = false>
 __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_tile, bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
 #pragma unroll
     for (int ks = 0; ks < kBlockN / 16; ++ks)
-        mma_ts(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
-               (accumulate || ks > 0) ? 1u : 0u);
+        mma_ts_any<kWarp>(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
+                          (accumulate || ks > 0) ? 1u : 0u);
 }
 
 // Half of O += P V: keys [64 half, 64 half + 64) of the tile (4 MMA steps of 16 keys).
-template <int D>
+template <int D, bool kWarp = false>
 __device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t v_tile, int half,
                                               bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
 #pragma unroll
     for (int k = 0; k < kBlockN / 32; ++k) {
         const int ks = half * (kBlockN / 32) + k;
-        mma_ts(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
-               (accumulate || ks > 0) ? 1u : 0u);
+        mma_ts_any<kWarp>(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 16 * 128, kBoxBytes, 1024), idesc,
+                          (accumulate || ks > 0) ? 1u : 0u);
     }
 }
 

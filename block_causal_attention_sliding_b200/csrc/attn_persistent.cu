@@ -21,6 +21,181 @@
 
 namespace swattn {
 
+// The MMA issuer runs as a converged warp (one lane issues each tcgen05 instruction, chosen by
+// elect.sync) rather than as one thread of a divergent branch.
+#ifndef SWATTN_MMA_WARP
+#define SWATTN_MMA_WARP 1
+#endif
+constexpr bool kMmaWarp = SWATTN_MMA_WARP != 0;
+
+// A bounded wait in the MMA issuer: warp-uniform when the whole warp runs the issuer, so that
+// every lane takes the same branch before the next elect.sync.
+template <bool kWarp>
+__device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t parity, volatile int* flag) {
+    if constexpr (kWarp) return warp_wait(bar, parity, flag);
+    else return wait_or_abort(bar, parity, flag);
+}
+
+// The TMA producer (one thread): Q tiles per piece, then the piece's K and V tiles in ring
+// order.  A function of its own, not inlined: the kernel's register budget is set by the softmax
+// warps, and the roles that hold little state must not have their loop state spilled for them.
+template <int D, bool kCommit, bool kQK8>
+__device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl, uint8_t* q_smem, uint8_t* kv_smem,
+                                             Sched sched, volatile int* abort_flag) {
+    constexpr int NQ = 2;
+    constexpr int kStages = TileCfg<D>::kStages;
+    constexpr int kTileBytes = TileCfg<D>::kTileBytes;
+    const uint32_t qbar = smem_u32(&ctl->q_full);
+    PieceIt pit;
+    Piece pc;
+    uint32_t it = 0;
+    int pi = 0;
+    bool ok = true;
+    // fused commit: the chunk's K_cur / V_cur tile j is stored by the piece of Q-tile pair
+    // j mod npairs that loads it, so the stores spread over the CTAs
+    const int cslot = kCommit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
+    CommitQueue<D, kStages> cq;
+    while (ok && next_piece(sched, pit, pc)) {
+        const int b = pc.bh / p.H, h = pc.bh % p.H;
+        // the Q buffers are reused: wait until every S MMA of the previous piece is done
+        if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(qbar, pc.live * QKTile<D, kQK8>::kBytes);
+        for (int qt = 0; qt < pc.live; ++qt) {
+            const QSrc qs = q_src(p, pc.pair * NQ + qt);
+            for (int c = 0; c < QKTile<D, kQK8>::kBoxes; ++c)
+                tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), qs.tm, qbar,
+                            c * QKTile<D, kQK8>::kBoxCols, h, qs.row0, b);
+        }
+        ++pi;
+        for (int j = pc.j0; j < pc.j1 && ok; ++j) {
+            for (int kv = 0; kv < 2; ++kv, ++it) {
+                const int s = it % kStages;
+                const uint32_t r = it / kStages;
+                if (!wait_or_abort(smem_u32(&ctl->kv_empty[s]), (r & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (kCommit) cq.before_refill(s);
+                const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
+                mbar_arrive_expect_tx(fbar, kv == 0 ? QKTile<D, kQK8>::kBytes : kTileBytes);
+                load_kv_tile<D, kQK8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                if (kCommit) {
+                    const bool mine = cslot >= 0 && pc.pair == j % sched.npairs &&
+                                      ctl->seg_kind[tile_seg(ctl, j)] == 2;
+                    if (!cq.step(p, ctl, kv_smem, cslot, it, CommitQueue<D, kStages>::pack(mine, j, kv, h, b),
+                                 abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                }
+            }
+        }
+    }
+    if (kCommit) {
+        if (ok) (void)cq.flush(p, ctl, kv_smem, cslot, it, abort_flag);
+        bulk_wait_all();
+    }
+    for (int s = 0; s < kStages; ++s) {
+        if (it > (uint32_t)s) {
+            const uint32_t uses = (it - 1 - s) / kStages + 1;
+            wait_drain(smem_u32(&ctl->kv_full[s]), (uses - 1) & 1);
+        }
+    }
+    if (pi > 0) wait_drain(qbar, (pi - 1) & 1);
+}
+
+// The MMA issuer (one thread): per piece, S of each live Q tile for the first key tile, then per
+// key tile P V and the next tile's S for each live Q tile, in issue order.  Not inlined, for the
+// same reason as the producer.
+template <int D, bool kQK8>
+__device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t* kv_smem, uint32_t tmem,
+                                        Sched sched, volatile int* abort_flag) {
+    constexpr int NQ = 2;
+    constexpr int kStages = TileCfg<D>::kStages;
+    constexpr int kTileBytes = TileCfg<D>::kTileBytes;
+    const uint32_t q_base = smem_u32(q_smem);
+    const uint32_t kv_base = smem_u32(kv_smem);
+    PieceIt pit;
+    Piece pc;
+    uint32_t it = 0;          // K/V tiles consumed so far (ring position)
+    int pi = 0;               // pieces started
+    uint32_t tcnt[2] = {0, 0};   // key tiles processed per Q tile (p_full phases)
+    uint32_t ucnt[2] = {0, 0};   // pieces finished per Q tile (o_empty phases)
+    bool ok = true;
+    while (ok && next_piece(sched, pit, pc)) {
+        const int n = pc.j1 - pc.j0;
+        const int live = pc.live;
+        if (!mma_wait<kMmaWarp>(smem_u32(&ctl->q_full), pi & 1, abort_flag)) break;
+        ++pi;
+        const int s0 = it % kStages;
+        if (!mma_wait<kMmaWarp>(smem_u32(&ctl->kv_full[s0]), (it / kStages) & 1, abort_flag)) break;
+        tc_fence_after();
+        for (int qt = 0; qt < live; ++qt) {
+            issue_s_qk<D, kQK8, kMmaWarp>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + s0 * kTileBytes);
+            mma_commit_any<kMmaWarp>(smem_u32(&ctl->s_full[qt]));
+        }
+        if (n == 1) mma_commit_any<kMmaWarp>(smem_u32(&ctl->q_empty));
+        mma_commit_any<kMmaWarp>(smem_u32(&ctl->kv_empty[s0]));
+        for (int jj = 0; jj < n && ok; ++jj) {
+            const uint32_t itV = it + 2 * jj + 1, itK = it + 2 * jj + 2;
+            const int sV = itV % kStages, sK = itK % kStages;
+            const bool more = jj + 1 < n;
+            if (!mma_wait<kMmaWarp>(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            for (int qt = 0; qt < live && ok; ++qt) {
+                const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
+                if (!mma_wait<kMmaWarp>(smem_u32(kSplitP ? &ctl->p_half[qt] : &ctl->p_full[qt]), tcnt[qt] & 1,
+                                   abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (jj == 0 && ucnt[qt] > 0) {
+                    // the previous piece's O must be out of TMEM before it is overwritten
+                    if (!mma_wait<kMmaWarp>(smem_u32(&ctl->o_empty[qt]), (ucnt[qt] - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                if (kSplitP) {
+                    issue_pv_half<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                    if (!mma_wait<kMmaWarp>(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv_half<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                } else {
+                    issue_pv<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
+                }
+                ++tcnt[qt];
+                if (!more) mma_commit_any<kMmaWarp>(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
+                if (more) {
+                    if (qt == 0 &&
+                        !mma_wait<kMmaWarp>(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    // in issue order after the PV that reads P_q from the same columns
+                    issue_s_qk<D, kQK8, kMmaWarp>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
+                    mma_commit_any<kMmaWarp>(smem_u32(&ctl->s_full[qt]));
+                }
+            }
+            if (!ok) break;
+            if (more && jj + 2 == n) mma_commit_any<kMmaWarp>(smem_u32(&ctl->q_empty));   // last S issued
+            mma_commit_any<kMmaWarp>(smem_u32(&ctl->kv_empty[sV]));
+            if (more) mma_commit_any<kMmaWarp>(smem_u32(&ctl->kv_empty[sK]));
+        }
+        for (int qt = 0; qt < live; ++qt) ++ucnt[qt];
+        it += 2 * n;
+    }
+    mma_commit_any<kMmaWarp>(smem_u32(&ctl->drain));
+    wait_drain(smem_u32(&ctl->drain), 0);
+}
+
 // kCommit: the launch also stores the chunk's K_cur / V_cur into the cache (fused commit); a
 // separate instantiation, so the plain forward carries none of that code.
 // kQK8: Q and K are e4m3 (d = 128), S = Q K^T on kind::f8f6f4; V, P and O as in the bf16 kernel.
@@ -72,150 +247,10 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && nt > 0) {
-            const uint32_t qbar = smem_u32(&ctl->q_full);
-            PieceIt pit;
-            Piece pc;
-            uint32_t it = 0;
-            int pi = 0;
-            bool ok = true;
-            // fused commit: the chunk's K_cur / V_cur tile j is stored by the piece of Q-tile pair
-            // j mod npairs that loads it, so the stores spread over the CTAs
-            const int cslot = kCommit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
-            CommitQueue<D, kStages> cq;
-            while (ok && next_piece(sched, pit, pc)) {
-                const int b = pc.bh / p.H, h = pc.bh % p.H;
-                // the Q buffers are reused: wait until every S MMA of the previous piece is done
-                if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(qbar, pc.live * QKTile<D, kQK8>::kBytes);
-                for (int qt = 0; qt < pc.live; ++qt) {
-                    const QSrc qs = q_src(p, pc.pair * NQ + qt);
-                    for (int c = 0; c < QKTile<D, kQK8>::kBoxes; ++c)
-                        tma_load_4d(smem_u32(q_smem + qt * kTileBytes + c * kBoxBytes), qs.tm, qbar,
-                                    c * QKTile<D, kQK8>::kBoxCols, h, qs.row0, b);
-                }
-                ++pi;
-                for (int j = pc.j0; j < pc.j1 && ok; ++j) {
-                    for (int kv = 0; kv < 2; ++kv, ++it) {
-                        const int s = it % kStages;
-                        const uint32_t r = it / kStages;
-                        if (!wait_or_abort(smem_u32(&ctl->kv_empty[s]), (r & 1) ^ 1, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        if (kCommit) cq.before_refill(s);
-                        const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
-                        mbar_arrive_expect_tx(fbar, kv == 0 ? QKTile<D, kQK8>::kBytes : kTileBytes);
-                        load_kv_tile<D, kQK8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
-                        if (kCommit) {
-                            const bool mine = cslot >= 0 && pc.pair == j % sched.npairs &&
-                                              ctl->seg_kind[tile_seg(ctl, j)] == 2;
-                            if (!cq.step(p, ctl, kv_smem, cslot, it, CommitQueue<D, kStages>::pack(mine, j, kv, h, b),
-                                         abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                        }
-                    }
-                }
-            }
-            if (kCommit) {
-                if (ok) (void)cq.flush(p, ctl, kv_smem, cslot, it, abort_flag);
-                bulk_wait_all();
-            }
-            for (int s = 0; s < kStages; ++s) {
-                if (it > (uint32_t)s) {
-                    const uint32_t uses = (it - 1 - s) / kStages + 1;
-                    wait_drain(smem_u32(&ctl->kv_full[s]), (uses - 1) & 1);
-                }
-            }
-            if (pi > 0) wait_drain(qbar, (pi - 1) & 1);
-        }
+        if (lane == 0 && nt > 0) persist_producer<D, kCommit, kQK8>(p, ctl, q_smem, kv_smem, sched, abort_flag);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nt > 0) {
-            const uint32_t q_base = smem_u32(q_smem);
-            const uint32_t kv_base = smem_u32(kv_smem);
-            PieceIt pit;
-            Piece pc;
-            uint32_t it = 0;          // K/V tiles consumed so far (ring position)
-            int pi = 0;               // pieces started
-            uint32_t tcnt[2] = {0, 0};   // key tiles processed per Q tile (p_full phases)
-            uint32_t ucnt[2] = {0, 0};   // pieces finished per Q tile (o_empty phases)
-            bool ok = true;
-            while (ok && next_piece(sched, pit, pc)) {
-                const int n = pc.j1 - pc.j0;
-                const int live = pc.live;
-                if (!wait_or_abort(smem_u32(&ctl->q_full), pi & 1, abort_flag)) break;
-                ++pi;
-                const int s0 = it % kStages;
-                if (!wait_or_abort(smem_u32(&ctl->kv_full[s0]), (it / kStages) & 1, abort_flag)) break;
-                tc_fence_after();
-                for (int qt = 0; qt < live; ++qt) {
-                    issue_s_qk<D, kQK8>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + s0 * kTileBytes);
-                    mma_commit(smem_u32(&ctl->s_full[qt]));
-                }
-                if (n == 1) mma_commit(smem_u32(&ctl->q_empty));
-                mma_commit(smem_u32(&ctl->kv_empty[s0]));
-                for (int jj = 0; jj < n && ok; ++jj) {
-                    const uint32_t itV = it + 2 * jj + 1, itK = it + 2 * jj + 2;
-                    const int sV = itV % kStages, sK = itK % kStages;
-                    const bool more = jj + 1 < n;
-                    if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    for (int qt = 0; qt < live && ok; ++qt) {
-                        const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
-                        if (!wait_or_abort(smem_u32(kSplitP ? &ctl->p_half[qt] : &ctl->p_full[qt]), tcnt[qt] & 1,
-                                           abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (jj == 0 && ucnt[qt] > 0) {
-                            // the previous piece's O must be out of TMEM before it is overwritten
-                            if (!wait_or_abort(smem_u32(&ctl->o_empty[qt]), (ucnt[qt] - 1) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                        }
-                        if (kSplitP) {
-                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
-                            if (!wait_or_abort(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
-                        } else {
-                            issue_pv<D>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
-                        }
-                        ++tcnt[qt];
-                        if (!more) mma_commit(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
-                        if (more) {
-                            if (qt == 0 &&
-                                !wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            // in issue order after the PV that reads P_q from the same columns
-                            issue_s_qk<D, kQK8>(tmem + qt * kBlockN, q_base + qt * kTileBytes, kv_base + sK * kTileBytes);
-                            mma_commit(smem_u32(&ctl->s_full[qt]));
-                        }
-                    }
-                    if (!ok) break;
-                    if (more && jj + 2 == n) mma_commit(smem_u32(&ctl->q_empty));   // last S issued
-                    mma_commit(smem_u32(&ctl->kv_empty[sV]));
-                    if (more) mma_commit(smem_u32(&ctl->kv_empty[sK]));
-                }
-                for (int qt = 0; qt < live; ++qt) ++ucnt[qt];
-                it += 2 * n;
-            }
-            mma_commit(smem_u32(&ctl->drain));
-            wait_drain(smem_u32(&ctl->drain), 0);
-        }
+        if ((kMmaWarp || lane == 0) && nt > 0) persist_mma<D, kQK8>(ctl, q_smem, kv_smem, tmem, sched, abort_flag);
     } else {
         // ------------------------------------------------------------ softmax warpgroups
         const int qt = (warp - 2) >> 2;
