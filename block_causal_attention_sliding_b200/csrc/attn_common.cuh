@@ -49,6 +49,7 @@ struct SmemCtl {
     uint64_t o_full[2];
     uint64_t o_empty[2];
     uint64_t drain;
+    uint64_t merge_bar[2][3];   // staged merge of split-piece partials: per Q tile, three buffers
     uint32_t tmem_base;
     int abort_flag;
     int n_seg;
@@ -507,6 +508,8 @@ __device__ __forceinline__ void init_barriers(SmemCtl* ctl, int stages) {
         mbar_init(smem_u32(&ctl->o_empty[q]), 4);
     }
     mbar_init(smem_u32(&ctl->drain), 1);
+    for (int q = 0; q < 2; ++q)
+        for (int b = 0; b < 3; ++b) mbar_init(smem_u32(&ctl->merge_bar[q][b]), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
 }

@@ -28,12 +28,31 @@ namespace swattn {
 #endif
 constexpr bool kMmaWarp = SWATTN_MMA_WARP != 0;
 
+// The merge of a split pair at the merging CTA's last piece is staged through idle shared memory
+// by bulk copies (see the epilogue).
+#ifndef SWATTN_STAGED_MERGE
+#define SWATTN_STAGED_MERGE 1
+#endif
+constexpr bool kStagedMerge = SWATTN_STAGED_MERGE != 0;
+
 // A bounded wait in the MMA issuer: warp-uniform when the whole warp runs the issuer, so that
 // every lane takes the same branch before the next elect.sync.
 template <bool kWarp>
 __device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t parity, volatile int* flag) {
     if constexpr (kWarp) return warp_wait(bar, parity, flag);
     else return wait_or_abort(bar, parity, flag);
+}
+
+// Two waits of the issuer at once: both phases are tested in one block first (the common case,
+// both long complete, then costs one round trip), and only if that fails are they waited for one
+// after the other, bounded as usual.
+template <bool kWarp>
+__device__ __forceinline__ bool mma_wait2(uint32_t bar_a, uint32_t parity_a, uint32_t bar_b, uint32_t parity_b,
+                                          volatile int* flag) {
+    bool both = mbar_try_wait2(bar_a, parity_a, bar_b, parity_b);
+    if constexpr (kWarp) both = __all_sync(0xffffffffu, both);
+    if (both) return true;
+    return mma_wait<kWarp>(bar_a, parity_a, flag) && mma_wait<kWarp>(bar_b, parity_b, flag);
 }
 
 // The TMA producer (one thread): Q tiles per piece, then the piece's K and V tiles in ring
@@ -140,14 +159,15 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
             const uint32_t itV = it + 2 * jj + 1, itK = it + 2 * jj + 2;
             const int sV = itV % kStages, sK = itK % kStages;
             const bool more = jj + 1 < n;
-            if (!mma_wait<kMmaWarp>(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
             for (int qt = 0; qt < live && ok; ++qt) {
                 const uint32_t tO = tmem + NQ * kBlockN + qt * D, tP = tmem + qt * kBlockN;
-                if (!mma_wait<kMmaWarp>(smem_u32(kSplitP ? &ctl->p_half[qt] : &ctl->p_full[qt]), tcnt[qt] & 1,
-                                   abort_flag)) {
+                const uint32_t pbar = smem_u32(kSplitP ? &ctl->p_half[qt] : &ctl->p_full[qt]);
+                const uint32_t fbar = smem_u32(&ctl->p_full[qt]), ppar = tcnt[qt] & 1;
+                const uint32_t vbar = smem_u32(&ctl->kv_full[sV]), vpar = (itV / kStages) & 1;
+                const uint32_t kbar = smem_u32(&ctl->kv_full[sK]), kpar = (itK / kStages) & 1;
+                // V of this key tile is waited for together with the first Q tile's P
+                if (!(qt == 0 ? mma_wait2<kMmaWarp>(vbar, vpar, pbar, ppar, abort_flag)
+                              : mma_wait<kMmaWarp>(pbar, ppar, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -162,7 +182,9 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
                 }
                 if (kSplitP) {
                     issue_pv_half<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
-                    if (!mma_wait<kMmaWarp>(smem_u32(&ctl->p_full[qt]), tcnt[qt] & 1, abort_flag)) {
+                    // the first Q tile's full P is waited for together with the next K tile
+                    if (!(qt == 0 && more ? mma_wait2<kMmaWarp>(fbar, ppar, kbar, kpar, abort_flag)
+                                          : mma_wait<kMmaWarp>(fbar, ppar, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -174,8 +196,7 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
                 ++tcnt[qt];
                 if (!more) mma_commit_any<kMmaWarp>(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
                 if (more) {
-                    if (qt == 0 &&
-                        !mma_wait<kMmaWarp>(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) {
+                    if (qt == 0 && !kSplitP && !mma_wait<kMmaWarp>(kbar, kpar, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -265,12 +286,15 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
         int sk_pi = 0;            // stream-K pieces seen (the first and last may be split)
         uint32_t tcnt = 0;        // key tiles processed (s_full phases)
         uint32_t ucnt = 0;        // pieces processed (o_full phases: one per piece)
+        uint32_t it_base = 0;     // K/V ring items of the pieces before this one
         bool ok = nt > 0;
         while (ok && next_piece(sched, pit, pc)) {
             const bool first_sk = pc.sk && sk_pi == 0;
             if (pc.sk) ++sk_pi;
-            if (qt >= pc.live) continue;
             const int n = pc.j1 - pc.j0;
+            const uint32_t it_piece = it_base;
+            it_base += 2 * n;
+            if (qt >= pc.live) continue;
             float m_ref = -INFINITY, l = 0.f;
             for (int jj = 0; jj < n; ++jj) {
                 int seg, row0, valid;
@@ -347,27 +371,94 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             }
             // merge every piece -- this one's too, read back -- in slot order, so the result
             // does not depend on which piece happened to arrive last
+            const auto slot_of = [&](int gg) {
+                return gg == g ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
+            };
             float M = -INFINITY;
-            for (int gg = g_first; gg <= g_last; ++gg) {
-                const int sl = gg == g ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
-                M = fmaxf(M, __ldcg(p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2));
-            }
+            for (int gg = g_first; gg <= g_last; ++gg)
+                M = fmaxf(M, __ldcg(p.sk_ml + ((size_t)slot_of(gg) * 2 + qt) * kBlockM * 2 + row * 2));
             float L_ = 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[c][i] = 0u;
-            for (int gg = g_first; gg <= g_last; ++gg) {
-                const int sl = gg == g ? slot : ((gg > g_first || opens_first) ? 2 * gg : 2 * gg + 1);
-                const float* pml = p.sk_ml + ((size_t)sl * 2 + qt) * kBlockM * 2 + row * 2;
-                const float w = ex2_approx(__ldcg(pml) - M);
-                L_ += w * __ldcg(pml + 1);
-                const float* po = p.sk_o + ((size_t)sl * 2 + qt) * D * kBlockM + row;
+            // At this CTA's last piece the producer is done and no MMA reads this Q tile's buffer
+            // or any ring stage but the one of the piece's last V (and that one neither, once this
+            // group's own last P V has completed): the partials are then staged through those
+            // buffers with bulk copies, three in flight, instead of loaded by each thread -- the
+            // direct loads are latency-bound at ~30 in flight per thread.  Same additions in the
+            // same order either way, so the result is bit-identical.
+            PieceIt after = pit;
+            Piece nxt;
+            const bool staged = kStagedMerge && !kCommit && !next_piece(sched, after, nxt);
+            if (staged) {
+                constexpr int kChunkCols = kTileBytes / (kBlockM * 4);   // partial columns per buffer
+                constexpr int kChunksPerSlot = D / kChunkCols;
+                const int s_last = (int)((it_piece + 2 * n - 1) % kStages);
+                int fs0 = -1, fs1 = -1, fs2 = -1;   // the stages other than s_last, in order
+                for (int st = 0; st < kStages; ++st) {
+                    if (st == s_last) continue;
+                    if (fs0 < 0) fs0 = st;
+                    else if (fs1 < 0) fs1 = st;
+                    else if (fs2 < 0) fs2 = st;
+                }
+                uint8_t* const b0 = q_smem + qt * kTileBytes;
+                uint8_t* const b1 = kv_smem + (qt == 0 ? fs0 : fs2) * kTileBytes;
+                uint8_t* const b2 = kv_smem + (qt == 0 ? fs1 : s_last) * kTileBytes;
+                const auto buf = [&](int b) { return b == 0 ? b0 : (b == 1 ? b1 : b2); };
+                const int nchunks = npieces * kChunksPerSlot;
+                const bool issuer = row == 0;
+                const auto issue = [&](int k) {
+                    const int gg = g_first + k / kChunksPerSlot, part = k % kChunksPerSlot;
+                    const float* src = p.sk_o + ((size_t)slot_of(gg) * 2 + qt) * D * kBlockM +
+                                       (size_t)part * kChunkCols * kBlockM;
+                    const uint32_t bar = smem_u32(&ctl->merge_bar[qt][k % 3]);
+                    mbar_arrive_expect_tx(bar, kTileBytes);
+                    bulk_load_1d(smem_u32(buf(k % 3)), src, kTileBytes, bar);
+                };
+                int issued = 0;
+                if (issuer) {
+                    fence_proxy_async_global();
+                    for (; issued < 3 && issued < nchunks; ++issued) issue(issued);
+                }
+                int k = 0;
+                for (; k < nchunks; ++k) {
+                    const int gg = g_first + k / kChunksPerSlot, part = k % kChunksPerSlot;
+                    bool mok = warp_wait(smem_u32(&ctl->merge_bar[qt][k % 3]), (k / 3) & 1, abort_flag);
+                    if (mok) {
+                        const float w = ex2_approx(__ldcg(p.sk_ml + ((size_t)slot_of(gg) * 2 + qt) * kBlockM * 2 + row * 2) - M);
+                        const float* bf = reinterpret_cast<const float*>(buf(k % 3)) + row;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
+                        for (int c = 0; c < D / 32; ++c) {
+                            if (c / (kChunkCols / 32) != part) continue;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[c][i] = __float_as_uint(fmaf(w, __ldcg(po + (c * 32 + i) * kBlockM), __uint_as_float(o[c][i])));
+                            for (int i = 0; i < 32; ++i)
+                                o[c][i] = __float_as_uint(fmaf(w, bf[(c * 32 + i - part * kChunkCols) * kBlockM],
+                                                               __uint_as_float(o[c][i])));
+                        }
+                    }
+                    // every thread of the group is done with this buffer before it is refilled
+                    if (!wg_all(qt, mok)) break;
+                    if (issuer && issued < nchunks) issue(issued++);
+                }
+                if (issuer)   // a failed wait leaves copies in flight: let them land before leaving
+                    for (int kk = k; kk < issued; ++kk) wait_drain(smem_u32(&ctl->merge_bar[qt][kk % 3]), (kk / 3) & 1);
+                for (int gg = g_first; gg <= g_last; ++gg) {
+                    const float* pml = p.sk_ml + ((size_t)slot_of(gg) * 2 + qt) * kBlockM * 2 + row * 2;
+                    L_ += ex2_approx(__ldcg(pml) - M) * __ldcg(pml + 1);
+                }
+            } else {
+                for (int gg = g_first; gg <= g_last; ++gg) {
+                    const float* pml = p.sk_ml + ((size_t)slot_of(gg) * 2 + qt) * kBlockM * 2 + row * 2;
+                    const float w = ex2_approx(__ldcg(pml) - M);
+                    L_ += w * __ldcg(pml + 1);
+                    const float* po = p.sk_o + ((size_t)slot_of(gg) * 2 + qt) * D * kBlockM + row;
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[c][i] = __float_as_uint(fmaf(w, __ldcg(po + (c * 32 + i) * kBlockM), __uint_as_float(o[c][i])));
+                }
             }
             const float inv = 1.f / L_;
             if (m_row < qs.rows) {

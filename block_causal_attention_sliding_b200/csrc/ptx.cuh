@@ -47,6 +47,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Two phases tested in one block, so their latencies overlap: true iff both have completed.
+__device__ __forceinline__ bool mbar_try_wait2(uint32_t bar_a, uint32_t parity_a, uint32_t bar_b, uint32_t parity_b) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred pa, pb, p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 pa, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 pb, [%3], %4;\n\t"
+        "and.pred p, pa, pb;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar_a), "r"(parity_a), "r"(bar_b), "r"(parity_b) : "memory");
+    return ok != 0;
+}
+
 // Non-blocking: has the phase with the given parity completed?
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -110,6 +123,17 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* map, uint3
           "r"(c4)
         : "memory");
 }
+
+// Contiguous bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global
+// to shared memory, completing on bar (which must expect the bytes).  No multicast.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Order this thread's view of global memory (generic proxy) before its later async-proxy reads.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // Tiled bulk store of one box from shared memory to global memory (5-D tensor map), in the
 // thread's bulk-async group.  Coordinates must be non-negative; rows past the tensor's extent
