@@ -50,6 +50,7 @@ struct SmemCtl {
     uint64_t o_empty[2];
     uint64_t drain;
     uint64_t merge_bar[2][3];   // staged merge of split-piece partials: per Q tile, three buffers
+    uint64_t prod_done;         // the producer has issued its last copy and every copy has landed
     uint32_t tmem_base;
     int abort_flag;
     int n_seg;
@@ -510,6 +511,7 @@ __device__ __forceinline__ void init_barriers(SmemCtl* ctl, int stages) {
     mbar_init(smem_u32(&ctl->drain), 1);
     for (int q = 0; q < 2; ++q)
         for (int b = 0; b < 3; ++b) mbar_init(smem_u32(&ctl->merge_bar[q][b]), 1);
+    mbar_init(smem_u32(&ctl->prod_done), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
 }

@@ -121,6 +121,7 @@ __device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl,
         }
     }
     if (pi > 0) wait_drain(qbar, (pi - 1) & 1);
+    mbar_arrive(smem_u32(&ctl->prod_done));   // no copy of this CTA reads or writes shared memory any more
 }
 
 // The MMA issuer (one thread): per piece, S of each live Q tile for the first key tile, then per
@@ -390,7 +391,10 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             // same order either way, so the result is bit-identical.
             PieceIt after = pit;
             Piece nxt;
-            const bool staged = kStagedMerge && !kCommit && !next_piece(sched, after, nxt);
+            // (at the last piece the producer has finished, or is about to: its fused-commit stores
+            // may still read ring stages until it signals prod_done)
+            bool staged = kStagedMerge && !next_piece(sched, after, nxt);   // the same in every warp
+            if (staged) staged = wg_all(qt, warp_wait(smem_u32(&ctl->prod_done), 0, abort_flag));
             if (staged) {
                 constexpr int kChunkCols = kTileBytes / (kBlockM * 4);   // partial columns per buffer
                 constexpr int kChunksPerSlot = D / kChunkCols;
