@@ -34,7 +34,7 @@ class SwAttnConfig(ctypes.Structure):
                 ("sink", ctypes.c_int), ("out_dtype", ctypes.c_int), ("scale", ctypes.c_float),
                 ("max_short_q", ctypes.c_int), ("schedule", ctypes.c_int), ("commit_in_forward", ctypes.c_int),
                 ("qk_fp8", ctypes.c_int), ("q_scale", ctypes.c_float), ("k_scale", ctypes.c_float),
-                ("commit_path", ctypes.c_int)]
+                ("commit_path", ctypes.c_int), ("pv_fp8", ctypes.c_int), ("v_scale", ctypes.c_float)]
 
 
 class SwAttnError(RuntimeError):

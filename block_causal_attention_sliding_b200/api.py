@@ -35,7 +35,7 @@ class SlidingWindowAttention:
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
                  max_short_q: int = 0, schedule: str = "auto", commit_in_forward: bool = False,
                  qk_fp8: bool = False, q_scale: float = 1.0, k_scale: float = 1.0, commit_path: str = "auto",
-                 device=None):
+                 pv_fp8: bool = False, v_scale: float = 1.0, device=None):
         self._lib = N.lib()
         cfg = N.SwAttnConfig(B=B, H=H, d=d, tokens_per_chunk=T, W=W, n_cond=n_cond,
                              sink=int(bool(sink)),
@@ -46,7 +46,8 @@ class SlidingWindowAttention:
                              commit_in_forward=int(bool(commit_in_forward)), qk_fp8=int(bool(qk_fp8)),
                              q_scale=float(q_scale), k_scale=float(k_scale),
                              commit_path={"auto": N.SW_COMMIT_AUTO, "copy": N.SW_COMMIT_COPY,
-                                          "tma": N.SW_COMMIT_TMA}[commit_path])
+                                          "tma": N.SW_COMMIT_TMA}[commit_path],
+                             pv_fp8=int(bool(pv_fp8)), v_scale=float(v_scale))
         if out_dtype not in (torch.float32, torch.bfloat16):
             raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
         h = ctypes.c_void_p()
@@ -58,6 +59,9 @@ class SlidingWindowAttention:
         # e4m3 queries and keys (FP8 handle), bf16 otherwise; V is always bf16
         self.qk_fp8 = bool(qk_fp8)
         self.qk_dtype = torch.float8_e4m3fn if self.qk_fp8 else torch.bfloat16
+        # e4m3 V as well (pv_fp8), bf16 otherwise
+        self.pv_fp8 = bool(pv_fp8)
+        self.v_dtype = torch.float8_e4m3fn if self.pv_fp8 else torch.bfloat16
         self.out_dtype = out_dtype
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         nbytes = int(self._lib.sw_attn_workspace_bytes(h))
@@ -87,7 +91,7 @@ class SlidingWindowAttention:
             if tuple(t.shape) != shape:
                 raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
         N.check(self._lib.sw_attn_set_cond(self._h, _dev_ptr(K_cond, "K_cond", self.qk_dtype),
-                                           _dev_ptr(V_cond, "V_cond", torch.bfloat16), _stream_ptr(stream)))
+                                           _dev_ptr(V_cond, "V_cond", self.v_dtype), _stream_ptr(stream)))
 
     def append_chunk(self, K: torch.Tensor, V: torch.Tensor, stream=None) -> None:
         shape = (self.B, self.T, self.H, self.d)
@@ -95,7 +99,7 @@ class SlidingWindowAttention:
             if tuple(t.shape) != shape:
                 raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
         N.check(self._lib.sw_attn_append_chunk(self._h, _dev_ptr(K, "K", self.qk_dtype),
-                                               _dev_ptr(V, "V", torch.bfloat16), _stream_ptr(stream)))
+                                               _dev_ptr(V, "V", self.v_dtype), _stream_ptr(stream)))
 
     def forward(self, Q: torch.Tensor, K_cur: torch.Tensor, V_cur: torch.Tensor,
                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -112,7 +116,7 @@ class SlidingWindowAttention:
             raise ValueError("out must match Q's shape and the handle's out_dtype")
         N.check(self._lib.sw_attn_forward(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
                                           _dev_ptr(K_cur, "K_cur", self.qk_dtype),
-                                          _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                          _dev_ptr(V_cur, "V_cur", self.v_dtype),
                                           _dev_ptr(out, "out"), n_q, _stream_ptr(stream)))
         return out
 
@@ -132,7 +136,7 @@ class SlidingWindowAttention:
             raise ValueError("out must be [B, T, H, d] in the handle's out_dtype")
         N.check(self._lib.sw_attn_forward_commit(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
                                                  _dev_ptr(K_cur, "K_cur", self.qk_dtype),
-                                                 _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                                 _dev_ptr(V_cur, "V_cur", self.v_dtype),
                                                  _dev_ptr(out, "out"), _stream_ptr(stream)))
         return out
 
@@ -157,7 +161,7 @@ class SlidingWindowAttention:
         N.check(self._lib.sw_attn_forward_joint(self._h, _dev_ptr(Q, "Q", self.qk_dtype),
                                                 _dev_ptr(Q_cond, "Q_cond", self.qk_dtype),
                                                 _dev_ptr(K_cur, "K_cur", self.qk_dtype),
-                                                _dev_ptr(V_cur, "V_cur", torch.bfloat16),
+                                                _dev_ptr(V_cur, "V_cur", self.v_dtype),
                                                 _dev_ptr(out, "out"), _dev_ptr(out_cond, "out_cond"),
                                                 _stream_ptr(stream)))
         return out, out_cond
@@ -187,8 +191,9 @@ class SlidingWindowAttention:
         n = 2 * self.B * self.H * S * self.T * self.d
         shape = (self.B, self.H, S, self.T, self.d)
         nk = n // 2 if self.qk_fp8 else n
+        nv = n // 2 if self.pv_fp8 else n
         kc = self.workspace[ko.value: ko.value + nk].view(self.qk_dtype).view(shape)
-        vc = self.workspace[vo.value: vo.value + n].view(torch.bfloat16).view(shape)
+        vc = self.workspace[vo.value: vo.value + nv].view(self.v_dtype).view(shape)
         return kc, vc
 
     def close(self) -> None:
@@ -216,6 +221,6 @@ def append_chunk_batched(handles, Ks, Vs, stream=None) -> None:
     lib = handles[0]._lib
     hp = (ctypes.c_void_p * n)(*[h._h.value for h in handles])
     kp = (ctypes.c_void_p * n)(*[_dev_ptr(K, "K", h.qk_dtype) for h, K in zip(handles, Ks)])
-    vp = (ctypes.c_void_p * n)(*[_dev_ptr(V, "V", torch.bfloat16) for V in Vs])
+    vp = (ctypes.c_void_p * n)(*[_dev_ptr(V, "V", h.v_dtype) for h, V in zip(handles, Vs)])
     N.check(lib.sw_attn_append_chunk_batched(ctypes.cast(hp, ctypes.c_void_p), n, ctypes.cast(kp, ctypes.c_void_p),
                                              ctypes.cast(vp, ctypes.c_void_p), _stream_ptr(stream)))

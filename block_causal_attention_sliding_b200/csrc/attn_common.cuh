@@ -11,6 +11,13 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: far above any legitim
 constexpr int kBoxCols = 64;                        // 128-byte swizzle atom = 64 bf16
 constexpr int kBoxBytes = kBlockM * kBoxCols * 2;   // 16 KB: one TMA box (128 rows x 64 cols)
 constexpr float kRescaleThreshold = 8.0f;           // log2 units: rescale O when max grows > 2^8
+// e4m3 P: weights are formed as 2^(s*sl2 - m + kP8Offset) and O is rescaled when the max grows
+// by more than 2^kP8Threshold, so P <= 2^(offset + threshold) = 256 stays below the e4m3 limit
+// (448) while the typical weight of a row (2^-6 .. 2^-2 of the max for Gaussian scores) lands in
+// e4m3's normal range, not its subnormals.  The factor 2^kP8Offset is common to l and O of every
+// partial, so it cancels in O / l and in the merge of split partials.
+constexpr float kP8Offset = 4.0f;
+constexpr float kP8Threshold = 4.0f;
 // One in kPolyEvery pairs of exponentials runs on the FMA pipe (exp2_poly) instead of MUFU
 // (0: none).  At two Q tiles per CTA the exponentials alone keep MUFU as busy as the tensor
 // core, but the softmax step is bound by issue and latency first; measured, not assumed.
@@ -167,15 +174,16 @@ __device__ __forceinline__ QSrc q_src(const AttnParams& p, int u) {
 
 // TMA loads of one 128-row K (kv = 0) or V (kv = 1) tile of key tile j of (b, h) into dst,
 // completing on bar: condition tokens, a ring slot, or the caller's current chunk.
-template <int D, bool kQK8 = false>
+template <int D, bool kQK8 = false, bool kPV8 = false>
 __device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl* ctl, int j, int kv,
                                              int h, int b, uint32_t dst, uint32_t bar) {
     int seg, row0, valid;
     tile_of(ctl, j, seg, row0, valid);
     const int kind = ctl->seg_kind[seg];
     const int slot = ctl->seg_slot[seg];
-    // an e4m3 K tile is one box of 128-byte rows; V (bf16) keeps its 64-column boxes
-    const int boxes = (kQK8 && kv == 0) ? 1 : TileCfg<D>::kBoxes;
+    // an e4m3 tile (K, or V on a pv_fp8 handle) is one box of 128-byte rows; bf16 keeps its
+    // 64-column boxes
+    const int boxes = ((kQK8 && kv == 0) || (kPV8 && kv == 1)) ? 1 : TileCfg<D>::kBoxes;
 #pragma unroll
     for (int c = 0; c < TileCfg<D>::kBoxes; ++c) {
         if (c >= boxes) break;
@@ -187,6 +195,12 @@ __device__ __forceinline__ void load_kv_tile(const AttnParams& p, const SmemCtl*
         else
             tma_load_4d(d, kv ? &p.tm_vcur : &p.tm_kcur, bar, c * kBoxCols, h, row0, b);
     }
+}
+
+// Bytes one K (kv = 0) or V (kv = 1) tile occupies in its ring stage.
+template <int D, bool kQK8, bool kPV8>
+__host__ __device__ constexpr int kv_tile_bytes(int kv) {
+    return ((kQK8 && kv == 0) || (kPV8 && kv == 1)) ? kBlockN * D : TileCfg<D>::kTileBytes;
 }
 
 // Fused commit: the producer stores the active chunk's K_cur / V_cur tiles, which it has just
@@ -286,6 +300,12 @@ __device__ __forceinline__ void mma_ts_any(uint32_t d, uint32_t a, uint64_t b, u
     if constexpr (kWarp) mma_ts_warp(d, a, b, idesc, acc);
     else mma_ts(d, a, b, idesc, acc);
 }
+// D (+)= A[tmem] * B[smem desc] with 8-bit floating-point operands (kind::f8f6f4).
+template <bool kWarp>
+__device__ __forceinline__ void mma_ss_f8_tmem_any(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if constexpr (kWarp) mma_ts_f8_warp(d, a, b, idesc, acc);
+    else mma_ts_f8(d, a, b, idesc, acc);
+}
 template <bool kWarp>
 __device__ __forceinline__ void mma_commit_any(uint32_t bar) {
     if constexpr (kWarp) mma_commit_warp(bar);
@@ -345,6 +365,20 @@ __device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t
     }
 }
 
+// Half of O += P V with e4m3 P (in TMEM, four keys per 32-bit column) and an e4m3 V tile (one box
+// of 128-byte rows, MN-major: d contiguous per key): keys [64 half, 64 half + 64), two kind::f8f6f4
+// MMA steps of 32 keys (32 rows of V = 4 KB apart; d = 128 is one 128-byte swizzle atom wide).
+template <bool kWarp = false>
+__device__ __forceinline__ void issue_pv_f8_half(uint32_t tO, uint32_t tP, uint32_t v_tile, int half, bool accumulate) {
+    constexpr uint32_t idesc = idesc_e4m3_f32(kBlockM, 128, true);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int ks = half * 2 + k;
+        mma_ss_f8_tmem_any<kWarp>(tO, tP + ks * 8, smem_desc_sw128(v_tile + ks * 32 * 128, kBlockN * 128, 1024), idesc,
+                                  (accumulate || ks > 0) ? 1u : 0u);
+    }
+}
+
 // One online-softmax step for this thread's query row over one key tile:
 //   read the S row from TMEM, mask keys past the segment's end, update the reference max
 //   (lazily: only when it grows by more than 2^kRescaleThreshold), write P = exp2(s*sl2 - m)
@@ -357,7 +391,13 @@ __device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint32_t
 // kWaitO: S was computed ahead of the previous tile's PV (double-buffered S), so before an O
 // rescale the warp waits for that PV on o_bar (phase parity o_parity).  Without it, the
 // previous PV is known complete (it was issued before this tile's S).
-template <int D, bool kWaitO = false>
+// kP8: P is written as e4m3 (four keys per 32-bit column, over S columns 0..31, for the
+// kind::f8f6f4 P V), rounded to nearest, offset by 2^kP8Offset with its own rescale threshold;
+// the row sum adds the fp32 weights before rounding.  Widening the bytes back to sum exactly the
+// quantised weights costs ten instructions per four keys on an issue-bound loop; the fp32 sum
+// leaves a common factor sum(q(p)) / sum(p) on the row, within the same 2^-4 relative bound as
+// each quantised weight and, over many keys, far inside it (the rounding errors average out).
+template <int D, bool kWaitO = false, bool kP8 = false>
 __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid, bool first,
                                              uint32_t p_half_bar, float sl2, float& m_ref, float& l,
                                              uint32_t o_bar = 0, uint32_t o_parity = 0,
@@ -397,7 +437,7 @@ __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid
     if (first) {
         m_ref = m_new;
     } else {
-        const bool need = m_new > m_ref + kRescaleThreshold;
+        const bool need = m_new > m_ref + (kP8 ? kP8Threshold : kRescaleThreshold);
         rescale = __any_sync(0xffffffffu, need);
         if (need) {
             f = ex2_approx(m_ref - m_new);
@@ -407,31 +447,52 @@ __device__ __forceinline__ void softmax_step(uint32_t tS, uint32_t tO, int valid
     float suma[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) suma[a] = 0.f;
-    const float neg_m = -m_ref;
+    const float neg_m = kP8 ? kP8Offset - m_ref : -m_ref;
     const uint64_t sl2_2 = bcast2(sl2), neg_m2 = bcast2(neg_m);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        if constexpr (kP8) {
+            uint32_t pk[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                // x = s * scale * log2(e) - m for two columns in one packed FMA
-                float x0, x1;
-                fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
-                const bool poly = kPolyEvery > 0 && ((i >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-                const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-                const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-                const uint32_t pp = pack_bf16x2(p0, p1);
-                // the row sum adds the same bf16-rounded weights the PV MMA multiplies, so
-                // out is an exact weighted mean of V under those weights (8 accumulators)
-                const int a = (i >> 1) & 7;
-                suma[a] = add_bf16x2_f32(pp, suma[a]);
-                pk[cc * 16 + (i >> 1)] = pp;
+                for (int i = 0; i < 32; i += 4) {
+                    float x0, x1, x2, x3;
+                    fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
+                    fma2_bcast(x2, x3, __uint_as_float(sr[c][i + 2]), __uint_as_float(sr[c][i + 3]), sl2_2, neg_m2);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+                    pk[cc * 8 + (i >> 2)] = pack_e4m3x4(p0, p1, p2, p3);
+                    // the row sum adds the fp32 weights (two packed adds per four keys)
+                    const int a = 4 * ((i >> 2) & 1);
+                    add2_f32(suma[a], suma[a + 1], p0, p1);
+                    add2_f32(suma[a + 2], suma[a + 3], p2, p3);
+                }
             }
+            tmem_st16(tS + half * 16, pk);   // over S columns this thread has already read
+        } else {
+            uint32_t pk[32];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    // x = s * scale * log2(e) - m for two columns in one packed FMA
+                    float x0, x1;
+                    fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
+                    const bool poly = kPolyEvery > 0 && ((i >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+                    const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+                    const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+                    const uint32_t pp = pack_bf16x2(p0, p1);
+                    // the row sum adds the same bf16-rounded weights the PV MMA multiplies, so
+                    // out is an exact weighted mean of V under those weights (8 accumulators)
+                    const int a = (i >> 1) & 7;
+                    suma[a] = add_bf16x2_f32(pp, suma[a]);
+                    pk[cc * 16 + (i >> 1)] = pp;
+                }
+            }
+            tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
         }
-        tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
         if (half == 0 && !rescale && kSplitP) {
             tmem_wait_st();
             tc_fence_before();

@@ -35,6 +35,14 @@ constexpr bool kMmaWarp = SWATTN_MMA_WARP != 0;
 #endif
 constexpr bool kStagedMerge = SWATTN_STAGED_MERGE != 0;
 
+// Half of O += P V (keys [64 half, 64 half + 64) of the tile): bf16 P and V on kind::f16, or e4m3
+// P and V on kind::f8f6f4.
+template <int D, bool kPV8>
+__device__ __forceinline__ void pv_half(uint32_t tO, uint32_t tP, uint32_t v_tile, int half, bool accumulate) {
+    if constexpr (kPV8) issue_pv_f8_half<kMmaWarp>(tO, tP, v_tile, half, accumulate);
+    else issue_pv_half<D, kMmaWarp>(tO, tP, v_tile, half, accumulate);
+}
+
 // A bounded wait in the MMA issuer: warp-uniform when the whole warp runs the issuer, so that
 // every lane takes the same branch before the next elect.sync.
 template <bool kWarp>
@@ -58,7 +66,7 @@ __device__ __forceinline__ bool mma_wait2(uint32_t bar_a, uint32_t parity_a, uin
 // The TMA producer (one thread): Q tiles per piece, then the piece's K and V tiles in ring
 // order.  A function of its own, not inlined: the kernel's register budget is set by the softmax
 // warps, and the roles that hold little state must not have their loop state spilled for them.
-template <int D, bool kCommit, bool kQK8>
+template <int D, bool kCommit, bool kQK8, bool kPV8>
 __device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl, uint8_t* q_smem, uint8_t* kv_smem,
                                              Sched sched, volatile int* abort_flag) {
     constexpr int NQ = 2;
@@ -96,8 +104,8 @@ __device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl,
                 }
                 if (kCommit) cq.before_refill(s);
                 const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
-                mbar_arrive_expect_tx(fbar, kv == 0 ? QKTile<D, kQK8>::kBytes : kTileBytes);
-                load_kv_tile<D, kQK8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                mbar_arrive_expect_tx(fbar, kv_tile_bytes<D, kQK8, kPV8>(kv));
+                load_kv_tile<D, kQK8, kPV8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
                 if (kCommit) {
                     const bool mine = cslot >= 0 && pc.pair == j % sched.npairs &&
                                       ctl->seg_kind[tile_seg(ctl, j)] == 2;
@@ -127,7 +135,7 @@ __device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl,
 // The MMA issuer (one thread): per piece, S of each live Q tile for the first key tile, then per
 // key tile P V and the next tile's S for each live Q tile, in issue order.  Not inlined, for the
 // same reason as the producer.
-template <int D, bool kQK8>
+template <int D, bool kQK8, bool kPV8>
 __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t* kv_smem, uint32_t tmem,
                                         Sched sched, volatile int* abort_flag) {
     constexpr int NQ = 2;
@@ -182,7 +190,7 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
                     tc_fence_after();
                 }
                 if (kSplitP) {
-                    issue_pv_half<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                    pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
                     // the first Q tile's full P is waited for together with the next K tile
                     if (!(qt == 0 && more ? mma_wait2<kMmaWarp>(fbar, ppar, kbar, kpar, abort_flag)
                                           : mma_wait<kMmaWarp>(fbar, ppar, abort_flag))) {
@@ -190,9 +198,10 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
                         break;
                     }
                     tc_fence_after();
-                    issue_pv_half<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                    pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                 } else {
-                    issue_pv<D, kMmaWarp>(tO, tP, kv_base + sV * kTileBytes, jj > 0);
+                    pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                    pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                 }
                 ++tcnt[qt];
                 if (!more) mma_commit_any<kMmaWarp>(smem_u32(&ctl->o_full[qt]));   // O complete: epilogue
@@ -221,7 +230,9 @@ __device__ __noinline__ void persist_mma(SmemCtl* ctl, uint8_t* q_smem, uint8_t*
 // kCommit: the launch also stores the chunk's K_cur / V_cur into the cache (fused commit); a
 // separate instantiation, so the plain forward carries none of that code.
 // kQK8: Q and K are e4m3 (d = 128), S = Q K^T on kind::f8f6f4; V, P and O as in the bf16 kernel.
-template <int D, bool kCommit, bool kQK8>
+// kPV8 (with kQK8): V is e4m3 too and O += P V runs on kind::f8f6f4 with P quantised to e4m3; the
+// V scale is applied with the final normalisation.
+template <int D, bool kCommit, bool kQK8, bool kPV8>
 __global__ void __launch_bounds__(AttnLayout<D, 2>::kThreads, 1)
 attn_persistent_kernel(const __grid_constant__ AttnParams p) {
     constexpr int NQ = 2;
@@ -269,10 +280,10 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && nt > 0) persist_producer<D, kCommit, kQK8>(p, ctl, q_smem, kv_smem, sched, abort_flag);
+        if (lane == 0 && nt > 0) persist_producer<D, kCommit, kQK8, kPV8>(p, ctl, q_smem, kv_smem, sched, abort_flag);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if ((kMmaWarp || lane == 0) && nt > 0) persist_mma<D, kQK8>(ctl, q_smem, kv_smem, tmem, sched, abort_flag);
+        if ((kMmaWarp || lane == 0) && nt > 0) persist_mma<D, kQK8, kPV8>(ctl, q_smem, kv_smem, tmem, sched, abort_flag);
     } else {
         // ------------------------------------------------------------ softmax warpgroups
         const int qt = (warp - 2) >> 2;
@@ -303,7 +314,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                 ok = warp_wait(smem_u32(&ctl->s_full[qt]), tcnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                softmax_step<D>(tS, tO, valid, jj == 0, smem_u32(&ctl->p_half[qt]), p.scale_log2, m_ref, l);
+                softmax_step<D, false, kPV8>(tS, tO, valid, jj == 0, smem_u32(&ctl->p_half[qt]), p.scale_log2, m_ref, l);
                 warp_arrive(smem_u32(&ctl->p_full[qt]));
                 ++tcnt;
             }
@@ -329,7 +340,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
             const int m_row = qs.row0 + row;
             const size_t orow = ((size_t)b * qs.rows + m_row) * p.H + h;
             if (pc.j0 == 0 && pc.j1 == nt) {
-                const float inv = 1.f / l;
+                const float inv = kPV8 ? p.out_scale / l : 1.f / l;
                 if (m_row < qs.rows) {
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(qs.out, p.out_f32, orow, c, o[c], inv);
@@ -464,7 +475,7 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
                             o[c][i] = __float_as_uint(fmaf(w, __ldcg(po + (c * 32 + i) * kBlockM), __uint_as_float(o[c][i])));
                 }
             }
-            const float inv = 1.f / L_;
+            const float inv = kPV8 ? p.out_scale / L_ : 1.f / L_;
             if (m_row < qs.rows) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) store_row_chunk<D>(qs.out, p.out_f32, orow, c, o[c], inv);
@@ -485,9 +496,9 @@ attn_persistent_kernel(const __grid_constant__ AttnParams p) {
 template <int D>
 static cudaError_t launch_persistent_d(const AttnParams& p, int ctas, cudaStream_t stream) {
     using L = AttnLayout<D, 2>;
-    auto kern = p.commit ? attn_persistent_kernel<D, true, false> : attn_persistent_kernel<D, false, false>;
+    auto kern = p.commit ? attn_persistent_kernel<D, true, false, false> : attn_persistent_kernel<D, false, false, false>;
     if constexpr (D == 128) {
-        if (p.qk_fp8) kern = attn_persistent_kernel<D, false, true>;
+        if (p.qk_fp8) kern = p.pv_fp8 ? attn_persistent_kernel<D, false, true, true> : attn_persistent_kernel<D, false, true, false>;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;

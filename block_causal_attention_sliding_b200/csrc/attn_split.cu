@@ -51,7 +51,16 @@ struct SplitLayout {
     static_assert(kNeed <= 227 * 1024, "shared memory");
 };
 
-template <int D>
+// Half of O += P V: bf16 P and V on kind::f16, or e4m3 on kind::f8f6f4.
+template <int D, bool kPV8>
+__device__ __forceinline__ void split_pv_half(uint32_t tO, uint32_t tP, uint32_t v_tile, int half, bool accumulate) {
+    if constexpr (kPV8) issue_pv_f8_half(tO, tP, v_tile, half, accumulate);
+    else issue_pv_half<D>(tO, tP, v_tile, half, accumulate);
+}
+
+// kQK8: e4m3 Q and K (S on kind::f8f6f4); kPV8 (with kQK8): e4m3 V and P too (O += P V on
+// kind::f8f6f4), the partials then carry the V scale, which the combine applies.
+template <int D, bool kQK8, bool kPV8>
 __global__ void __launch_bounds__(SplitLayout<D>::kThreads, 1)
 attn_split_kernel(const __grid_constant__ AttnParams p) {
     using L = SplitLayout<D>;
@@ -127,9 +136,9 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && n > 0) {
             const uint32_t qbar = smem_u32(&ctl->q_full);
-            mbar_arrive_expect_tx(qbar, kTileBytes);
-            for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
-                tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * kBoxCols, h, 0, b);
+            mbar_arrive_expect_tx(qbar, QKTile<D, kQK8>::kBytes);
+            for (int c = 0; c < QKTile<D, kQK8>::kBoxes; ++c)
+                tma_load_4d(smem_u32(q_smem + c * kBoxBytes), &p.tm_q, qbar, c * QKTile<D, kQK8>::kBoxCols, h, 0, b);
             uint32_t it = 0;
             bool ok = true;
             for (int jj = 0, j = sl; jj < n && ok; ++jj, j += ns) {
@@ -140,8 +149,8 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
                         break;
                     }
                     const uint32_t fbar = smem_u32(&ctl->kv_full[s]);
-                    mbar_arrive_expect_tx(fbar, kTileBytes);
-                    load_kv_tile<D>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
+                    mbar_arrive_expect_tx(fbar, kv_tile_bytes<D, kQK8, kPV8>(kv));
+                    load_kv_tile<D, kQK8, kPV8>(p, ctl, j, kv, h, b, smem_u32(kv_smem + s * kTileBytes), fbar);
                 }
             }
             // never leave while copies are in flight: the last fill of every stage has landed
@@ -163,7 +172,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
             if (ok) ok = wait_or_abort(smem_u32(&ctl->kv_full[0]), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_s<D>(tmem, q_base, kv_base);   // S_0 into buffer 0
+                issue_s_qk<D, kQK8>(tmem, q_base, kv_base);   // S_0 into buffer 0
                 mma_commit(smem_u32(&ctl->s_full[0]));
                 mma_commit(smem_u32(&ctl->kv_empty[0]));
             }
@@ -176,7 +185,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
                     if (!wait_or_abort(smem_u32(&ctl->kv_full[sK]), (itK / kStages) & 1, abort_flag)) break;
                     tc_fence_after();
                     const int nb = (jj + 1) & 1;
-                    issue_s<D>(tmem + nb * kBlockN, q_base, kv_base + sK * kTileBytes);
+                    issue_s_qk<D, kQK8>(tmem + nb * kBlockN, q_base, kv_base + sK * kTileBytes);
                     mma_commit(smem_u32(&ctl->s_full[nb]));
                     mma_commit(smem_u32(&ctl->kv_empty[sK]));
                 }
@@ -188,10 +197,10 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
                 if (!wait_or_abort(smem_u32(&ctl->kv_full[sV]), (itV / kStages) & 1, abort_flag)) break;
                 if (!wait_or_abort(smem_u32(&ctl->p_half[buf]), ph, abort_flag)) break;
                 tc_fence_after();
-                issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
+                split_pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 0, jj > 0);
                 if (!wait_or_abort(smem_u32(&ctl->p_full[buf]), ph, abort_flag)) break;
                 tc_fence_after();
-                issue_pv_half<D>(tO, tP, kv_base + sV * kTileBytes, 1, true);
+                split_pv_half<D, kPV8>(tO, tP, kv_base + sV * kTileBytes, 1, true);
                 mma_commit(smem_u32(&x->pv_done));
                 mma_commit(smem_u32(&ctl->kv_empty[sV]));
                 if (jj + 1 == n) mma_commit(smem_u32(&ctl->o_full[0]));   // O complete: epilogue
@@ -208,7 +217,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         const uint32_t tO = lane_base + L::kColO;
         float m_ref = -INFINITY;   // reference max, log2-scaled
-        float l = 0.f;             // row sum of the bf16-rounded exp2(s*sl2 - m_ref)
+        float l = 0.f;             // row sum of the weights (see softmax_step)
         bool ok = true;
         for (int jj = 0; jj < n; ++jj) {
             int seg, row0, valid;
@@ -217,7 +226,7 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
             ok = warp_wait(smem_u32(&ctl->s_full[buf]), (jj >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            softmax_step<D, true>(lane_base + buf * kBlockN, tO, valid, jj == 0, smem_u32(&ctl->p_half[buf]),
+            softmax_step<D, true, kPV8>(lane_base + buf * kBlockN, tO, valid, jj == 0, smem_u32(&ctl->p_half[buf]),
                                   p.scale_log2, m_ref, l, smem_u32(&x->pv_done), (uint32_t)((jj - 1) & 1),
                                   abort_flag);
             warp_arrive(smem_u32(&ctl->p_full[buf]));
@@ -282,10 +291,10 @@ static cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 blo
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int D>
+template <int D, bool kQK8, bool kPV8>
 static cudaError_t launch_split_d(const AttnParams& p, int splits, cudaStream_t stream) {
     using L = SplitLayout<D>;
-    auto kern = attn_split_kernel<D>;
+    auto kern = attn_split_kernel<D, kQK8, kPV8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     return launch_dependent(kern, dim3(splits, p.H, p.B), dim3(L::kThreads), L::kSmemBytes, stream, p);
@@ -293,8 +302,12 @@ static cudaError_t launch_split_d(const AttnParams& p, int splits, cudaStream_t 
 
 cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream) {
     if (p.n_q < 1 || p.n_q > kBlockM || splits < 1) return cudaErrorInvalidValue;
-    if (d == 128) return launch_split_d<128>(p, splits, stream);
-    if (d == 64) return launch_split_d<64>(p, splits, stream);
+    if (d == 128) {
+        if (p.qk_fp8) return p.pv_fp8 ? launch_split_d<128, true, true>(p, splits, stream)
+                                      : launch_split_d<128, true, false>(p, splits, stream);
+        return launch_split_d<128, false, false>(p, splits, stream);
+    }
+    if (d == 64 && !p.qk_fp8) return launch_split_d<64, false, false>(p, splits, stream);
     return cudaErrorInvalidValue;
 }
 
@@ -304,7 +317,8 @@ cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t st
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
                                                       const float* __restrict__ ml_part, void* out,
-                                                      int B, int H, int n_q, int splits, int out_f32) {
+                                                      int B, int H, int n_q, int splits, int out_f32,
+                                                      float out_scale) {
     // one warp per output row; each lane owns D / 32 consecutive columns.  The splits are read
     // eight at a time with every load of a group issued before any is used (one memory round
     // trip per group), and merged with a running max like the online softmax.
@@ -371,7 +385,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         }
         M = Mg;
     }
-    const float inv = 1.f / den;
+    const float inv = out_scale / den;   // out_scale: the V scale of e4m3 V, else 1
     const size_t orow = ((size_t)b * n_q + row) * H + h;
     if (out_f32) {
         float* dst = static_cast<float*>(out) + orow * D + lane * V;
@@ -385,17 +399,17 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
-                           int n_q, int d, int splits, int out_f32, cudaStream_t stream) {
+                           int n_q, int d, int splits, int out_f32, float out_scale, cudaStream_t stream) {
     const long long warps = (long long)B * H * n_q;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     // programmatic dependent launch: the combine's blocks are scheduled while the split kernel
     // finishes, and wait on the device (griddepcontrol.wait) instead of behind a launch gap
     if (d == 128)
         return launch_dependent(combine_kernel<128>, dim3(blocks), dim3(256), 0, stream, o_part, ml_part, out, B, H,
-                                n_q, splits, out_f32);
+                                n_q, splits, out_f32, out_scale);
     if (d == 64)
         return launch_dependent(combine_kernel<64>, dim3(blocks), dim3(256), 0, stream, o_part, ml_part, out, B, H,
-                                n_q, splits, out_f32);
+                                n_q, splits, out_f32, out_scale);
     return cudaErrorInvalidValue;
 }
 

@@ -287,11 +287,12 @@ static int vpr_log2_of(int d, int esz) {
     return (vpr >= 1 && (1 << l) == vpr) ? l : -1;
 }
 
-cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, cudaStream_t stream) {
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, int v_esz,
+                                cudaStream_t stream) {
     if (a.n < 1 || a.n > kMaxBatch) return cudaErrorInvalidValue;
-    const int vpr_log2 = vpr_log2_of(d, 2), vpr_log2_k = vpr_log2_of(d, k_esz);
+    const int vpr_log2 = vpr_log2_of(d, v_esz), vpr_log2_k = vpr_log2_of(d, k_esz);
     if (vpr_log2 < 0 || vpr_log2_k < 0) return cudaErrorInvalidValue;
-    const int vpr = 1 << vpr_log2;
+    const int vpr = 1 << (vpr_log2 > vpr_log2_k ? vpr_log2 : vpr_log2_k);   // the wider of K and V rows
     const long long rows = (long long)B * T;
     if (rows < 1 || rows > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int per_row = H * vpr;
@@ -305,10 +306,10 @@ cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d
 
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int S, int32_t* state, const TableAdvance& ta,
-                            int advance, cudaStream_t stream, int k_esz) {
-    const int vpr_log2 = vpr_log2_of(d, 2), vpr_log2_k = vpr_log2_of(d, k_esz);   // 16-byte vectors per row
-    if (vpr_log2 < 0 || vpr_log2_k < 0) return cudaErrorInvalidValue;              // d is 64 or 128
-    const int vpr = 1 << vpr_log2;
+                            int advance, cudaStream_t stream, int k_esz, int v_esz) {
+    const int vpr_log2 = vpr_log2_of(d, v_esz), vpr_log2_k = vpr_log2_of(d, k_esz);   // 16-byte vectors per row
+    if (vpr_log2 < 0 || vpr_log2_k < 0) return cudaErrorInvalidValue;                  // d is 64 or 128
+    const int vpr = 1 << (vpr_log2 > vpr_log2_k ? vpr_log2 : vpr_log2_k);   // the wider of K and V rows
     const long long rows = (long long)B * N;
     if (rows < 1 || rows > 0x7fffffffLL || (advance && !ring)) return cudaErrorInvalidValue;
     const int per_row = H * vpr;
@@ -320,9 +321,10 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
     return cudaGetLastError();
 }
 
-cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int32_t* state,
-                              const TableAdvance& ta, int S, int ctas, cudaStream_t stream) {
-    if (B < 1 || T < 1 || H < 1 || ctas < 1 || (d * k_esz) % 16 != 0 || d * 2 > 256) return cudaErrorInvalidValue;
+cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int v_esz,
+                              int32_t* state, const TableAdvance& ta, int S, int ctas, cudaStream_t stream) {
+    if (B < 1 || T < 1 || H < 1 || ctas < 1 || (d * k_esz) % 16 != 0 || (d * v_esz) % 16 != 0 || d * 2 > 256)
+        return cudaErrorInvalidValue;
     CommitItems it;
     it.B = B;
     it.T = T;
@@ -330,7 +332,7 @@ cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d
     it.nt = (T + kCommitRows - 1) / kCommitRows;
     it.nh = (H + kCommitHeads - 1) / kCommitHeads;
     const int h_box = H < kCommitHeads ? H : kCommitHeads;
-    const int box_k = d * k_esz * kCommitRows * h_box, box_v = d * 2 * kCommitRows * h_box;
+    const int box_k = d * k_esz * kCommitRows * h_box, box_v = d * v_esz * kCommitRows * h_box;
     const int smem = kCommitBufs * (box_k > box_v ? box_k : box_v) + 1024;
     cudaError_t e = cudaFuncSetAttribute(commit_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

@@ -17,8 +17,9 @@ constexpr int kCommitHeads = 24;
 constexpr int kCommitBufs = 8;   // buffers per CTA (one CTA per SM)
 
 // Copy the finished chunk into the ring slot the device counter names, then (last CTA) advance
-// the counter and rebuild the table.  ctas: one per SM.  k_esz: bytes per K element (1: e4m3).
-cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int32_t* state,
-                              const TableAdvance& ta, int S, int ctas, cudaStream_t stream);
+// the counter and rebuild the table.  ctas: one per SM.  k_esz, v_esz: bytes per K and V element
+// (1: e4m3, 2: bf16).
+cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int v_esz,
+                              int32_t* state, const TableAdvance& ta, int S, int ctas, cudaStream_t stream);
 
 }  // namespace swattn

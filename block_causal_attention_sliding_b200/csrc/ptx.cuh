@@ -235,6 +235,23 @@ __device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
         ::"r"(bar) : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc] with 8-bit floating-point operands (kind::f8f6f4), one
+// thread and converged-warp forms.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // Arrive (once) on an mbarrier when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -299,6 +316,31 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+          "r"(r[15])
+        : "memory");
+}
+
+// ------------------------------------------------------------------ e4m3
+
+// Four fp32 values rounded to nearest (saturating at the largest finite e4m3) and packed as
+// e4m3 bytes, p0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r) : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
+    return r;
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and stride byte
@@ -323,11 +365,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | ((uint32_t)(M >> 4) << 24);
 }
 
-// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (both K-major), fp32 D.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B, fp32 D; A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major = false) {
     return (1u << 4)                      // D format: f32
          | (0u << 7)                      // A format: e4m3
          | (0u << 10)                     // B format: e4m3
+         | ((b_mn_major ? 1u : 0u) << 16) // B major
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
 }
@@ -360,6 +403,13 @@ __device__ __forceinline__ void fma2_bcast(float& x0, float& x1, float a0, float
     asm("{\n\t.reg .b64 a, d;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 d, a, %4, %5;\n\t"
         "mov.b64 {%0, %1}, d;\n\t}"
         : "=f"(x0), "=f"(x1) : "f"(a0), "f"(a1), "l"(s2), "l"(b2));
+}
+
+// (s0, s1) += (a0, a1) as one packed two-lane fp32 add (sm_100 f32x2 form, round to nearest).
+__device__ __forceinline__ void add2_f32(float& s0, float& s1, float a0, float a1) {
+    asm("{\n\t.reg .b64 s, a;\n\tmov.b64 s, {%0, %1};\n\tmov.b64 a, {%2, %3};\n\t"
+        "add.rn.f32x2 s, s, a;\n\tmov.b64 {%0, %1}, s;\n\t}"
+        : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
 }
 
 // v in both lanes of a packed f32x2 operand.

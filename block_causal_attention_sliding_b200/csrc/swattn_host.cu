@@ -129,6 +129,9 @@ int check_cfg(const sw_attn_config& c) {
     if (c.qk_fp8 && c.d != 128) return fail(SW_ESHAPE, "e4m3 Q/K need d = 128");
     if (c.qk_fp8 && c.commit_in_forward) return fail(SW_ESHAPE, "commit_in_forward is not available with e4m3 Q/K");
     if (!std::isfinite(c.q_scale) || !std::isfinite(c.k_scale)) return fail(SW_EINVAL, "scales must be finite");
+    if (c.pv_fp8 != 0 && c.pv_fp8 != 1) return fail(SW_EINVAL, "pv_fp8 must be 0 or 1");
+    if (c.pv_fp8 && !c.qk_fp8) return fail(SW_ESHAPE, "pv_fp8 requires qk_fp8 (e4m3 Q and K)");
+    if (!std::isfinite(c.v_scale)) return fail(SW_EINVAL, "v_scale must be finite");
     if (c.commit_path != SW_COMMIT_AUTO && c.commit_path != SW_COMMIT_COPY && c.commit_path != SW_COMMIT_TMA)
         return fail(SW_EINVAL, "bad commit_path");
     const double elems = (double)c.B * c.H * (c.W + 2) * c.tokens_per_chunk * c.d;
@@ -155,9 +158,9 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->cfg = *cfg;
     if (h->cfg.scale <= 0.f) h->cfg.scale = 1.0f / std::sqrt((float)cfg->d);
     h->short_q = cfg->max_short_q == 0 ? kMaxShortQ : (cfg->max_short_q < 0 ? 0 : cfg->max_short_q);
-    if (cfg->qk_fp8) h->short_q = 0;   // e4m3 Q/K run on the persistent kernel only
     if (h->cfg.q_scale <= 0.f) h->cfg.q_scale = 1.f;
     if (h->cfg.k_scale <= 0.f) h->cfg.k_scale = 1.f;
+    if (h->cfg.v_scale <= 0.f) h->cfg.v_scale = 1.f;
     // window slots: W, or W + 1 to keep a spare slot for commits during the chunk's own forward
     h->R = cfg->commit_in_forward && cfg->W > 0 ? cfg->W + 1 : cfg->W;
     h->S = h->R + (cfg->sink ? 1 : 0);
@@ -167,10 +170,11 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     const size_t B = cfg->B, H = cfg->H, d = cfg->d, T = cfg->tokens_per_chunk;
     size_t off = align_up(sizeof(int32_t) * (kStateHeaderInts + h->table_ints), 1024);
     const size_t ek = cfg->qk_fp8 ? 1 : 2;   // bytes per K element (e4m3 on an FP8 handle)
+    const size_t ev = cfg->pv_fp8 ? 1 : 2;   // bytes per V element
     h->off_kcache = off; off = align_up(off + B * H * h->S * T * d * ek, 1024);
-    h->off_vcache = off; off = align_up(off + B * H * h->S * T * d * 2, 1024);
+    h->off_vcache = off; off = align_up(off + B * H * h->S * T * d * ev, 1024);
     h->off_kcond = off;  off = align_up(off + B * H * cfg->n_cond * d * ek, 1024);
-    h->off_vcond = off;  off = align_up(off + B * H * cfg->n_cond * d * 2, 1024);
+    h->off_vcond = off;  off = align_up(off + B * H * cfg->n_cond * d * ev, 1024);
     h->off_opart = off;
     if (h->short_q > 0) off = align_up(off + (size_t)h->max_splits * bh * kBlockM * d * 4, 1024);
     h->off_ml = off;
@@ -194,6 +198,7 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     c.sink = 1; c.out_dtype = SW_OUT_BF16; c.scale = 0.f; c.max_short_q = 0; c.schedule = SW_SCHED_AUTO;
     c.commit_in_forward = 0;
     c.qk_fp8 = 0; c.q_scale = 0.f; c.k_scale = 0.f; c.commit_path = SW_COMMIT_AUTO;
+    c.pv_fp8 = 0; c.v_scale = 0.f;
     return sw_attn_create_ex(&c, out);
 }
 
@@ -221,17 +226,19 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         // ring [B][H][S][T][d]: dims {d, T, S, H, B}; rows past T read as zero
         const uint64_t dims[5] = {(uint64_t)c.d, (uint64_t)c.tokens_per_chunk, (uint64_t)h->S, (uint64_t)c.H,
                                   (uint64_t)c.B};
-        const uint64_t row = (uint64_t)c.d * 2;
-        const uint64_t strides[4] = {row, row * c.tokens_per_chunk, row * c.tokens_per_chunk * h->S,
-                                     row * c.tokens_per_chunk * h->S * c.H};
-        const uint32_t box[5] = {64, (uint32_t)kBlockN, 1, 1, 1};
+        // boxes of 128-byte rows (64 bf16 or 128 e4m3 columns), 128-byte swizzle
         const int ek = c.qk_fp8 ? 1 : 2;   // K in e4m3 on an FP8 handle
         const uint64_t rowk = (uint64_t)c.d * ek;
         const uint64_t stridesk[4] = {rowk, rowk * c.tokens_per_chunk, rowk * c.tokens_per_chunk * h->S,
                                       rowk * c.tokens_per_chunk * h->S * c.H};
         const uint32_t boxk[5] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1, 1};
+        const int ev = c.pv_fp8 ? 1 : 2;   // V in e4m3 on a pv_fp8 handle
+        const uint64_t rowv = (uint64_t)c.d * ev;
+        const uint64_t stridesv[4] = {rowv, rowv * c.tokens_per_chunk, rowv * c.tokens_per_chunk * h->S,
+                                      rowv * c.tokens_per_chunk * h->S * c.H};
+        const uint32_t boxv[5] = {(uint32_t)(128 / ev), (uint32_t)kBlockN, 1, 1, 1};
         if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, stridesk, boxk, "K cache", ek))) return rc;
-        if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, strides, box, "V cache"))) return rc;
+        if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, stridesv, boxv, "V cache", ev))) return rc;
         // chunk commits by TMA: the ring with a box of d x kCommitRows rows x up to kCommitHeads
         // heads (unswizzled), and a trial map of the caller side (permuted strides); where the
         // driver declines either, commits use the copy kernel
@@ -246,22 +253,23 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         h->commit_tma = want &&
             encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cbox, "K cache", ek,
                    CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
-            encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, strides, cbox, "V cache", 2,
+            encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, stridesv, cbox, "V cache", ev,
                    CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
             encode_commit_src(&trial, ws + h->off_kcache, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek) == SW_OK;
         g_err.clear();
     }
     if (c.n_cond > 0) {
         const uint64_t dims[4] = {(uint64_t)c.d, (uint64_t)c.n_cond, (uint64_t)c.H, (uint64_t)c.B};
-        const uint64_t row = (uint64_t)c.d * 2;
-        const uint64_t strides[3] = {row, row * c.n_cond, row * c.n_cond * c.H};
-        const uint32_t box[4] = {64, (uint32_t)kBlockN, 1, 1};
         const int ek = c.qk_fp8 ? 1 : 2;
         const uint64_t rowk = (uint64_t)c.d * ek;
         const uint64_t stridesk[3] = {rowk, rowk * c.n_cond, rowk * c.n_cond * c.H};
         const uint32_t boxk[4] = {(uint32_t)(128 / ek), (uint32_t)kBlockN, 1, 1};
+        const int ev = c.pv_fp8 ? 1 : 2;
+        const uint64_t rowv = (uint64_t)c.d * ev;
+        const uint64_t stridesv[3] = {rowv, rowv * c.n_cond, rowv * c.n_cond * c.H};
+        const uint32_t boxv[4] = {(uint32_t)(128 / ev), (uint32_t)kBlockN, 1, 1};
         if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, stridesk, boxk, "K cond", ek))) return rc;
-        if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, strides, box, "V cond"))) return rc;
+        if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, stridesv, boxv, "V cond", ev))) return rc;
     }
     e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk,
                            reinterpret_cast<int32_t*>(ws + h->off_sk_cnt), h->n_counters,
@@ -302,7 +310,7 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
     if (!aligned16(K_cond) || !aligned16(V_cond)) return fail(SW_EALIGN, "condition tensors must be 16-byte aligned");
     cudaError_t e = launch_relayout(K_cond, V_cond, h->ws + h->off_kcond, h->ws + h->off_vcond, c.B, c.n_cond,
                                     c.H, c.d, c.n_cond, 0, h->S, reinterpret_cast<int32_t*>(h->ws), table_advance(h),
-                                    0, static_cast<cudaStream_t>(stream), c.qk_fp8 ? 1 : 2);
+                                    0, static_cast<cudaStream_t>(stream), c.qk_fp8 ? 1 : 2, c.pv_fp8 ? 1 : 2);
     if (e != cudaSuccess) return cuda_fail(e, "condition copy launch");
     h->cond_set = true;
     return SW_OK;
@@ -313,20 +321,21 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
 // or the copy kernel where the handle's maps could not be made.
 static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_t st) {
     const sw_attn_config& c = h->cfg;
-    const int ek = c.qk_fp8 ? 1 : 2;
+    const int ek = c.qk_fp8 ? 1 : 2, ev = c.pv_fp8 ? 1 : 2;
     int32_t* state = reinterpret_cast<int32_t*>(h->ws);
     cudaError_t e;
     if (h->commit_tma) {
         CommitMaps m;
         int rc;
         if ((rc = encode_commit_src(&m.src_k, K, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek))) return rc;
-        if ((rc = encode_commit_src(&m.src_v, V, c.B, c.tokens_per_chunk, c.H, c.d, "V", 2))) return rc;
+        if ((rc = encode_commit_src(&m.src_v, V, c.B, c.tokens_per_chunk, c.H, c.d, "V", ev))) return rc;
         m.dst_k = h->tm_commit_k;
         m.dst_v = h->tm_commit_v;
-        e = launch_commit_tma(m, c.B, c.tokens_per_chunk, c.H, c.d, ek, state, table_advance(h), h->S, h->num_sms, st);
+        e = launch_commit_tma(m, c.B, c.tokens_per_chunk, c.H, c.d, ek, ev, state, table_advance(h), h->S, h->num_sms,
+                              st);
     } else {
         e = launch_relayout(K, V, h->ws + h->off_kcache, h->ws + h->off_vcache, c.B, c.tokens_per_chunk, c.H, c.d,
-                            h->S * c.tokens_per_chunk, 1, h->S, state, table_advance(h), 1, st, ek);
+                            h->S * c.tokens_per_chunk, 1, h->S, state, table_advance(h), 1, st, ek, ev);
     }
     return e == cudaSuccess ? SW_OK : cuda_fail(e, "append launch");
 }
@@ -382,7 +391,7 @@ static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const v
     const int eqk = c.qk_fp8 ? 1 : 2;
     if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q", eqk))) return rc;
     if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur", eqk))) return rc;
-    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur"))) return rc;
+    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur", c.pv_fp8 ? 1 : 2))) return rc;
     // maps for regions this handle does not have are never read; fill them with a valid map
     p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
     p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
@@ -400,6 +409,8 @@ static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const v
     p.n_qc = 0;
     p.commit = 0;
     p.qk_fp8 = c.qk_fp8;
+    p.pv_fp8 = c.pv_fp8;
+    p.out_scale = c.pv_fp8 ? c.v_scale : 1.f;
     p.ring_R = h->R;
     p.sink = c.sink;
     p.out_f32 = c.out_dtype == SW_OUT_F32;
@@ -466,7 +477,7 @@ int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* 
         p.ml_part = reinterpret_cast<float*>(h->ws + h->off_ml);
         cudaError_t e = launch_split(p, c.d, splits, st);
         if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
-        e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, st);
+        e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, splits, p.out_f32, p.out_scale, st);
         if (e != cudaSuccess) return cuda_fail(e, "combine launch");
         return SW_OK;
     }
@@ -487,8 +498,8 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
         if (h->device != h0->device) return fail(SW_ESTATE, "handle %d is on another device", l);
         const sw_attn_config& c = h->cfg;
         if (c.B != c0.B || c.H != c0.H || c.d != c0.d || c.tokens_per_chunk != c0.tokens_per_chunk ||
-            c.qk_fp8 != c0.qk_fp8)
-            return fail(SW_ESHAPE, "handle %d: B, H, d, T and the K format must match handle 0", l);
+            c.qk_fp8 != c0.qk_fp8 || c.pv_fp8 != c0.pv_fp8)
+            return fail(SW_ESHAPE, "handle %d: B, H, d, T and the K and V formats must match handle 0", l);
         if (!K[l] || !V[l]) return fail(SW_EINVAL, "null K or V for handle %d", l);
         if (!aligned16(K[l]) || !aligned16(V[l])) return fail(SW_EALIGN, "K and V of handle %d must be 16-byte aligned", l);
         for (int m = 0; m < l; ++m)
@@ -512,7 +523,8 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
             a.sink[q] = h->cfg.sink;
             a.n_cond[q] = h->cfg.n_cond;
         }
-        cudaError_t e = launch_append_batch(a, c0.B, c0.tokens_per_chunk, c0.H, c0.d, c0.qk_fp8 ? 1 : 2, st);
+        cudaError_t e = launch_append_batch(a, c0.B, c0.tokens_per_chunk, c0.H, c0.d, c0.qk_fp8 ? 1 : 2,
+                                            c0.pv_fp8 ? 1 : 2, st);
         if (e != cudaSuccess) return cuda_fail(e, "batched append launch");
     }
     return SW_OK;
@@ -633,7 +645,6 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
     const sw_attn_config& c = h->cfg;
-    if (c.qk_fp8) return fail(SW_ESTATE, "the split-K path has no e4m3 Q/K form");
     if (n_q < 1 || n_q > kMaxShortQ || n_q > c.tokens_per_chunk)
         return fail(SW_ESHAPE, "n_q must be in [1, min(%d, T)] (n_q=%d)", kMaxShortQ, n_q);
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))
@@ -673,7 +684,7 @@ extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     e = launch_split(p, c.d, (int)splits, st);
     if (e != cudaSuccess) return cuda_fail(e, "split-K attention launch");
-    e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, (int)splits, p.out_f32, st);
+    e = launch_combine(p.o_part, p.ml_part, out, c.B, c.H, n_q, c.d, (int)splits, p.out_f32, p.out_scale, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return SW_OK;
 }

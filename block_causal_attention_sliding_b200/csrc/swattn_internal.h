@@ -67,6 +67,8 @@ struct alignas(64) AttnParams {
     int n_qc;                // condition-stream query rows (0: none); their Q tiles follow the chunk's
     int commit;              // 1: also store K_cur / V_cur into the ring slot of the active chunk
     int qk_fp8;              // 1: Q and K (current, cache, condition) are e4m3, scales folded into scale_log2
+    int pv_fp8;              // 1: V (current, cache, condition) is e4m3 and P V runs on kind::f8f6f4
+    float out_scale;         // applied with the final normalisation (the e4m3 V's scale; 1 otherwise)
     int ring_R;              // window slots of the ring (for the commit slot)
     int sink;
     int out_f32;
@@ -93,7 +95,7 @@ struct TableAdvance {
 // only) the same launch then advances the counter and rebuilds the table (a chunk commit).
 cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV, int B, int N,
                             int H, int d, int rows_per_bh, int ring, int S, int32_t* state, const TableAdvance& ta,
-                            int advance, cudaStream_t stream, int k_esz = 2);
+                            int advance, cudaStream_t stream, int k_esz = 2, int v_esz = 2);
 // One chunk commit for each of up to kMaxBatch handles (layers) of the same B, T, H, d, in one
 // copy launch and one table launch (the per-handle window, sink, slots and counter stay apart).
 constexpr int kMaxBatch = 32;
@@ -106,7 +108,8 @@ struct AppendBatch {
     int R[kMaxBatch], S[kMaxBatch], W[kMaxBatch], sink[kMaxBatch], n_cond[kMaxBatch];
     int n;                       // handles in this launch
 };
-cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, cudaStream_t stream);
+cudaError_t launch_append_batch(const AppendBatch& a, int B, int T, int H, int d, int k_esz, int v_esz,
+                                cudaStream_t stream);
 
 cudaError_t launch_attention(const AttnParams& p, int d, int grid_x, cudaStream_t stream);
 cudaError_t launch_persistent(const AttnParams& p, int d, int ctas, cudaStream_t stream);
@@ -114,6 +117,6 @@ cudaError_t launch_tri(const AttnParams& p, int d, int ctas, cudaStream_t stream
 cudaError_t launch_split(const AttnParams& p, int d, int splits, cudaStream_t stream);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
-                           int n_q, int d, int splits, int out_f32, cudaStream_t stream);
+                           int n_q, int d, int splits, int out_f32, float out_scale, cudaStream_t stream);
 
 }  // namespace swattn

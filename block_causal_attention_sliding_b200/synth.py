@@ -12,9 +12,10 @@ bf16 inputs.  Recipe (stated once, used everywhere):
     queries = 5; condition K/V use chunk 0, step 0 for the first prompt and chunk v, step 0 for
     prompt version v (a prompt changed mid-stream); condition queries use the (chunk, step) of
     the forward they belong to.
-  * FP8 inputs (queries and keys of an e4m3 handle): the same draws divided by a power-of-two
-    scale (FP8_SCALE, exact) and rounded to OCP e4m3 (float8_e4m3fn, round to nearest even);
-    the dequantised values x8 * FP8_SCALE are what the attention sees.
+  * FP8 inputs (queries and keys of an e4m3 handle, and values too on a handle with e4m3 V): the
+    same draws divided by a power-of-two scale (FP8_SCALE, exact) and rounded to OCP e4m3
+    (float8_e4m3fn, round to nearest even); the dequantised values x8 * FP8_SCALE are what the
+    attention sees.
 The user layout is [B, N, H, d] contiguous.
 """
 from __future__ import annotations
@@ -81,13 +82,14 @@ def from_e4m3(x8: torch.Tensor, scale: float = FP8_SCALE) -> torch.Tensor:
     return x8.float() * scale
 
 
-def chunk_inputs_fp8(wl, chunk: int, step: int, *, seed: int = 0, device="cpu"):
-    """Q and K_cur in e4m3, V_cur in bf16, for one (chunk, step) of an e4m3 handle."""
-    Q, K, V = chunk_inputs(wl, chunk, step, seed=seed, device=device)
-    return to_e4m3(Q), to_e4m3(K), V
+def chunk_inputs_fp8(wl, chunk: int, step: int, *, seed: int = 0, n_q: int | None = None, device="cpu",
+                     v8: bool = False):
+    """Q and K_cur in e4m3, V_cur in bf16 (e4m3 with v8), for one (chunk, step) of an e4m3 handle."""
+    Q, K, V = chunk_inputs(wl, chunk, step, seed=seed, n_q=n_q, device=device)
+    return to_e4m3(Q), to_e4m3(K), (to_e4m3(V) if v8 else V)
 
 
-def cond_inputs_fp8(wl, *, seed: int = 0, version: int = 0, device="cpu"):
-    """Condition K in e4m3, V in bf16."""
+def cond_inputs_fp8(wl, *, seed: int = 0, version: int = 0, device="cpu", v8: bool = False):
+    """Condition K in e4m3, V in bf16 (e4m3 with v8)."""
     Kc, Vc = cond_inputs(wl, seed=seed, version=version, device=device)
-    return to_e4m3(Kc), Vc
+    return to_e4m3(Kc), (to_e4m3(Vc) if v8 else Vc)

@@ -87,13 +87,22 @@ typedef struct {
                                 Q_cond, K_cur, the appended K and K_cond are e4m3 tensors of
                                 the same [B, N, H, d] shape, the K cache is kept in e4m3 (half
                                 the bytes) and S = Q K^T runs on kind::f8f6f4; V stays bf16.
-                                Requires d = 128; full path on the persistent schedule only
-                                (no split-K path, no commit_in_forward) */
+                                Requires d = 128; full path on the persistent schedule, short
+                                queries on the split-K path; no commit_in_forward */
     float q_scale, k_scale;  /* dequantisation scales of the e4m3 Q and K (per tensor; <= 0
                                 selects 1): the attention uses q * q_scale and k * k_scale */
     int   commit_path;       /* chunk commits: SW_COMMIT_AUTO (default; TMA bulk copies when
                                 the commit gives every SM at least a full ring of 8 items, else
                                 the copy kernel), SW_COMMIT_TMA or SW_COMMIT_COPY */
+    int   pv_fp8;            /* 1 (requires qk_fp8): V is e4m3 too -- V_cur, the appended V and
+                                V_cond are e4m3 tensors of the usual shapes, the V cache is kept in
+                                e4m3 (the whole K/V cache at half the bf16 bytes) -- and O = P V
+                                runs on kind::f8f6f4 with P quantised to e4m3.  A precision mode of
+                                its own: P in e4m3 carries 3 mantissa bits against bf16's 7, so
+                                the output's rounding error is about 16x that of bf16 P (a
+                                mean-relative error near 2.5e-2 on Gaussian inputs) */
+    float v_scale;           /* dequantisation scale of the e4m3 V (per tensor; <= 0 selects 1):
+                                the attention uses v * v_scale; applied once to the output */
 } sw_attn_config;
 
 /* schedules of the full path */
@@ -238,7 +247,6 @@ SW_API int sw_attn_forward_joint(sw_attn_t *h, const void *Q, const void *Q_cond
  *     may follow a reset of the device in the same process.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.  Same argument rules as
  *     sw_attn_forward; the caller's current device must be the workspace's device.
- *   - Handles with e4m3 Q/K (qk_fp8) have no split-K form: SW_ESTATE.
  */
 SW_API int sw_attn_forward_short_noalloc(sw_attn_t *h, const void *Q, const void *K_cur,
                                          const void *V_cur, void *out, int n_q, void *stream);

@@ -306,39 +306,52 @@ def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, 
     return results
 
 
+# The error an e4m3 P adds.  The kernel rounds P to the MMA's operand type and divides by the sum
+# of the rounded weights, so the output's error from P scales with that type's unit roundoff:
+# 2^-8 for bf16 (8 significant bits), 2^-4 for e4m3 (4).  The parity tolerance above is the one
+# bf16 P meets; with e4m3 P it is scaled by the ratio of the two, 2^4.
+E4M3_P_TOL = (MAX_ABS * 16, MEAN_REL * 16)
+
+
 def stream_and_check_fp8(wl, dev, *, chunks, check_at=None, n_rows=None, keep_last=None,
                          gen_on_device=False, out_dtype=torch.float32, seed=0, joint=False,
-                         tol=(MAX_ABS, MEAN_REL)):
-    """Stream through a handle with e4m3 queries and keys (V bf16): 2 forwards then an append
-    per chunk, all Q/K in e4m3 with scale FP8_SCALE.  The oracle computes the same attention on
-    the dequantised values (exact in float32).  With joint, the forward also carries e4m3
-    condition queries.  Returns a list of (k, step, which, max_abs, mean_rel)."""
+                         tol=None, pv8=False, n_q=None):
+    """Stream through a handle with e4m3 queries and keys (and, with pv8, e4m3 values: P V on
+    kind::f8f6f4): 2 forwards then an append per chunk, every e4m3 tensor with scale FP8_SCALE.
+    The oracle computes the same attention on the dequantised values (exact in float32).  With
+    joint, the forward also carries e4m3 condition queries; with n_q (<= 128) the forwards take
+    the chunk's first n_q queries (the split-K path).  Tolerance: the parity one, or E4M3_P_TOL
+    with pv8.  Returns a list of (k, step, which, max_abs, mean_rel)."""
     sc = synth.FP8_SCALE
+    if tol is None:
+        tol = E4M3_P_TOL if pv8 else (MAX_ABS, MEAN_REL)
     h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
-                               out_dtype=out_dtype, qk_fp8=True, q_scale=sc, k_scale=sc, device=dev)
+                               out_dtype=out_dtype, qk_fp8=True, q_scale=sc, k_scale=sc, pv_fp8=pv8,
+                               v_scale=sc, device=dev)
     gdev = dev if gen_on_device else "cpu"
-    Kc8, Vc = synth.cond_inputs_fp8(wl, seed=seed, device=gdev)
+    deq_v = (lambda t: synth.from_e4m3(t)) if pv8 else (lambda t: t)
+    Kc8, Vc = synth.cond_inputs_fp8(wl, seed=seed, device=gdev, v8=pv8)
     h.set_cond(Kc8.to(dev), Vc.to(dev))
     Kc = synth.from_e4m3(Kc8).cpu()
-    Vc = Vc.cpu()
+    Vc = deq_v(Vc).cpu()
     hist_K, hist_V, results = [], [], []
     for k in range(chunks):
         for step in range(wl.steps):
-            Q8, K8, V = synth.chunk_inputs_fp8(wl, k, step, seed=seed, device=gdev)
+            Q8, K8, V = synth.chunk_inputs_fp8(wl, k, step, seed=seed, n_q=n_q, device=gdev, v8=pv8)
             if joint:
                 Qc8 = synth.to_e4m3(synth.cond_queries(wl, k, step, seed=seed, device=gdev))
                 out, out_c = h.forward_joint(Q8.to(dev), Qc8.to(dev), K8.to(dev), V.to(dev))
                 sets = (("chunk", Q8, out, wl.T), ("cond", Qc8, out_c, wl.n_cond))
             else:
                 out = h.forward(Q8.to(dev), K8.to(dev), V.to(dev))
-                sets = (("chunk", Q8, out, wl.T),)
+                sets = (("chunk", Q8, out, Q8.shape[1]),)
             if check_at is None or k in check_at:
                 for which, q8, o, n in sets:
                     r = None if n_rows is None else sample_rows(n, n_rows, seed=1000 * k + step)
                     ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
                                            k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V,
                                            Q=synth.from_e4m3(q8).cpu(), K_cur=synth.from_e4m3(K8).cpu(),
-                                           V_cur=V.cpu(), rows=r)
+                                           V_cur=deq_v(V).cpu(), rows=r)
                     got = o.float().cpu().numpy()
                     if r is not None:
                         got = got[:, r]
@@ -346,7 +359,7 @@ def stream_and_check_fp8(wl, dev, *, chunks, check_at=None, n_rows=None, keep_la
                     results.append((k, step, which, ma, mr))
         h.append_chunk(K8.to(dev), V.to(dev))
         hist_K.append(synth.from_e4m3(K8).cpu())
-        hist_V.append(V.cpu())
+        hist_V.append(deq_v(V).cpu())
         if keep_last is not None:
             for c in range(1, max(1, len(hist_K) - keep_last)):
                 hist_K[c] = None

@@ -620,6 +620,78 @@ def test_fp8_qk_cache_bytes(dev, commit_path):
     assert h8.status() == 0
 
 
+@pytest.mark.parametrize("W,sink,n_cond", [(2, True, 40), (1, False, 130), (0, True, 0)])
+def test_fp8_pv_ragged(dev, W, sink, n_cond):
+    """e4m3 Q, K and V (P V on kind::f8f6f4 with e4m3 P, e4m3 K and V caches): every chunk and
+    step, all rows, against the oracle on the dequantised inputs at the e4m3-P tolerance."""
+    wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, pv8=True)
+    assert len(res) == wl.chunks * wl.steps
+
+
+def test_fp8_pv_joint(dev):
+    """e4m3 chunk and condition queries with e4m3 V in one joint launch."""
+    wl = dataclasses.replace(RAGGED, n_cond=130, chunks=4)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True, pv8=True)
+    assert len(res) == 2 * wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("commit_path", ["copy", "tma"])
+def test_fp8_pv_cache_bytes(dev, commit_path):
+    """With e4m3 V the V cache holds exactly the appended e4m3 values (bit for bit), and the whole
+    K/V cache takes half the bytes of the bf16 one, with either commit path."""
+    wl = dataclasses.replace(RAGGED, chunks=3)
+    sc = synth.FP8_SCALE
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    h = make_handle(wl, dev)
+    h8 = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                qk_fp8=True, q_scale=sc, k_scale=sc, pv_fp8=True, v_scale=sc,
+                                commit_path=commit_path, device=dev)
+    assert h8.commit_kind() == commit_path
+    kc, vc = h8.cache_views()
+    kb, vb = h.cache_views()
+    assert kc.numel() * kc.element_size() * 2 == kb.numel() * kb.element_size()
+    assert vc.numel() * vc.element_size() * 2 == vb.numel() * vb.element_size()
+    for c in range(wl.chunks):
+        _, K8, V8 = synth.chunk_inputs_fp8(wl, c, 1, v8=True)
+        h8.append_chunk(K8.to(dev), V8.to(dev))
+        torch.cuda.synchronize()
+        s_ = oracle.slot(c, wl.W, wl.sink)
+        assert torch.equal(kc[:, :, s_].cpu().view(torch.uint8), K8.permute(0, 2, 1, 3).contiguous().view(torch.uint8))
+        assert torch.equal(vc[:, :, s_].cpu().view(torch.uint8), V8.permute(0, 2, 1, 3).contiguous().view(torch.uint8))
+    assert h8.status() == 0
+
+
+def test_fp8_pv_720p_sampled(dev):
+    """720p with e4m3 Q, K and V: sampled rows at chunks 0, W + 1 and the last of 7."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_fp8(wl, dev, chunks=7, check_at={0, 4, 6}, n_rows=32, keep_last=wl.W + 1,
+                               gen_on_device=True, pv8=True)
+    assert len(res) == 6
+
+
+@pytest.mark.parametrize("pv8", [False, True])
+@pytest.mark.parametrize("n_q", [1, 128])
+def test_fp8_short_queries_720p(dev, n_q, pv8):
+    """Split-K path with e4m3 Q and K (and V, P with pv8) against the steady-state 720p cache,
+    all n_q rows at chunks 0 and 5."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_fp8(wl, dev, chunks=6, check_at={0, 5}, keep_last=wl.W + 1, gen_on_device=True,
+                               pv8=pv8, n_q=n_q)
+    assert len(res) == 2 * wl.steps
+
+
+@pytest.mark.parametrize("pv8", [False, True])
+@pytest.mark.parametrize("H", [3, 24])
+@pytest.mark.parametrize("n_q", [1, 33, 100])
+def test_fp8_short_queries_ragged(dev, H, n_q, pv8):
+    """Split-K path with e4m3 inputs on ragged shapes, every chunk and step: H = 3 leaves most
+    slices empty or one tile long, H = 24 gives slices of several tiles."""
+    wl = dataclasses.replace(RAGGED, H=H, chunks=5)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, pv8=pv8, n_q=n_q)
+    assert len(res) == wl.chunks * wl.steps
+
+
 def test_fp8_qk_720p_sampled(dev):
     """720p with e4m3 Q and K: sampled rows at chunks 0, W + 1 and the last of 7."""
     wl = WORKLOADS["720p"]
