@@ -272,25 +272,6 @@ attn_split_kernel(const __grid_constant__ AttnParams p) {
     if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
 }
 
-// A launch that may begin while the stream's previous kernel finishes (programmatic stream
-// serialization); the kernel itself waits for that kernel's completion (griddepcontrol.wait)
-// before it touches memory the previous kernel may write.
-template <typename... Params, typename... Args>
-static cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t stream, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 template <int D, bool kQK8, bool kPV8>
 static cudaError_t launch_split_d(const AttnParams& p, int splits, cudaStream_t stream) {
     using L = SplitLayout<D>;

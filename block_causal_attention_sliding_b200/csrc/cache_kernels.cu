@@ -224,6 +224,11 @@ __global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant
                                                            int box_k, int box_v, int32_t* state, TableAdvance ta,
                                                            int S) {
     const int box_bytes = box_k > box_v ? box_k : box_v;   // buffer stride (K may be e4m3)
+    // launched as a programmatic dependent: nothing the previous kernel may touch (the caller's
+    // K/V, the ring, the counter, the table) is read or written before it has completed; the
+    // next kernel may be scheduled at once, it waits for this grid's completion itself
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kCommitBufs];
@@ -336,8 +341,8 @@ cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d
     const int smem = kCommitBufs * (box_k > box_v ? box_k : box_v) + 1024;
     cudaError_t e = cudaFuncSetAttribute(commit_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    commit_tma_kernel<<<ctas, 32, smem, stream>>>(maps, it, box_k, box_v, state, ta, S);
-    return cudaGetLastError();
+    return launch_dependent(commit_tma_kernel, dim3(ctas), dim3(32), (size_t)smem, stream, maps, it, box_k, box_v,
+                            state, ta, S);
 }
 
 }  // namespace swattn

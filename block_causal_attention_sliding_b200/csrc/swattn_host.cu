@@ -38,6 +38,16 @@ struct sw_attn {
     CUtensorMap tm_cache_k, tm_cache_v, tm_cond_k, tm_cond_v;
     CUtensorMap tm_commit_k, tm_commit_v;   // the ring with the TMA commit's box
     bool commit_tma = false;                // chunk commits by TMA bulk copies (else the copy kernel)
+    // tensor maps over the caller's last Q, Q_cond, K_cur and V_cur: a map depends only on the
+    // pointer and the row count (B, H, d and the element size are the handle's), so it is encoded
+    // again only when one of them changes
+    struct MapMemo {
+        const void* ptr = nullptr;
+        int rows = -1;
+        CUtensorMap map;
+    };
+    MapMemo memo_q, memo_qc, memo_kcur, memo_vcur;
+    MapMemo memo_commit_k, memo_commit_v;   // the same for a TMA commit's source K and V
 };
 
 namespace {
@@ -99,6 +109,18 @@ int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, con
     const uint64_t strides[3] = {(uint64_t)d * esz, (uint64_t)H * d * esz, (uint64_t)N * H * d * esz};
     const uint32_t box[4] = {(uint32_t)(128 / esz), 1, (uint32_t)kBlockN, 1};
     return encode(m, ptr, 4, dims, strides, box, what, esz);
+}
+
+// encode_user through a one-entry memo keyed by (pointer, rows).
+int encode_user_memo(sw_attn::MapMemo& m, const void* ptr, int B, int N, int H, int d, const char* what, int esz) {
+    if (m.ptr == ptr && m.rows == N) return SW_OK;
+    m.ptr = nullptr;
+    m.rows = -1;
+    const int rc = encode_user(&m.map, ptr, B, N, H, d, what, esz);
+    if (rc) return rc;
+    m.ptr = ptr;
+    m.rows = N;
+    return SW_OK;
 }
 
 // The caller's [B, T, H, d] K or V for a TMA chunk commit: dims ordered {d, t, h, b} (strides
@@ -327,8 +349,19 @@ static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_
     if (h->commit_tma) {
         CommitMaps m;
         int rc;
-        if ((rc = encode_commit_src(&m.src_k, K, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek))) return rc;
-        if ((rc = encode_commit_src(&m.src_v, V, c.B, c.tokens_per_chunk, c.H, c.d, "V", ev))) return rc;
+        for (int kv = 0; kv < 2; ++kv) {
+            sw_attn::MapMemo& mm = kv ? h->memo_commit_v : h->memo_commit_k;
+            const void* src = kv ? V : K;
+            if (mm.ptr != src) {
+                mm.ptr = nullptr;
+                if ((rc = encode_commit_src(&mm.map, src, c.B, c.tokens_per_chunk, c.H, c.d, kv ? "V" : "K",
+                                            kv ? ev : ek)))
+                    return rc;
+                mm.ptr = src;
+            }
+        }
+        m.src_k = h->memo_commit_k.map;
+        m.src_v = h->memo_commit_v.map;
         m.dst_k = h->tm_commit_k;
         m.dst_v = h->tm_commit_v;
         e = launch_commit_tma(m, c.B, c.tokens_per_chunk, c.H, c.d, ek, ev, state, table_advance(h), h->S, h->num_sms,
@@ -383,15 +416,19 @@ int sw_attn_commit_kind(const sw_attn_t* h) {
 }
 
 // Tensor maps, pointers and scalars every forward shares (the chunk's own n_q queries).
-static int fill_params(const sw_attn_t* h, AttnParams& p, const void* Q, const void* K_cur, const void* V_cur,
+static int fill_params(sw_attn_t* h, AttnParams& p, const void* Q, const void* K_cur, const void* V_cur,
                        void* out, int n_q) {
     const sw_attn_config& c = h->cfg;
     std::memset(&p, 0, sizeof p);
     int rc;
     const int eqk = c.qk_fp8 ? 1 : 2;
-    if ((rc = encode_user(&p.tm_q, Q, c.B, n_q, c.H, c.d, "Q", eqk))) return rc;
-    if ((rc = encode_user(&p.tm_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur", eqk))) return rc;
-    if ((rc = encode_user(&p.tm_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur", c.pv_fp8 ? 1 : 2))) return rc;
+    if ((rc = encode_user_memo(h->memo_q, Q, c.B, n_q, c.H, c.d, "Q", eqk))) return rc;
+    if ((rc = encode_user_memo(h->memo_kcur, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur", eqk))) return rc;
+    if ((rc = encode_user_memo(h->memo_vcur, V_cur, c.B, c.tokens_per_chunk, c.H, c.d, "V_cur", c.pv_fp8 ? 1 : 2)))
+        return rc;
+    p.tm_q = h->memo_q.map;
+    p.tm_kcur = h->memo_kcur.map;
+    p.tm_vcur = h->memo_vcur.map;
     // maps for regions this handle does not have are never read; fill them with a valid map
     p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
     p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
@@ -577,7 +614,8 @@ int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const
     AttnParams p;
     int rc;
     if ((rc = fill_params(h, p, Q, K_cur, V_cur, out, c.tokens_per_chunk))) return rc;
-    if ((rc = encode_user(&p.tm_qc, Q_cond, c.B, c.n_cond, c.H, c.d, "Q_cond", c.qk_fp8 ? 1 : 2))) return rc;
+    if ((rc = encode_user_memo(h->memo_qc, Q_cond, c.B, c.n_cond, c.H, c.d, "Q_cond", c.qk_fp8 ? 1 : 2))) return rc;
+    p.tm_qc = h->memo_qc.map;
     p.out_c = out_cond;
     p.n_qc = c.n_cond;
     return launch_full(h, p, static_cast<cudaStream_t>(stream));

@@ -119,4 +119,23 @@ cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStre
 cudaError_t launch_combine(const float* o_part, const float* ml_part, void* out, int B, int H,
                            int n_q, int d, int splits, int out_f32, float out_scale, cudaStream_t stream);
 
+// A launch that may begin while the stream's previous kernel finishes (programmatic stream
+// serialization).  Only kernels that call griddepcontrol.wait before they touch memory the
+// previous kernel may write are launched this way.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace swattn

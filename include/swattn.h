@@ -29,7 +29,9 @@
  *     then returns a message (thread-local, valid until the next call on that thread).
  *   - Problems found on the device (a wait that ran out, an impossible slot) set bits in a
  *     status word on the device; kernels never trap.  Read it with sw_attn_get_status.
- *   - One handle holds one layer's cache.  Calls on one handle must be ordered on one stream.
+ *   - One handle holds one layer's cache.  Calls on one handle must be ordered on one stream
+ *     and made from one host thread at a time (the handle keeps host-side state: the tensor
+ *     maps of the last inputs, reused while their pointers and row counts repeat).
  */
 #ifndef SWATTN_H
 #define SWATTN_H
