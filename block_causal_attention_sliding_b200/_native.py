@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswattn.s
 SW_OK, SW_EINVAL, SW_ESHAPE, SW_EALIGN, SW_ESTATE, SW_ECUDA = 0, -1, -2, -3, -4, -5
 SW_STATUS_TIMEOUT, SW_STATUS_BAD_SLOT, SW_STATUS_OVERFLOW = 0x1, 0x2, 0x4
 SW_OUT_BF16, SW_OUT_F32 = 0, 1
-SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO = 0, 1, 2, 3
+SW_SCHED_PERSISTENT, SW_SCHED_GRID, SW_SCHED_TRI, SW_SCHED_AUTO, SW_SCHED_PAIR = 0, 1, 2, 3, 4
 SW_COMMIT_AUTO, SW_COMMIT_COPY, SW_COMMIT_TMA = 0, 1, 2
 
 # every symbol include/swattn.h declares

@@ -42,7 +42,8 @@ class SlidingWindowAttention:
                              out_dtype=N.SW_OUT_F32 if out_dtype == torch.float32 else N.SW_OUT_BF16,
                              scale=0.0 if scale is None else float(scale), max_short_q=max_short_q,
                              schedule={"persistent": N.SW_SCHED_PERSISTENT, "grid": N.SW_SCHED_GRID,
-                                       "tri": N.SW_SCHED_TRI, "auto": N.SW_SCHED_AUTO}[schedule],
+                                       "tri": N.SW_SCHED_TRI, "pair": N.SW_SCHED_PAIR,
+                                       "auto": N.SW_SCHED_AUTO}[schedule],
                              commit_in_forward=int(bool(commit_in_forward)), qk_fp8=int(bool(qk_fp8)),
                              q_scale=float(q_scale), k_scale=float(k_scale),
                              commit_path={"auto": N.SW_COMMIT_AUTO, "copy": N.SW_COMMIT_COPY,
@@ -82,7 +83,8 @@ class SlidingWindowAttention:
         r = int(self._lib.sw_attn_schedule_for(self._h, self.T if n_q is None else n_q))
         if r < 0:
             N.check(r)
-        return {N.SW_SCHED_PERSISTENT: "persistent", N.SW_SCHED_GRID: "grid", N.SW_SCHED_TRI: "tri"}[r]
+        return {N.SW_SCHED_PERSISTENT: "persistent", N.SW_SCHED_GRID: "grid", N.SW_SCHED_TRI: "tri",
+                N.SW_SCHED_PAIR: "pair"}[r]
 
     # -- stream control
     def set_cond(self, K_cond: torch.Tensor, V_cond: torch.Tensor, stream=None) -> None:

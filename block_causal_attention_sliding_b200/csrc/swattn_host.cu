@@ -36,6 +36,9 @@ struct sw_attn {
     int num_sms = 148;
     bool cond_set = false;
     CUtensorMap tm_cache_k, tm_cache_v, tm_cond_k, tm_cond_v;
+    CUtensorMap tm_cache_kh, tm_cond_kh;    // the K maps with 64-row boxes (CTA-pair kernel)
+    bool pair_ok = false;                   // bf16, d = 128: the CTA-pair kernel can run
+    int pair_clusters = -1;                 // CTA pairs that fit at once (-1: not yet queried)
     CUtensorMap tm_commit_k, tm_commit_v;   // the ring with the TMA commit's box
     bool commit_tma = false;                // chunk commits by TMA bulk copies (else the copy kernel)
     // tensor maps over the caller's last Q, Q_cond, K_cur and V_cur: a map depends only on the
@@ -48,6 +51,7 @@ struct sw_attn {
     };
     MapMemo memo_q, memo_qc, memo_kcur, memo_vcur;
     MapMemo memo_commit_k, memo_commit_v;   // the same for a TMA commit's source K and V
+    MapMemo memo_kcur_h;                    // K_cur with 64-row boxes (CTA-pair kernel)
 };
 
 namespace {
@@ -103,20 +107,23 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, cons
     return SW_OK;
 }
 
-// user layout [B, N, H, d]: dims {d, H, N, B}; box (128 bytes) x 1 x 128 x 1 (128 rows of one head)
-int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, const char* what, int esz = 2) {
+// user layout [B, N, H, d]: dims {d, H, N, B}; box (128 bytes) x 1 x rows x 1 (rows of one head;
+// 128 by default, 64 for the CTA-pair kernel's K halves)
+int encode_user(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, const char* what, int esz = 2,
+                int rows = kBlockN) {
     const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)N, (uint64_t)B};
     const uint64_t strides[3] = {(uint64_t)d * esz, (uint64_t)H * d * esz, (uint64_t)N * H * d * esz};
-    const uint32_t box[4] = {(uint32_t)(128 / esz), 1, (uint32_t)kBlockN, 1};
+    const uint32_t box[4] = {(uint32_t)(128 / esz), 1, (uint32_t)rows, 1};
     return encode(m, ptr, 4, dims, strides, box, what, esz);
 }
 
 // encode_user through a one-entry memo keyed by (pointer, rows).
-int encode_user_memo(sw_attn::MapMemo& m, const void* ptr, int B, int N, int H, int d, const char* what, int esz) {
+int encode_user_memo(sw_attn::MapMemo& m, const void* ptr, int B, int N, int H, int d, const char* what, int esz,
+                     int box_rows = kBlockN) {
     if (m.ptr == ptr && m.rows == N) return SW_OK;
     m.ptr = nullptr;
     m.rows = -1;
-    const int rc = encode_user(&m.map, ptr, B, N, H, d, what, esz);
+    const int rc = encode_user(&m.map, ptr, B, N, H, d, what, esz, box_rows);
     if (rc) return rc;
     m.ptr = ptr;
     m.rows = N;
@@ -143,7 +150,10 @@ int check_cfg(const sw_attn_config& c) {
     if (c.out_dtype != SW_OUT_BF16 && c.out_dtype != SW_OUT_F32) return fail(SW_EINVAL, "bad out_dtype");
     if (c.max_short_q > kMaxShortQ) return fail(SW_ESHAPE, "max_short_q must be <= %d", kMaxShortQ);
     if (!std::isfinite(c.scale)) return fail(SW_EINVAL, "scale must be finite");
+    if (c.schedule == SW_SCHED_PAIR && (c.d != 128 || c.qk_fp8))
+        return fail(SW_ESHAPE, "the CTA-pair schedule needs d = 128 and bf16 Q/K/V");
     if (c.schedule != SW_SCHED_PERSISTENT && c.schedule != SW_SCHED_GRID && c.schedule != SW_SCHED_TRI &&
+        c.schedule != SW_SCHED_PAIR &&
         c.schedule != SW_SCHED_AUTO)
         return fail(SW_EINVAL, "bad schedule");
     if (c.commit_in_forward != 0 && c.commit_in_forward != 1) return fail(SW_EINVAL, "commit_in_forward must be 0 or 1");
@@ -241,6 +251,9 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    // the CTA-pair kernel: bf16 with d = 128, and only where pairs of its CTAs fit the device
+    h->pair_ok = h->cfg.d == 128 && !h->cfg.qk_fp8 && !h->cfg.pv_fp8;
+    h->pair_clusters = h->pair_ok ? pair_max_clusters() : 0;
     const sw_attn_config& c = h->cfg;
     char* ws = static_cast<char*>(dev_ptr);
     int rc;
@@ -260,6 +273,10 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
                                       rowv * c.tokens_per_chunk * h->S * c.H};
         const uint32_t boxv[5] = {(uint32_t)(128 / ev), (uint32_t)kBlockN, 1, 1, 1};
         if ((rc = encode(&h->tm_cache_k, ws + h->off_kcache, 5, dims, stridesk, boxk, "K cache", ek))) return rc;
+        if (h->pair_ok) {
+            const uint32_t boxkh[5] = {64u, (uint32_t)(kBlockN / 2), 1, 1, 1};
+            if ((rc = encode(&h->tm_cache_kh, ws + h->off_kcache, 5, dims, stridesk, boxkh, "K cache", ek))) return rc;
+        }
         if ((rc = encode(&h->tm_cache_v, ws + h->off_vcache, 5, dims, stridesv, boxv, "V cache", ev))) return rc;
         // chunk commits by TMA: the ring with a box of d x kCommitRows rows x up to kCommitHeads
         // heads (unswizzled), and a trial map of the caller side (permuted strides); where the
@@ -291,6 +308,10 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
         const uint64_t stridesv[3] = {rowv, rowv * c.n_cond, rowv * c.n_cond * c.H};
         const uint32_t boxv[4] = {(uint32_t)(128 / ev), (uint32_t)kBlockN, 1, 1};
         if ((rc = encode(&h->tm_cond_k, ws + h->off_kcond, 4, dims, stridesk, boxk, "K cond", ek))) return rc;
+        if (h->pair_ok) {
+            const uint32_t boxkh[4] = {64u, (uint32_t)(kBlockN / 2), 1, 1};
+            if ((rc = encode(&h->tm_cond_kh, ws + h->off_kcond, 4, dims, stridesk, boxkh, "K cond", ek))) return rc;
+        }
         if ((rc = encode(&h->tm_cond_v, ws + h->off_vcond, 4, dims, stridesv, boxv, "V cond", ev))) return rc;
     }
     e = launch_state_reset(reinterpret_cast<int32_t*>(ws), c.W, h->R, c.sink, c.n_cond, c.tokens_per_chunk,
@@ -393,6 +414,7 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
 static int resolve_schedule_tiles(const sw_attn_t* h, long long nqt) {
     const sw_attn_config& c = h->cfg;
     if (c.qk_fp8) return SW_SCHED_PERSISTENT;   // the one kernel with an e4m3 Q/K form
+    if (c.schedule == SW_SCHED_PAIR) return h->pair_clusters > 0 ? SW_SCHED_PAIR : SW_SCHED_TRI;
     if (c.schedule != SW_SCHED_AUTO) return c.schedule;
     const long long pairs = (long long)c.B * c.H * ((nqt + 1) / 2);
     return pairs < h->num_sms ? SW_SCHED_TRI : SW_SCHED_PERSISTENT;
@@ -433,6 +455,15 @@ static int fill_params(sw_attn_t* h, AttnParams& p, const void* Q, const void* K
     p.tm_cache_k = h->S > 0 ? h->tm_cache_k : p.tm_kcur;
     p.tm_cache_v = h->S > 0 ? h->tm_cache_v : p.tm_vcur;
     p.tm_cond_k = c.n_cond > 0 ? h->tm_cond_k : p.tm_kcur;
+    if (h->pair_ok) {
+        if ((rc = encode_user_memo(h->memo_kcur_h, K_cur, c.B, c.tokens_per_chunk, c.H, c.d, "K_cur", 2, kBlockN / 2)))
+            return rc;
+        p.tm_kcur_h = h->memo_kcur_h.map;
+        p.tm_cache_kh = h->S > 0 ? h->tm_cache_kh : p.tm_kcur_h;
+        p.tm_cond_kh = c.n_cond > 0 ? h->tm_cond_kh : p.tm_kcur_h;
+    } else {
+        p.tm_kcur_h = p.tm_cache_kh = p.tm_cond_kh = p.tm_kcur;   // never read
+    }
     p.tm_cond_v = c.n_cond > 0 ? h->tm_cond_v : p.tm_vcur;
     p.tm_qc = p.tm_q;   // no condition queries unless a joint forward sets them
     int32_t* state = reinterpret_cast<int32_t*>(h->ws);
@@ -482,6 +513,14 @@ static int launch_full(sw_attn_t* h, AttnParams& p, cudaStream_t st) {
     if (sched == SW_SCHED_TRI) {
         e = launch_tri(p, c.d, (int)ctas, st);
         if (e != cudaSuccess) return cuda_fail(e, "three-buffer attention launch");
+        return SW_OK;
+    }
+    if (sched == SW_SCHED_PAIR) {
+        // one CTA pair per two SMs, with the same floor of two items per pair
+        long long pairs = std::min<long long>(h->pair_clusters, kMaxPersistentCtas / 2);
+        pairs = std::max<long long>(1, std::min<long long>(pairs, c_min / 4));
+        e = launch_pair(p, (int)pairs, st);
+        if (e != cudaSuccess) return cuda_fail(e, "CTA-pair attention launch");
         return SW_OK;
     }
     e = launch_persistent(p, c.d, (int)ctas, st);
@@ -586,8 +625,9 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const long long nqt = (c.tokens_per_chunk + kBlockM - 1) / kBlockM;
     int32_t* state = reinterpret_cast<int32_t*>(h->ws);
-    if (resolve_schedule_tiles(h, nqt) == SW_SCHED_TRI) {
-        // the three-buffer kernel does not store K/V: forward, then the copy into the same slot
+    const int sched = resolve_schedule_tiles(h, nqt);
+    if (sched == SW_SCHED_TRI || sched == SW_SCHED_PAIR) {
+        // the three-buffer kernels do not store K/V: forward, then the copy into the same slot
         if ((rc = launch_full(h, p, st))) return rc;
         if (h->S > 0) return launch_commit(h, K_cur, V_cur, st);   // the copy launch also advances the table
     } else {

@@ -57,6 +57,8 @@ struct alignas(64) AttnParams {
     CUtensorMap tm_cond_k;   // K cond  [B][H][n_cond][d] dims {d, n_cond, H, B}
     CUtensorMap tm_cond_v;
     CUtensorMap tm_qc;       // condition-stream queries [B, n_qc, H, d] (joint forward)
+    // the same K maps with boxes of 64 rows (half a key tile), for the CTA-pair kernel
+    CUtensorMap tm_kcur_h, tm_cache_kh, tm_cond_kh;
     void* out;               // [B, n_q, H, d] bf16 or f32 (full mode)
     void* out_c;             // [B, n_qc, H, d] (joint forward)
     float* o_part;           // split mode: [splits][B*H][kBlockM][d] unnormalised fp32
@@ -82,6 +84,10 @@ struct alignas(64) AttnParams {
 };
 
 // kernel launchers (defined in the .cu files)
+// CTA-pair three-buffer kernel (d = 128, bf16): `clusters` pairs of CTAs.
+cudaError_t launch_pair(const AttnParams& p, int clusters, cudaStream_t stream);
+// Pairs of CTAs of that kernel that fit on the device at once (0 if none or on error).
+int pair_max_clusters();
 cudaError_t launch_table_build(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
                                cudaStream_t stream);
 cudaError_t launch_state_reset(int32_t* state, int W, int R, int sink, int n_cond, int T,

@@ -81,7 +81,7 @@ typedef struct {
     int   max_short_q;       /* n_q <= this uses the split-K path; 0 selects 128, max 128,
                                 negative disables the split-K path */
     int   schedule;          /* full path: SW_SCHED_AUTO (default), SW_SCHED_PERSISTENT,
-                                SW_SCHED_GRID or SW_SCHED_TRI */
+                                SW_SCHED_GRID, SW_SCHED_TRI or SW_SCHED_PAIR */
     int   commit_in_forward; /* 1: keep one spare window slot (W + 1 in all) so that
                                 sw_attn_forward_commit can write the chunk's K/V into the cache
                                 while its own forward runs; 0 (default): W window slots */
@@ -115,6 +115,11 @@ typedef struct {
 #define SW_SCHED_AUTO       3   /* per launch: SW_SCHED_TRI when the pairs of 128-row Q tiles
                                    (B * H * ceil(n_q / 256)) are fewer than the SMs, else
                                    SW_SCHED_PERSISTENT (see sw_attn_schedule_for) */
+#define SW_SCHED_PAIR       4   /* clusters of two CTAs on two SMs, one 256-row tcgen05 MMA
+                                   (cta_group::2) per key tile over two Q tiles, three S
+                                   accumulators per SM; d = 128 and bf16 only (SW_ESHAPE
+                                   otherwise at create); SW_SCHED_TRI where the device cannot
+                                   hold a pair of its CTAs */
 
 /*
  * Create a handle with B = 1, sink on, bf16 output, scale 1/sqrt(d).  Host only: allocates

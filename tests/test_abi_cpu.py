@@ -88,6 +88,7 @@ def test_workspace_constant_in_stream_length(native):
     (dict(tokens_per_chunk=0), -2), (dict(W=-1), -2), (dict(W=65), -2), (dict(n_cond=-3), -2),
     (dict(sink=2), -1), (dict(out_dtype=7), -1), (dict(max_short_q=129), -2),
     (dict(scale=float("inf")), -1), (dict(schedule=5), -1),
+    (dict(schedule=4, d=64), -2),   # the CTA-pair schedule is d = 128 only
 ])
 def test_create_rejects_bad_config(native, kw, code):
     rc, h = _create(native, **kw)
@@ -132,6 +133,9 @@ def test_schedule_resolution(native):
         (dict(schedule=native.SW_SCHED_AUTO, H=16, tokens_per_chunk=1400), 1400, native.SW_SCHED_TRI),  # 96
         (dict(schedule=native.SW_SCHED_GRID), 3180, native.SW_SCHED_GRID),
         (dict(schedule=native.SW_SCHED_TRI), 3180, native.SW_SCHED_TRI),
+        # the CTA-pair kernel needs a device that holds a pair of its CTAs: before a workspace is
+        # bound (no device known) it resolves to the three-buffer kernel
+        (dict(schedule=native.SW_SCHED_PAIR), 3180, native.SW_SCHED_TRI),
     ]
     for kw, n_q, want in cases:
         rc, h = _create(native, **kw)

@@ -158,24 +158,26 @@ def test_tiny_full_stream(dev, out_dtype, max_short_q):
     assert len(res) == wl.chunks * wl.steps
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri", "pair"])
 @pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("max_short_q", [-1, 0])
 def test_ragged_multi_tile(dev, d, max_short_q, schedule):
     """T = 300 gives one full pair and one single-tile pair per head; with the persistent
     schedule the few items per CTA force many-way splits of every pair's key tiles."""
+    if schedule == "pair" and d != 128:
+        pytest.skip("the CTA-pair schedule is d = 128 only (refused at create otherwise)")
     wl = dataclasses.replace(RAGGED, d=d)
     stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=max_short_q, schedule=schedule)
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri", "pair"])
 @pytest.mark.parametrize("W,sink,n_cond", [(0, False, 40), (0, True, 0), (4, False, 7), (1, True, 130)])
 def test_ragged_other_windows(dev, W, sink, n_cond, schedule):
     wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
     stream_and_check(wl, dev, chunks=wl.chunks, max_short_q=-1, schedule=schedule)
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "tri", "pair"])
 @pytest.mark.parametrize("H,T", [(1, 300), (1, 129), (5, 640), (2, 1400), (7, 3180)])
 def test_persistent_split_shapes(dev, H, T, schedule):
     """Shapes whose cost line cuts units into 2, 3 or more pieces (one head: a handful of CTAs
@@ -185,7 +187,7 @@ def test_persistent_split_shapes(dev, H, T, schedule):
                      check_at=None if T < 3000 else {0, 3}, n_rows=None if T < 3000 else 48)
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "tri", "pair"])
 def test_persistent_repeatable(dev, schedule):
     """The merge counters return to zero after every launch, and split pieces are merged in a
     fixed order whichever arrives last: repeated forwards give bit-identical output."""
@@ -286,6 +288,30 @@ def test_720p_sampled_tri(dev):
     assert len(res) == 6
 
 
+def test_720p_sampled_pair(dev):
+    """The 720p workload on the CTA-pair kernel: chunks 0, W+1 and the last of 12, rows in every
+    32-row quarter of every tile (25 Q tiles per head: the last pair has one tile)."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check(wl, dev, chunks=12, check_at={0, 4, 11}, n_rows=104, keep_last=wl.W + 1,
+                           gen_on_device=True, schedule="pair")
+    assert len(res) == 6
+
+
+def test_480p_sampled_pair(dev):
+    wl = WORKLOADS["480p"]
+    res = stream_and_check(wl, dev, chunks=6, check_at={0, 1, 3, 5}, n_rows=64, keep_last=wl.W + 1,
+                           gen_on_device=True, schedule="pair")
+    assert len(res) == 8
+
+
+def test_stress_sampled_pair(dev):
+    """Four streams, 32 heads, W = 6, sigma-4 key outliers (O rescales) on the CTA-pair kernel."""
+    wl = WORKLOADS["stress"]
+    res = stream_and_check(wl, dev, chunks=8, check_at={0, 7}, n_rows=0, keep_last=wl.W + 1,
+                           gen_on_device=True, schedule="pair")
+    assert len(res) == 4
+
+
 def test_stress_sampled_tri(dev):
     wl = WORKLOADS["stress"]
     res = stream_and_check(wl, dev, chunks=8, check_at={7}, n_rows=0, keep_last=wl.W + 1,
@@ -356,12 +382,14 @@ def test_joint_tiny_stream(dev, schedule):
     assert len(res) == 2 * wl.chunks * wl.steps
 
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri", "pair"])
 @pytest.mark.parametrize("d,T,n_cond", [(128, 300, 40), (128, 256, 130), (64, 300, 200), (128, 129, 1)])
 def test_joint_ragged(dev, d, T, n_cond, schedule):
     """Ragged tails in both query sets: the chunk's last Q tile and a condition tile share a
     pair (T = 300, n_cond = 40: 3 + 1 tiles), two condition tiles form a pair (n_cond = 130),
     an odd tile total (T = 300, n_cond = 200 at d = 64: 3 + 2 tiles), one condition query."""
+    if schedule == "pair" and d != 128:
+        pytest.skip("the CTA-pair schedule is d = 128 only (refused at create otherwise)")
     wl = dataclasses.replace(RAGGED, d=d, T=T, n_cond=n_cond, chunks=4)
     res = stream_and_check_joint(wl, dev, chunks=wl.chunks, schedule=schedule)
     assert len(res) == 2 * wl.chunks * wl.steps
@@ -388,7 +416,7 @@ def test_joint_720p_sampled(dev):
 
 # ------------------------------------------------------------------ fused clean-KV commit
 
-@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri"])
+@pytest.mark.parametrize("schedule", ["persistent", "grid", "tri", "pair"])
 @pytest.mark.parametrize("W,sink", [(2, True), (1, False), (3, True), (0, True)])
 def test_commit_in_forward_stream(dev, W, sink, schedule):
     """The clean pass commits its own K/V: tables and cache contents bit-exact against the
