@@ -426,7 +426,7 @@ def run_cuda(args, wl, world, rank, local):
             h = None
             paths["long_horizon"] = long_horizon(args, dev, stream, pool)
             paths["commit"] = commit_path(args, dev, stream, pool)
-            paths["layers"] = layers_path(args, dev, stream)
+            paths["layers"] = layers_path(args, dev, stream, peaks=peaks)
             paths["fp8"] = fp8_path(args, dev, stream, peaks)
             paths["workloads"] = other_workloads(args, dev, stream, peaks)
 
@@ -693,10 +693,11 @@ def fp8_path(args, dev, stream, peaks):
     return res
 
 
-def layers_path(args, dev, stream, n_layers=8):
+def layers_path(args, dev, stream, n_layers=8, peaks=None):
     """A chunk step of an n-layer model at 480p: each layer (one handle, its own cache) runs its
     two forwards, then every layer commits the chunk.  Timed with per-layer appends, with one
-    batched append for all layers, and with the whole step replayed from a CUDA graph."""
+    batched append for all layers, and with the whole step replayed from a CUDA graph; and the
+    batched commit alone (HBM-bound: every layer's K/V read once and written once)."""
     from block_causal_attention_sliding_b200.api import SlidingWindowAttention, append_chunk_batched
     wl = WORKLOADS["480p"]
     hs, ins, outs = [], [], []
@@ -741,6 +742,17 @@ def layers_path(args, dev, stream, n_layers=8):
 
     t_each = timed(step_each)
     t_batched = timed(step_batched)
+    # the batched commit alone, alternating each layer's two (K, V) sets: 2 x 8 x 11.5 MB of
+    # sources, more than L2 holds, so the copies read from HBM
+    flip = [0]
+
+    def commit_only():
+        s = flip[0] % wl.steps
+        flip[0] += 1
+        append_chunk_batched(hs, [x[s][1] for x in ins], [x[s][2] for x in ins])
+
+    t_commit = timed(commit_only)
+    commit_bytes = 2 * 2 * n_layers * ins[0][0][1].numel() * ins[0][0][1].element_size()
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream())
@@ -753,9 +765,12 @@ def layers_path(args, dev, stream, n_layers=8):
     del graph
     for h in hs:
         h.close()
+    commit = {"us": round(t_commit * 1e3, 2), "GB/s": round(commit_bytes / t_commit / 1e6, 1), "bytes": commit_bytes}
+    if peaks:
+        commit["frac_hbm"] = round(commit_bytes / t_commit / 1e6 / peaks["hbm_gbs"], 3)
     return {"workload": wl.name, "layers": n_layers, "ms_per_chunk_appends_each": round(t_each, 4),
             "ms_per_chunk_batched_append": round(t_batched, 4), "ms_per_chunk_graph": round(t_graph, 4),
-            "status": status}
+            "batched_commit_alone": commit, "status": status}
 
 
 def other_workloads(args, dev, stream, peaks):

@@ -149,11 +149,13 @@ __device__ __forceinline__ void relayout_rows(const uint4* __restrict__ srcK, co
 // complete before the barrier below (its value decided the thread's stores, or its return), so
 // every block has read the counter before it is counted; state[2] counts the finished blocks and
 // is back at zero when the launch ends.
-__device__ __forceinline__ void advance_after_commit(int32_t* state, const TableAdvance& ta) {
+// blocks: the blocks of this handle's grid (all of the launch unless a batch gives each handle
+// a part of it).
+__device__ __forceinline__ void advance_after_commit(int32_t* state, const TableAdvance& ta, unsigned blocks = 0) {
     __syncthreads();
     if (threadIdx.x != 0) return;
     __threadfence();
-    const unsigned total = gridDim.x * gridDim.y;
+    const unsigned total = blocks ? blocks : gridDim.x * gridDim.y;
     const unsigned done = atomicAdd(reinterpret_cast<unsigned*>(state + 2), 1u) + 1u;
     if (done == total) {
         __threadfence();
@@ -220,23 +222,18 @@ struct CommitItems {
     }
 };
 
-__global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant__ CommitMaps m, CommitItems it,
-                                                           int box_k, int box_v, int32_t* state, TableAdvance ta,
-                                                           int S) {
+// One handle's commit: part `part` of `parts` of its items, by thread 0 of the block.
+__device__ __forceinline__ void commit_tma_part(const CommitMaps& m, const CommitItems& it, int box_k, int box_v,
+                                                int32_t* state, const TableAdvance& ta, int S, int part, int parts) {
     const int box_bytes = box_k > box_v ? box_k : box_v;   // buffer stride (K may be e4m3)
-    // launched as a programmatic dependent: nothing the previous kernel may touch (the caller's
-    // K/V, the ring, the counter, the table) is read or written before it has completed; the
-    // next kernel may be scheduled at once, it waits for this grid's completion itself
-    grid_dependency_wait();
-    grid_dependents_launch();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kCommitBufs];
     if (threadIdx.x == 0) {
         const int slot = commit_slot(state, ta.R, ta.sink, S);
         const long long total = it.total();
-        const long long i0 = slot >= 0 ? (long long)blockIdx.x * total / gridDim.x : 0;
-        const long long i1 = slot >= 0 ? (long long)(blockIdx.x + 1) * total / gridDim.x : 0;
+        const long long i0 = slot >= 0 ? (long long)part * total / parts : 0;
+        const long long i1 = slot >= 0 ? (long long)(part + 1) * total / parts : 0;
         for (int q = 0; q < kCommitBufs; ++q) mbar_init(smem_u32(&full[q]), 1);
         fence_mbar_init();
         auto load = [&](long long i) {
@@ -281,7 +278,30 @@ __global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant
         }
         bulk_wait_all();   // every store complete before the buffers go away
     }
+}
+
+__global__ void __launch_bounds__(32, 1) commit_tma_kernel(const __grid_constant__ CommitMaps m, CommitItems it,
+                                                           int box_k, int box_v, int32_t* state, TableAdvance ta,
+                                                           int S) {
+    // launched as a programmatic dependent: nothing the previous kernel may touch (the caller's
+    // K/V, the ring, the counter, the table) is read or written before it has completed; the
+    // next kernel may be scheduled at once, it waits for this grid's completion itself
+    grid_dependency_wait();
+    grid_dependents_launch();
+    commit_tma_part(m, it, box_k, box_v, state, ta, S, blockIdx.x, gridDim.x);
     advance_after_commit(state, ta);
+}
+
+// The chunk commit of several handles (layers) in one launch: blockIdx.y selects the handle,
+// whose gridDim.x blocks split its items; each handle's last block advances its own counter and
+// table, exactly as commit_tma_kernel does for one handle.
+__global__ void __launch_bounds__(32, 1) commit_tma_batch_kernel(const __grid_constant__ CommitBatch cb,
+                                                                 CommitItems it, int box_k, int box_v) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int l = blockIdx.y;
+    commit_tma_part(cb.maps[l], it, box_k, box_v, cb.state[l], cb.ta[l], cb.S[l], blockIdx.x, gridDim.x);
+    advance_after_commit(cb.state[l], cb.ta[l], gridDim.x);
 }
 
 // 16-byte vectors per head row of d elements of esz bytes, as a power of two (-1: not one).
@@ -324,6 +344,26 @@ cudaError_t launch_relayout(const void* K, const void* V, void* dstK, void* dstV
         static_cast<const uint4*>(K), static_cast<const uint4*>(V), static_cast<uint4*>(dstK),
         static_cast<uint4*>(dstV), N, rows, H, vpr_log2_k, vpr_log2, rows_per_bh, ring, S, state, ta, advance);
     return cudaGetLastError();
+}
+
+cudaError_t launch_commit_tma_batch(const CommitBatch& cb, int B, int T, int H, int d, int k_esz, int v_esz,
+                                    int ctas_per_handle, cudaStream_t stream) {
+    if (cb.n < 1 || cb.n > kCommitBatch || B < 1 || T < 1 || H < 1 || ctas_per_handle < 1 || (d * k_esz) % 16 != 0 ||
+        (d * v_esz) % 16 != 0 || d * 2 > 256)
+        return cudaErrorInvalidValue;
+    CommitItems it;
+    it.B = B;
+    it.T = T;
+    it.H = H;
+    it.nt = (T + kCommitRows - 1) / kCommitRows;
+    it.nh = (H + kCommitHeads - 1) / kCommitHeads;
+    const int h_box = H < kCommitHeads ? H : kCommitHeads;
+    const int box_k = d * k_esz * kCommitRows * h_box, box_v = d * v_esz * kCommitRows * h_box;
+    const int smem = kCommitBufs * (box_k > box_v ? box_k : box_v) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(commit_tma_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    return launch_dependent(commit_tma_batch_kernel, dim3(ctas_per_handle, cb.n), dim3(32), (size_t)smem, stream, cb,
+                            it, box_k, box_v);
 }
 
 cudaError_t launch_commit_tma(const CommitMaps& maps, int B, int T, int H, int d, int k_esz, int v_esz,

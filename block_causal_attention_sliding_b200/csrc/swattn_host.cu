@@ -41,6 +41,7 @@ struct sw_attn {
     int pair_clusters = -1;                 // CTA pairs that fit at once (-1: not yet queried)
     CUtensorMap tm_commit_k, tm_commit_v;   // the ring with the TMA commit's box
     bool commit_tma = false;                // chunk commits by TMA bulk copies (else the copy kernel)
+    bool commit_maps_ok = false;            // the commit's ring maps exist (a batch may use them)
     // tensor maps over the caller's last Q, Q_cond, K_cur and V_cur: a map depends only on the
     // pointer and the row count (B, H, d and the element size are the handle's), so it is encoded
     // again only when one of them changes
@@ -289,12 +290,15 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
                                 ((c.H + kCommitHeads - 1) / kCommitHeads);
         const bool want = c.commit_path == SW_COMMIT_TMA ||
                           (c.commit_path == SW_COMMIT_AUTO && items >= (long long)kCommitBufs * sms);
-        h->commit_tma = want &&
+        // the maps are made whenever TMA commits are allowed: a batched commit of several handles
+        // may have enough items together where one handle alone has not
+        h->commit_maps_ok = c.commit_path != SW_COMMIT_COPY &&
             encode(&h->tm_commit_k, ws + h->off_kcache, 5, dims, stridesk, cbox, "K cache", ek,
                    CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
             encode(&h->tm_commit_v, ws + h->off_vcache, 5, dims, stridesv, cbox, "V cache", ev,
                    CU_TENSOR_MAP_SWIZZLE_NONE) == SW_OK &&
             encode_commit_src(&trial, ws + h->off_kcache, c.B, c.tokens_per_chunk, c.H, c.d, "K", ek) == SW_OK;
+        h->commit_tma = want && h->commit_maps_ok;
         g_err.clear();
     }
     if (c.n_cond > 0) {
@@ -362,6 +366,28 @@ int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void*
 // One chunk commit of K and V ([B, T, H, d]) into the ring slot the device counter names, with
 // the counter advance and table rebuild in the same launch: TMA bulk copies (one CTA per SM),
 // or the copy kernel where the handle's maps could not be made.
+// The four maps of a TMA chunk commit of K, V into h's ring (source maps memoised by pointer).
+static int commit_maps(sw_attn_t* h, const void* K, const void* V, CommitMaps& m) {
+    const sw_attn_config& c = h->cfg;
+    const int ek = c.qk_fp8 ? 1 : 2, ev = c.pv_fp8 ? 1 : 2;
+    int rc;
+    for (int kv = 0; kv < 2; ++kv) {
+        sw_attn::MapMemo& mm = kv ? h->memo_commit_v : h->memo_commit_k;
+        const void* src = kv ? V : K;
+        if (mm.ptr != src) {
+            mm.ptr = nullptr;
+            if ((rc = encode_commit_src(&mm.map, src, c.B, c.tokens_per_chunk, c.H, c.d, kv ? "V" : "K", kv ? ev : ek)))
+                return rc;
+            mm.ptr = src;
+        }
+    }
+    m.src_k = h->memo_commit_k.map;
+    m.src_v = h->memo_commit_v.map;
+    m.dst_k = h->tm_commit_k;
+    m.dst_v = h->tm_commit_v;
+    return SW_OK;
+}
+
 static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_t st) {
     const sw_attn_config& c = h->cfg;
     const int ek = c.qk_fp8 ? 1 : 2, ev = c.pv_fp8 ? 1 : 2;
@@ -370,21 +396,7 @@ static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_
     if (h->commit_tma) {
         CommitMaps m;
         int rc;
-        for (int kv = 0; kv < 2; ++kv) {
-            sw_attn::MapMemo& mm = kv ? h->memo_commit_v : h->memo_commit_k;
-            const void* src = kv ? V : K;
-            if (mm.ptr != src) {
-                mm.ptr = nullptr;
-                if ((rc = encode_commit_src(&mm.map, src, c.B, c.tokens_per_chunk, c.H, c.d, kv ? "V" : "K",
-                                            kv ? ev : ek)))
-                    return rc;
-                mm.ptr = src;
-            }
-        }
-        m.src_k = h->memo_commit_k.map;
-        m.src_v = h->memo_commit_v.map;
-        m.dst_k = h->tm_commit_k;
-        m.dst_v = h->tm_commit_v;
+        if ((rc = commit_maps(h, K, V, m))) return rc;
         e = launch_commit_tma(m, c.B, c.tokens_per_chunk, c.H, c.d, ek, ev, state, table_advance(h), h->S, h->num_sms,
                               st);
     } else {
@@ -582,6 +594,36 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
             if (hs[m] == h) return fail(SW_EINVAL, "handle %d appears twice", l);
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // TMA bulk copies when every handle has its commit maps and either forces them or the batch
+    // as a whole gives every SM a full ring of items (the single-commit rule, over all handles)
+    bool tma = true, forced = true;
+    for (int l = 0; l < n; ++l) {
+        tma = tma && hs[l]->commit_maps_ok && hs[l]->S > 0;
+        forced = forced && hs[l]->cfg.commit_path == SW_COMMIT_TMA;
+    }
+    const long long items = 2LL * c0.B * ((c0.tokens_per_chunk + kCommitRows - 1) / kCommitRows) *
+                            ((c0.H + kCommitHeads - 1) / kCommitHeads) * n;
+    tma = tma && (forced || items >= (long long)kCommitBufs * h0->num_sms);
+    if (tma) {
+        const int ek = c0.qk_fp8 ? 1 : 2, ev = c0.pv_fp8 ? 1 : 2;
+        for (int l0 = 0; l0 < n; l0 += kCommitBatch) {
+            CommitBatch cb;
+            std::memset(&cb, 0, sizeof cb);
+            cb.n = std::min(kCommitBatch, n - l0);
+            for (int q = 0; q < cb.n; ++q) {
+                sw_attn_t* h = hs[l0 + q];
+                int rc;
+                if ((rc = commit_maps(h, K[l0 + q], V[l0 + q], cb.maps[q]))) return rc;
+                cb.state[q] = reinterpret_cast<int32_t*>(h->ws);
+                cb.ta[q] = table_advance(h);
+                cb.S[q] = h->S;
+            }
+            const int per = std::max(1, h0->num_sms / cb.n);
+            cudaError_t e = launch_commit_tma_batch(cb, c0.B, c0.tokens_per_chunk, c0.H, c0.d, ek, ev, per, st);
+            if (e != cudaSuccess) return cuda_fail(e, "batched TMA commit launch");
+        }
+        return SW_OK;
+    }
     for (int l0 = 0; l0 < n; l0 += kMaxBatch) {
         AppendBatch a;
         std::memset(&a, 0, sizeof a);

@@ -176,7 +176,11 @@ SW_API int sw_attn_forward(sw_attn_t *h, const void *Q, const void *K_cur, const
 /*
  * Commit the finished chunk of n handles at once -- typically the n layers of one model, each
  * with its own cache: the same effect as sw_attn_append_chunk(handles[l], K[l], V[l]) for every
- * l, in one launch per 32 handles (each handle's copy, then its counter and table) instead of one per handle
+ * l, in one launch (each handle's copy, then its counter and table) instead of one per handle.
+ * The copies are TMA bulk copies (16 handles per launch, the SMs split between them) when every
+ * handle has a ring and allows TMA commits (commit_path not SW_COMMIT_COPY) and either all force
+ * them (SW_COMMIT_TMA) or the batch together gives every SM a full ring of copies; otherwise
+ * the copy kernel (32 handles per launch)
  * (the clean-KV cache build of a chunk covers every layer: tutorial, section "软硬件协同部署";
  * neurohive review, section "Откуда берётся 30 FPS").  All handles share B, H, d and T; window,
  * sink, condition count and chunk counter are each handle's own.  K[l], V[l]: [B, T, H, d] bf16.

@@ -458,16 +458,19 @@ LAYERS = [dict(W=2, sink=True, n_cond=40, commit_in_forward=False), dict(W=1, si
           dict(W=2, sink=False, n_cond=130, commit_in_forward=True)]
 
 
-def test_append_batched_matches_ring(dev):
+@pytest.mark.parametrize("commit_path,d", [("copy", 64), ("tma", 64), ("tma", 128)])
+def test_append_batched_matches_ring(dev, commit_path, d):
     """Five layers with different windows, sinks, condition counts and slot counts, committed
-    together: every layer's table and cache equal its own oracle model, bit for bit."""
+    together: every layer's table and cache equal its own oracle model, bit for bit, with the
+    copy kernel and with the batched TMA bulk copies (every handle forcing them)."""
     from block_causal_attention_sliding_b200.api import append_chunk_batched
     from parity_util import check_cache_against_ring
-    B, H, d, T, chunks = 2, 3, 64, 40, 9
+    B, H, T, chunks = 2, 3, 40, 9
     hs, rings, held = [], [], []
     for cfg in LAYERS:
         wl = Workload("l", B=B, H=H, d=d, T=T, n_cond=cfg["n_cond"], W=cfg["W"], sink=cfg["sink"], chunks=chunks, steps=1)
-        h = make_handle(wl, dev, commit_in_forward=cfg["commit_in_forward"])
+        h = make_handle(wl, dev, commit_in_forward=cfg["commit_in_forward"], commit_path=commit_path)
+        assert h.commit_kind() == commit_path
         kc, vc = h.cache_views()
         kc.fill_(float("nan"))
         vc.fill_(float("nan"))
