@@ -626,68 +626,74 @@ def commit_path(args, dev, stream, pool):
 
 
 def fp8_path(args, dev, stream, peaks):
-    """The 720p steady-state forward with e4m3 queries and keys (S on kind::f8f6f4, e4m3 K
-    cache) and bf16 V, and with e4m3 V as well (e4m3 V cache, P in e4m3, PV on kind::f8f6f4),
-    against the bf16 forward of the same draws, each timed alone."""
+    """The steady-state forward with e4m3 queries and keys (S on kind::f8f6f4, e4m3 K cache) and
+    bf16 V, and with e4m3 V as well (e4m3 V cache, P in e4m3, PV on kind::f8f6f4), against the
+    bf16 forward of the same draws, each timed alone: at 720p (the persistent kernel) with the
+    split-K path beside it, and at 480p (the three-buffer kernel)."""
     from block_causal_attention_sliding_b200.api import SlidingWindowAttention
-    wl = WORKLOADS["720p"]
     sc = synth.FP8_SCALE
     res = {}
     # read (not written) to flush L2: a written buffer would leave dirty lines whose write-backs
     # land inside the timed launch
     flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MiB, twice the L2
-    for name, fp8, v8 in (("bf16", False, False), ("e4m3_qk", True, False), ("e4m3_qkv", True, True)):
-        h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
-                                   out_dtype=torch.bfloat16, qk_fp8=fp8, q_scale=sc, k_scale=sc,
-                                   pv_fp8=v8, v_scale=sc, device=dev)
-        if fp8:
-            Kc, Vc = synth.cond_inputs_fp8(wl, seed=11, device=dev, v8=v8)
-            Q, K, V = synth.chunk_inputs_fp8(wl, 0, 0, seed=11, device=dev, v8=v8)
-        else:
-            Kc, Vc = synth.cond_inputs(wl, seed=11, device=dev)
-            Q, K, V = synth.chunk_inputs(wl, 0, 0, seed=11, device=dev)
-        h.set_cond(Kc, Vc)
-        for _ in range(wl.steady_k()):
-            h.append_chunk(K, V)
-        out = torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            h.forward(Q, K, V, out=out)
-        torch.cuda.synchronize(dev)
-        reps = 50
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(torch.cuda.current_stream())
-        for _ in range(reps):
-            h.forward(Q, K, V, out=out)
-        e1.record(torch.cuda.current_stream())
-        torch.cuda.synchronize(dev)
-        t = e0.elapsed_time(e1) / 1e3 / reps
-        tf = wl.flops_forward(wl.steady_k()) / t / 1e12
-        kc, vc = h.cache_views()
-        rec = {"ms_per_forward": round(t * 1e3, 4), "TFLOP/s": round(tf, 2), "workspace_bytes": h.workspace_bytes(),
-               "cache_bytes": kc.numel() * kc.element_size() + vc.numel() * vc.element_size()}
-        # split-K with 128 queries: HBM-bound, so the e4m3 cache shows up as time.  The e4m3 key
-        # set fits in L2, so L2 is flushed before every launch and each launch timed alone.
-        q = Q[:, :128].contiguous()
-        o = torch.empty((wl.B, 128, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            h.forward(q, K, V, out=o)
-        ts = []
-        for _ in range(20):
-            flush.amax()
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(torch.cuda.current_stream())
-            h.forward(q, K, V, out=o)
-            a1.record(torch.cuda.current_stream())
+    for wname in ("720p", "480p"):
+        wl = WORKLOADS[wname]
+        res_w = {}
+        for name, fp8, v8 in (("bf16", False, False), ("e4m3_qk", True, False), ("e4m3_qkv", True, True)):
+            h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                       out_dtype=torch.bfloat16, qk_fp8=fp8, q_scale=sc, k_scale=sc,
+                                       pv_fp8=v8, v_scale=sc, device=dev)
+            if fp8:
+                Kc, Vc = synth.cond_inputs_fp8(wl, seed=11, device=dev, v8=v8)
+                Q, K, V = synth.chunk_inputs_fp8(wl, 0, 0, seed=11, device=dev, v8=v8)
+            else:
+                Kc, Vc = synth.cond_inputs(wl, seed=11, device=dev)
+                Q, K, V = synth.chunk_inputs(wl, 0, 0, seed=11, device=dev)
+            h.set_cond(Kc, Vc)
+            for _ in range(wl.steady_k()):
+                h.append_chunk(K, V)
+            out = torch.empty((wl.B, wl.T, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+            for _ in range(3):
+                h.forward(Q, K, V, out=out)
             torch.cuda.synchronize(dev)
-            ts.append(a0.elapsed_time(a1) / 1e3)
-        tq = statistics.median(ts)
-        kv_bytes = wl.B * wl.H * wl.n_vis(wl.steady_k()) * wl.d * (K.element_size() + V.element_size())
-        rec["split_k_128"] = {"us": round(tq * 1e6, 2), "GB/s": round(kv_bytes / tq / 1e9, 1),
-                              "frac_hbm": round(kv_bytes / tq / 1e9 / peaks["hbm_gbs"], 3), "bytes": kv_bytes,
-                              "timing": "L2 flushed by a 256 MiB read before each launch, median of 20"}
-        rec["status"] = h.status()
-        res[name] = rec
-        h.close()
+            reps = 50
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(torch.cuda.current_stream())
+            for _ in range(reps):
+                h.forward(Q, K, V, out=out)
+            e1.record(torch.cuda.current_stream())
+            torch.cuda.synchronize(dev)
+            t = e0.elapsed_time(e1) / 1e3 / reps
+            tf = wl.flops_forward(wl.steady_k()) / t / 1e12
+            kc, vc = h.cache_views()
+            rec = {"ms_per_forward": round(t * 1e3, 4), "TFLOP/s": round(tf, 2), "schedule": h.schedule_for(),
+                   "workspace_bytes": h.workspace_bytes(),
+                   "cache_bytes": kc.numel() * kc.element_size() + vc.numel() * vc.element_size()}
+            if wname == "720p":
+                # split-K with 128 queries: HBM-bound, so the e4m3 cache shows up as time.  The e4m3
+                # key set fits in L2, so L2 is flushed before every launch and each launch timed alone.
+                q = Q[:, :128].contiguous()
+                o = torch.empty((wl.B, 128, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+                for _ in range(3):
+                    h.forward(q, K, V, out=o)
+                ts = []
+                for _ in range(20):
+                    flush.amax()
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(torch.cuda.current_stream())
+                    h.forward(q, K, V, out=o)
+                    a1.record(torch.cuda.current_stream())
+                    torch.cuda.synchronize(dev)
+                    ts.append(a0.elapsed_time(a1) / 1e3)
+                tq = statistics.median(ts)
+                kv_bytes = wl.B * wl.H * wl.n_vis(wl.steady_k()) * wl.d * (K.element_size() + V.element_size())
+                rec["split_k_128"] = {"us": round(tq * 1e6, 2), "GB/s": round(kv_bytes / tq / 1e9, 1),
+                                      "frac_hbm": round(kv_bytes / tq / 1e9 / peaks["hbm_gbs"], 3), "bytes": kv_bytes,
+                                      "timing": "L2 flushed by a 256 MiB read before each launch, median of 20"}
+            rec["status"] = h.status()
+            res_w[name] = rec
+            h.close()
+        res[wname] = res_w
     res["note"] = ("e4m3 inputs with per-tensor scale 2^-4; e4m3_qk: bf16 V and P; e4m3_qkv: e4m3 V and P; "
                    "FLOPs counted as for bf16")
     return res

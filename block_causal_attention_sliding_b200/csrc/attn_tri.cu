@@ -40,13 +40,18 @@ namespace swattn {
 
 namespace tri {
 
-template <int D>
+// kQK8: e4m3 Q and K (16 KB tiles, S on kind::f8f6f4); kPV8 (with kQK8): e4m3 V as well, P in
+// e4m3 and O += P V on kind::f8f6f4.  Stages are sized by the operand format, so with e4m3 K
+// the K ring holds three stages where bf16 at d = 128 fits two.
+template <int D, bool kQK8 = false, bool kPV8 = false>
 struct Cfg {
-    static constexpr int kTileBytes = TileCfg<D>::kTileBytes;
-    static constexpr int kKSt = D == 128 ? 2 : 3;    // K ring stages (at most 3, see above)
-    static constexpr int kVSt = 3;                  // V ring stages (at most 3)
-    static constexpr int kQBytes = kTileBytes;
-    static constexpr int kKVBytes = (kKSt + kVSt) * kTileBytes;
+    static constexpr int kKBytes = kv_tile_bytes<D, kQK8, kPV8>(0);   // one K stage
+    static constexpr int kVBytes = kv_tile_bytes<D, kQK8, kPV8>(1);   // one V stage
+    static constexpr int kKSt = (D == 128 && !kQK8) ? 2 : 3;          // K ring stages (at most 3, see above)
+    static constexpr int kVSt = 3;                                    // V ring stages (at most 3)
+    static constexpr int kQBytes = QKTile<D, kQK8>::kBytes;
+    static constexpr int kVOffset = kKSt * kKBytes;                   // V ring after the K ring
+    static constexpr int kKVBytes = kVOffset + kVSt * kVBytes;
     static_assert(kKSt <= 3 && kVSt <= 3 && kKSt + kVSt <= 8, "ring stages");
     static constexpr int kCtlOffset = kQBytes + kKVBytes;
     static constexpr int kThreads = 64 + 2 * 128 + 32;   // + the load-completion helper warp
@@ -75,19 +80,21 @@ struct Ext {
     float lsum[2][2][kBlockM];   // [piece parity][group][row] row sums at the final reference
 };
 
-template <int D>
+template <int D, bool kQK8 = false, bool kPV8 = false>
 constexpr int smem_bytes() {
-    return ((Cfg<D>::kCtlOffset + (int)sizeof(SmemCtl) + 15) & ~15) + (int)sizeof(Ext) + 1024;
+    // at least 120 KB: one CTA per SM, so no CTA waits on another's tensor memory
+    constexpr int need = ((Cfg<D, kQK8, kPV8>::kCtlOffset + (int)sizeof(SmemCtl) + 15) & ~15) + (int)sizeof(Ext) + 1024;
+    return need > 120 * 1024 ? need : 120 * 1024;
 }
 
 }  // namespace tri
 
 
-template <int D>
+template <int D, bool kQK8, bool kPV8>
 __global__ void __launch_bounds__(tri::Cfg<D>::kThreads, 1)
 attn_tri_kernel(const __grid_constant__ AttnParams p) {
-    using C = tri::Cfg<D>;
-    constexpr int kTileBytes = C::kTileBytes;
+    using C = tri::Cfg<D, kQK8, kPV8>;
+    using QT = QKTile<D, kQK8>;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -153,10 +160,10 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                 const int b = bh / p.H, h = bh % p.H;
                 // the Q buffer is reused: every S MMA of the previous piece has completed
                 if (pi > 0 && !wait_or_abort(smem_u32(&ctl->q_empty), (pi - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(qbar, kTileBytes);
+                mbar_arrive_expect_tx(qbar, QT::kBytes);
                 const QSrc qs = q_src(p, qtile);
-                for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
-                    tma_load_4d(smem_u32(q_smem + c * kBoxBytes), qs.tm, qbar, c * kBoxCols, h, qs.row0, b);
+                for (int c = 0; c < QT::kBoxes; ++c)
+                    tma_load_4d(smem_u32(q_smem + c * kBoxBytes), qs.tm, qbar, c * QT::kBoxCols, h, qs.row0, b);
                 ++pi;
                 const int n = pc.j1 - pc.j0;
                 // K(u): its stage last held K(u - kKSt), free once S(u - kKSt) has completed
@@ -169,8 +176,8 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                     }
                     const int st = u % C::kKSt;
                     const uint32_t fbar = smem_u32(&ctl->kv_full[st]);
-                    mbar_arrive_expect_tx(fbar, kTileBytes);
-                    load_kv_tile<D>(p, ctl, pc.j0 + jrel, 0, h, b, smem_u32(kv_smem + st * kTileBytes), fbar);
+                    mbar_arrive_expect_tx(fbar, C::kKBytes);
+                    load_kv_tile<D, kQK8, kPV8>(p, ctl, pc.j0 + jrel, 0, h, b, smem_u32(kv_smem + st * C::kKBytes), fbar);
                     return true;
                 };
                 // V(u): its stage last held V(u - kVSt), free once PV(u - kVSt) has completed
@@ -181,10 +188,11 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                         if (!wait_or_abort(smem_u32(&ex->o_full[v % tri::kSBufs]), (v / tri::kSBufs) & 1, abort_flag))
                             return false;
                     }
-                    const int st = C::kKSt + (int)(u % C::kVSt);
-                    const uint32_t fbar = smem_u32(&ctl->kv_full[st]);
-                    mbar_arrive_expect_tx(fbar, kTileBytes);
-                    load_kv_tile<D>(p, ctl, pc.j0 + jrel, 1, h, b, smem_u32(kv_smem + st * kTileBytes), fbar);
+                    const int vs = (int)(u % C::kVSt);
+                    const uint32_t fbar = smem_u32(&ctl->kv_full[C::kKSt + vs]);
+                    mbar_arrive_expect_tx(fbar, C::kVBytes);
+                    load_kv_tile<D, kQK8, kPV8>(p, ctl, pc.j0 + jrel, 1, h, b,
+                                                smem_u32(kv_smem + C::kVOffset + vs * C::kVBytes), fbar);
                     return true;
                 };
                 // consumption order: K(0..2), then V(jj), K(jj + 3)
@@ -227,7 +235,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                     }
                     tc_fence_after();
                     // buffer u % 3 last held P(u - 3), read by a PV issued before this S
-                    issue_s<D>(tmem + (u % tri::kSBufs) * kBlockN, q_base, kv_base + (u % C::kKSt) * kTileBytes);
+                    issue_s_qk<D, kQK8>(tmem + (u % tri::kSBufs) * kBlockN, q_base, kv_base + (u % C::kKSt) * C::kKBytes);
                     mma_commit(smem_u32(&ex->s_full[u % tri::kSBufs]));
                     if (k == n - 1) mma_commit(smem_u32(&ctl->q_empty));   // last S of the piece
                 }
@@ -244,11 +252,17 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                     }
                     tc_fence_after();
                     const uint32_t tP = tmem + bu * kBlockN;
-                    issue_pv<D>(tO, tP, kv_base + (C::kKSt + u % C::kVSt) * kTileBytes, jj > 0);
+                    const uint32_t v_tile = kv_base + C::kVOffset + (u % C::kVSt) * C::kVBytes;
+                    if constexpr (kPV8) {
+                        issue_pv_f8_half(tO, tP, v_tile, 0, jj > 0);
+                        issue_pv_f8_half(tO, tP, v_tile, 1, true);
+                    } else {
+                        issue_pv<D>(tO, tP, v_tile, jj > 0);
+                    }
                     mma_commit(smem_u32(&ex->o_full[bu]));   // PV(u) done: V stage, rescale, epilogue
                     if (more) {
                         // S(u + 3) into the same buffer, in issue order after PV(u) read P(u)
-                        issue_s<D>(tP, q_base, kv_base + ((u + 3) % C::kKSt) * kTileBytes);
+                        issue_s_qk<D, kQK8>(tP, q_base, kv_base + ((u + 3) % C::kKSt) * C::kKBytes);
                         mma_commit(smem_u32(&ex->s_full[bu]));
                         if (jj + 3 == n - 1) mma_commit(smem_u32(&ctl->q_empty));
                     }
@@ -326,7 +340,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t up = u - 1;   // unused when jj == 0
-                ok = tri::softmax_tile<D>(lane_base + bu * kBlockN, tO, valid, jj == 0, u, &ex->ref[up & 1][row],
+                ok = tri::softmax_tile<D, false, kPV8>(lane_base + bu * kBlockN, tO, valid, jj == 0, u, &ex->ref[up & 1][row],
                                           &ex->ref[u & 1][row], smem_u32(&ex->o_full[up % tri::kSBufs]),
                                           (up / tri::kSBufs) & 1, smem_u32(&ex->p_cnt[bu]), p.scale_log2, m_g,
                                           l_g, has_g, abort_flag);
@@ -369,7 +383,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
             const int m_row = qs.row0 + row;
             const size_t orow = ((size_t)b * qs.rows + m_row) * p.H + h;
             if (pc.j0 == 0 && pc.j1 == nt) {
-                const float inv = 1.f / l_row;
+                const float inv = (kPV8 ? p.out_scale : 1.f) / l_row;   // e4m3 V: its scale, once
                 if (m_row < qs.rows) {
 #pragma unroll
                     for (int c = 0; c < D / 64; ++c)
@@ -417,7 +431,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                 const float* pml = p.sk_ml + (size_t)sl * 2 * kBlockM * 2 + row * 2;
                 L_ += ex2_approx(__ldcg(pml) - M) * __ldcg(pml + 1);
             }
-            const float inv = 1.f / L_;
+            const float inv = (kPV8 ? p.out_scale : 1.f) / L_;
 #pragma unroll 1
             for (int c = 0; c < D / 64; ++c) {      // 32 columns at a time
                 uint32_t acc[32];
@@ -446,21 +460,25 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
     if (threadIdx.x == 0 && ctl->abort_flag) atomicOr(p.status, SW_STATUS_TIMEOUT);
 }
 
-template <int D>
+template <int D, bool kQK8, bool kPV8>
 static cudaError_t launch_tri_d(const AttnParams& p, int ctas, cudaStream_t stream) {
-    constexpr int smem = tri::smem_bytes<D>();
+    constexpr int smem = tri::smem_bytes<D, kQK8, kPV8>();
     static_assert(smem <= 227 * 1024, "shared memory budget");
-    auto kern = attn_tri_kernel<D>;
+    auto kern = attn_tri_kernel<D, kQK8, kPV8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, tri::Cfg<D>::kThreads, smem, stream>>>(p);
+    kern<<<ctas, tri::Cfg<D, kQK8, kPV8>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_tri(const AttnParams& p, int d, int ctas, cudaStream_t stream) {
     if (ctas < 1 || ctas > kMaxPersistentCtas) return cudaErrorInvalidValue;
-    if (d == 128) return launch_tri_d<128>(p, ctas, stream);
-    if (d == 64) return launch_tri_d<64>(p, ctas, stream);
+    if (d == 128) {
+        if (p.qk_fp8) return p.pv_fp8 ? launch_tri_d<128, true, true>(p, ctas, stream)
+                                      : launch_tri_d<128, true, false>(p, ctas, stream);
+        return launch_tri_d<128, false, false>(p, ctas, stream);
+    }
+    if (d == 64 && !p.qk_fp8) return launch_tri_d<64, false, false>(p, ctas, stream);
     return cudaErrorInvalidValue;
 }
 

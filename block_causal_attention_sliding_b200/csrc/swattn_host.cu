@@ -161,6 +161,7 @@ int check_cfg(const sw_attn_config& c) {
     if (c.qk_fp8 != 0 && c.qk_fp8 != 1) return fail(SW_EINVAL, "qk_fp8 must be 0 or 1");
     if (c.qk_fp8 && c.d != 128) return fail(SW_ESHAPE, "e4m3 Q/K need d = 128");
     if (c.qk_fp8 && c.commit_in_forward) return fail(SW_ESHAPE, "commit_in_forward is not available with e4m3 Q/K");
+    if (c.qk_fp8 && c.schedule == SW_SCHED_GRID) return fail(SW_ESHAPE, "the grid schedule has no e4m3 Q/K form");
     if (!std::isfinite(c.q_scale) || !std::isfinite(c.k_scale)) return fail(SW_EINVAL, "scales must be finite");
     if (c.pv_fp8 != 0 && c.pv_fp8 != 1) return fail(SW_EINVAL, "pv_fp8 must be 0 or 1");
     if (c.pv_fp8 && !c.qk_fp8) return fail(SW_ESHAPE, "pv_fp8 requires qk_fp8 (e4m3 Q and K)");
@@ -425,7 +426,8 @@ int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* strea
 // tiles than SMs, the three-buffer kernel (one tile per unit balances better); else persistent.
 static int resolve_schedule_tiles(const sw_attn_t* h, long long nqt) {
     const sw_attn_config& c = h->cfg;
-    if (c.qk_fp8) return SW_SCHED_PERSISTENT;   // the one kernel with an e4m3 Q/K form
+    // e4m3 handles: the persistent and three-buffer kernels have e4m3 forms (grid and pair do not,
+    // refused at create), and the automatic choice below is the same as for bf16
     if (c.schedule == SW_SCHED_PAIR) return h->pair_clusters > 0 ? SW_SCHED_PAIR : SW_SCHED_TRI;
     if (c.schedule != SW_SCHED_AUTO) return c.schedule;
     const long long pairs = (long long)c.B * c.H * ((nqt + 1) / 2);

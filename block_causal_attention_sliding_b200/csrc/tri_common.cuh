@@ -177,7 +177,10 @@ __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" 
 // Returns false on abort.
 // p_sig: the P counter's address, a shared::cta one, or (kRemote, in a CTA pair) the
 // shared::cluster address of the leader's counter.
-template <int D, bool kRemote = false>
+// kP8: P is written as e4m3 (four keys per 32-bit column over S columns 0..31, for an e4m3 P V on
+// kind::f8f6f4), formed as 2^(s sl2 - m + kP8Offset) with the rescale threshold kP8Threshold, and
+// the row sum adds the fp32 weights -- as in the two-tile kernel's softmax step.
+template <int D, bool kRemote = false, bool kP8 = false>
 __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid, bool first, uint32_t u,
                                              const unsigned long long* ref_prev, unsigned long long* ref_mine,
                                              uint32_t o_full_prev, uint32_t o_full_prev_parity,
@@ -216,7 +219,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid
     if (!first) {
         float m_prev;
         if (!ref_get(ref_prev, u, m_prev, abort_flag)) return false;
-        const bool need = m_loc > m_prev + kRescaleThreshold;
+        const bool need = m_loc > m_prev + (kP8 ? kP8Threshold : kRescaleThreshold);
         m_new = need ? m_loc : m_prev;
         if (need) f_o = ex2_approx(m_prev - m_new);
         rescale = __any_sync(0xffffffffu, need);
@@ -228,26 +231,46 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid
     float suma[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) suma[a] = 0.f;
-    const float neg_m = -m_new;
+    const float neg_m = kP8 ? kP8Offset - m_new : -m_new;
     const uint64_t sl2_2 = bcast2(sl2), neg_m2 = bcast2(neg_m);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        if constexpr (kP8) {
+            uint32_t pk[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                float x0, x1;   // s * scale * log2(e) - m for two columns in one packed FMA
-                fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
-                const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
-                // the row sum adds the same bf16-rounded weights the PV MMA multiplies
-                const int a = (i >> 1) & 7;
-                suma[a] = add_bf16x2_f32(pp, suma[a]);
-                pk[cc * 16 + (i >> 1)] = pp;
+                for (int i = 0; i < 32; i += 4) {
+                    float x0, x1, x2, x3;
+                    fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
+                    fma2_bcast(x2, x3, __uint_as_float(sr[c][i + 2]), __uint_as_float(sr[c][i + 3]), sl2_2, neg_m2);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+                    pk[cc * 8 + (i >> 2)] = pack_e4m3x4(p0, p1, p2, p3);
+                    const int a = 4 * ((i >> 2) & 1);
+                    add2_f32(suma[a], suma[a + 1], p0, p1);
+                    add2_f32(suma[a + 2], suma[a + 3], p2, p3);
+                }
             }
+            tmem_st16(tS + half * 16, pk);   // over S columns this thread has already read
+        } else {
+            uint32_t pk[32];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    float x0, x1;   // s * scale * log2(e) - m for two columns in one packed FMA
+                    fma2_bcast(x0, x1, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]), sl2_2, neg_m2);
+                    const uint32_t pp = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+                    // the row sum adds the same bf16-rounded weights the PV MMA multiplies
+                    const int a = (i >> 1) & 7;
+                    suma[a] = add_bf16x2_f32(pp, suma[a]);
+                    pk[cc * 16 + (i >> 1)] = pp;
+                }
+            }
+            tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
         }
-        tmem_st32(tS + half * 32, pk);   // over S columns this thread has already read
     }
 #pragma unroll
     for (int w = 4; w >= 1; w >>= 1)

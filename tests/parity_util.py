@@ -315,7 +315,7 @@ E4M3_P_TOL = (MAX_ABS * 16, MEAN_REL * 16)
 
 def stream_and_check_fp8(wl, dev, *, chunks, check_at=None, n_rows=None, keep_last=None,
                          gen_on_device=False, out_dtype=torch.float32, seed=0, joint=False,
-                         tol=None, pv8=False, n_q=None):
+                         tol=None, pv8=False, n_q=None, schedule="auto"):
     """Stream through a handle with e4m3 queries and keys (and, with pv8, e4m3 values: P V on
     kind::f8f6f4): 2 forwards then an append per chunk, every e4m3 tensor with scale FP8_SCALE.
     The oracle computes the same attention on the dequantised values (exact in float32).  With
@@ -327,7 +327,7 @@ def stream_and_check_fp8(wl, dev, *, chunks, check_at=None, n_rows=None, keep_la
         tol = E4M3_P_TOL if pv8 else (MAX_ABS, MEAN_REL)
     h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
                                out_dtype=out_dtype, qk_fp8=True, q_scale=sc, k_scale=sc, pv_fp8=pv8,
-                               v_scale=sc, device=dev)
+                               v_scale=sc, schedule=schedule, device=dev)
     gdev = dev if gen_on_device else "cpu"
     deq_v = (lambda t: synth.from_e4m3(t)) if pv8 else (lambda t: t)
     Kc8, Vc = synth.cond_inputs_fp8(wl, seed=seed, device=gdev, v8=pv8)

@@ -89,6 +89,7 @@ def test_workspace_constant_in_stream_length(native):
     (dict(sink=2), -1), (dict(out_dtype=7), -1), (dict(max_short_q=129), -2),
     (dict(scale=float("inf")), -1), (dict(schedule=5), -1),
     (dict(schedule=4, d=64), -2),   # the CTA-pair schedule is d = 128 only
+    (dict(schedule=1, qk_fp8=1), -2),   # no e4m3 form of the grid schedule
 ])
 def test_create_rejects_bad_config(native, kw, code):
     rc, h = _create(native, **kw)

@@ -612,19 +612,21 @@ def test_chunk_step_graph_capture(dev):
 
 # ------------------------------------------------------------------ e4m3 queries and keys
 
+@pytest.mark.parametrize("schedule", ["tri", "persistent"])
 @pytest.mark.parametrize("W,sink,n_cond", [(2, True, 40), (1, False, 130), (0, True, 0)])
-def test_fp8_qk_ragged(dev, W, sink, n_cond):
+def test_fp8_qk_ragged(dev, W, sink, n_cond, schedule):
     """e4m3 Q and K (S on kind::f8f6f4, e4m3 K cache), bf16 V: every chunk and step, all rows,
-    against the oracle on the dequantised inputs."""
+    against the oracle on the dequantised inputs, on both kernels with an e4m3 form."""
     wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
-    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, schedule=schedule)
     assert len(res) == wl.chunks * wl.steps
 
 
-def test_fp8_qk_joint(dev):
+@pytest.mark.parametrize("schedule", ["tri", "persistent"])
+def test_fp8_qk_joint(dev, schedule):
     """e4m3 chunk and condition queries in one joint launch."""
     wl = dataclasses.replace(RAGGED, n_cond=130, chunks=4)
-    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True, schedule=schedule)
     assert len(res) == 2 * wl.chunks * wl.steps
 
 
@@ -651,19 +653,21 @@ def test_fp8_qk_cache_bytes(dev, commit_path):
     assert h8.status() == 0
 
 
+@pytest.mark.parametrize("schedule", ["tri", "persistent"])
 @pytest.mark.parametrize("W,sink,n_cond", [(2, True, 40), (1, False, 130), (0, True, 0)])
-def test_fp8_pv_ragged(dev, W, sink, n_cond):
+def test_fp8_pv_ragged(dev, W, sink, n_cond, schedule):
     """e4m3 Q, K and V (P V on kind::f8f6f4 with e4m3 P, e4m3 K and V caches): every chunk and
     step, all rows, against the oracle on the dequantised inputs at the e4m3-P tolerance."""
     wl = dataclasses.replace(RAGGED, W=W, sink=sink, n_cond=n_cond, chunks=6)
-    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, pv8=True)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, pv8=True, schedule=schedule)
     assert len(res) == wl.chunks * wl.steps
 
 
-def test_fp8_pv_joint(dev):
+@pytest.mark.parametrize("schedule", ["tri", "persistent"])
+def test_fp8_pv_joint(dev, schedule):
     """e4m3 chunk and condition queries with e4m3 V in one joint launch."""
     wl = dataclasses.replace(RAGGED, n_cond=130, chunks=4)
-    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True, pv8=True)
+    res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, joint=True, pv8=True, schedule=schedule)
     assert len(res) == 2 * wl.chunks * wl.steps
 
 
@@ -721,6 +725,16 @@ def test_fp8_short_queries_ragged(dev, H, n_q, pv8):
     wl = dataclasses.replace(RAGGED, H=H, chunks=5)
     res = stream_and_check_fp8(wl, dev, chunks=wl.chunks, pv8=pv8, n_q=n_q)
     assert len(res) == wl.chunks * wl.steps
+
+
+@pytest.mark.parametrize("pv8", [False, True])
+def test_fp8_480p_sampled(dev, pv8):
+    """480p with e4m3 inputs on the automatic schedule (the three-buffer kernel: 96 Q-tile pairs
+    on 148 SMs), sampled rows at chunks 0, W + 1 and the last of 6."""
+    wl = WORKLOADS["480p"]
+    res = stream_and_check_fp8(wl, dev, chunks=6, check_at={0, 3, 5}, n_rows=64, keep_last=wl.W + 1,
+                               gen_on_device=True, pv8=pv8)
+    assert len(res) == 6
 
 
 def test_fp8_qk_720p_sampled(dev):
