@@ -472,7 +472,7 @@ def run_cuda(args, wl, world, rank, local):
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
                          "kernel": {"persistent": "attn_persistent_kernel<128, false, false, false>", "tri": "attn_tri_kernel<128, false, false>",
-                                    "grid": "attn_fwd_kernel<128,2>"}[sched],
+                                    "grid": "attn_fwd_kernel<128,2>", "pair": "attn_pair_kernel"}[sched],
                          "achieved": round(achieved, 2),
                          # the launches are timed inside a continuous, power-capped stream of chunk
                          # steps (no idle gap before the timed region), so the sustained GEMM figure
@@ -999,7 +999,7 @@ def main(argv=None):
     ap.add_argument("--warm-seconds", type=float, default=4.0,
                     help="seconds of chunk steps before the timed long-horizon stream")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", choices=["auto", "persistent", "grid", "tri"], default="auto")
+    ap.add_argument("--schedule", choices=["auto", "persistent", "grid", "tri", "pair"], default="auto")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the long-horizon and other-workload side measurements")
     args = ap.parse_args(argv)
