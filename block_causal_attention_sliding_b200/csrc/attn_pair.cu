@@ -84,7 +84,9 @@ __device__ __forceinline__ void st_release_cluster(uint32_t addr, uint32_t v) {
 
 // S = Q K^T over the pair: 8 MMAs of 16 columns of d.  Q: two 16 KB boxes (128 rows x 64
 // columns); this CTA's K half: two 8 KB boxes (64 keys x 64 columns); K-major, 128-byte swizzle.
-__device__ __forceinline__ void issue_s_pair(uint32_t tS, uint32_t q_tile, uint32_t k_half) {
+// The two issue sequences are out of line: measured on B200, that keeps the issuer's code apart
+// from the unrolled softmax and the forward takes 3% less time (0.829 against 0.857 ms at 720p).
+__device__ __noinline__ void issue_s_pair(uint32_t tS, uint32_t q_tile, uint32_t k_half) {
     constexpr uint32_t idesc = idesc_bf16_f32(2 * kBlockM, kBlockN, false);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
@@ -96,7 +98,7 @@ __device__ __forceinline__ void issue_s_pair(uint32_t tS, uint32_t q_tile, uint3
 
 // O (+)= P V over the pair: 8 MMAs of 16 keys.  P: bf16 pairs in each CTA's tensor memory; this
 // CTA's V half: one 16 KB box of 128 keys x 64 columns, MN-major (one 128-byte swizzle atom wide).
-__device__ __forceinline__ void issue_pv_pair(uint32_t tO, uint32_t tP, uint32_t v_half, bool accumulate) {
+__device__ __noinline__ void issue_pv_pair(uint32_t tO, uint32_t tP, uint32_t v_half, bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(2 * kBlockM, D, true);
 #pragma unroll
     for (int ks = 0; ks < kBlockN / 16; ++ks)
