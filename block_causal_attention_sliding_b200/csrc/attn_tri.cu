@@ -340,7 +340,7 @@ attn_tri_kernel(const __grid_constant__ AttnParams p) {
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t up = u - 1;   // unused when jj == 0
-                ok = tri::softmax_tile<D, false, kPV8>(lane_base + bu * kBlockN, tO, valid, jj == 0, u, &ex->ref[up & 1][row],
+                ok = tri::softmax_tile<D, kPV8>(lane_base + bu * kBlockN, tO, valid, jj == 0, u, &ex->ref[up & 1][row],
                                           &ex->ref[u & 1][row], smem_u32(&ex->o_full[up % tri::kSBufs]),
                                           (up / tri::kSBufs) & 1, smem_u32(&ex->p_cnt[bu]), p.scale_log2, m_g,
                                           l_g, has_g, abort_flag);

@@ -76,21 +76,15 @@ __device__ __forceinline__ void st_release(uint32_t* a, uint32_t v) {
     asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
 }
 
-// One release increment per warp, after the warp's lanes have finished (and fenced) their work:
-// on a word of this CTA (kRemote = false: a shared::cta address) or, in a CTA pair, on a word
-// of the pair's leader (kRemote = true: a shared::cluster address, cluster scope).
-template <bool kRemote = false>
+// One release increment per warp on a word of this CTA (shared::cta address), after the warp's
+// lanes have finished (and fenced) their work.
 __device__ __forceinline__ void warp_signal(uint32_t addr) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) {
-        if constexpr (kRemote)
-            asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], 1;" ::"r"(addr) : "memory");
-        else
-            asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(addr) : "memory");
-    }
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// Acquire load at cluster scope (pairs with the remote signals above).
+// Acquire load at cluster scope (pairs with a release from the peer CTA of a pair).
 __device__ __forceinline__ uint32_t ld_acquire_cluster(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
@@ -175,12 +169,11 @@ __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" 
 // has had a tile in this piece).  P is published once it is written in full and O, if the
 // reference moved, has been rescaled.
 // Returns false on abort.
-// p_sig: the P counter's address, a shared::cta one, or (kRemote, in a CTA pair) the
-// shared::cluster address of the leader's counter.
+// p_sig: the shared::cta address of the P counter.
 // kP8: P is written as e4m3 (four keys per 32-bit column over S columns 0..31, for an e4m3 P V on
 // kind::f8f6f4), formed as 2^(s sl2 - m + kP8Offset) with the rescale threshold kP8Threshold, and
 // the row sum adds the fp32 weights -- as in the two-tile kernel's softmax step.
-template <int D, bool kRemote = false, bool kP8 = false>
+template <int D, bool kP8 = false>
 __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid, bool first, uint32_t u,
                                              const unsigned long long* ref_prev, unsigned long long* ref_mine,
                                              uint32_t o_full_prev, uint32_t o_full_prev_parity,
@@ -294,7 +287,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int valid
     }
     tmem_wait_st();
     tc_fence_before();
-    warp_signal<kRemote>(p_sig);   // P(u) written and O ready for PV(u)
+    warp_signal(p_sig);   // P(u) written and O ready for PV(u)
     return true;
 }
 
