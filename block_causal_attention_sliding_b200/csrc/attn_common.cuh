@@ -212,7 +212,8 @@ __host__ __device__ constexpr int kv_tile_bytes(int kv) {
 // the producer flushes them and waits for the stores to complete before it finishes.  The
 // per-item work is kept out of line: inlined, it changed the register allocation of the whole
 // kernel and cost more (measured) than the stores themselves.
-template <int D, int kStages>
+// kQK8 / kPV8: K / V tiles are e4m3, one box of 128-byte rows each (bf16: kBoxes boxes).
+template <int D, int kStages, bool kQK8 = false, bool kPV8 = false>
 struct CommitQueue {
     static constexpr int kLag = kStages - 1;
     static_assert(kLag >= 1 && kLag <= 7, "commit history");
@@ -241,9 +242,12 @@ struct CommitQueue {
         tile_of(ctl, j, seg, row0, valid);
         fence_proxy_async_smem();
         const uint32_t src = smem_u32(kv_smem + (size_t)s * TileCfg<D>::kTileBytes);
+        const int boxes = ((kQK8 && kv == 0) || (kPV8 && kv == 1)) ? 1 : TileCfg<D>::kBoxes;
 #pragma unroll
-        for (int c = 0; c < TileCfg<D>::kBoxes; ++c)
+        for (int c = 0; c < TileCfg<D>::kBoxes; ++c) {
+            if (c >= boxes) break;
             tma_store_5d(kv ? &p.tm_cache_v : &p.tm_cache_k, src + c * kBoxBytes, c * kBoxCols, row0, slot, h, b);
+        }
         bulk_commit_group();
         pending |= 1u << s;
         return true;

@@ -81,7 +81,7 @@ __device__ __noinline__ void persist_producer(const AttnParams& p, SmemCtl* ctl,
     // fused commit: the chunk's K_cur / V_cur tile j is stored by the piece of Q-tile pair
     // j mod npairs that loads it, so the stores spread over the CTAs
     const int cslot = kCommit ? ring_slot(__ldg(p.table), p.ring_R, p.sink) : -1;
-    CommitQueue<D, kStages> cq;
+    CommitQueue<D, kStages, kQK8, kPV8> cq;
     while (ok && next_piece(sched, pit, pc)) {
         const int b = pc.bh / p.H, h = pc.bh % p.H;
         // the Q buffers are reused: wait until every S MMA of the previous piece is done
@@ -507,7 +507,10 @@ static cudaError_t launch_persistent_d(const AttnParams& p, int ctas, cudaStream
     using L = AttnLayout<D, 2>;
     auto kern = p.commit ? attn_persistent_kernel<D, true, false, false> : attn_persistent_kernel<D, false, false, false>;
     if constexpr (D == 128) {
-        if (p.qk_fp8) kern = p.pv_fp8 ? attn_persistent_kernel<D, false, true, true> : attn_persistent_kernel<D, false, true, false>;
+        if (p.qk_fp8) {
+            if (p.commit) kern = p.pv_fp8 ? attn_persistent_kernel<D, true, true, true> : attn_persistent_kernel<D, true, true, false>;
+            else kern = p.pv_fp8 ? attn_persistent_kernel<D, false, true, true> : attn_persistent_kernel<D, false, true, false>;
+        }
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -160,7 +160,6 @@ int check_cfg(const sw_attn_config& c) {
     if (c.commit_in_forward != 0 && c.commit_in_forward != 1) return fail(SW_EINVAL, "commit_in_forward must be 0 or 1");
     if (c.qk_fp8 != 0 && c.qk_fp8 != 1) return fail(SW_EINVAL, "qk_fp8 must be 0 or 1");
     if (c.qk_fp8 && c.d != 128) return fail(SW_ESHAPE, "e4m3 Q/K need d = 128");
-    if (c.qk_fp8 && c.commit_in_forward) return fail(SW_ESHAPE, "commit_in_forward is not available with e4m3 Q/K");
     if (c.qk_fp8 && c.schedule == SW_SCHED_GRID) return fail(SW_ESHAPE, "the grid schedule has no e4m3 Q/K form");
     if (!std::isfinite(c.q_scale) || !std::isfinite(c.k_scale)) return fail(SW_EINVAL, "scales must be finite");
     if (c.pv_fp8 != 0 && c.pv_fp8 != 1) return fail(SW_EINVAL, "pv_fp8 must be 0 or 1");
@@ -658,7 +657,6 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     const sw_attn_config& c = h->cfg;
     if (!c.commit_in_forward) return fail(SW_ESTATE, "the handle was not created with commit_in_forward");
-    if (c.qk_fp8) return fail(SW_ESTATE, "no committing forward with e4m3 Q/K");
     if (c.B > 32767 || c.H > 65535) return fail(SW_ESHAPE, "a committing forward supports B <= 32767, H <= 65535");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
     if (!aligned16(Q) || !aligned16(K_cur) || !aligned16(V_cur) || !aligned16(out))

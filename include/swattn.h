@@ -91,7 +91,7 @@ typedef struct {
                                 the bytes) and S = Q K^T runs on kind::f8f6f4; V stays bf16.
                                 Requires d = 128; full path on the persistent or three-buffer
                                 schedule (SW_SCHED_GRID and SW_SCHED_PAIR: SW_ESHAPE at create),
-                                short queries on the split-K path; no commit_in_forward */
+                                short queries on the split-K path */
     float q_scale, k_scale;  /* dequantisation scales of the e4m3 Q and K (per tensor; <= 0
                                 selects 1): the attention uses q * q_scale and k * k_scale */
     int   commit_path;       /* chunk commits: SW_COMMIT_AUTO (default; TMA bulk copies when

@@ -229,9 +229,24 @@ def stream_and_check_joint(wl, dev, *, chunks, check_at=None, n_rows=None, promp
     return results
 
 
+def _bits(t):
+    """The raw bits of a bf16 (int16 view) or e4m3 (uint8 view) tensor."""
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.uint8)
+
+
+def poison_cache(h):
+    """Fill the handle's K/V cache with NaN (bf16 or e4m3)."""
+    for t in h.cache_views():
+        if t.element_size() == 2:
+            t.fill_(float("nan"))
+        else:
+            t.view(torch.uint8).fill_(0x7F)   # e4m3 NaN
+
+
 def check_cache_against_ring(h, ring, chunks):
     """Every slot of the handle's cache holds, bit for bit, the chunk the oracle's ring model
-    puts there; slots the model leaves empty still hold the NaN poison."""
+    puts there (the tensors appended, bf16 or e4m3); slots the model leaves empty still hold the
+    NaN poison."""
     kc, vc = h.cache_views()
     held = ring.slot_chunks()
     assert len(held) == kc.shape[2]
@@ -241,36 +256,53 @@ def check_cache_against_ring(h, ring, chunks):
             assert torch.isnan(gk.float()).all() and torch.isnan(gv.float()).all(), f"slot {s} written"
         else:
             ek, ev = chunks[c]
-            assert torch.equal(gk.view(torch.int16), ek.permute(0, 2, 1, 3).contiguous().view(torch.int16)), s
-            assert torch.equal(gv.view(torch.int16), ev.permute(0, 2, 1, 3).contiguous().view(torch.int16)), s
+            assert torch.equal(_bits(gk), _bits(ek.permute(0, 2, 1, 3).contiguous())), s
+            assert torch.equal(_bits(gv), _bits(ev.permute(0, 2, 1, 3).contiguous())), s
 
 
 def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, n_rows=None,
                             check_cache=True, append_at=(), keep_last=None, gen_on_device=False,
-                            out_dtype=torch.float32, seed=0, tol=(MAX_ABS, MEAN_REL)):
+                            out_dtype=torch.float32, seed=0, tol=None, fp8=None):
     """Stream through a handle created with commit_in_forward: per chunk, the first step's
     forward, then the last step's forward_commit (its K_cur / V_cur become the chunk's cache
     entry) -- or, at the chunks in `append_at`, a plain forward plus append_chunk.  After every
     chunk the table is compared with the oracle's table for the ring with a spare slot and (with
     check_cache) the cache with the oracle's ring model, bit for bit; at the chunks in
-    `check_at` (all if None) both outputs are compared with the oracle.
+    `check_at` (all if None) both outputs are compared with the oracle.  fp8 = "qk" or "qkv": an
+    e4m3 handle (e4m3 Q/K, and V too with "qkv"); the cache is compared with the e4m3 tensors
+    committed, the outputs with the oracle on the dequantised inputs (E4M3_P_TOL with "qkv").
     Returns a list of (k, step, max_abs, mean_rel)."""
-    h = make_handle(wl, dev, out_dtype=out_dtype, max_short_q=-1, schedule=schedule, commit_in_forward=True)
+    pv8 = fp8 == "qkv"
+    if tol is None:
+        tol = E4M3_P_TOL if pv8 else (MAX_ABS, MEAN_REL)
+    if fp8:
+        sc = synth.FP8_SCALE
+        h = SlidingWindowAttention(B=wl.B, H=wl.H, d=wl.d, T=wl.T, W=wl.W, n_cond=wl.n_cond, sink=wl.sink,
+                                   out_dtype=out_dtype, max_short_q=-1, schedule=schedule, commit_in_forward=True,
+                                   qk_fp8=True, q_scale=sc, k_scale=sc, pv_fp8=pv8, v_scale=sc, device=dev)
+    else:
+        h = make_handle(wl, dev, out_dtype=out_dtype, max_short_q=-1, schedule=schedule, commit_in_forward=True)
+    deq_qk = synth.from_e4m3 if fp8 else (lambda t: t)
+    deq_v = synth.from_e4m3 if pv8 else (lambda t: t)
     R = h.R
     if check_cache:
-        kc, vc = h.cache_views()
-        kc.fill_(float("nan"))
-        vc.fill_(float("nan"))
+        poison_cache(h)
     gdev = dev if gen_on_device else "cpu"
-    Kc, Vc = synth.cond_inputs(wl, seed=seed, device=gdev)
+    if fp8:
+        Kc, Vc = synth.cond_inputs_fp8(wl, seed=seed, device=gdev, v8=pv8)
+    else:
+        Kc, Vc = synth.cond_inputs(wl, seed=seed, device=gdev)
     h.set_cond(Kc.to(dev), Vc.to(dev))
-    Kc, Vc = Kc.cpu(), Vc.cpu()
+    Kc, Vc = deq_qk(Kc.cpu()), deq_v(Vc.cpu())
     ring = oracle.Ring(B=wl.B, H=wl.H, d=wl.d, T=wl.T, n_cond=0, W=wl.W, sink=wl.sink, Kc=None, Vc=None, R=R) \
         if check_cache else None
     hist_K, hist_V, committed, results = [], [], {}, []
     for k in range(chunks):
         for step in range(wl.steps):
-            Q, K, V = synth.chunk_inputs(wl, k, step, seed=seed, device=gdev)
+            if fp8:
+                Q, K, V = synth.chunk_inputs_fp8(wl, k, step, seed=seed, device=gdev, v8=pv8)
+            else:
+                Q, K, V = synth.chunk_inputs(wl, k, step, seed=seed, device=gdev)
             last = step == wl.steps - 1
             if last and k not in append_at:
                 out = h.forward_commit(Q.to(dev), K.to(dev), V.to(dev))
@@ -279,8 +311,8 @@ def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, 
             if check_at is None or k in check_at:
                 r = None if n_rows is None else sample_rows(wl.T, n_rows, seed=1000 * k + step)
                 ref = oracle.attention(H=wl.H, d=wl.d, T=wl.T, n_cond=wl.n_cond, W=wl.W, sink=wl.sink,
-                                       k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V, Q=Q.cpu(),
-                                       K_cur=K.cpu(), V_cur=V.cpu(), rows=r)
+                                       k=k, Kc=Kc, Vc=Vc, hist_K=hist_K, hist_V=hist_V, Q=deq_qk(Q.cpu()),
+                                       K_cur=deq_qk(K.cpu()), V_cur=deq_v(V.cpu()), rows=r)
                 got = out.float().cpu().numpy()
                 if r is not None:
                     got = got[:, r]
@@ -289,12 +321,12 @@ def stream_and_check_commit(wl, dev, *, chunks, schedule="auto", check_at=None, 
         if k in append_at:
             h.append_chunk(K.to(dev), V.to(dev))
         Kh, Vh = K.cpu(), V.cpu()
-        hist_K.append(Kh)
-        hist_V.append(Vh)
+        hist_K.append(deq_qk(Kh))
+        hist_V.append(deq_v(Vh))
         torch.cuda.synchronize()
         check_table(h.table().cpu().numpy(), k + 1, wl.W, wl.sink, wl.n_cond, wl.T, R=R)
         if check_cache:
-            ring.append(Kh, Vh)
+            ring.append(deq_qk(Kh), deq_v(Vh))
             committed[k] = (Kh, Vh)
             check_cache_against_ring(h, ring, committed)
         if keep_last is not None:

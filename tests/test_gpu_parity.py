@@ -426,6 +426,28 @@ def test_commit_in_forward_stream(dev, W, sink, schedule):
     assert len(res) == wl.chunks * wl.steps
 
 
+@pytest.mark.parametrize("schedule", ["persistent", "tri"])
+@pytest.mark.parametrize("fp8", ["qk", "qkv"])
+@pytest.mark.parametrize("W,sink", [(2, True), (1, False)])
+def test_fp8_commit_in_forward_stream(dev, W, sink, fp8, schedule):
+    """The committing forward on e4m3 handles (e4m3 K, and V with "qkv"): the cache holds the
+    committed e4m3 tensors bit for bit after every chunk, tables exact, both outputs against the
+    oracle on the dequantised inputs.  The persistent kernel stores the tiles itself (one box of
+    128-byte rows per e4m3 tile); the three-buffer kernel's forward is followed by the copy."""
+    wl = dataclasses.replace(RAGGED, W=W, sink=sink, chunks=6)
+    res = stream_and_check_commit(wl, dev, chunks=wl.chunks, schedule=schedule, fp8=fp8)
+    assert len(res) == wl.chunks * wl.steps
+
+
+def test_fp8_commit_720p_sampled(dev):
+    """720p, e4m3 Q/K/V, the clean pass committing on the persistent kernel: sampled rows at
+    chunks 0, W + 1 and the last of 6; cache and table checked after every chunk."""
+    wl = WORKLOADS["720p"]
+    res = stream_and_check_commit(wl, dev, chunks=6, check_at={0, 4, 5}, n_rows=32, keep_last=wl.W + 2,
+                                  gen_on_device=True, fp8="qkv")
+    assert len(res) == 6
+
+
 @pytest.mark.parametrize("schedule", ["persistent", "grid"])
 def test_commit_mixed_with_append(dev, schedule):
     """Commits in the forward and plain appends interleaved on one handle: the same cache."""
