@@ -98,6 +98,22 @@ def test_create_rejects_bad_config(native, kw, code):
     assert native.lib().sw_attn_last_error().decode()
 
 
+def test_fp8_configs_accepted(native):
+    """e4m3 handles are accepted with the committing forward and with the schedules that have an
+    e4m3 form (automatic, persistent, three-buffer), e4m3 V only on top of e4m3 Q/K."""
+    L = native.lib()
+    for kw in (dict(qk_fp8=1), dict(qk_fp8=1, pv_fp8=1), dict(qk_fp8=1, commit_in_forward=1),
+               dict(qk_fp8=1, pv_fp8=1, commit_in_forward=1), dict(qk_fp8=1, schedule=native.SW_SCHED_TRI),
+               dict(qk_fp8=1, schedule=native.SW_SCHED_AUTO)):
+        rc, h = _create(native, **kw)
+        assert rc == 0, (kw, L.sw_attn_last_error())
+        L.sw_attn_destroy(h)
+    for kw in (dict(pv_fp8=1), dict(qk_fp8=1, d=64), dict(qk_fp8=1, schedule=native.SW_SCHED_PAIR)):
+        rc, h = _create(native, **kw)
+        assert rc == native.SW_ESHAPE, kw
+        assert not h.value
+
+
 def test_calls_before_workspace_fail_cleanly(native):
     L = native.lib()
     rc, h = _create(native, H=2, d=64, tokens_per_chunk=16, W=1, n_cond=8)
