@@ -23,7 +23,7 @@ EXPORTS = (
     "sw_attn_forward_commit", "sw_attn_append_chunk_batched",
     "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
-    "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc",
+    "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc", "sw_attn_schedule_pieces",
     "sw_attn_selftest_timeout", "sw_attn_schedule_for", "sw_attn_commit_kind",
 )
 
@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_destroy.restype = None
     L.sw_attn_cache_offsets.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.sw_attn_cache_offsets.restype = i32
+    L.sw_attn_schedule_pieces.argtypes = [i32, i32, i32, i32, i32, vp, i32]
+    L.sw_attn_schedule_pieces.restype = i32
     L.sw_attn_last_error.argtypes = []
     L.sw_attn_last_error.restype = ctypes.c_char_p
     _lib = L

@@ -15,17 +15,18 @@ struct Piece {
     bool sk;    // from the stream-K phase (may be split) rather than a whole-pair round
 };
 
-// The two-phase schedule, identical in every role of every CTA.
+// The two-phase schedule, identical in every role of every CTA (and callable on the host, where
+// an inspection hook enumerates its pieces for the tests).
 struct Sched {
     int nqt, nt, npairs, P, G, g, rounds, p0, Gsk;
     long long Csk, c0, c1;   // stream-K line length and this CTA's range of it
-    __device__ int live(int p) const { return min(2, nqt - 2 * (p % npairs)); }
+    __host__ __device__ int live(int p) const { return min(2, nqt - 2 * (p % npairs)); }
     // cost position of pair p (p >= p0) on the stream-K line: 2 nt per pair, nt for the
     // single-tile last pair of a head (when nqt is odd)
-    __device__ long long cstart(int p) const {
+    __host__ __device__ long long cstart(int p) const {
         return 2LL * nt * (p - p0) - (long long)(nqt & 1) * nt * (p / npairs - p0 / npairs);
     }
-    __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
+    __host__ __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
         nqt = nqt_; nt = nt_; npairs = (nqt + 1) / 2; P = BH * npairs; G = G_; g = g_;
         rounds = P / G;
         p0 = rounds * G;
@@ -35,12 +36,12 @@ struct Sched {
         Gsk = Csk > 0 ? (int)min((long long)G, max(1LL, Csk / 2)) : 0;
         set_range(g);
     }
-    __device__ void set_range(int cta) {
+    __host__ __device__ void set_range(int cta) {
         c0 = cta < Gsk ? (long long)cta * Csk / Gsk : 0;
         c1 = cta < Gsk ? (long long)(cta + 1) * Csk / Gsk : 0;
     }
     // the stream-K CTA whose range holds cost position s
-    __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
+    __host__ __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
 };
 
 struct PieceIt {
@@ -49,7 +50,7 @@ struct PieceIt {
     int p = 0;             // stream-K pair the cursor is in
 };
 
-__device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
+__host__ __device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
     if (it.r < s.rounds) {
         const int p = s.g + it.r * s.G;
         ++it.r;

@@ -14,8 +14,8 @@ constexpr int kSBufs = 3;   // S accumulators in tensor memory: S of tile u + 3 
 struct Sched {
     int nqt, nt, U, G, g, rounds, u0, Gsk;
     long long Csk, c0, c1;   // stream-K line length and this CTA's range of it
-    __device__ long long cstart(int u) const { return (long long)(u - u0) * nt; }
-    __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
+    __host__ __device__ long long cstart(int u) const { return (long long)(u - u0) * nt; }
+    __host__ __device__ void init(int nqt_, int nt_, int BH, int G_, int g_) {
         nqt = nqt_; nt = nt_; U = BH * nqt; G = G_; g = g_;
         rounds = U / G;
         u0 = rounds * G;
@@ -24,11 +24,11 @@ struct Sched {
         Gsk = Csk > 0 ? (int)min((long long)G, max(1LL, Csk / 2)) : 0;
         set_range(g);
     }
-    __device__ void set_range(int cta) {
+    __host__ __device__ void set_range(int cta) {
         c0 = cta < Gsk ? (long long)cta * Csk / Gsk : 0;
         c1 = cta < Gsk ? (long long)(cta + 1) * Csk / Gsk : 0;
     }
-    __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
+    __host__ __device__ int cta_of(long long s) const { return (int)(((s + 1) * Gsk - 1) / Csk); }
 };
 
 struct Piece {
@@ -42,7 +42,7 @@ struct PieceIt {
     long long cur = -1;
 };
 
-__device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
+__host__ __device__ __forceinline__ bool next_piece(const Sched& s, PieceIt& it, Piece& pc) {
     if (it.r < s.rounds) {
         pc.unit = s.g + it.r * s.G;
         ++it.r;

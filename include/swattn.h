@@ -288,6 +288,18 @@ SW_API int sw_attn_get_table(const sw_attn_t *h, int32_t *dev_table, void *strea
 SW_API int sw_attn_cache_offsets(const sw_attn_t *h, size_t *k_offset, size_t *v_offset);
 
 /*
+ * Test hook: the pieces of the full-path schedules, enumerated on the host with the schedule code
+ * the kernels run.  schedule: SW_SCHED_PERSISTENT (units are pairs of 128-row Q tiles), SW_SCHED_TRI
+ * (units are Q tiles) or SW_SCHED_PAIR (units are pairs of Q tiles, ctas counts CTA pairs); nqt Q
+ * tiles and nt key tiles per (b, h), bh = B * H.  Writes up to cap rows of 6 int32 -- CTA (or
+ * pair) index, unit (bh-major), first and one-past-last key tile, 1 if from the stream-K phase,
+ * Q tiles of the unit that hold queries -- in CTA order and, within a CTA, in processing order.
+ * Returns the number of rows, SW_EINVAL for bad arguments, SW_ESHAPE if cap is too small.
+ * No device memory is touched.
+ */
+SW_API int sw_attn_schedule_pieces(int schedule, int nqt, int nt, int bh, int ctas, int32_t *out, int cap);
+
+/*
  * Failure-detection self-test.  Enqueues one tiny kernel that waits on an mbarrier nothing
  * will ever complete, through the same bounded wait every attention kernel uses, with a limit
  * of limit_ns (1e6 .. 2e9 ns) instead of the kernels' 1 s.  When the wait gives up it sets
