@@ -29,7 +29,12 @@ def _dev_ptr(t: torch.Tensor, name: str, dtype=None) -> int:
 
 
 class SlidingWindowAttention:
-    """Streaming block-causal attention over [condition ; sink ; window ; current chunk]."""
+    """Streaming block-causal attention over [condition ; sink ; window ; current chunk].
+
+    One handle holds one layer's cache (sw_attn_create_ex + a torch-allocated workspace).
+    schedule: "auto", "persistent", "tri", "grid" or "pair" (the full-path kernel); qk_fp8 /
+    pv_fp8: e4m3 queries and keys / values with per-tensor scales; commit_in_forward: keep a spare
+    window slot for forward_commit; commit_path: "auto", "tma" or "copy" for chunk commits."""
 
     def __init__(self, *, H: int, d: int, T: int, W: int, n_cond: int, B: int = 1,
                  sink: bool = True, out_dtype=torch.bfloat16, scale: float | None = None,
@@ -57,7 +62,7 @@ class SlidingWindowAttention:
         self.B, self.H, self.d, self.T, self.W, self.n_cond, self.sink = B, H, d, T, W, n_cond, bool(sink)
         # window slots of the ring: W, or W + 1 (a spare slot) with commit_in_forward
         self.R = W + 1 if (commit_in_forward and W > 0) else W
-        # e4m3 queries and keys (FP8 handle), bf16 otherwise; V is always bf16
+        # e4m3 queries and keys (FP8 handle), bf16 otherwise
         self.qk_fp8 = bool(qk_fp8)
         self.qk_dtype = torch.float8_e4m3fn if self.qk_fp8 else torch.bfloat16
         # e4m3 V as well (pv_fp8), bf16 otherwise

@@ -88,7 +88,8 @@ typedef struct {
     int   qk_fp8;            /* 1: queries and keys are e4m3 (OCP FP8, 1 byte per element): Q,
                                 Q_cond, K_cur, the appended K and K_cond are e4m3 tensors of
                                 the same [B, N, H, d] shape, the K cache is kept in e4m3 (half
-                                the bytes) and S = Q K^T runs on kind::f8f6f4; V stays bf16.
+                                the bytes) and S = Q K^T runs on kind::f8f6f4; V stays bf16
+                                unless pv_fp8 is set.
                                 Requires d = 128; full path on the persistent or three-buffer
                                 schedule (SW_SCHED_GRID and SW_SCHED_PAIR: SW_ESHAPE at create),
                                 short queries on the split-K path */
