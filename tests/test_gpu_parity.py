@@ -5,7 +5,10 @@ attention outputs (fp32) within max-abs 1e-2 and mean-relative 2e-3, bf16 output
 tolerance derived from those (parity_util.bf16_out_tol).  Full rows for the small workloads
 (several 128-row tiles with ragged tails); on the 480p, 720p and stress workloads, sampled rows:
 both ends, every tile edge, one random row in every 32-row quarter of every tile (every softmax
-warp of every tile), plus random rows on top.
+warp of every tile), plus random rows on top.  Every full-path schedule (persistent, grid,
+three-buffer, CTA pair) is covered, as are the split-K path, the joint and committing forwards,
+batched commits, and e4m3 handles (compared on their dequantised inputs; e4m3 P at its own
+tolerance, parity_util.E4M3_P_TOL).
 """
 from __future__ import annotations
 
