@@ -14,6 +14,8 @@ Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (b
 tiny inputs, closed forms, a library special case, four invariants).  The pages print no
 worked numeric example, so nothing is pinned against printed values; the visibility tables
 are pinned against a hand enumeration of the pages' rule in ``tests/golden/``.
+``tests/test_oracle_mutants.py`` plants plausible mistakes in a private copy of this package and
+checks that each one fails a pin.
 """
 from __future__ import annotations
 

@@ -185,6 +185,8 @@ def test_tables_brute_force(oracle_mod, W, sink):
     for k in range(40):
         vis = brute_visible(k, W, sink)
         assert [j for j in range(k) if oracle_mod.visible(k, W, sink, j)] == vis
+        # causal across chunks: neither the active chunk itself nor a later one is history
+        assert not any(oracle_mod.visible(k, W, sink, j) for j in (k, k + 1, k + W + 2, -1))
         tab = oracle_mod.table(k, W, sink, n_cond=3, T=11)
         segs = tab[3:].reshape(-1, 4)
         assert tab[0] == k and tab[1] == len(segs)
