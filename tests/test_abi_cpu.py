@@ -169,3 +169,49 @@ def test_schedule_resolution(native):
     assert L.sw_attn_schedule_for(h, 0) == native.SW_EINVAL
     assert L.sw_attn_schedule_for(None, 10) == native.SW_EINVAL
     L.sw_attn_destroy(h)
+
+
+def test_fp8_handles_halve_the_cache(native):
+    """An e4m3 K (and V) cache takes one byte per element: the K cache of a qk_fp8 handle and the
+    K and V caches of a qk_fp8 + pv_fp8 handle are half their bf16 sizes, and nothing else in the
+    workspace changes.  Host only."""
+    L = native.lib()
+    ring_half = 24 * 4 * 3180 * 128          # one of K or V in the ring, bytes at 2 B per element / 2
+    cond_half = 24 * 256 * 128
+
+    def layout(**kw):
+        rc, h = _create(native, **kw)
+        assert rc == 0, L.sw_attn_last_error()
+        ko, vo = ctypes.c_size_t(), ctypes.c_size_t()
+        assert L.sw_attn_cache_offsets(h, ctypes.byref(ko), ctypes.byref(vo)) == 0
+        ws = L.sw_attn_workspace_bytes(h)
+        L.sw_attn_destroy(h)
+        return ws, ko.value, vo.value
+
+    ws16, ko16, vo16 = layout()
+    ws8k, ko8k, vo8k = layout(qk_fp8=1)
+    ws8, ko8, vo8 = layout(qk_fp8=1, pv_fp8=1)
+    assert ko16 == ko8k == ko8                               # the state header comes first, unchanged
+    assert vo16 - ko16 == 2 * ring_half                      # bf16 K cache (already 1 KB aligned)
+    assert vo8k - ko8k == ring_half and vo8 - ko8 == ring_half
+    # K ring + K cond halve on the qk_fp8 handle; V ring + V cond too with pv_fp8
+    assert ws16 - ws8k == ring_half + cond_half
+    assert ws16 - ws8 == 2 * (ring_half + cond_half)
+
+
+def test_commit_in_forward_keeps_one_spare_slot(native):
+    """The committing forward writes the chunk into a slot its own forward does not read, so the
+    ring has W + 1 window slots (plus the sink): one more slot of K and V.  W = 0 keeps none."""
+    L = native.lib()
+    slot = 2 * 24 * 3180 * 128 * 2           # one slot of K and V, bf16
+
+    def ws(**kw):
+        rc, h = _create(native, **kw)
+        assert rc == 0, L.sw_attn_last_error()
+        n = L.sw_attn_workspace_bytes(h)
+        L.sw_attn_destroy(h)
+        return n
+
+    assert ws(commit_in_forward=1) - ws() == slot
+    assert ws(commit_in_forward=1, W=0) == ws(W=0)
+    assert ws(commit_in_forward=1, qk_fp8=1, pv_fp8=1) - ws(qk_fp8=1, pv_fp8=1) == slot // 2
