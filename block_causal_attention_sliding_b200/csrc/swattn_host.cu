@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <unordered_set>
 
 #include <cudaTypedefs.h>
 
@@ -71,6 +72,23 @@ int fail(int code, const char* fmt, ...) {
 
 int cuda_fail(cudaError_t e, const char* what) {
     return fail(SW_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// The handles created and not yet destroyed.  Every call checks its handle against this set, so
+// a destroyed (or never created) handle is refused instead of dereferenced, and a second destroy
+// does nothing.  The check cannot tell a stale handle from a newer one that was given the same
+// address by a later create.
+std::mutex g_live_mu;
+std::unordered_set<const sw_attn*> g_live;
+
+bool live(const sw_attn* h) {
+    if (!h) return false;
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    return g_live.count(h) != 0;
+}
+
+int bad_handle(const sw_attn* h) {
+    return fail(SW_EINVAL, h ? "unknown or destroyed handle" : "null handle");
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -220,6 +238,10 @@ int sw_attn_create_ex(const sw_attn_config* cfg, sw_attn_t** out) {
     h->off_sk_ml = off;  off = align_up(off + (size_t)2 * kMaxPersistentCtas * 2 * kBlockM * 2 * 4, 1024);
     h->off_sk_cnt = off; off = align_up(off + (size_t)h->n_counters * 4, 1024);
     h->total = off;
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        g_live.insert(h);
+    }
     *out = h;
     return SW_OK;
 }
@@ -235,15 +257,23 @@ int sw_attn_create(int H, int d, int tokens_per_chunk, int W, int n_cond, sw_att
     return sw_attn_create_ex(&c, out);
 }
 
-size_t sw_attn_workspace_bytes(const sw_attn_t* h) { return h ? h->total : 0; }
+size_t sw_attn_workspace_bytes(const sw_attn_t* h) { return live(h) ? h->total : 0; }
 
-int sw_attn_table_ints(const sw_attn_t* h) { return h ? h->table_ints : 0; }
+int sw_attn_table_ints(const sw_attn_t* h) { return live(h) ? h->table_ints : 0; }
 
-void sw_attn_destroy(sw_attn_t* h) { delete h; }
+void sw_attn_destroy(sw_attn_t* h) {
+    if (!h) return;
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        if (!g_live.erase(h)) return;   // unknown or already destroyed
+    }
+    delete h;
+}
 
 int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stream) {
     g_err.clear();
-    if (!h || !dev_ptr) return fail(SW_EINVAL, "null argument");
+    if (!live(h)) return bad_handle(h);
+    if (!dev_ptr) return fail(SW_EINVAL, "null argument");
     if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u) return fail(SW_EALIGN, "workspace must be 256-byte aligned");
     if (bytes < h->total) return fail(SW_ESHAPE, "workspace too small: %zu < %zu", bytes, h->total);
     int dev = 0;
@@ -332,7 +362,7 @@ int sw_attn_bind_workspace(sw_attn_t* h, void* dev_ptr, size_t bytes, void* stre
 
 int sw_attn_reset(sw_attn_t* h, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     const sw_attn_config& c = h->cfg;
     cudaError_t e = launch_state_reset(reinterpret_cast<int32_t*>(h->ws), c.W, h->R, c.sink, c.n_cond,
@@ -349,7 +379,7 @@ static TableAdvance table_advance(const sw_attn_t* h) {
 
 int sw_attn_set_cond(sw_attn_t* h, const void* K_cond, const void* V_cond, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     const sw_attn_config& c = h->cfg;
     if (c.n_cond == 0) return SW_OK;
@@ -408,7 +438,7 @@ static int launch_commit(sw_attn_t* h, const void* K, const void* V, cudaStream_
 
 int sw_attn_append_chunk(sw_attn_t* h, const void* K, const void* V, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (!K || !V) return fail(SW_EINVAL, "null K or V");
     if (!aligned16(K) || !aligned16(V)) return fail(SW_EALIGN, "K and V must be 16-byte aligned");
@@ -439,13 +469,14 @@ static int resolve_schedule(const sw_attn_t* h, int n_q) {
 
 int sw_attn_schedule_for(const sw_attn_t* h, int n_q) {
     g_err.clear();
-    if (!h || n_q < 1) return fail(SW_EINVAL, "null handle or n_q < 1");
+    if (!live(h)) return bad_handle(h);
+    if (n_q < 1) return fail(SW_EINVAL, "n_q < 1");
     return resolve_schedule(h, n_q);
 }
 
 int sw_attn_commit_kind(const sw_attn_t* h) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     return h->commit_tma ? SW_COMMIT_TMA : SW_COMMIT_COPY;
 }
@@ -544,7 +575,7 @@ static int launch_full(sw_attn_t* h, AttnParams& p, cudaStream_t st) {
 int sw_attn_forward(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out, int n_q,
                     void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");
@@ -578,11 +609,11 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
     g_err.clear();
     if (!hs || !K || !V || n < 1) return fail(SW_EINVAL, "null array or n < 1");
     const sw_attn_t* h0 = hs[0];
-    if (!h0) return fail(SW_EINVAL, "null handle 0");
+    if (!live(h0)) return fail(SW_EINVAL, h0 ? "unknown or destroyed handle 0" : "null handle 0");
     const sw_attn_config& c0 = h0->cfg;
     for (int l = 0; l < n; ++l) {
         const sw_attn_t* h = hs[l];
-        if (!h) return fail(SW_EINVAL, "null handle %d", l);
+        if (!live(h)) return fail(SW_EINVAL, h ? "unknown or destroyed handle %d" : "null handle %d", l);
         if (!h->ws) return fail(SW_ESTATE, "handle %d has no workspace bound", l);
         if (h->device != h0->device) return fail(SW_ESTATE, "handle %d is on another device", l);
         const sw_attn_config& c = h->cfg;
@@ -652,7 +683,7 @@ int sw_attn_append_chunk_batched(sw_attn_t* const* hs, int n, const void* const*
 int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur, void* out,
                            void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     const sw_attn_config& c = h->cfg;
@@ -684,7 +715,7 @@ int sw_attn_forward_commit(sw_attn_t* h, const void* Q, const void* K_cur, const
 int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const void* K_cur, const void* V_cur,
                           void* out, void* out_cond, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     const sw_attn_config& c = h->cfg;
@@ -705,7 +736,8 @@ int sw_attn_forward_joint(sw_attn_t* h, const void* Q, const void* Q_cond, const
 
 int sw_attn_get_table(const sw_attn_t* h, int32_t* dev_table, void* stream) {
     g_err.clear();
-    if (!h || !dev_table) return fail(SW_EINVAL, "null argument");
+    if (!live(h)) return bad_handle(h);
+    if (!dev_table) return fail(SW_EINVAL, "null argument");
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     cudaError_t e = cudaMemcpyAsync(dev_table, h->ws + sizeof(int32_t) * kStateHeaderInts,
                                     sizeof(int32_t) * h->table_ints, cudaMemcpyDeviceToDevice,
@@ -715,7 +747,8 @@ int sw_attn_get_table(const sw_attn_t* h, int32_t* dev_table, void* stream) {
 
 int sw_attn_cache_offsets(const sw_attn_t* h, size_t* k_offset, size_t* v_offset) {
     g_err.clear();
-    if (!h || !k_offset || !v_offset) return fail(SW_EINVAL, "null argument");
+    if (!live(h)) return bad_handle(h);
+    if (!k_offset || !v_offset) return fail(SW_EINVAL, "null argument");
     *k_offset = h->off_kcache;
     *v_offset = h->off_vcache;
     return SW_OK;
@@ -723,7 +756,7 @@ int sw_attn_cache_offsets(const sw_attn_t* h, size_t* k_offset, size_t* v_offset
 
 int sw_attn_selftest_timeout(sw_attn_t* h, int64_t limit_ns, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (limit_ns < 1000000 || limit_ns > 2000000000LL) return fail(SW_EINVAL, "limit_ns must be in [1e6, 2e9]");
     cudaError_t e = launch_selftest_timeout(reinterpret_cast<int32_t*>(h->ws) + 1, (uint64_t)limit_ns,
@@ -733,7 +766,8 @@ int sw_attn_selftest_timeout(sw_attn_t* h, int64_t limit_ns, void* stream) {
 
 int sw_attn_get_status(sw_attn_t* h, int32_t* host_status) {
     g_err.clear();
-    if (!h || !host_status) return fail(SW_EINVAL, "null argument");
+    if (!live(h)) return bad_handle(h);
+    if (!host_status) return fail(SW_EINVAL, "null argument");
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
@@ -760,7 +794,7 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 extern "C" int sw_attn_forward_short_noalloc(sw_attn_t* h, const void* Q, const void* K_cur, const void* V_cur,
                                              void* out, int n_q, void* stream) {
     g_err.clear();
-    if (!h) return fail(SW_EINVAL, "null handle");
+    if (!live(h)) return bad_handle(h);
     if (!h->ws) return fail(SW_ESTATE, "no workspace bound");
     if (!h->cond_set) return fail(SW_ESTATE, "condition tokens not set");
     if (!Q || !K_cur || !V_cur || !out) return fail(SW_EINVAL, "null tensor");

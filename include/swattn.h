@@ -32,6 +32,10 @@
  *   - One handle holds one layer's cache.  Calls on one handle must be ordered on one stream
  *     and made from one host thread at a time (the handle keeps host-side state: the tensor
  *     maps of the last inputs, reused while their pointers and row counts repeat).
+ *   - Every call checks its handle against the library's set of live handles: a null,
+ *     destroyed or never-created handle gives SW_EINVAL (0 from the size queries) and is never
+ *     dereferenced.  A later create may be given a destroyed handle's address, and the check
+ *     cannot tell the two apart, so a destroyed handle must still not be used.
  */
 #ifndef SWATTN_H
 #define SWATTN_H
@@ -53,7 +57,7 @@ typedef struct sw_attn sw_attn_t;   /* opaque handle, created and destroyed by t
 
 /* return codes */
 #define SW_OK       0
-#define SW_EINVAL  (-1)   /* null handle or pointer, bad enum, bad number */
+#define SW_EINVAL  (-1)   /* null, destroyed or unknown handle; null pointer, bad enum, bad number */
 #define SW_ESHAPE  (-2)   /* unsupported or inconsistent size */
 #define SW_EALIGN  (-3)   /* pointer or size not aligned as required */
 #define SW_ESTATE  (-4)   /* call not valid in the handle's state (no workspace, no cond) */
@@ -336,7 +340,8 @@ SW_API int sw_attn_get_status(sw_attn_t *h, int32_t *host_status);
 /* Start a new stream on the same handle: counter and status to 0, table for chunk 0. */
 SW_API int sw_attn_reset(sw_attn_t *h, void *stream);
 
-/* Free the handle (host memory only; the workspace stays the caller's). NULL is ignored. */
+/* Free the handle (host memory only; the workspace stays the caller's).  NULL, an unknown
+ * handle and a second destroy of the same handle are ignored. */
 SW_API void sw_attn_destroy(sw_attn_t *h);
 
 /* Message for the last failed call on this thread ("" if none). */

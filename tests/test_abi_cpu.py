@@ -215,3 +215,48 @@ def test_commit_in_forward_keeps_one_spare_slot(native):
     assert ws(commit_in_forward=1) - ws() == slot
     assert ws(commit_in_forward=1, W=0) == ws(W=0)
     assert ws(commit_in_forward=1, qk_fp8=1, pv_fp8=1) - ws(qk_fp8=1, pv_fp8=1) == slot // 2
+
+
+def test_destroyed_and_unknown_handles_are_refused(native):
+    """A destroyed handle, or a pointer that never was a handle, is refused by every call with
+    SW_EINVAL (0 from the size queries) before anything is dereferenced; a second destroy and the
+    destroy of an unknown pointer are ignored.  Host only."""
+    L = native.lib()
+    rc, h = _create(native, H=2, d=64, tokens_per_chunk=16, W=1, n_cond=8)
+    assert rc == 0 and L.sw_attn_workspace_bytes(h) > 0
+    L.sw_attn_destroy(h)
+    fake = ctypes.c_void_p(0x7000)           # never dereferenced: the set of live handles says no
+    dummy = ctypes.c_void_p(0x1000)
+    st = ctypes.c_int32()
+    ko, vo = ctypes.c_size_t(), ctypes.c_size_t()
+    for bad in (h, fake):
+        assert L.sw_attn_workspace_bytes(bad) == 0
+        assert L.sw_attn_table_ints(bad) == 0
+        calls = [
+            L.sw_attn_bind_workspace(bad, ctypes.c_void_p(0x10000), 1 << 30, None),
+            L.sw_attn_set_cond(bad, dummy, dummy, None),
+            L.sw_attn_append_chunk(bad, dummy, dummy, None),
+            L.sw_attn_forward(bad, dummy, dummy, dummy, dummy, 16, None),
+            L.sw_attn_forward_commit(bad, dummy, dummy, dummy, dummy, None),
+            L.sw_attn_forward_joint(bad, dummy, dummy, dummy, dummy, dummy, dummy, None),
+            L.sw_attn_forward_short_noalloc(bad, dummy, dummy, dummy, dummy, 16, None),
+            L.sw_attn_reset(bad, None),
+            L.sw_attn_get_table(bad, dummy, None),
+            L.sw_attn_get_status(bad, ctypes.byref(st)),
+            L.sw_attn_cache_offsets(bad, ctypes.byref(ko), ctypes.byref(vo)),
+            L.sw_attn_schedule_for(bad, 16),
+            L.sw_attn_commit_kind(bad),
+            L.sw_attn_selftest_timeout(bad, 1000, None),
+        ]
+        assert calls == [native.SW_EINVAL] * len(calls)
+        assert b"unknown or destroyed handle" in L.sw_attn_last_error()
+        arr = (ctypes.c_void_p * 1)(bad)
+        ptrs = (ctypes.c_void_p * 1)(dummy)
+        assert L.sw_attn_append_chunk_batched(arr, 1, ptrs, ptrs, None) == native.SW_EINVAL
+        assert b"unknown or destroyed handle 0" in L.sw_attn_last_error()
+        L.sw_attn_destroy(bad)                # ignored: destroyed before, or never created
+    # another handle created afterwards is unaffected, and is refused once destroyed in turn
+    rc, h2 = _create(native, H=2, d=64, tokens_per_chunk=16, W=1, n_cond=8)
+    assert rc == 0 and L.sw_attn_workspace_bytes(h2) > 0
+    L.sw_attn_destroy(h2)
+    assert L.sw_attn_workspace_bytes(h2) == 0
