@@ -7,7 +7,8 @@ CTA-pair (pairs of Q tiles over CTA pairs) kernels:
     slots the merging piece reads (two per CTA: 2g for its first stream-K piece, 2g + 1 for the
     other) are exactly the slots the unit's pieces wrote;
   * the live Q tiles of a unit are what its position in the head gives.
-Host only: no device memory is touched.
+Checked on the workloads' shapes, on small shapes cut into many pieces, and on 300 seeded random
+shapes per schedule.  Host only: no device memory is touched.
 """
 from __future__ import annotations
 
@@ -38,6 +39,24 @@ def pieces(kind, nqt, nt, bh, ctas):
 @pytest.mark.parametrize("nqt,nt,bh,sms", SHAPES)
 def test_schedule_covers_and_merges(name, kind, nqt, nt, bh, sms):
     ctas = sms // 2 if kind == N.SW_SCHED_PAIR else sms   # the pair kernel runs one cluster per 2 SMs
+    check_schedule(kind, nqt, nt, bh, ctas)
+
+
+@pytest.mark.parametrize("name,kind", KINDS)
+def test_schedule_random_shapes(name, kind):
+    """The same checks on 300 seeded random shapes per schedule: small and large tile counts,
+    CTA counts from 1 to above the number of units, so every mix of whole rounds, many-way
+    splits and idle CTAs comes up."""
+    rng = np.random.default_rng(20260 + kind)
+    for _ in range(300):
+        nqt = int(rng.integers(1, 40))
+        nt = int(rng.integers(1, 150))
+        bh = int(rng.integers(1, 40))
+        ctas = int(rng.integers(1, 200))
+        check_schedule(kind, nqt, nt, bh, ctas)
+
+
+def check_schedule(kind, nqt, nt, bh, ctas):
     per_bh = nqt if kind == N.SW_SCHED_TRI else (nqt + 1) // 2
     rows = pieces(kind, nqt, nt, bh, ctas)
     assert len(rows) > 0
