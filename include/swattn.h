@@ -140,7 +140,7 @@ SW_API int sw_attn_create_ex(const sw_attn_config *cfg, sw_attn_t **out);
  * Bytes of device memory the handle needs: the K and V ring caches [B][H][S][T][d] bf16 with
  * S = W + sink slots, the condition K/V [B][H][n_cond][d] bf16, the split-K partials, the
  * chunk counter, the status word and the visibility table.  Constant for the handle's life.
- * Returns 0 for a NULL handle.
+ * Returns 0 for a NULL, destroyed or unknown handle.
  */
 SW_API size_t sw_attn_workspace_bytes(const sw_attn_t *h);
 
