@@ -4,6 +4,11 @@ exp2_poly (csrc/ptx.cuh) replaces a share of the MUFU exponentials with FMA-pipe
 a Cody-Waite split x = j + f, |f| <= 1/2, a cubic for 2^f, and j added into the exponent bits.
 Its bound is pinned here by replaying the same float32 steps (fused multiply-adds rounded once)
 against numpy's exp2 in float64 over the whole input range the softmax can produce.
+
+Also here: a float64 model of the rounding of P to e4m3 (the e4m3-P tolerance), and of the
+kernels' online softmax with its lazy rescale thresholds and e4m3 weight offset (read from the
+kernel source) together with the merge of split pieces, which must give exact softmax attention
+for any split of the key tiles and keep every weight inside e4m3's range.
 """
 from __future__ import annotations
 
@@ -106,3 +111,107 @@ def test_e4m3_p_tolerance_model():
     assert eb < 2e-3, eb
     assert e8 < 3.2e-2, e8
     assert 8.0 < e8 / eb < 24.0, (eb, e8, e8 / eb)
+
+
+# ------------------------------------------------------------------ online softmax and merges
+
+def _softmax_constants():
+    """The kernels' lazy-rescale thresholds and e4m3 weight offset (log2 units), read from the
+    source so that a change there is checked here."""
+    src = open(os.path.join(ROOT, "block_causal_attention_sliding_b200", "csrc", "attn_common.cuh")).read()
+
+    def get(name):
+        return float(re.search(rf"constexpr float {name} = ([0-9.]+)f;", src).group(1))
+
+    return get("kRescaleThreshold"), get("kP8Offset"), get("kP8Threshold")
+
+
+def _online_piece(x, V, tiles, tau, off):
+    """One piece of the kernels' online softmax over the key tiles `tiles` ((lo, hi) ranges, in
+    order) for one query row, in float64: x holds the row's scores in log2 units (s * scale *
+    log2 e).  The reference max moves only when a tile's max exceeds it by more than tau; the
+    weights are 2^(x - m_ref + off).  Returns the partial (O, m_ref, l) and the largest weight."""
+    m_ref, O, l, pmax = None, np.zeros(V.shape[1]), 0.0, 0.0
+    for lo, hi in tiles:
+        m_new = x[lo:hi].max()
+        if m_ref is None:
+            m_ref = m_new
+        elif m_new > m_ref + tau:
+            f = 2.0 ** (m_ref - m_new)
+            O *= f
+            l *= f
+            m_ref = m_new
+        p = 2.0 ** (x[lo:hi] - m_ref + off)
+        pmax = max(pmax, float(p.max()))
+        O += p @ V[lo:hi]
+        l += p.sum()
+    return O, m_ref, l, pmax
+
+
+def _merge(parts):
+    """The split-K / stream-K merge of partials (O_i, m_i, l_i): rescale each to the largest m."""
+    M = max(m for _, m, _ in parts)
+    O = sum(2.0 ** (m - M) * o for o, m, _ in parts)
+    l = sum(2.0 ** (m - M) * li for _, m, li in parts)
+    return O / l
+
+
+def _score_rows(rng, n):
+    """Score rows (log2 units) that exercise the lazy rescale: Gaussian rows at the workloads'
+    logit spread, rows that climb by just under and just over the threshold per tile, a single
+    huge outlier late in the row, and falling rows."""
+    tile = 128
+    steps = np.repeat(np.arange((n + tile - 1) // tile), tile)[:n]
+    return [
+        rng.standard_normal(n) * 1.5,
+        rng.standard_normal(n) * 0.3 + steps * 7.9,          # climbs just under 2^8 per tile
+        rng.standard_normal(n) * 0.3 + steps * 8.1,          # climbs just over it
+        rng.standard_normal(n) * 0.3 + steps * 3.9,          # just under 2^4 per tile
+        np.where(np.arange(n) == n - 77, 60.0, rng.standard_normal(n)),
+        -steps * 5.0 + rng.standard_normal(n),
+    ]
+
+
+def test_online_softmax_and_merge_are_exact():
+    """The kernels' online softmax -- lazy rescale at 2^kRescaleThreshold (bf16 P) or
+    2^kP8Threshold with weights offset by 2^kP8Offset (e4m3 P) -- and the merge of split pieces
+    give exact softmax attention whatever the split, and keep every weight at most
+    2^(threshold + offset): 256 for both, below e4m3's largest finite value 448, with each row's
+    largest weight at 2^offset or more (inside e4m3's normal range, which starts at 2^-6)."""
+    tau16, off8, tau8 = _softmax_constants()
+    assert (tau16, off8, tau8) == (8.0, 4.0, 4.0)
+    rng = np.random.default_rng(11)
+    n, d = 1000, 16                       # 8 key tiles, the last one ragged (104 keys)
+    V = rng.standard_normal((n, d))
+    tiles = [(lo, min(lo + 128, n)) for lo in range(0, n, 128)]
+    for x in _score_rows(rng, n):
+        w = np.exp2(x - x.max())
+        exact = (w @ V) / w.sum()
+        for tau, off in ((tau16, 0.0), (tau8, off8)):
+            # whole row in one piece, then several random splits of the tile sequence
+            cuts_list = [[]] + [sorted(rng.choice(np.arange(1, len(tiles)), size=k, replace=False).tolist())
+                                for k in (1, 2, 4, 7) for _ in range(3)]
+            for cuts in cuts_list:
+                bounds = [0] + cuts + [len(tiles)]
+                parts, pmax = [], 0.0
+                for a, b in zip(bounds, bounds[1:]):
+                    O, m, l, pm = _online_piece(x, V, tiles[a:b], tau, off)
+                    parts.append((O, m, l))
+                    pmax = max(pmax, pm)
+                got = _merge(parts)
+                np.testing.assert_allclose(got, exact, rtol=1e-12, atol=1e-12)
+                assert pmax <= 2.0 ** (tau + off) * (1 + 1e-12)
+                assert pmax >= 2.0 ** off
+    assert 2.0 ** (tau8 + off8) < 448.0
+
+
+def test_online_softmax_threshold_is_needed():
+    """Guard for the test above: without the rescale (a reference max that never moves) the
+    weights of a climbing row overflow any bound, so the threshold is what keeps them small."""
+    rng = np.random.default_rng(3)
+    n = 1000
+    steps = np.repeat(np.arange(8), 128)[:n]
+    x = rng.standard_normal(n) * 0.3 + steps * 8.1
+    tiles = [(lo, min(lo + 128, n)) for lo in range(0, n, 128)]
+    _, _, _, pmax = _online_piece(x, np.ones((n, 1)), tiles, tau=np.inf, off=0.0)
+    assert pmax > 2.0 ** 50
