@@ -260,3 +260,31 @@ def test_destroyed_and_unknown_handles_are_refused(native):
     assert rc == 0 and L.sw_attn_workspace_bytes(h2) > 0
     L.sw_attn_destroy(h2)
     assert L.sw_attn_workspace_bytes(h2) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without the built library the binding raises at first use: there is no fallback."""
+    from block_causal_attention_sliding_b200 import _native as N
+    monkeypatch.setattr(N, "_lib", None)
+    monkeypatch.setattr(N, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libswattn.so"))
+    with pytest.raises(ImportError, match="not built"):
+        N.lib()
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package (binding, API, build, inputs) imports, loads and names nothing under oracle/."""
+    pkg = os.path.join(ROOT, "block_causal_attention_sliding_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, name), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), name
+                assert "swattn_oracle" not in text and "libswattn_oracle" not in text, name
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_api_without_a_gpu_raises():
+    """On a machine without a GPU the Python API raises when it needs the device: no CPU path."""
+    from block_causal_attention_sliding_b200.api import SlidingWindowAttention
+    with pytest.raises((RuntimeError, AssertionError)):
+        SlidingWindowAttention(H=2, d=64, T=16, W=1, n_cond=8)
