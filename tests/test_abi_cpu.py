@@ -288,3 +288,24 @@ def test_api_without_a_gpu_raises():
     from block_causal_attention_sliding_b200.api import SlidingWindowAttention
     with pytest.raises((RuntimeError, AssertionError)):
         SlidingWindowAttention(H=2, d=64, T=16, W=1, n_cond=8)
+
+
+def test_bench_reaches_the_oracle_only_from_its_baseline_legs():
+    """bench.py imports the oracle only inside the functions of its CPU-baseline and reference
+    legs, never at module level or in the CUDA arm."""
+    import ast
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py"), encoding="utf-8").read())
+    allowed = {"oracle_inputs", "cpu_baseline", "cpu_stream_ms"}
+    found = []
+
+    def visit(node, func):
+        for child in ast.iter_child_nodes(node):
+            f = child.name if isinstance(child, (ast.FunctionDef, ast.AsyncFunctionDef)) else func
+            if isinstance(child, ast.Import) and any(a.name.split(".")[0] == "oracle" for a in child.names):
+                found.append(func)
+            if isinstance(child, ast.ImportFrom) and (child.module or "").split(".")[0] == "oracle":
+                found.append(func)
+            visit(child, f)
+
+    visit(tree, None)
+    assert found and set(found) <= allowed, found
