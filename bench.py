@@ -955,6 +955,10 @@ def run_reference(args, wl, world, rank):
     would take is given separately, extrapolated from the measured throughput."""
     if rank != 0:
         return
+    # rank 0 runs alone: every host core it may run on, whatever thread count a multi-process
+    # launcher set for the job's processes
+    import oracle
+    oracle.set_num_threads(len(os.sched_getaffinity(0)))
     k = wl.steady_k()
     x = oracle_inputs(wl, k)   # the workload's inputs, resident on the host like the GPU arm's
     per_row = None

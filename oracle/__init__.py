@@ -77,6 +77,8 @@ def _load():
     lib.swo_ring_forward.argtypes = [vp, vp, i32, vp, vp, dbl, vp]
     lib.swo_ring_forward.restype = i32
     lib.swo_num_threads.restype = i32
+    lib.swo_set_num_threads.argtypes = [i32]
+    lib.swo_set_num_threads.restype = None
     _lib = lib
     return lib
 
@@ -98,6 +100,11 @@ def _ptr(a: np.ndarray | None):
 
 def num_threads() -> int:
     return int(_load().swo_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads for the oracle's calls made from this thread from now on."""
+    _load().swo_set_num_threads(int(n))
 
 
 def visible(k: int, W: int, sink: bool, j: int) -> bool:

@@ -405,3 +405,14 @@ int swo_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads for the calling thread's later parallel regions (a launcher may have set
+ * OMP_NUM_THREADS=1 for every process of a multi-process job). */
+void swo_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
