@@ -444,7 +444,7 @@ def run_cuda(args, wl, world, rank, local):
         paths["chunk_ms"] = {"median": round(statistics.median(chunk_ms), 4),
                              "p95": round(sorted(chunk_ms)[min(len(chunk_ms) - 1, int(0.95 * len(chunk_ms)))], 4),
                              "chunks": len(chunk_ms)}
-        if not args.no_extra:
+        if not args.no_extra and world == 1:   # side measurements at N = 1 only: all N GPUs are held
             h.close()
             h = None
             paths["long_horizon"] = long_horizon(args, dev, stream, pool)
@@ -455,7 +455,7 @@ def run_cuda(args, wl, world, rank, local):
 
     if rank == 0:
         cpu = None
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:   # the CPU baseline is an N = 1 figure
             try:
                 cpu = cpu_baseline_record(wl, k_start)
             except Exception as e:   # the baseline never blocks the GPU line
