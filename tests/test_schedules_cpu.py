@@ -27,11 +27,22 @@ SHAPES = [
 KINDS = [("persistent", N.SW_SCHED_PERSISTENT), ("tri", N.SW_SCHED_TRI), ("pair", N.SW_SCHED_PAIR)]
 
 
-def pieces(kind, nqt, nt, bh, ctas):
+def load_schedule_lib(path):
+    """A library built from other copies of the schedule sources (the mutation check), typed
+    like the package's own."""
+    import ctypes
+    L = ctypes.CDLL(path)
+    L.sw_attn_schedule_pieces.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int]
+    L.sw_attn_schedule_pieces.restype = ctypes.c_int
+    return L
+
+
+def pieces(kind, nqt, nt, bh, ctas, lib=None):
+    L = lib if lib is not None else N.lib()
     cap = 1 << 20
     out = np.zeros((cap, 6), dtype=np.int32)
-    n = N.lib().sw_attn_schedule_pieces(kind, nqt, nt, bh, ctas, out.ctypes.data, cap)
-    assert n >= 0, N.lib().sw_attn_last_error()
+    n = L.sw_attn_schedule_pieces(kind, nqt, nt, bh, ctas, out.ctypes.data, cap)
+    assert n >= 0, n
     return out[:n]
 
 
@@ -56,9 +67,20 @@ def test_schedule_random_shapes(name, kind):
         check_schedule(kind, nqt, nt, bh, ctas)
 
 
-def check_schedule(kind, nqt, nt, bh, ctas):
+def check_all(lib=None, n_random=100):
+    """Every check above on every fixed shape and n_random seeded random shapes per schedule."""
+    for _, kind in KINDS:
+        for nqt, nt, bh, sms in SHAPES:
+            check_schedule(kind, nqt, nt, bh, sms // 2 if kind == N.SW_SCHED_PAIR else sms, lib)
+        rng = np.random.default_rng(20260 + kind)
+        for _ in range(n_random):
+            check_schedule(kind, int(rng.integers(1, 40)), int(rng.integers(1, 150)), int(rng.integers(1, 40)),
+                           int(rng.integers(1, 200)), lib)
+
+
+def check_schedule(kind, nqt, nt, bh, ctas, lib=None):
     per_bh = nqt if kind == N.SW_SCHED_TRI else (nqt + 1) // 2
-    rows = pieces(kind, nqt, nt, bh, ctas)
+    rows = pieces(kind, nqt, nt, bh, ctas, lib)
     assert len(rows) > 0
 
     # every (unit, key tile) exactly once; a unit's pieces in consecutive CTAs, in key-tile order
