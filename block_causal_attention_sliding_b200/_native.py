@@ -24,6 +24,7 @@ EXPORTS = (
     "sw_attn_table_ints",
     "sw_attn_get_table", "sw_attn_get_status", "sw_attn_reset", "sw_attn_destroy",
     "sw_attn_last_error", "sw_attn_cache_offsets", "sw_attn_forward_short_noalloc", "sw_attn_schedule_pieces",
+    "sw_attn_table_host",
     "sw_attn_selftest_timeout", "sw_attn_schedule_for", "sw_attn_commit_kind",
 )
 
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
     L.sw_attn_cache_offsets.restype = i32
     L.sw_attn_schedule_pieces.argtypes = [i32, i32, i32, i32, i32, vp, i32]
     L.sw_attn_schedule_pieces.restype = i32
+    L.sw_attn_table_host.argtypes = [i32] * 7 + [vp, i32]
+    L.sw_attn_table_host.restype = i32
     L.sw_attn_last_error.argtypes = []
     L.sw_attn_last_error.restype = ctypes.c_char_p
     _lib = L

@@ -14,8 +14,10 @@ namespace swattn {
 // K1: advance the counter (after an append) and write the visibility table of the active
 // chunk k: [k, n_segments, N_vis, (kind, chunk_id, slot, n_tokens)...], in the order
 // condition, sink, window ascending, current; slots of a ring with R window slots; then the
-// chunk bitmap row (see table_vis_offset).  One thread: a few dozen integers.
-__device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance, int reset) {
+// chunk bitmap row (see table_vis_offset).  One thread: a few dozen integers.  Also compiled
+// for the host, where sw_attn_table_host runs it for the tests.
+__host__ __device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
+                                     int reset) {
     int32_t* tab = state + kStateHeaderInts;
     if (reset) {
         state[0] = 0;
@@ -54,6 +56,25 @@ __device__ void build_table(int32_t* state, int W, int R, int sink, int n_cond, 
     tab[cap + 1] = (int32_t)w[0];
     tab[cap + 2] = (int32_t)w[1];
 }
+
+}  // namespace swattn
+
+// Host hook: the state header and table that build_table writes for active chunk k (after an
+// advance if `advance`), run on the host with the device's own code.
+extern "C" int sw_attn_table_host(int k, int W, int R, int sink, int n_cond, int T, int advance, int32_t* out,
+                                  int cap) {
+    if (!out || k < 0 || W < 0 || W > 64 || (R != W && R != W + 1) || (W == 0 && R != 0) ||
+        (sink != 0 && sink != 1) || n_cond < 0 || T < 1 || (advance != 0 && advance != 1))
+        return SW_EINVAL;
+    const int n = swattn::kStateHeaderInts + swattn::table_ints_for(W);
+    if (cap < n) return SW_ESHAPE;
+    for (int i = 0; i < n; ++i) out[i] = 0;
+    out[0] = k;
+    swattn::build_table(out, W, R, sink, n_cond, T, advance, 0);
+    return n;
+}
+
+namespace swattn {
 
 __global__ void table_build_kernel(int32_t* state, int W, int R, int sink, int n_cond, int T, int advance,
                                    int reset) {

@@ -305,6 +305,18 @@ SW_API int sw_attn_cache_offsets(const sw_attn_t *h, size_t *k_offset, size_t *v
 SW_API int sw_attn_schedule_pieces(int schedule, int nqt, int nt, int bh, int ctas, int32_t *out, int cap);
 
 /*
+ * Test hook: the device state the table builder writes, computed on the host with the builder's
+ * own code -- the header of 16 int32 ([0] chunks committed, [1] status bits) followed by the
+ * visibility table as sw_attn_get_table returns it -- for active chunk k (k + 1 after an advance,
+ * advance = 1, as a chunk commit does), a window of W <= 64 chunks kept in R = W or W + 1 window
+ * slots (R = 0 when W = 0), sink 0 or 1, n_cond condition tokens and T tokens per chunk.
+ * Returns the number of int32 written (16 + sw_attn_table_ints for W), SW_EINVAL for bad
+ * arguments, SW_ESHAPE if cap is too small.  No device memory is touched.
+ */
+SW_API int sw_attn_table_host(int k, int W, int R, int sink, int n_cond, int T, int advance, int32_t *out,
+                              int cap);
+
+/*
  * Failure-detection self-test.  Enqueues one tiny kernel that waits on an mbarrier nothing
  * will ever complete, through the same bounded wait every attention kernel uses, with a limit
  * of limit_ns (1e6 .. 2e9 ns) instead of the kernels' 1 s.  When the wait gives up it sets
