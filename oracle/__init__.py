@@ -1,8 +1,8 @@
 """FP64 CPU oracle for block-causal sink + sliding-window attention (test infrastructure).
 
-Only the tests, the package's smoke check and the benchmark's CPU-baseline leg may import
-this package.  The product path (the CUDA library and its binding) never touches it, and it
-shares no code with that path.
+Only the tests, the package's smoke check and the benchmark's CPU-baseline and reference legs
+may import this package.  The product path (the CUDA library and its binding) never touches it,
+and it shares no code with that path.
 
 The arithmetic lives in ``swattn_oracle.c`` (plain C, double precision, OpenMP); this module
 only builds it with gcc and marshals numpy arrays.  What it computes follows the JoyAI-Video-Edit

@@ -2,7 +2,8 @@
  * swattn_oracle.c -- plain FP64 CPU oracle for block-causal sink + sliding-window attention.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call this file:
- * only the tests, the package's smoke check and the benchmark's CPU-baseline leg use it.
+ * only the tests, the package's smoke check and the benchmark's CPU-baseline and reference legs
+ * use it.
  * It shares no code, header or constant with the CUDA library.
  *
  * What it computes follows two pages about JoyAI-Video-Edit:
@@ -25,7 +26,7 @@
  *            the mask is the same for every query row (bidirectional inside the chunk).
  *   out[i]   = sum_{M[j]=1} exp(s q_i.k_j - m_i) v_j / sum_{M[j]=1} exp(s q_i.k_j - m_i)
  *
- * Readings taken where the pages are silent (each is listed in the design notes):
+ * Readings taken where the pages are silent:
  *   - W counts recent chunks only; the sink is a set union with the window, so chunk 0 is
  *     never counted twice and steady state sees W+1 history chunks.
  *   - the sink is exactly chunk 0 (all T tokens); chunk 0 as the active chunk sees the
